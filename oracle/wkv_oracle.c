@@ -1,0 +1,164 @@
+/*
+ * CPU oracle for the RWKV WKV operator: the float64 recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg load this library. The product path (the CUDA library) never
+ * links, loads or calls it, and this file shares no code with it.
+ *
+ * What it computes. "Linear attention without writing a CUDA kernel" (page 1),
+ * section "The recurrence", defines wkv_t as a weighted mean of the values: the
+ * current token enters with weight e^{u+k_t}, an earlier token i with weight
+ * e^{-(t-1-i)w + k_i}. The same section gives the constant-cost form: a carried
+ * state (numerator, denominator, max_exponent), where the max exponent is
+ * subtracted before every exponential, as in a stable softmax. One step:
+ *
+ *   output  : e = max(m, k+u);  a = exp(m-e);  b = exp(k+u-e);
+ *             out = (a*num + b*v) / (a*den + b)
+ *   advance : e' = max(m-w, k); a' = exp(m-w-e'); b' = exp(k-e');
+ *             num' = a'*num + b'*v;  den' = a'*den + b';  m' = e'
+ *
+ * This file runs that step in float64, in the order given there, one channel
+ * at a time (channels are independent: w and u are per channel). The empty
+ * state is (0, 0, -inf): the page leaves it open, and -inf makes exp(m-e) = 0,
+ * so the first output is v_1 and the first state is (v_1, 1, k_1).
+ *
+ * Inputs are fp32 or bf16 codes (widened to float64 exactly); everything after
+ * that is float64 with IEEE semantics (build without fast-math).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* element type codes of the k, v inputs */
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+static double widen(const void *p, int dtype, size_t i)
+{
+    if (dtype == ORACLE_BF16) {
+        uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)p)[i];
+}
+
+/* One token for one channel: writes the output and advances (num, den, m). */
+static double wkv_token(double kt, double vt, double w, double u,
+                        double *num, double *den, double *m)
+{
+    double kb = kt + u;                 /* exponent of the current token (with bonus) */
+    double top = fmax(*m, kb);          /* the larger exponent is subtracted from both */
+    double past = exp(*m - top);
+    double cur = exp(kb - top);
+    double out = (past * *num + cur * vt) / (past * *den + cur);
+
+    double decayed = *m - w;            /* the carried exponent after one step of decay */
+    double top2 = fmax(decayed, kt);
+    double keep = exp(decayed - top2);
+    double add = exp(kt - top2);
+    *num = keep * *num + add * vt;
+    *den = keep * *den + add;
+    *m = top2;
+    return out;
+}
+
+/*
+ * Sequence forward over k, v laid out [B, T, C] (C fastest).
+ *
+ * state_in: three [B, C] float64 arrays (num, den, max_e), or all NULL for the
+ * empty state. out: [B, T, C] float64. state_out: three [B, C] float64 arrays
+ * (may be NULL). nthreads <= 0 uses the OpenMP default.
+ */
+void wkv_oracle_forward(int64_t B, int64_t T, int64_t C,
+                        const void *k, const void *v, int kv_dtype,
+                        const float *w, const float *u,
+                        const double *num_in, const double *den_in, const double *max_in,
+                        double *out,
+                        double *num_out, double *den_out, double *max_out,
+                        int nthreads)
+{
+    const int64_t CB = 16;                       /* channels per work item */
+    const int64_t nblk = (C + CB - 1) / CB;
+    const int64_t items = B * nblk;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t it = 0; it < items; ++it) {
+        const int64_t b = it / nblk;
+        const int64_t c0 = (it % nblk) * CB;
+        const int64_t nc = (C - c0) < CB ? (C - c0) : CB;
+        double num[16], den[16], m[16], wc[16], uc[16];
+        for (int64_t j = 0; j < nc; ++j) {
+            const int64_t s = b * C + c0 + j;
+            wc[j] = (double)w[c0 + j];
+            uc[j] = (double)u[c0 + j];
+            if (num_in) {
+                num[j] = num_in[s];
+                den[j] = den_in[s];
+                m[j] = max_in[s];
+            } else {
+                num[j] = 0.0;
+                den[j] = 0.0;
+                m[j] = -INFINITY;
+            }
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            const size_t row = ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c0;
+            for (int64_t j = 0; j < nc; ++j) {
+                const double kt = widen(k, kv_dtype, row + (size_t)j);
+                const double vt = widen(v, kv_dtype, row + (size_t)j);
+                out[row + (size_t)j] = wkv_token(kt, vt, wc[j], uc[j], &num[j], &den[j], &m[j]);
+            }
+        }
+        if (num_out) {
+            for (int64_t j = 0; j < nc; ++j) {
+                const int64_t s = b * C + c0 + j;
+                num_out[s] = num[j];
+                den_out[s] = den[j];
+                max_out[s] = m[j];
+            }
+        }
+    }
+}
+
+/*
+ * One decode token for S independent streams: k, v [S, C] fp32; the state is
+ * read from (num_in, den_in, max_in) and written to (num_out, den_out,
+ * max_out), all float64 [S, C] (the two may be the same arrays).
+ */
+void wkv_oracle_step(int64_t S, int64_t C, const float *k, const float *v,
+                     const float *w, const float *u,
+                     const double *num_in, const double *den_in, const double *max_in,
+                     double *out, double *num_out, double *den_out, double *max_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < S * C; ++i) {
+        const int64_t c = i % C;
+        double num = num_in[i], den = den_in[i], m = max_in[i];
+        out[i] = wkv_token((double)k[i], (double)v[i], (double)w[c], (double)u[c], &num, &den, &m);
+        num_out[i] = num;
+        den_out[i] = den;
+        max_out[i] = m;
+    }
+}
+
+int wkv_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
