@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the WKV operator (libwkv.so) on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+wkv_forward over the workload's [B, T, C] sequence (chunked scan or
+sequential kernel, as dispatched), then one batched wkv_step decode token for
+the B streams from the returned state. Metric: WKV channel-steps per second
+(B*T*C + B*C per step), and the forward kernel's achieved HBM bandwidth against
+the measured B200 copy bandwidth.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload layer]
+    python -m torch.distributed.run --nproc-per-node N bench.py --gpus N ...
+    python bench.py --impl reference ...     # the float64 CPU oracle, timed
+
+Each rank processes its own batch (seed = rank): the work per GPU is fixed as N
+grows (weak scaling) and no collective touches the data path; ranks only meet
+at the barriers around the timed region and for the max-over-ranks timing.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "WKV channel-steps/sec (B*T*C per s) and achieved HBM GB/s vs B200 peak"
+UNIT = "channel-steps/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (also exercised on CPU with gloo by the tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def dist_init(backend: str, timeout_s: float = 120.0):
+    import datetime
+
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[int(str(device).split(":")[1])])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# workload bookkeeping
+# ---------------------------------------------------------------------------
+
+def workload_desc(wl):
+    return (f"wkv_forward {wl.kv_dtype} B={wl.B} T={wl.T} C={wl.C}"
+            f"{' (state in)' if wl.state != 'zero' else ''} + 1 wkv_step decode token")
+
+
+def units_per_step(wl) -> int:
+    return wl.B * wl.T * wl.C + wl.B * wl.C
+
+
+def forward_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one wkv_forward launch: k, v read once, out
+    written once, w and u read once, the state read (if any) and written once."""
+    kv_es = 2 if wl.kv_dtype == "bf16" else 4
+    out_es = 2 if wl.out_dtype == "bf16" else 4
+    n = wl.B * wl.T * wl.C
+    state = 12 * wl.B * wl.C
+    return n * (2 * kv_es + out_es) + state * (2 if wl.state != "zero" else 1) + 8 * wl.C
+
+
+def step_bytes(wl) -> int:
+    """One wkv_step over B x C: k, v, out and the 3-word state read and written (fp32)."""
+    return 36 * wl.B * wl.C + 8 * wl.C
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "wkv_recurrence_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded by an ncu capture under profiles/, if it
+    was taken on the current kernel sources (else None)."""
+    digest = source_digest()
+    for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        with open(p) as f:
+            for line in f:
+                m = re.match(r"traffic:\s*kernel=(\S+)\s+workload=(\S+)\s+source=(\S+)\s+bytes_per_launch=(\d+)",
+                             line.strip())
+                if m and m.group(1) == kernel and m.group(2) == workload and m.group(3) == digest:
+                    return int(m.group(4))
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="wkv_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, val in zip(names, r[5:9]) if val.lower() == "active"})
+        busy = [x for x in sm if smax and x >= 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import wkv_recurrence_b200 as W
+    from wkv_recurrence_b200 import inputs as I
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist_init("nccl")
+    wl = I.WORKLOADS[args.workload]
+    options = json.loads(args.options) if args.options else None
+
+    # synthetic inputs, one batch per rank
+    k, v = I.draw_kv(wl, seed=rank)
+    w, u = I.draw_w(wl, seed=0), I.draw_u(wl, seed=0)
+    st = I.draw_state(wl, seed=rank)
+    k1, v1 = I.draw_decode_token(wl, 0, seed=rank)
+    bf16 = wl.kv_dtype == "bf16"
+
+    def to_dev(x, as_bf16=False):
+        t = torch.from_numpy(np.ascontiguousarray(x.view(np.int16) if as_bf16 else x))
+        t = t.to(device)
+        return t.view(torch.bfloat16) if as_bf16 else t
+
+    K, V = to_dev(k, bf16), to_dev(v, bf16)
+    Wt, U = to_dev(w), to_dev(u)
+    S_in = None if st is None else tuple(to_dev(s) for s in st)
+    K1, V1 = to_dev(k1), to_dev(v1)
+    out_dtype = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
+    out = torch.empty(wl.B, wl.T, wl.C, dtype=out_dtype, device=device)
+    state = tuple(torch.empty(wl.B, wl.C, device=device) for _ in range(3))
+    out1 = torch.empty(wl.B, wl.C, device=device)
+    ws = W.make_workspace(wl.B, wl.T, wl.C, options=options, device=device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def one_step():
+        W.forward(K, V, Wt, U, S_in, out=out, state_out=state, workspace=ws, options=options)
+        W.step(state, K1, V1, Wt, U, out=out1, inplace=True)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        one_step()
+    torch.cuda.synchronize(device)
+    if W.query_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
+    sampler = ClockSampler(local_rank) if not args.no_clocks else None
+    if sampler:
+        sampler.start()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    t_wall0 = time.perf_counter()
+    for i in range(K_steps):
+        flush.zero_()  # L2 flushed between timed steps (outside the events)
+        ev[i][0].record(stream)
+        W.forward(K, V, Wt, U, S_in, out=out, state_out=state, workspace=ws, options=options)
+        ev[i][1].record(stream)
+        W.step(state, K1, V1, Wt, U, out=out1, inplace=True)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    t_wall = time.perf_counter() - t_wall0
+    clocks = sampler.stop() if sampler else None
+    if W.query_status(ws) != 0:
+        raise RuntimeError("device-side wait timed out during the timed steps")
+
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    step_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(e[0].elapsed_time(e[2]) for e in ev)
+    total_ms_max = max_over_ranks(total_ms, device)
+    units = units_per_step(wl) * K_steps * world
+    value = units / (total_ms_max / 1e3)
+
+    # roofline of the dominant kernel (the forward launch)
+    peak, peak_kind = measured_peaks()
+    fwd_mean_ms = max_over_ranks(statistics.mean(fwd_ms), device)
+    algo = forward_bytes(wl)
+    achieved = algo / (fwd_mean_ms / 1e3) / 1e9
+    kernel_name = "wkv_fwd_chunk" if (options or {}).get("kernel", 0) == 2 or (
+        (options or {}).get("kernel", 0) == 0 and not (wl.B * wl.C >= 65536 or wl.T <= 64)) else "wkv_fwd_seq"
+    traffic = recorded_traffic(kernel_name, wl.name)
+
+    # end to end through the public API: pinned host -> device, compute, device -> host
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda x: torch.from_numpy(np.ascontiguousarray(x)).pin_memory()  # noqa: E731
+        hk = pin(k.view(np.int16) if bf16 else k)
+        hv = pin(v.view(np.int16) if bf16 else v)
+        hk1, hv1 = pin(k1), pin(v1)
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hout1 = torch.empty(out1.shape).pin_memory()
+        hst = tuple(torch.empty(wl.B, wl.C).pin_memory() for _ in range(3))
+        n_e2e = max(3, min(K_steps, args.e2e_steps))
+
+        def e2e_step():
+            K.view(torch.int16 if bf16 else torch.float32).copy_(hk, non_blocking=True)
+            V.view(torch.int16 if bf16 else torch.float32).copy_(hv, non_blocking=True)
+            K1.copy_(hk1, non_blocking=True)
+            V1.copy_(hv1, non_blocking=True)
+            one_step()
+            hout.copy_(out, non_blocking=True)
+            hout1.copy_(out1, non_blocking=True)
+            for h, s in zip(hst, state):
+                h.copy_(s, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+        h2d = k.nbytes + v.nbytes + k1.nbytes + v1.nbytes
+        d2h = hout.numel() * hout.element_size() + hout1.numel() * 4 + 3 * wl.B * wl.C * 4
+        e2e = {"value": units_per_step(wl) * n_e2e * world / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
+               "ms_per_step": e2e_ms / n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
+            "warmup": max(3, args.warmup), "ms_per_step": total_ms_max / K_steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if not bf16 else "bf16-io/f32",
+            "data": "synthetic (seeded numpy draws of the workload's distributions)",
+            "config": {"workload": workload_desc(wl), "name": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+                       "kv_dtype": wl.kv_dtype, "out_dtype": wl.out_dtype, "global_batch": wl.B * world,
+                       "seq_len": wl.T, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": "flushed between timed steps (write of a buffer >= 2x L2)",
+                       "options": options or "auto"},
+            "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
+                         "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "algorithmic_bytes": algo,
+                         "launch_ms": fwd_mean_ms},
+            "decode_step_ms": statistics.mean(step_ms),
+            "forward_ms": {"mean": statistics.mean(fwd_ms), "median": statistics.median(fwd_ms),
+                           "min": min(fwd_ms)},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * K_steps, "clocks": clocks,
+            "wall_s_timed_region": t_wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle, timed (cpu_baseline leg, and the reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(wl, rows, cols, seed=0):
+    from wkv_recurrence_b200 import inputs as I
+    k, v = I.draw_kv_rows(wl, range(rows), seed=seed)
+    k, v = k[:, :, :cols].copy(), v[:, :, :cols].copy()
+    w, u = I.draw_w(wl)[:cols].copy(), I.draw_u(wl)[:cols].copy()
+    st = I.draw_state(wl, rows=range(rows), seed=seed)
+    if st is not None:
+        st = tuple(s[:, :cols].copy() for s in st)
+    k1, v1 = I.draw_decode_token(wl, 0, rows=range(rows), seed=seed)
+    return k, v, w, u, st, k1[:, :cols].copy(), v1[:, :cols].copy()
+
+
+def _oracle_step(O, sample):
+    k, v, w, u, st, k1, v1 = sample
+    _, s = O.recurrence_forward(k, v, w, u, st)
+    O.recurrence_step(s, k1, v1, w, u)
+
+
+def _pick_sample(wl, max_units):
+    """Largest (rows, channels) slice of the workload with at most max_units channel-steps."""
+    rows = wl.B
+    cols = wl.C
+    per = wl.T + 1
+    while rows * cols * per > max_units and rows > 1:
+        rows = max(1, rows // 2)
+    while rows * cols * per > max_units and cols > 16:
+        cols = max(16, cols // 2)
+    return rows, cols
+
+
+def cpu_baseline(wl, budget_s=10.0):
+    from oracle import oracle as O
+    O.build()
+    # calibrate on a small slice, then size the sample to ~budget_s of CPU work
+    rows, cols = _pick_sample(wl, 2_000_000)
+    sample = _oracle_sample(wl, rows, cols)
+    t0 = time.perf_counter()
+    _oracle_step(O, sample)
+    dt = time.perf_counter() - t0
+    rate = rows * cols * (wl.T + 1) / max(dt, 1e-6)
+    rows, cols = _pick_sample(wl, int(rate * budget_s / 3))
+    sample = _oracle_sample(wl, rows, cols)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        _oracle_step(O, sample)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    units = rows * cols * (wl.T + 1) * reps
+    return {"value": units / dt, "unit": UNIT, "cores": O.max_threads(), "kind": "oracle",
+            "sample": f"float64 C recurrence (OpenMP) on rows 0..{rows - 1}, channels 0..{cols - 1} of the "
+                      f"{wl.name} workload (T={wl.T}, plus one decode token), {reps} repetition(s), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    from wkv_recurrence_b200 import inputs as I
+    O.build()
+    wl = I.WORKLOADS[args.workload]
+    steps, warm = args.steps, max(3, args.warmup)
+    budget = float(args.reference_seconds)
+    # size each step so that warm-up + timed steps take about `budget` seconds
+    rows, cols = _pick_sample(wl, 200_000)
+    sample = _oracle_sample(wl, rows, cols)
+    t0 = time.perf_counter()
+    _oracle_step(O, sample)
+    rate = rows * cols * (wl.T + 1) / max(time.perf_counter() - t0, 1e-6)
+    per_step = max(2_000, int(rate * budget / (steps + warm)))
+    rows, cols = _pick_sample(wl, per_step)
+    sample = _oracle_sample(wl, rows, cols)
+    for _ in range(warm):
+        _oracle_step(O, sample)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        _oracle_step(O, sample)
+    dt = time.perf_counter() - t0
+    units = rows * cols * (wl.T + 1) * steps
+    value = units / dt
+    desc = (f"float64 C recurrence (OpenMP) per step on rows 0..{rows - 1}, channels 0..{cols - 1} of the "
+            f"{wl.name} workload (T={wl.T}) plus one decode token")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(wl), "name": wl.name, "B": wl.B, "T": wl.T, "C": wl.C},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.max_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="layer", help="tiny|small|layer|decode|long|mixed")
+    ap.add_argument("--options", default="", help='JSON wkv_options, e.g. {"kernel": 2, "chunk_len": 64}')
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-seconds", type=float, default=60.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    _, _, world = dist_env()
+    if world != args.gpus and args.impl == "ours" and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

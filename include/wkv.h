@@ -1,0 +1,184 @@
+/*
+ * wkv.h -- C ABI of libwkv.so, a Blackwell (sm_100a) implementation of the RWKV
+ * time-mixing WKV operator.
+ *
+ * The operation. "Linear attention without writing a CUDA kernel"
+ * (anshulranjan.vercel.app), section "The recurrence", defines for each channel
+ * c, with a per-channel decay w_c and bonus u_c,
+ *
+ *     wkv_t = ( sum_{i<t} e^{-(t-1-i)w + k_i} v_i + e^{u + k_t} v_t )
+ *           / ( sum_{i<t} e^{-(t-1-i)w + k_i}     + e^{u + k_t}     )
+ *
+ * and the same section carries the two sums forward as a state
+ * (numerator, denominator, max_exponent): the true pair is
+ * N = num * e^{max_e}, D = den * e^{max_e}. One token first forms the output
+ * from the state and the bonus-weighted current token, then decays the state by
+ * e^{-w} and adds the current token (without the bonus). A state passed in is
+ * used at the first token before any decay, exactly as the recurrence does.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers (memory the caller allocated with
+ *     cudaMalloc or a caching allocator on the current device), unless a
+ *     comment says otherwise. The caller owns every buffer; the library keeps
+ *     no pointer after the call returns and allocates no device memory.
+ *   - Layouts are dense and row-major: k, v, out are [B, T, C] with the channel
+ *     axis fastest (element (b,t,c) at (b*T + t)*C + c); w, u are [C]; each of
+ *     the three state arrays is [B, C] (or [S, C] for decode).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream). The return value reports argument checks and launch
+ *     errors only. Arguments are checked before anything is launched; a call
+ *     that returns an error has launched nothing and written nothing.
+ *   - Inputs must be finite. The empty state is (0, 0, -inf); any state with
+ *     den <= 0 or max_e = -inf is treated as empty.
+ *   - out must not overlap k, v, w, u or the state arrays.
+ *   - Results are bitwise reproducible for fixed shapes, dtypes, options and
+ *     device.
+ */
+#ifndef WKV_H
+#define WKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WKV_API __attribute__((visibility("default")))
+#else
+#define WKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WKV_OK = 0,
+    WKV_ERR_INVALID_ARG = 1,        /* negative size, NULL pointer, bad option value */
+    WKV_ERR_UNSUPPORTED_DTYPE = 2,  /* dtype combination not in the list below */
+    WKV_ERR_MISALIGNED = 3,         /* reserved: misaligned inputs take a slower path instead */
+    WKV_ERR_WORKSPACE_TOO_SMALL = 4,
+    WKV_ERR_CUDA = 5,               /* a CUDA runtime call failed (no device, launch error) */
+    WKV_ERR_WAIT_TIMEOUT = 6        /* device side: a bounded wait gave up (see wkv_query_status) */
+} wkv_status;
+
+typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
+
+/* State read by a call: three fp32 arrays (num, den, max_e), each [B, C]. */
+typedef struct {
+    const float *num;
+    const float *den;
+    const float *max_e;
+} wkv_cstate;
+
+/* State written by a call: three fp32 arrays, each [B, C]. They may be the
+ * very same arrays as a wkv_cstate of the same call (in-place update). */
+typedef struct {
+    float *num;
+    float *den;
+    float *max_e;
+} wkv_state;
+
+/*
+ * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
+ * zero-filled struct also means "defaults".
+ *   kernel          0 = choose by shape, 1 = sequential-over-T kernel,
+ *                   2 = chunked-scan kernel
+ *   chunk_len       tokens per chunk for the chunked kernel (0 = choose;
+ *                   otherwise 32, 64 or 128)
+ *   lookback_group  G: the chunked kernel publishes a running prefix every G
+ *                   chunks and each chunk combines at most G-1 chunk totals
+ *                   after the last one (0 = choose; otherwise 1..1024)
+ *   wait_timeout_ns limit of every device-side wait (0 = 1 second)
+ *   inject_enable, inject_unpublished_tile
+ *                   tests of the bounded waits only: with inject_enable = 1,
+ *                   chunk-scan tile number inject_unpublished_tile computes
+ *                   but never publishes its result, so the tiles that wait for
+ *                   it reach their wait limit, carry on, and the call reports
+ *                   WKV_ERR_WAIT_TIMEOUT through wkv_query_status. 0 = off.
+ */
+typedef struct {
+    int32_t kernel;
+    int32_t chunk_len;
+    int32_t lookback_group;
+    int32_t inject_enable;
+    int64_t wait_timeout_ns;
+    int64_t inject_unpublished_tile;
+} wkv_options;
+
+/*
+ * Bytes of workspace that wkv_forward needs for these sizes and options.
+ * Host-only; touches no device. The workspace must be zero-filled before its
+ * first use; the library leaves it ready for the next call. One workspace must
+ * not be used by two calls that may run at the same time.
+ */
+WKV_API size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const wkv_options *opts);
+
+/*
+ * Sequence forward: for every (b, c), run the recurrence over t = 0..T-1,
+ * starting from state_in (NULL = the empty state), write wkv_t to out and the
+ * state after the last token to state_out (NULL = not written).
+ *
+ *   k, v       [B, T, C], element type kv_dtype
+ *   w, u       [C] fp32: decay (the state is multiplied by e^{-w} per token)
+ *              and bonus of the current token
+ *   out        [B, T, C], element type out_dtype
+ *   state_in   NULL, or three fp32 [B, C] arrays
+ *   state_out  NULL, or three fp32 [B, C] arrays; may alias state_in
+ *   workspace  device buffer of at least wkv_forward_workspace_size() bytes,
+ *              zero-filled before its first use; it also carries the
+ *              device-side status word read by wkv_query_status
+ *   stream     cudaStream_t
+ *   opts       NULL for defaults
+ *
+ * Supported dtypes: (kv F32, out F32), (kv BF16, out BF16), (kv BF16, out F32).
+ * Sizes: B, T, C >= 0, T < 2^24, B*T*C < 2^62. T = 0 copies state_in to
+ * state_out (or writes the empty state when state_in is NULL).
+ * The state is always fp32 and the arithmetic is fp32.
+ */
+WKV_API wkv_status wkv_forward(int64_t B, int64_t T, int64_t C,
+                       const void *k, const void *v, wkv_dtype kv_dtype,
+                       const float *w, const float *u,
+                       void *out, wkv_dtype out_dtype,
+                       const wkv_cstate *state_in, const wkv_state *state_out,
+                       void *workspace, size_t workspace_bytes,
+                       void *stream, const wkv_options *opts);
+
+/*
+ * Batched one-token decode (the constant-cost step of the recurrence): S
+ * independent streams of C channels each take one token.
+ *
+ *   k, v       [S, C], element type kv_dtype
+ *   w, u       [C] fp32
+ *   out        [S, C], element type out_dtype
+ *   state_in   required: three fp32 [S, C] arrays (the empty state is allowed)
+ *   state_out  required: three fp32 [S, C] arrays; may alias state_in (in place)
+ *   stream     cudaStream_t
+ *
+ * Needs no workspace and has no device-side waits. Capture-safe: no host
+ * synchronisation and no allocation.
+ */
+WKV_API wkv_status wkv_step(int64_t S, int64_t C,
+                    const void *k, const void *v, wkv_dtype kv_dtype,
+                    const float *w, const float *u,
+                    void *out, wkv_dtype out_dtype,
+                    const wkv_cstate *state_in, const wkv_state *state_out,
+                    void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-side status word in
+ * `workspace` (a wkv_forward workspace). Returns WKV_OK, WKV_ERR_WAIT_TIMEOUT
+ * if a device-side wait of an earlier call gave up (its outputs are then not
+ * valid), or WKV_ERR_CUDA if the synchronisation itself failed.
+ */
+WKV_API wkv_status wkv_query_status(void *workspace, void *stream);
+
+/* Static English text for a status code. Host-only. */
+WKV_API const char *wkv_status_string(wkv_status status);
+
+/* Library version as 10000*major + 100*minor + patch. Host-only. */
+WKV_API int32_t wkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_H */

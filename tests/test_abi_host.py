@@ -1,0 +1,116 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/wkv.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from wkv_recurrence_b200 import _abi
+from wkv_recurrence_b200 import build as wbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wkv.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    wbuild.build()
+    return _abi.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"WKV_API\s+[\w\s\*]+?\b(wkv_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(_abi.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(7):
+        s = _abi.status_string(code)
+        assert s and s != "unknown status"
+    assert _abi.status_string(99) == "unknown status"
+    assert L.wkv_version() >= 100
+
+
+def test_workspace_size(L):
+    # sequential kernel: the 256-byte header only
+    assert L.wkv_forward_workspace_size(16, 4096, 4096, None) == 256
+    # chunked kernel: header + flags + chunk totals; grows with T
+    a = L.wkv_forward_workspace_size(8, 1024, 768, None)
+    b = L.wkv_forward_workspace_size(8, 2048, 768, None)
+    assert 256 < a < b
+    assert L.wkv_forward_workspace_size(-1, 4, 4, None) == 0
+    o = _abi.wkv_options(kernel=2, chunk_len=48)
+    assert L.wkv_forward_workspace_size(1, 64, 64, ctypes.byref(o)) == 0
+    o = _abi.wkv_options(kernel=2, chunk_len=32, lookback_group=4)
+    assert L.wkv_forward_workspace_size(1, 64, 64, ctypes.byref(o)) > 256
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails its checks first
+
+
+def fwd(L, B=1, T=4, C=8, k=FAKE, v=FAKE, kvd=0, w=FAKE, u=FAKE, out=FAKE, od=0, sin=None, sout=None,
+        ws=ctypes.c_void_p(0x100000), wsb=1 << 20, opts=None):
+    return L.wkv_forward(B, T, C, k, v, kvd, w, u, out, od, sin, sout, ws, wsb, None, opts)
+
+
+def test_forward_rejects_bad_arguments(L):
+    assert fwd(L, B=-1) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, T=-3) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, T=1 << 24) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, kvd=7) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert fwd(L, kvd=_abi.WKV_F32, od=_abi.WKV_BF16) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert fwd(L, k=None) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, out=None) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, w=None) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, ws=None) == _abi.WKV_ERR_INVALID_ARG
+    assert fwd(L, ws=ctypes.c_void_p(0x100010)) == _abi.WKV_ERR_MISALIGNED
+    assert fwd(L, T=4096, C=8, wsb=16) == _abi.WKV_ERR_WORKSPACE_TOO_SMALL
+    bad_state = _abi.wkv_cstate(0x1000, None, 0x1000)
+    assert fwd(L, sin=ctypes.byref(bad_state)) == _abi.WKV_ERR_INVALID_ARG
+    bad_out = _abi.wkv_state(0x1000, 0x1000, None)
+    assert fwd(L, sout=ctypes.byref(bad_out)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(kernel=3)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(kernel=2, chunk_len=100)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(wait_timeout_ns=-5)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(inject_enable=2)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+
+
+def test_step_rejects_bad_arguments(L):
+    s = _abi.wkv_cstate(0x1000, 0x1000, 0x1000)
+    so = _abi.wkv_state(0x1000, 0x1000, 0x1000)
+    P = ctypes.byref
+    assert L.wkv_step(-1, 4, FAKE, FAKE, 0, FAKE, FAKE, FAKE, 0, P(s), P(so), None) == _abi.WKV_ERR_INVALID_ARG
+    assert L.wkv_step(2, 4, FAKE, FAKE, 0, FAKE, FAKE, FAKE, 0, None, P(so), None) == _abi.WKV_ERR_INVALID_ARG
+    assert L.wkv_step(2, 4, FAKE, FAKE, 0, FAKE, FAKE, FAKE, 0, P(s), None, None) == _abi.WKV_ERR_INVALID_ARG
+    assert L.wkv_step(2, 4, FAKE, FAKE, 3, FAKE, FAKE, FAKE, 0, P(s), P(so), None) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert L.wkv_step(2, 4, FAKE, FAKE, 0, FAKE, FAKE, FAKE, 1, P(s), P(so), None) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert L.wkv_step(2, 4, None, FAKE, 0, FAKE, FAKE, FAKE, 0, P(s), P(so), None) == _abi.WKV_ERR_INVALID_ARG
+    # nothing to do: no device needed
+    assert L.wkv_step(0, 4, None, None, 0, None, None, None, 0, P(s), P(so), None) == _abi.WKV_OK
+
+
+def test_zero_sized_forward_needs_no_device(L):
+    assert fwd(L, B=0, k=None, v=None, out=None) == _abi.WKV_OK
+    assert fwd(L, C=0, k=None, v=None, out=None, w=None, u=None) == _abi.WKV_OK
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    import wkv_recurrence_b200 as W
+    x = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        W.forward(x, x, torch.zeros(8), torch.zeros(8))

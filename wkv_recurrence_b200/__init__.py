@@ -1,0 +1,19 @@
+"""B200 (sm_100a) implementation of the RWKV time-mixing WKV operator.
+
+The operator is the per-channel decayed weighted mean of "Linear attention
+without writing a CUDA kernel", section "The recurrence", carried as a
+(numerator, denominator, max_exponent) state. The work runs in libwkv.so
+(hand-written CUDA, C ABI in include/wkv.h); this package is its Python
+binding:
+
+    out, state = wkv_recurrence_b200.forward(k, v, w, u, state=None)
+    out, state = wkv_recurrence_b200.step(state, k, v, w, u)
+
+Importing the package does not load the library; the first call does, and
+fails loudly if it is missing or no CUDA device is present.
+"""
+
+from .api import (WkvError, forward, make_workspace, query_status, step,  # noqa: F401
+                  workspace_size)
+
+__all__ = ["forward", "step", "workspace_size", "make_workspace", "query_status", "WkvError"]

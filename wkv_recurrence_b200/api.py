@@ -1,0 +1,186 @@
+"""Python binding of libwkv.so with the same entry points as include/wkv.h.
+
+Argument marshalling only: tensors -> device pointers, the current CUDA stream,
+dtype codes. PyTorch provides device memory and streams; every step of the
+operator runs in the library's kernels. There is no fallback path: without the
+built library or a CUDA device these functions raise.
+
+The names mirror the page's step function ``wkv_step(state, k, v, w, u) ->
+(out, state)`` ("Linear attention without writing a CUDA kernel", section "The
+recurrence"): ``step`` takes and returns the (num, den, max_e) state, and
+``forward`` runs the same recurrence over a [B, T, C] sequence.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+from ._abi import WkvError  # noqa: F401
+
+State = Tuple[torch.Tensor, torch.Tensor, torch.Tensor]
+
+_DT = {torch.float32: _abi.WKV_F32, torch.bfloat16: _abi.WKV_BF16}
+_workspaces = {}
+
+
+def _dtype_code(t: torch.Tensor, name: str) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"{name}: dtype {t.dtype} is not supported (float32 or bfloat16)")
+    return _DT[t.dtype]
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _options(options: Optional[dict]):
+    if not options:
+        return None
+    o = _abi.wkv_options()
+    for key, val in options.items():
+        if not hasattr(o, key):
+            raise KeyError(f"unknown option {key!r}")
+        setattr(o, key, int(val))
+    return ctypes.byref(o)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def workspace_size(B: int, T: int, C: int, options: Optional[dict] = None) -> int:
+    """Bytes of workspace ``forward`` needs for this shape (host-only)."""
+    n = _abi.lib().wkv_forward_workspace_size(int(B), int(T), int(C), _options(options))
+    if n == 0:
+        raise ValueError("invalid sizes or options")
+    return int(n)
+
+
+def make_workspace(B: int, T: int, C: int, options: Optional[dict] = None, device=None) -> torch.Tensor:
+    """A zero-filled workspace for ``forward`` (zero once; the library keeps it ready)."""
+    return torch.zeros(workspace_size(B, T, C, options), dtype=torch.uint8,
+                       device=device if device is not None else torch.device("cuda"))
+
+
+def _default_workspace(nbytes: int, device: torch.device) -> torch.Tensor:
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def forward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+            state: Optional[State] = None, *, out_dtype: Optional[torch.dtype] = None,
+            out: Optional[torch.Tensor] = None, state_out: Optional[State] = None,
+            workspace: Optional[torch.Tensor] = None, options: Optional[dict] = None,
+            return_state: bool = True):
+    """WKV over a sequence. k, v: [B, T, C] (float32 or bfloat16); w, u: [C] float32.
+
+    state: optional (num, den, max_e), each float32 [B, C]. Returns
+    (out [B, T, C], (num, den, max_e)) -- the state after the last token.
+    """
+    _need_cuda(k, "k")
+    _need_cuda(v, "v", k.dtype)
+    _need_cuda(w, "w", torch.float32)
+    _need_cuda(u, "u", torch.float32)
+    if k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, T, C]")
+    B, T, C = k.shape
+    if w.shape != (C,) or u.shape != (C,):
+        raise ValueError("w and u must be [C]")
+    dev = k.device
+    out_dtype = out_dtype or k.dtype
+    if out is None:
+        out = torch.empty((B, T, C), dtype=out_dtype, device=dev)
+    _need_cuda(out, "out", out_dtype)
+    sin = None
+    if state is not None:
+        for i, s in enumerate(state):
+            _need_cuda(s, f"state[{i}]", torch.float32)
+            if s.shape != (B, C):
+                raise ValueError("state arrays must be [B, C]")
+        sin = _abi.wkv_cstate(*(s.data_ptr() for s in state))
+    sout = None
+    if return_state or state_out is not None:
+        if state_out is None:
+            state_out = tuple(torch.empty((B, C), dtype=torch.float32, device=dev) for _ in range(3))
+        for i, s in enumerate(state_out):
+            _need_cuda(s, f"state_out[{i}]", torch.float32)
+        sout = _abi.wkv_state(*(s.data_ptr() for s in state_out))
+    opts = _options(options)
+    need = _abi.lib().wkv_forward_workspace_size(B, T, C, opts)
+    if need == 0:
+        raise ValueError("invalid sizes or options")
+    if workspace is None:
+        workspace = _default_workspace(need, dev)
+    _need_cuda(workspace, "workspace")
+    code = _abi.lib().wkv_forward(
+        B, T, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u),
+        _ptr(out), _dtype_code(out, "out"),
+        ctypes.byref(sin) if sin is not None else None,
+        ctypes.byref(sout) if sout is not None else None,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(), opts)
+    _abi.check(code, "wkv_forward")
+    return out, state_out
+
+
+def step(state: State, k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor, *,
+         out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
+         state_out: Optional[State] = None, inplace: bool = False):
+    """One decode token for S streams. k, v: [S, C]; state: (num, den, max_e) [S, C].
+
+    Returns (out [S, C], new state). With ``inplace=True`` the state tensors
+    are updated in place and returned.
+    """
+    _need_cuda(k, "k")
+    _need_cuda(v, "v", k.dtype)
+    _need_cuda(w, "w", torch.float32)
+    _need_cuda(u, "u", torch.float32)
+    if k.dim() != 2 or v.shape != k.shape:
+        raise ValueError("k and v must both be [S, C]")
+    S, C = k.shape
+    for i, s in enumerate(state):
+        _need_cuda(s, f"state[{i}]", torch.float32)
+        if s.shape != (S, C):
+            raise ValueError("state arrays must be [S, C]")
+    out_dtype = out_dtype or k.dtype
+    if out is None:
+        out = torch.empty((S, C), dtype=out_dtype, device=k.device)
+    _need_cuda(out, "out", out_dtype)
+    if inplace:
+        state_out = state
+    elif state_out is None:
+        state_out = tuple(torch.empty_like(s) for s in state)
+    sin = _abi.wkv_cstate(*(s.data_ptr() for s in state))
+    sout = _abi.wkv_state(*(s.data_ptr() for s in state_out))
+    code = _abi.lib().wkv_step(S, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u),
+                               _ptr(out), _dtype_code(out, "out"), ctypes.byref(sin),
+                               ctypes.byref(sout), _stream())
+    _abi.check(code, "wkv_step")
+    return out, state_out
+
+
+def query_status(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream; return and clear the device-side status of a workspace."""
+    return int(_abi.lib().wkv_query_status(_ptr(workspace), _stream()))
+
+
+def empty_state(B: int, C: int, device=None) -> State:
+    """The empty state (0, 0, -inf) as three float32 [B, C] tensors."""
+    dev = device if device is not None else torch.device("cuda")
+    return (torch.zeros(B, C, device=dev), torch.zeros(B, C, device=dev),
+            torch.full((B, C), float("-inf"), device=dev))

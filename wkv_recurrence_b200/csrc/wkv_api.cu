@@ -1,0 +1,440 @@
+// C ABI of libwkv.so (declared in include/wkv.h): argument checks, the choice
+// of kernel and tile sizes, workspace layout, TMA descriptors and launches.
+// Nothing here allocates device memory; the caller passes every buffer.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/wkv.h"
+#include "wkv_device.cuh"
+#include "wkv_fwd.cuh"
+#include "wkv_step.cuh"
+
+namespace wkv {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s
+
+// ---------------------------------------------------------------------------
+// kernel configurations
+// ---------------------------------------------------------------------------
+// sequential kernel: CTA = kSeqThreads threads x VEC channels, LT-token tiles
+constexpr int kSeqThreads = 128;
+constexpr int kSeqVecF32 = 2, kSeqLtF32 = 8, kSeqStagesF32 = 4;    // 256 ch, 4 x 16 KB
+constexpr int kSeqVecBf16 = 2, kSeqLtBf16 = 16, kSeqStagesBf16 = 4;  // 256 ch, 4 x 16 KB
+constexpr int kSeqFallbackVec = 1, kSeqFallbackLt = 16;
+
+// chunked kernel: a tile is 64 channels (32 threads x 2) by L = P x J tokens
+constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
+
+struct Plan {
+  int kernel;  // 1 seq, 2 chunk
+  int L;       // chunk length (chunk kernel)
+  int G;       // look-back group
+  int NG;      // channel groups per batch row
+  int nch;     // chunks per sequence
+  long long n_tiles;
+  long long nblk;  // look-back groups per sequence
+  size_t off_flags_a, off_flags_p, off_agg_a, off_agg_p, bytes;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl) {
+  std::memset(pl, 0, sizeof *pl);
+  const int want = o ? o->kernel : 0;
+  if (want < 0 || want > 2) return false;
+  const int64_t lanes = B * C;
+  int kernel = want;
+  if (kernel == 0) kernel = (lanes >= 65536 || T <= 64) ? 1 : 2;
+  pl->kernel = kernel;
+  pl->bytes = sizeof(WsHeader);
+  if (kernel == 1) return true;
+
+  int L = o ? o->chunk_len : 0;
+  if (L == 0) L = 64;
+  if (L != 32 && L != 64 && L != 128) return false;
+  int G = o ? o->lookback_group : 0;
+  if (G == 0) G = 16;
+  if (G < 1 || G > 1024) return false;
+  pl->L = L;
+  pl->G = G;
+  pl->NG = (int)((C + kChunkCG - 1) / kChunkCG);
+  pl->nch = (int)((T + L - 1) / L);
+  const long long BNG = (long long)B * pl->NG;
+  pl->n_tiles = (long long)pl->nch * BNG;
+  if (pl->n_tiles >= (1ll << 31)) return false;
+  pl->nblk = (pl->nch + G - 1) / G;
+  size_t off = sizeof(WsHeader);
+  pl->off_flags_a = off;
+  off = round_up(off + sizeof(uint32_t) * (size_t)pl->n_tiles, 256);
+  pl->off_flags_p = off;
+  off = round_up(off + sizeof(uint32_t) * (size_t)(pl->nblk * BNG), 256);
+  pl->off_agg_a = off;
+  off = round_up(off + sizeof(float4) * (size_t)pl->n_tiles * kChunkCG, 256);
+  pl->off_agg_p = off;
+  off = round_up(off + sizeof(float4) * (size_t)(pl->nblk * BNG) * kChunkCG, 256);
+  pl->bytes = off;
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// device facts and per-kernel setup, cached per device
+// ---------------------------------------------------------------------------
+struct DevInfo {
+  int sms = 0;
+  int smem_optin = 0;
+};
+std::mutex g_mu;
+DevInfo g_dev[kMaxDevices];
+bool g_dev_ok[kMaxDevices];
+
+bool dev_info(int dev, DevInfo* out) {
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev_ok[dev]) {
+    DevInfo d;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return false;
+    g_dev[dev] = d;
+    g_dev_ok[dev] = true;
+  }
+  *out = g_dev[dev];
+  return true;
+}
+
+// Sets the dynamic shared memory limit of kernel `fn` once per device and
+// returns how many CTAs of it fit on one SM (cached per kernel and device).
+struct KernelSetup {
+  const void* fn;
+  int dev;
+  size_t smem;
+  int occ;
+};
+std::vector<KernelSetup> g_setups;
+
+template <typename F>
+bool kernel_setup(F fn, int dev, int threads, size_t smem, int* blocks_per_sm) {
+  const void* key = reinterpret_cast<const void*>(fn);
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (const KernelSetup& s : g_setups) {
+    if (s.fn == key && s.dev == dev && s.smem == smem) {
+      *blocks_per_sm = s.occ;
+      return true;
+    }
+  }
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return false;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess) return false;
+  g_setups.push_back(KernelSetup{key, dev, smem, n});
+  *blocks_per_sm = n;
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B, T, C] tensor, box [1, rows, cols] (cols contiguous)
+bool make_tmap(CUtensorMap* m, const void* base, wkv_dtype dt, int64_t B, int64_t T, int64_t C, int rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const size_t es = dt == WKV_F32 ? 4 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)(C * es), (cuuint64_t)(T * C * es)};
+  cuuint32_t box[3] = {(cuuint32_t)cols, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt == WKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+template <typename KV, typename OUT, int VEC, int LT, int STAGES, bool kTMA>
+wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
+  constexpr int CG = kSeqThreads * VEC;
+  const size_t smem = (size_t)STAGES * 2 * LT * CG * sizeof(KV) + 64 * STAGES;
+  auto fn = wkv_fwd_seq<KV, OUT, VEC, kSeqThreads, LT, STAGES, kTMA>;
+  int occ = 0;
+  if (!kernel_setup(fn, dev, kSeqThreads, smem, &occ)) return WKV_ERR_CUDA;
+  FwdParams q = p;
+  q.NG = (p.C + CG - 1) / CG;
+  const long long grid = (long long)p.B * q.NG;
+  if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  fn<<<(unsigned)grid, kSeqThreads, smem, st>>>(q, tk, tv);
+  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <typename KV, typename OUT, int P, int J, bool kTMA>
+wkv_status launch_chunk(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev,
+                        int sms) {
+  constexpr int L = P * J;
+  const size_t smem = 2ull * 2 * L * kChunkCG * sizeof(KV) + sizeof(float4) * P * kChunkCG + 64;
+  auto fn = wkv_fwd_chunk<KV, OUT, kChunkVec, kChunkRW, P, J, kTMA>;
+  int occ = 0;
+  if (!kernel_setup(fn, dev, kChunkRW * P, smem, &occ)) return WKV_ERR_CUDA;
+  if (occ < 1) return WKV_ERR_CUDA;
+  const long long grid = std::min<long long>((long long)occ * sms, p.n_tiles);
+  fn<<<(unsigned)grid, kChunkRW * P, smem, st>>>(p, tk, tv);
+  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <typename KV, typename OUT>
+wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kvdt, cudaStream_t st, int dev,
+                            int sms) {
+  CUtensorMap tk, tv;
+  std::memset(&tk, 0, sizeof tk);
+  std::memset(&tv, 0, sizeof tv);
+  if (pl.kernel == 1) {
+    constexpr bool kF32 = sizeof(KV) == 4;
+    constexpr int VEC = kF32 ? kSeqVecF32 : kSeqVecBf16;
+    constexpr int LT = kF32 ? kSeqLtF32 : kSeqLtBf16;
+    constexpr int STG = kF32 ? kSeqStagesF32 : kSeqStagesBf16;
+    if (tma) {
+      if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, kSeqThreads * VEC) ||
+          !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, kSeqThreads * VEC))
+        return WKV_ERR_CUDA;
+      return launch_seq<KV, OUT, VEC, LT, STG, true>(p, tk, tv, st, dev);
+    }
+    return launch_seq<KV, OUT, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
+  }
+  if (tma) {
+    if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
+        !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
+      return WKV_ERR_CUDA;
+    switch (pl.L) {
+      case 32: return launch_chunk<KV, OUT, 4, 8, true>(p, tk, tv, st, dev, sms);
+      case 64: return launch_chunk<KV, OUT, 8, 8, true>(p, tk, tv, st, dev, sms);
+      default: return launch_chunk<KV, OUT, 8, 16, true>(p, tk, tv, st, dev, sms);
+    }
+  }
+  switch (pl.L) {
+    case 32: return launch_chunk<KV, OUT, 4, 8, false>(p, tk, tv, st, dev, sms);
+    case 64: return launch_chunk<KV, OUT, 8, 8, false>(p, tk, tv, st, dev, sms);
+    default: return launch_chunk<KV, OUT, 8, 16, false>(p, tk, tv, st, dev, sms);
+  }
+}
+
+}  // namespace
+}  // namespace wkv
+
+using namespace wkv;
+
+extern "C" {
+
+int32_t wkv_version(void) { return 100; }
+
+const char* wkv_status_string(wkv_status s) {
+  switch (s) {
+    case WKV_OK: return "ok";
+    case WKV_ERR_INVALID_ARG: return "invalid argument";
+    case WKV_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype combination";
+    case WKV_ERR_MISALIGNED: return "misaligned pointer";
+    case WKV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case WKV_ERR_CUDA: return "CUDA runtime error";
+    case WKV_ERR_WAIT_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const wkv_options* opts) {
+  Plan pl;
+  if (B < 0 || T < 0 || C < 0 || !make_plan(B, T, C, opts, &pl)) return 0;
+  return pl.bytes;
+}
+
+wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
+                       const float* w, const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
+                       const wkv_state* state_out, void* workspace, size_t workspace_bytes, void* stream,
+                       const wkv_options* opts) {
+  // ---- argument checks: nothing is launched before they pass
+  if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
+  if (T >= (1ll << 24) || C >= (1ll << 31) || B >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  if (B > 0 && C > 0 && T > (int64_t)((1ull << 62) / (uint64_t)(B * C))) return WKV_ERR_INVALID_ARG;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (out_dtype != WKV_F32 && out_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (kv_dtype == WKV_F32 && out_dtype != WKV_F32) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (state_in && (!state_in->num || !state_in->den || !state_in->max_e)) return WKV_ERR_INVALID_ARG;
+  if (state_out && (!state_out->num || !state_out->den || !state_out->max_e)) return WKV_ERR_INVALID_ARG;
+  if (opts && opts->wait_timeout_ns < 0) return WKV_ERR_INVALID_ARG;
+  if (opts && (opts->inject_enable != 0 && opts->inject_enable != 1)) return WKV_ERR_INVALID_ARG;
+  Plan pl;
+  if (!make_plan(B, T, C, opts, &pl)) return WKV_ERR_INVALID_ARG;
+  if (!workspace) return WKV_ERR_INVALID_ARG;
+  if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
+  const int64_t n = B * T * C;
+  if (n > 0 && (!k || !v || !out)) return WKV_ERR_INVALID_ARG;
+  if (B * C > 0 && T > 0 && (!w || !u)) return WKV_ERR_INVALID_ARG;
+
+  const int64_t BC = B * C;
+  if (BC == 0) return WKV_OK;  // nothing to compute or write
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WKV_ERR_CUDA;
+  DevInfo di;
+  if (!dev_info(dev, &di)) return WKV_ERR_CUDA;
+  if (T == 0) {  // the state passes through unchanged
+    if (!state_out) return WKV_OK;
+    if (state_in) {
+      const float* src[3] = {state_in->num, state_in->den, state_in->max_e};
+      float* dst[3] = {state_out->num, state_out->den, state_out->max_e};
+      for (int i = 0; i < 3; ++i)
+        if (src[i] != dst[i] &&
+            cudaMemcpyAsync(dst[i], src[i], sizeof(float) * BC, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+          return WKV_ERR_CUDA;
+      return WKV_OK;
+    }
+    wkv_fill_empty_state<<<(unsigned)((BC + 255) / 256), 256, 0, st>>>(BC, state_out->num, state_out->den,
+                                                                      state_out->max_e);
+    return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  }
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.B = (int)B;
+  p.T = (int)T;
+  p.C = (int)C;
+  p.k = k;
+  p.v = v;
+  p.w = w;
+  p.u = u;
+  p.out = out;
+  if (state_in) {
+    p.s_num = state_in->num;
+    p.s_den = state_in->den;
+    p.s_max = state_in->max_e;
+  }
+  if (state_out) {
+    p.o_num = state_out->num;
+    p.o_den = state_out->den;
+    p.o_max = state_out->max_e;
+  }
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.hdr = reinterpret_cast<WsHeader*>(ws);
+  p.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? (uint64_t)opts->wait_timeout_ns : kDefaultTimeoutNs;
+  p.inject_tile = (opts && opts->inject_enable) ? (int)std::min<int64_t>(opts->inject_unpublished_tile, INT32_MAX) : -1;
+  if (pl.kernel == 2) {
+    p.NG = pl.NG;
+    p.nch = pl.nch;
+    p.G = pl.G;
+    p.n_tiles = (int)pl.n_tiles;
+    p.flags_a = reinterpret_cast<uint32_t*>(ws + pl.off_flags_a);
+    p.flags_p = reinterpret_cast<uint32_t*>(ws + pl.off_flags_p);
+    p.agg_a = reinterpret_cast<float4*>(ws + pl.off_agg_a);
+    p.agg_p = reinterpret_cast<float4*>(ws + pl.off_agg_p);
+  }
+  const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
+  const size_t oes = out_dtype == WKV_F32 ? 4 : 2;
+  // TMA needs 16-byte aligned bases and row pitches; otherwise the same
+  // kernels fill their tiles with plain loads
+  const bool tma = aligned(k, 16) && aligned(v, 16) && (C * kes) % 16 == 0;
+  const int vec = pl.kernel == 1 ? (tma ? (kv_dtype == WKV_F32 ? kSeqVecF32 : kSeqVecBf16) : kSeqFallbackVec)
+                                 : kChunkVec;
+  p.vec_store = aligned(out, oes * vec) && (C % vec) == 0;
+
+  if (kv_dtype == WKV_F32) return dispatch_forward<float, float>(pl, p, tma, kv_dtype, st, dev, di.sms);
+  if (out_dtype == WKV_BF16)
+    return dispatch_forward<__nv_bfloat16, __nv_bfloat16>(pl, p, tma, kv_dtype, st, dev, di.sms);
+  return dispatch_forward<__nv_bfloat16, float>(pl, p, tma, kv_dtype, st, dev, di.sms);
+}
+
+wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype, const float* w,
+                    const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
+                    const wkv_state* state_out, void* stream) {
+  if (S < 0 || C < 0) return WKV_ERR_INVALID_ARG;
+  if (S > 0 && C > (int64_t)((1ull << 62) / (uint64_t)S)) return WKV_ERR_INVALID_ARG;
+  if (C >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (out_dtype != WKV_F32 && out_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (kv_dtype == WKV_F32 && out_dtype != WKV_F32) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (!state_in || !state_out) return WKV_ERR_INVALID_ARG;
+  if (!state_in->num || !state_in->den || !state_in->max_e) return WKV_ERR_INVALID_ARG;
+  if (!state_out->num || !state_out->den || !state_out->max_e) return WKV_ERR_INVALID_ARG;
+  const int64_t n = S * C;
+  if (n == 0) return WKV_OK;
+  if (!k || !v || !w || !u || !out) return WKV_ERR_INVALID_ARG;
+
+  StepParams p;
+  p.n = n;
+  p.C = (int)C;
+  p.k = k;
+  p.v = v;
+  p.w = w;
+  p.u = u;
+  p.out = out;
+  p.s_num = state_in->num;
+  p.s_den = state_in->den;
+  p.s_max = state_in->max_e;
+  p.o_num = state_out->num;
+  p.o_den = state_out->den;
+  p.o_max = state_out->max_e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t kes = kv_dtype == WKV_F32 ? 4 : 2, oes = out_dtype == WKV_F32 ? 4 : 2;
+  constexpr int VEC = 4;
+  const bool vec = (C % VEC) == 0 && aligned(k, kes * VEC) && aligned(v, kes * VEC) && aligned(out, oes * VEC) &&
+                   aligned(w, 16) && aligned(u, 16) && aligned(p.s_num, 16) && aligned(p.s_den, 16) &&
+                   aligned(p.s_max, 16) && aligned(p.o_num, 16) && aligned(p.o_den, 16) && aligned(p.o_max, 16);
+  const int per = vec ? VEC : 1;
+  const long long threads = (n + per - 1) / per;
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  if (kv_dtype == WKV_F32) {
+    if (vec) wkv_step_kernel<float, float, VEC><<<blocks, 256, 0, st>>>(p);
+    else wkv_step_kernel<float, float, 1><<<blocks, 256, 0, st>>>(p);
+  } else if (out_dtype == WKV_BF16) {
+    if (vec) wkv_step_kernel<__nv_bfloat16, __nv_bfloat16, VEC><<<blocks, 256, 0, st>>>(p);
+    else wkv_step_kernel<__nv_bfloat16, __nv_bfloat16, 1><<<blocks, 256, 0, st>>>(p);
+  } else {
+    if (vec) wkv_step_kernel<__nv_bfloat16, float, VEC><<<blocks, 256, 0, st>>>(p);
+    else wkv_step_kernel<__nv_bfloat16, float, 1><<<blocks, 256, 0, st>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+wkv_status wkv_query_status(void* workspace, void* stream) {
+  if (!workspace) return WKV_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return WKV_ERR_CUDA;
+  WsHeader* h = static_cast<WsHeader*>(workspace);
+  uint32_t bits = 0;
+  if (cudaMemcpy(&bits, &h->status, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess) return WKV_ERR_CUDA;
+  if (bits) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(&h->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return WKV_ERR_CUDA;
+  }
+  return (bits & kStatusWaitTimeout) ? WKV_ERR_WAIT_TIMEOUT : WKV_OK;
+}
+
+}  // extern "C"
