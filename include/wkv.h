@@ -164,6 +164,38 @@ WKV_API wkv_status wkv_step(int64_t S, int64_t C,
                     void *stream);
 
 /*
+ * wkv_forward without a caller-provided workspace. The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory themselves: hosts that hand a plug-in only its input and
+ * output buffers while their own pool owns the rest of the GPU, and code with
+ * hard latency limits, where cudaMalloc's implicit synchronisation of the
+ * device is not acceptable.
+ *
+ * Same arguments and results as wkv_forward with default options, except that
+ * the scratch memory lives in a fixed array of WKV_NOALLOC_SCRATCH_BYTES bytes
+ * inside the library (every GPU that loads the library holds it until the
+ * process exits). The call allocates nothing.
+ *   - Shapes whose scratch need (wkv_forward_workspace_size(B, T, C, NULL))
+ *     exceeds WKV_NOALLOC_SCRATCH_BYTES are rejected with
+ *     WKV_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call zeroes the array's counters and flags on `stream` before its
+ *     kernel runs. All calls share the one array: two calls that may overlap on
+ *     the GPU (different streams, or different host threads) race and give
+ *     wrong results; serialise them.
+ *   - Device-side wait timeouts are not reported through this entry point
+ *     (there is no workspace to query); the waits still end at their limit.
+ */
+#define WKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+WKV_API wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C,
+                               const void *k, const void *v, wkv_dtype kv_dtype,
+                               const float *w, const float *u,
+                               void *out, wkv_dtype out_dtype,
+                               const wkv_cstate *state_in, const wkv_state *state_out,
+                               void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device-side status word in
  * `workspace` (a wkv_forward workspace). Returns WKV_OK, WKV_ERR_WAIT_TIMEOUT
  * if a device-side wait of an earlier call gave up (its outputs are then not

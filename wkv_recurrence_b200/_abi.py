@@ -24,7 +24,10 @@ WKV_BF16 = 1
 
 # entry points declared in include/wkv.h
 EXPORTS = ("wkv_forward_workspace_size", "wkv_forward", "wkv_step", "wkv_query_status",
-           "wkv_status_string", "wkv_version")
+           "wkv_status_string", "wkv_version", "wkv_forward_noalloc")
+
+# size of the library's built-in scratch array used by wkv_forward_noalloc
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class wkv_cstate(ctypes.Structure):
@@ -67,6 +70,9 @@ def lib() -> ctypes.CDLL:
         L.wkv_step.argtypes = [I64, I64, P, P, I, P, P, P, I,
                                ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P]
         L.wkv_step.restype = I
+        L.wkv_forward_noalloc.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
+                                          ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P]
+        L.wkv_forward_noalloc.restype = I
         L.wkv_query_status.argtypes = [P, P]
         L.wkv_query_status.restype = I
         L.wkv_status_string.argtypes = [I]

@@ -437,4 +437,60 @@ wkv_status wkv_query_status(void* workspace, void* stream) {
   return (bits & kStatusWaitTimeout) ? WKV_ERR_WAIT_TIMEOUT : WKV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// wkv_forward_noalloc: wkv_forward with its scratch in a fixed device array
+// ---------------------------------------------------------------------------
+// For callers that cannot allocate device memory (a host that owns all of it
+// and passes in only inputs and outputs; latency-bound code that must not take
+// cudaMalloc's device-wide synchronisation). The array is zero at module load;
+// each call zeroes the counters and flags its kernel relies on, then runs the
+// ordinary forward path on the array. Calls share the array, so calls that
+// overlap on the GPU race.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[WKV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[wkv::kMaxDevices];
+
+// Device address of g_noalloc_scratch on `dev` (the current device), looked up
+// once per device. In host code the array's name is only a stand-in for the
+// symbol, never a usable device address.
+bool noalloc_scratch(int dev, void** ptr) {
+  if (dev < 0 || dev >= wkv::kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(wkv::g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return false;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return true;
+}
+}  // namespace
+
+wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
+                               const float* w, const float* u, void* out, wkv_dtype out_dtype,
+                               const wkv_cstate* state_in, const wkv_state* state_out, void* stream) {
+  if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
+  Plan pl;
+  if (!make_plan(B, T, C, nullptr, &pl)) return WKV_ERR_INVALID_ARG;
+  if (pl.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_WORKSPACE_TOO_SMALL;
+  if (B * C == 0) {
+    // nothing to compute: wkv_forward checks the other arguments and returns
+    // before it would look at a workspace, so no device (and no scratch
+    // address) is needed; 256 only satisfies its alignment check
+    return wkv_forward(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out,
+                       reinterpret_cast<void*>(uintptr_t(256)), WKV_NOALLOC_SCRATCH_BYTES, stream, nullptr);
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WKV_ERR_CUDA;
+  void* scratch = nullptr;
+  if (!noalloc_scratch(dev, &scratch)) return WKV_ERR_CUDA;
+  // counters, epoch, status and flags start at zero for this call
+  const size_t clear = pl.kernel == 2 ? pl.off_agg_a : sizeof(WsHeader);
+  if (cudaMemsetAsync(scratch, 0, clear, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WKV_ERR_CUDA;
+  return wkv_forward(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, scratch,
+                     WKV_NOALLOC_SCRATCH_BYTES, stream, nullptr);
+}
+
 }  // extern "C"
