@@ -96,6 +96,17 @@ def workload_desc(wl):
             f"{' (state in)' if wl.state != 'zero' else ''} + 1 wkv_step decode token")
 
 
+def workload(args):
+    """The named workload, with B and/or T overridden for profiling runs."""
+    import dataclasses
+
+    from wkv_recurrence_b200 import inputs as I
+    wl = I.WORKLOADS[args.workload]
+    if args.batch or args.tokens:
+        wl = dataclasses.replace(wl, B=args.batch or wl.B, T=args.tokens or wl.T)
+    return wl
+
+
 def units_per_step(wl) -> int:
     return wl.B * wl.T * wl.C + wl.B * wl.C
 
@@ -219,7 +230,7 @@ def run_ours(args):
     device = torch.device("cuda", local_rank)
     if world > 1:
         dist_init("nccl")
-    wl = I.WORKLOADS[args.workload]
+    wl = workload(args)
     options = json.loads(args.options) if args.options else None
 
     # synthetic inputs, one batch per rank
@@ -247,9 +258,13 @@ def run_ours(args):
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
+    # arguments checked and marshalled once; each call below is one C-ABI call
+    fwd = W.PreparedForward(K, V, Wt, U, S_in, out=out, state_out=state, workspace=ws, options=options)
+    dec = W.PreparedStep(state, K1, V1, Wt, U, out=out1)
+
     def one_step():
-        W.forward(K, V, Wt, U, S_in, out=out, state_out=state, workspace=ws, options=options)
-        W.step(state, K1, V1, Wt, U, out=out1, inplace=True)
+        fwd()
+        dec()
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -269,9 +284,9 @@ def run_ours(args):
     for i in range(K_steps):
         flush.zero_()  # L2 flushed between timed steps (outside the events)
         ev[i][0].record(stream)
-        W.forward(K, V, Wt, U, S_in, out=out, state_out=state, workspace=ws, options=options)
+        fwd()
         ev[i][1].record(stream)
-        W.step(state, K1, V1, Wt, U, out=out1, inplace=True)
+        dec()
         ev[i][2].record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -436,7 +451,7 @@ def run_reference(args):
     from oracle import oracle as O
     from wkv_recurrence_b200 import inputs as I
     O.build()
-    wl = I.WORKLOADS[args.workload]
+    wl = workload(args)
     steps, warm = args.steps, max(3, args.warmup)
     budget = float(args.reference_seconds)
     # size each step so that warm-up + timed steps take about `budget` seconds
@@ -476,6 +491,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="layer", help="tiny|small|layer|decode|long|mixed")
     ap.add_argument("--options", default="", help='JSON wkv_options, e.g. {"kernel": 2, "chunk_len": 64}')
+    ap.add_argument("--batch", type=int, default=0, help="override B of the workload (profiling)")
+    ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)

@@ -81,13 +81,19 @@ typedef struct {
  * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
  * zero-filled struct also means "defaults".
  *   kernel          0 = choose by shape, 1 = sequential-over-T kernel,
- *                   2 = chunked-scan kernel
- *   chunk_len       tokens per chunk for the chunked kernel (0 = choose;
+ *                   2 = chunked scan in one launch (look-back between CTAs),
+ *                   3 = chunked scan in two launches (chunk totals, then
+ *                   replay; for inputs that stay in L2 between them)
+ *   chunk_len       tokens per chunk for the chunked kernels (0 = choose;
  *                   otherwise 32, 64 or 128)
  *   lookback_group  G: the chunked kernel publishes a running prefix every G
  *                   chunks and each chunk combines at most G-1 chunk totals
  *                   after the last one (0 = choose; otherwise 1..1024)
  *   wait_timeout_ns limit of every device-side wait (0 = 1 second)
+ *   span            tokens per warp in a chunk-scan tile, 8 or 16 (0 = choose);
+ *                   chunk_len / span warps share a tile
+ *   seq_threads     threads per CTA of the sequential kernel: 32, 64 or 128
+ *                   (0 = choose); each thread carries 2 channels
  *   inject_enable, inject_unpublished_tile
  *                   tests of the bounded waits only: with inject_enable = 1,
  *                   chunk-scan tile number inject_unpublished_tile computes
@@ -102,6 +108,8 @@ typedef struct {
     int32_t inject_enable;
     int64_t wait_timeout_ns;
     int64_t inject_unpublished_tile;
+    int32_t span;
+    int32_t seq_threads;
 } wkv_options;
 
 /*

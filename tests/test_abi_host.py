@@ -79,13 +79,17 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, sin=ctypes.byref(bad_state)) == _abi.WKV_ERR_INVALID_ARG
     bad_out = _abi.wkv_state(0x1000, 0x1000, None)
     assert fwd(L, sout=ctypes.byref(bad_out)) == _abi.WKV_ERR_INVALID_ARG
-    o = _abi.wkv_options(kernel=3)
+    o = _abi.wkv_options(kernel=4)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(kernel=2, chunk_len=100)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(wait_timeout_ns=-5)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(inject_enable=2)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(kernel=2, span=12)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(kernel=1, seq_threads=48)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
 
 

@@ -20,6 +20,9 @@ pytestmark = pytest.mark.gpu
 
 SEQ = {"kernel": 1}
 CHUNK = {"kernel": 2}
+TWO = {"kernel": 3}
+KERNELS = [SEQ, CHUNK, TWO]
+KIDS = ["seq", "chunk", "two"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -58,8 +61,12 @@ def compare(oracle, k, v, w, u, state=None, kv="f32", out_dtype=None, options=No
 
 @pytest.mark.parametrize("opts", [None, SEQ, CHUNK, {"kernel": 2, "chunk_len": 32, "lookback_group": 1},
                                   {"kernel": 2, "chunk_len": 128, "lookback_group": 3},
-                                  {"kernel": 2, "chunk_len": 32, "lookback_group": 5}],
-                         ids=["auto", "seq", "chunk64", "chunk32g1", "chunk128g3", "chunk32g5"])
+                                  {"kernel": 2, "chunk_len": 32, "lookback_group": 5, "span": 8},
+                                  {"kernel": 2, "chunk_len": 64, "span": 8},
+                                  TWO, {"kernel": 3, "chunk_len": 32, "span": 8},
+                                  {"kernel": 3, "chunk_len": 64}],
+                         ids=["auto", "seq", "chunk128", "chunk32g1", "chunk128g3", "chunk32g5s8", "chunk64s8",
+                              "two128", "two32s8", "two64"])
 @pytest.mark.parametrize("shape", [(1, 1, 64), (2, 33, 64), (3, 1000, 128), (2, 517, 200), (1, 2048, 64)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_random_f32(oracle, opts, shape):
@@ -69,7 +76,7 @@ def test_random_f32(oracle, opts, shape):
     compare(oracle, k, v, w, u, st, options=opts)
 
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("C", [1, 5, 127, 130])
 def test_ragged_channels_plain_load_path(oracle, opts, C):
     """C * 4 bytes not a multiple of 16: the kernels fill tiles with plain loads."""
@@ -77,7 +84,7 @@ def test_ragged_channels_plain_load_path(oracle, opts, C):
     compare(oracle, k, v, w, u, st, options=opts)
 
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_misaligned_pointers(oracle, opts):
     B, T, C = 2, 257, 64
     k, v, w, u, _ = I.random_case(B, T, C, seed=77)
@@ -92,7 +99,7 @@ def test_misaligned_pointers(oracle, opts):
 
 
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_bf16_inputs(oracle, out_dtype, opts):
     k, v, w, u, st = I.random_case(2, 700, 128, seed=5, k_scale=4.0, state=True)
     kb, vb = I.f32_to_bf16_bits(2.0 * k), I.f32_to_bf16_bits(v)
@@ -104,7 +111,7 @@ def test_bf16_inputs(oracle, out_dtype, opts):
 # special cases with closed forms
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_first_token_and_constant_v(oracle, opts):
     k, v, w, u, _ = I.random_case(1, 200, 64, seed=9, k_scale=3.0)
     v[:] = np.float32(0.625)
@@ -116,14 +123,14 @@ def test_first_token_and_constant_v(oracle, opts):
     assert np.allclose(st1[2], k[:, 0], rtol=1e-6, atol=1e-6)
 
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("mag", [60.0, 100.0, 1000.0])
 def test_extreme_keys_stay_finite(oracle, opts, mag):
     k, v, w, u, st = I.random_case(2, 600, 64, seed=int(mag), k_spike=mag, w_range=(1e-4, 4.0), state=True)
     compare(oracle, k, v, w, u, st, options=opts, rtol=RTOL_F32 if mag < 200 else 1e-4)
 
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_large_decay_and_bonus_limits(oracle, opts):
     k, v, w, u, _ = I.random_case(1, 300, 64, seed=11, k_scale=3.0)
     w[:] = np.float32(1e4)
@@ -136,7 +143,7 @@ def test_large_decay_and_bonus_limits(oracle, opts):
     compare(oracle, k, v, w, u, options=opts)
 
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_empty_sequence(oracle, opts):
     B, C = 3, 64
     st = tuple(dev_f32(np.full((B, C), x, np.float32)) for x in (0.5, 2.0, 1.25))
@@ -149,7 +156,7 @@ def test_empty_sequence(oracle, opts):
     assert torch.all(so[0] == 0) and torch.all(so[1] == 0) and torch.all(so[2] == float("-inf"))
 
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_empty_state_forms_are_equivalent(oracle, opts):
     """An explicit (0, 0, -inf) state behaves like no state."""
     k, v, w, u, _ = I.random_case(2, 130, 64, seed=13)
@@ -165,7 +172,7 @@ def test_empty_state_forms_are_equivalent(oracle, opts):
 # structure: resume from a state, step vs forward, kernels agree, determinism
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("opts", [SEQ, CHUNK], ids=["seq", "chunk"])
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
 def test_split_and_resume(oracle, opts):
     k, v, w, u, st = I.random_case(2, 1500, 128, seed=17, k_spike=40.0, w_range=(1e-4, 4.0), state=True)
     o1, s1 = run_forward(k[:, :611], v[:, :611], w, u, st, options=opts)
@@ -177,10 +184,13 @@ def test_split_and_resume(oracle, opts):
     assert_state(s2, rst, sst[0], RTOL_F32)
 
 
-def test_in_place_state(oracle):
-    k, v, w, u, st = I.random_case(2, 400, 64, seed=19, state=True)
+@pytest.mark.parametrize("opts", [SEQ, {"kernel": 2, "chunk_len": 32}, {"kernel": 3, "chunk_len": 32}],
+                         ids=KIDS)
+def test_in_place_state(oracle, opts):
+    """state_out aliases state_in; the chunked kernels use many chunks here."""
+    k, v, w, u, st = I.random_case(2, 1000, 128, seed=19, state=True)
     S = tuple(dev_f32(s) for s in st)
-    out, so = W.forward(dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u), S, state_out=S)
+    out, so = W.forward(dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u), S, state_out=S, options=opts)
     assert all(a.data_ptr() == b.data_ptr() for a, b in zip(so, S))
     ref, rst = oracle.recurrence_forward(k, v, w, u, st)
     sc, sst = oracle.abs_scale_forward(k, v, w, u, st)
@@ -240,23 +250,24 @@ def test_step_from_empty_state(oracle):
 
 def test_kernels_agree_and_are_deterministic(oracle):
     k, v, w, u, st = I.random_case(4, 3000, 192, seed=37, k_spike=50.0, w_range=(1e-4, 8.0), state=True)
-    a1, sa1 = run_forward(k, v, w, u, st, options=SEQ)
-    a2, sa2 = run_forward(k, v, w, u, st, options=SEQ)
-    c1, sc1 = run_forward(k, v, w, u, st, options=CHUNK)
-    c2, sc2 = run_forward(k, v, w, u, st, options=CHUNK)
-    assert np.array_equal(a1, a2) and np.array_equal(c1, c2)
-    for x, y in zip(sc1, sc2):
-        assert np.array_equal(x, y)
     sc, _ = oracle.abs_scale_forward(k, v, w, u, st)
-    assert np.all(np.abs(a1 - c1) <= 2 * RTOL_F32 * sc)
+    a1, _ = run_forward(k, v, w, u, st, options=SEQ)
+    for opts in KERNELS + [{"kernel": 2, "chunk_len": 32, "lookback_group": 3}]:
+        r1, s1 = run_forward(k, v, w, u, st, options=opts)
+        r2, s2 = run_forward(k, v, w, u, st, options=opts)
+        assert np.array_equal(r1, r2), opts
+        for x, y in zip(s1, s2):
+            assert np.array_equal(x, y), opts
+        assert np.all(np.abs(a1 - r1) <= 2 * RTOL_F32 * sc), opts
 
 
-def test_workspace_reuse_across_shapes(oracle):
+@pytest.mark.parametrize("opts", [CHUNK, TWO], ids=["chunk", "two"])
+def test_workspace_reuse_across_shapes(oracle, opts):
     """One workspace serves successive calls of different shapes (the epoch scheme)."""
-    ws = W.make_workspace(4, 4096, 256, options=CHUNK)
+    ws = W.make_workspace(4, 4096, 256, options=opts)
     for (B, T, C) in [(4, 4096, 256), (2, 1000, 64), (4, 4096, 256), (1, 2500, 192)]:
         k, v, w, u, _ = I.random_case(B, T, C, seed=B + T + C)
-        out, _ = W.forward(dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u), workspace=ws, options=CHUNK)
+        out, _ = W.forward(dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u), workspace=ws, options=opts)
         assert W.query_status(ws) == 0
         ref, _ = oracle.recurrence_forward(k, v, w, u)
         sc, _ = oracle.abs_scale_forward(k, v, w, u)
@@ -319,7 +330,7 @@ def test_workload_full_size(oracle, name):
 def test_tiny_against_decimal_golden():
     from test_oracle_pins import load_golden
     k, v, w, u, ref = load_golden()
-    for opts in (None, SEQ, CHUNK):
+    for opts in (None, SEQ, CHUNK, TWO):
         out, _ = run_forward(k, v, w, u, options=opts)
         assert np.allclose(out, ref, rtol=RTOL_F32, atol=RTOL_F32 * np.abs(v).max())
 

@@ -13,7 +13,8 @@ Importing the package does not load the library; the first call does, and
 fails loudly if it is missing or no CUDA device is present.
 """
 
-from .api import (WkvError, forward, make_workspace, query_status, step,  # noqa: F401
-                  workspace_size)
+from .api import (PreparedForward, PreparedStep, WkvError, empty_state, forward,  # noqa: F401
+                  make_workspace, query_status, step, workspace_size)
 
-__all__ = ["forward", "step", "workspace_size", "make_workspace", "query_status", "WkvError"]
+__all__ = ["forward", "step", "workspace_size", "make_workspace", "query_status", "empty_state",
+           "PreparedForward", "PreparedStep", "WkvError"]

@@ -184,3 +184,92 @@ def empty_state(B: int, C: int, device=None) -> State:
     dev = device if device is not None else torch.device("cuda")
     return (torch.zeros(B, C, device=dev), torch.zeros(B, C, device=dev),
             torch.full((B, C), float("-inf"), device=dev))
+
+
+class PreparedForward:
+    """``forward`` with its arguments checked and marshalled once.
+
+    For loops that call the operator on the same buffers again and again
+    (benchmarks, decode loops, CUDA-graph capture): ``__call__`` is a single
+    C-ABI call with the stored pointers, on the stream current at preparation
+    time unless another is passed.
+    """
+
+    def __init__(self, k, v, w, u, state=None, *, out, state_out=None, workspace=None,
+                 options: Optional[dict] = None):
+        _need_cuda(k, "k")
+        _need_cuda(v, "v", k.dtype)
+        _need_cuda(w, "w", torch.float32)
+        _need_cuda(u, "u", torch.float32)
+        B, T, C = k.shape
+        if v.shape != k.shape or w.shape != (C,) or u.shape != (C,) or out.shape != k.shape:
+            raise ValueError("shapes must be k, v, out [B, T, C] and w, u [C]")
+        _need_cuda(out, "out")
+        self._keep = [k, v, w, u, out]
+        self._sin = self._sout = None
+        if state is not None:
+            for i, s in enumerate(state):
+                _need_cuda(s, f"state[{i}]", torch.float32)
+            self._sin = _abi.wkv_cstate(*(s.data_ptr() for s in state))
+            self._keep += list(state)
+        if state_out is not None:
+            for i, s in enumerate(state_out):
+                _need_cuda(s, f"state_out[{i}]", torch.float32)
+            self._sout = _abi.wkv_state(*(s.data_ptr() for s in state_out))
+            self._keep += list(state_out)
+        self._opts_struct = None
+        if options:
+            self._opts_struct = _abi.wkv_options()
+            for key, val in options.items():
+                setattr(self._opts_struct, key, int(val))
+        opts = ctypes.byref(self._opts_struct) if self._opts_struct is not None else None
+        need = _abi.lib().wkv_forward_workspace_size(B, T, C, opts)
+        if need == 0:
+            raise ValueError("invalid sizes or options")
+        if workspace is None:
+            workspace = make_workspace(B, T, C, options, device=k.device)
+        _need_cuda(workspace, "workspace")
+        self.workspace = workspace
+        self._keep.append(workspace)
+        self._fn = _abi.lib().wkv_forward
+        self._args = (B, T, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u), _ptr(out),
+                      _dtype_code(out, "out"),
+                      ctypes.byref(self._sin) if self._sin is not None else None,
+                      ctypes.byref(self._sout) if self._sout is not None else None,
+                      _ptr(workspace), workspace.numel() * workspace.element_size())
+        self._stream = _stream()
+        self._opts = opts
+
+    def __call__(self, stream=None) -> None:
+        code = self._fn(*self._args, self._stream if stream is None else stream, self._opts)
+        if code:
+            _abi.check(code, "wkv_forward")
+
+
+class PreparedStep:
+    """``step`` with its arguments checked and marshalled once (see PreparedForward)."""
+
+    def __init__(self, state, k, v, w, u, *, out, state_out=None):
+        _need_cuda(k, "k")
+        _need_cuda(v, "v", k.dtype)
+        _need_cuda(w, "w", torch.float32)
+        _need_cuda(u, "u", torch.float32)
+        _need_cuda(out, "out")
+        S, C = k.shape
+        state_out = state if state_out is None else state_out
+        for i, s in enumerate(tuple(state) + tuple(state_out)):
+            _need_cuda(s, f"state[{i}]", torch.float32)
+            if s.shape != (S, C):
+                raise ValueError("state arrays must be [S, C]")
+        self._keep = [k, v, w, u, out, *state, *state_out]
+        self._sin = _abi.wkv_cstate(*(s.data_ptr() for s in state))
+        self._sout = _abi.wkv_state(*(s.data_ptr() for s in state_out))
+        self._fn = _abi.lib().wkv_step
+        self._args = (S, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u), _ptr(out),
+                      _dtype_code(out, "out"), ctypes.byref(self._sin), ctypes.byref(self._sout))
+        self._stream = _stream()
+
+    def __call__(self, stream=None) -> None:
+        code = self._fn(*self._args, self._stream if stream is None else stream)
+        if code:
+            _abi.check(code, "wkv_step")

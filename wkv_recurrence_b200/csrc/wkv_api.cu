@@ -27,46 +27,67 @@ constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s
 // ---------------------------------------------------------------------------
 // kernel configurations
 // ---------------------------------------------------------------------------
-// sequential kernel: CTA = kSeqThreads threads x VEC channels, LT-token tiles
-constexpr int kSeqThreads = 128;
-constexpr int kSeqVecF32 = 2, kSeqLtF32 = 8, kSeqStagesF32 = 4;    // 256 ch, 4 x 16 KB
-constexpr int kSeqVecBf16 = 2, kSeqLtBf16 = 16, kSeqStagesBf16 = 4;  // 256 ch, 4 x 16 KB
+// sequential kernel: CTA = 32, 64 or 128 threads x VEC channels, LT-token tiles
+constexpr int kSeqVecF32 = 2, kSeqLtF32 = 8, kSeqStagesF32 = 4;    // 4 stages of 64 B x CG
+constexpr int kSeqVecBf16 = 2, kSeqLtBf16 = 16, kSeqStagesBf16 = 4;  // 4 stages of 64 B x CG
 constexpr int kSeqFallbackVec = 1, kSeqFallbackLt = 16;
 
-// chunked kernel: a tile is 64 channels (32 threads x 2) by L = P x J tokens
+// chunked kernel: a tile is 64 channels (32 lanes x 2) by L = NW x 16 tokens
 constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 
 struct Plan {
-  int kernel;  // 1 seq, 2 chunk
+  int kernel;  // 1 seq, 2 chunked single launch, 3 chunked two launches (L2-resident inputs)
+  int seq_threads;  // CTA width of the sequential kernel
   int L;       // chunk length (chunk kernel)
+  int J;       // tokens per warp (chunk kernel)
   int G;       // look-back group
   int NG;      // channel groups per batch row
   int nch;     // chunks per sequence
   long long n_tiles;
   long long nblk;  // look-back groups per sequence
-  size_t off_flags_a, off_flags_p, off_agg_a, off_agg_p, bytes;
+  size_t off_flags_a, off_flags_p, off_agg_a, off_agg_p, off_x0, bytes;
 };
+
+// Inputs up to this size take the two-launch scan (they stay in L2 between
+// the launches; B200 has 126 MB of L2).
+constexpr int64_t kL2ResidentBytes = 64ll << 20;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl) {
+bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, int kv_bytes = 4) {
   std::memset(pl, 0, sizeof *pl);
   const int want = o ? o->kernel : 0;
-  if (want < 0 || want > 2) return false;
+  if (want < 0 || want > 3) return false;
   const int64_t lanes = B * C;
   int kernel = want;
-  if (kernel == 0) kernel = (lanes >= 65536 || T <= 64) ? 1 : 2;
+  if (kernel == 0) {
+    if (lanes >= 65536 || T <= 64) {
+      kernel = 1;
+    } else {
+      const int Ld = (o && o->chunk_len) ? o->chunk_len : 128;
+      const int64_t nch = (T + Ld - 1) / Ld;
+      kernel = (2 * B * T * C * kv_bytes <= kL2ResidentBytes && nch <= 64) ? 3 : 2;
+    }
+  }
   pl->kernel = kernel;
   pl->bytes = sizeof(WsHeader);
+  int sth = o ? o->seq_threads : 0;
+  if (sth == 0) sth = 128;
+  if (sth != 32 && sth != 64 && sth != 128) return false;
+  pl->seq_threads = sth;
   if (kernel == 1) return true;
 
   int L = o ? o->chunk_len : 0;
-  if (L == 0) L = 64;
+  if (L == 0) L = 128;
   if (L != 32 && L != 64 && L != 128) return false;
+  int J = o ? o->span : 0;
+  if (J == 0) J = 16;
+  if (J != 8 && J != 16) return false;
   int G = o ? o->lookback_group : 0;
   if (G == 0) G = 16;
   if (G < 1 || G > 1024) return false;
   pl->L = L;
+  pl->J = J;
   pl->G = G;
   pl->NG = (int)((C + kChunkCG - 1) / kChunkCG);
   pl->nch = (int)((T + L - 1) / L);
@@ -74,6 +95,17 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl) 
   pl->n_tiles = (long long)pl->nch * BNG;
   if (pl->n_tiles >= (1ll << 31)) return false;
   pl->nblk = (pl->nch + G - 1) / G;
+  if (kernel == 3) {
+    size_t off = sizeof(WsHeader);
+    pl->off_agg_a = off;
+    off = round_up(off + sizeof(float4) * (size_t)pl->n_tiles * kChunkCG, 256);
+    pl->off_agg_p = off;
+    off = round_up(off + sizeof(float4) * (size_t)pl->n_tiles * (L / J) * kChunkCG, 256);
+    pl->off_x0 = off;
+    off = round_up(off + sizeof(float4) * (size_t)BNG * kChunkCG, 256);
+    pl->bytes = off;
+    return true;
+  }
   size_t off = sizeof(WsHeader);
   pl->off_flags_a = off;
   off = round_up(off + sizeof(uint32_t) * (size_t)pl->n_tiles, 256);
@@ -181,33 +213,93 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-template <typename KV, typename OUT, int VEC, int LT, int STAGES, bool kTMA>
+template <typename KV, typename OUT, int THREADS, int VEC, int LT, int STAGES, bool kTMA>
 wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
-  constexpr int CG = kSeqThreads * VEC;
+  constexpr int CG = THREADS * VEC;
   const size_t smem = (size_t)STAGES * 2 * LT * CG * sizeof(KV) + 64 * STAGES;
-  auto fn = wkv_fwd_seq<KV, OUT, VEC, kSeqThreads, LT, STAGES, kTMA>;
+  auto fn = wkv_fwd_seq<KV, OUT, VEC, THREADS, LT, STAGES, kTMA>;
   int occ = 0;
-  if (!kernel_setup(fn, dev, kSeqThreads, smem, &occ)) return WKV_ERR_CUDA;
+  if (!kernel_setup(fn, dev, THREADS, smem, &occ)) return WKV_ERR_CUDA;
   FwdParams q = p;
   q.NG = (p.C + CG - 1) / CG;
   const long long grid = (long long)p.B * q.NG;
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  fn<<<(unsigned)grid, kSeqThreads, smem, st>>>(q, tk, tv);
+  fn<<<(unsigned)grid, THREADS, smem, st>>>(q, tk, tv);
   return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
-template <typename KV, typename OUT, int P, int J, bool kTMA>
-wkv_status launch_chunk(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev,
-                        int sms) {
-  constexpr int L = P * J;
-  const size_t smem = 2ull * 2 * L * kChunkCG * sizeof(KV) + sizeof(float4) * P * kChunkCG + 64;
-  auto fn = wkv_fwd_chunk<KV, OUT, kChunkVec, kChunkRW, P, J, kTMA>;
+template <typename KV, typename OUT, int NW, int J, bool kTMA>
+wkv_status launch_chunk(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
+  constexpr int L = NW * J;
+  const size_t smem = 2ull * L * kChunkCG * sizeof(KV) + sizeof(float4) * (NW + 1) * kChunkCG + 64;
+  auto fn = wkv_fwd_chunk<KV, OUT, NW, J, kTMA>;
   int occ = 0;
-  if (!kernel_setup(fn, dev, kChunkRW * P, smem, &occ)) return WKV_ERR_CUDA;
-  if (occ < 1) return WKV_ERR_CUDA;
-  const long long grid = std::min<long long>((long long)occ * sms, p.n_tiles);
-  fn<<<(unsigned)grid, kChunkRW * P, smem, st>>>(p, tk, tv);
+  if (!kernel_setup(fn, dev, (NW + 1) * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  fn<<<(unsigned)p.n_tiles, (NW + 1) * 32, smem, st>>>(p, tk, tv);
   return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <typename KV, typename OUT, int NW, int J, bool kTMA>
+wkv_status launch_two(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
+  constexpr int L = NW * J;
+  const size_t tile = 2ull * L * kChunkCG * sizeof(KV);
+  const size_t smem_a = tile + sizeof(float4) * NW * kChunkCG + 64;
+  const size_t smem_b = tile + sizeof(float4) * kChunkCG + 64;
+  auto fa = wkv_chunk_totals<KV, NW, J, kTMA>;
+  auto fb = wkv_chunk_replay<KV, OUT, NW, J, kTMA>;
+  int occ = 0;
+  if (!kernel_setup(fa, dev, NW * 32, smem_a, &occ) || occ < 1) return WKV_ERR_CUDA;
+  if (!kernel_setup(fb, dev, (NW + 1) * 32, smem_b, &occ) || occ < 1) return WKV_ERR_CUDA;
+  fa<<<(unsigned)p.n_tiles, NW * 32, smem_a, st>>>(p, tk, tv);
+  if (cudaGetLastError() != cudaSuccess) return WKV_ERR_CUDA;
+  // the replay launch may begin while the totals launch drains: it copies its
+  // inputs first and waits (griddepcontrol.wait) before reading any total
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.n_tiles);
+  cfg.blockDim = dim3((NW + 1) * 32);
+  cfg.dynamicSmemBytes = smem_b;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fb, p, tk, tv) != cudaSuccess) return WKV_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <typename KV, typename OUT, bool kTMA>
+wkv_status launch_two_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                            cudaStream_t st, int dev) {
+  if (pl.J == 8) {
+    switch (pl.L) {
+      case 32: return launch_two<KV, OUT, 4, 8, kTMA>(p, tk, tv, st, dev);
+      case 64: return launch_two<KV, OUT, 8, 8, kTMA>(p, tk, tv, st, dev);
+      default: return launch_two<KV, OUT, 16, 8, kTMA>(p, tk, tv, st, dev);
+    }
+  }
+  switch (pl.L) {
+    case 32: return launch_two<KV, OUT, 2, 16, kTMA>(p, tk, tv, st, dev);
+    case 64: return launch_two<KV, OUT, 4, 16, kTMA>(p, tk, tv, st, dev);
+    default: return launch_two<KV, OUT, 8, 16, kTMA>(p, tk, tv, st, dev);
+  }
+}
+
+template <typename KV, typename OUT, bool kTMA>
+wkv_status launch_chunk_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                              cudaStream_t st, int dev) {
+  if (pl.J == 8) {
+    switch (pl.L) {
+      case 32: return launch_chunk<KV, OUT, 4, 8, kTMA>(p, tk, tv, st, dev);
+      case 64: return launch_chunk<KV, OUT, 8, 8, kTMA>(p, tk, tv, st, dev);
+      default: return launch_chunk<KV, OUT, 16, 8, kTMA>(p, tk, tv, st, dev);
+    }
+  }
+  switch (pl.L) {
+    case 32: return launch_chunk<KV, OUT, 2, 16, kTMA>(p, tk, tv, st, dev);
+    case 64: return launch_chunk<KV, OUT, 4, 16, kTMA>(p, tk, tv, st, dev);
+    default: return launch_chunk<KV, OUT, 8, 16, kTMA>(p, tk, tv, st, dev);
+  }
 }
 
 template <typename KV, typename OUT>
@@ -222,28 +314,27 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
     constexpr int LT = kF32 ? kSeqLtF32 : kSeqLtBf16;
     constexpr int STG = kF32 ? kSeqStagesF32 : kSeqStagesBf16;
     if (tma) {
-      if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, kSeqThreads * VEC) ||
-          !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, kSeqThreads * VEC))
+      const int cg = pl.seq_threads * VEC;
+      if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, cg) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, cg))
         return WKV_ERR_CUDA;
-      return launch_seq<KV, OUT, VEC, LT, STG, true>(p, tk, tv, st, dev);
+      switch (pl.seq_threads) {
+        case 32: return launch_seq<KV, OUT, 32, VEC, LT, STG, true>(p, tk, tv, st, dev);
+        case 64: return launch_seq<KV, OUT, 64, VEC, LT, STG, true>(p, tk, tv, st, dev);
+        default: return launch_seq<KV, OUT, 128, VEC, LT, STG, true>(p, tk, tv, st, dev);
+      }
     }
-    return launch_seq<KV, OUT, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
+    return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
   }
+  (void)sms;
   if (tma) {
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
         !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
       return WKV_ERR_CUDA;
-    switch (pl.L) {
-      case 32: return launch_chunk<KV, OUT, 4, 8, true>(p, tk, tv, st, dev, sms);
-      case 64: return launch_chunk<KV, OUT, 8, 8, true>(p, tk, tv, st, dev, sms);
-      default: return launch_chunk<KV, OUT, 8, 16, true>(p, tk, tv, st, dev, sms);
-    }
+    if (pl.kernel == 3) return launch_two_shape<KV, OUT, true>(pl, p, tk, tv, st, dev);
+    return launch_chunk_shape<KV, OUT, true>(pl, p, tk, tv, st, dev);
   }
-  switch (pl.L) {
-    case 32: return launch_chunk<KV, OUT, 4, 8, false>(p, tk, tv, st, dev, sms);
-    case 64: return launch_chunk<KV, OUT, 8, 8, false>(p, tk, tv, st, dev, sms);
-    default: return launch_chunk<KV, OUT, 8, 16, false>(p, tk, tv, st, dev, sms);
-  }
+  if (pl.kernel == 3) return launch_two_shape<KV, OUT, false>(pl, p, tk, tv, st, dev);
+  return launch_chunk_shape<KV, OUT, false>(pl, p, tk, tv, st, dev);
 }
 
 }  // namespace
@@ -269,9 +360,11 @@ const char* wkv_status_string(wkv_status s) {
 }
 
 size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const wkv_options* opts) {
-  Plan pl;
-  if (B < 0 || T < 0 || C < 0 || !make_plan(B, T, C, opts, &pl)) return 0;
-  return pl.bytes;
+  // the automatic choice of kernel may depend on the input dtype, which is
+  // not an argument here: return what either choice needs
+  Plan a, b;
+  if (B < 0 || T < 0 || C < 0 || !make_plan(B, T, C, opts, &a, 4) || !make_plan(B, T, C, opts, &b, 2)) return 0;
+  return std::max(a.bytes, b.bytes);
 }
 
 wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
@@ -290,7 +383,7 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   if (opts && opts->wait_timeout_ns < 0) return WKV_ERR_INVALID_ARG;
   if (opts && (opts->inject_enable != 0 && opts->inject_enable != 1)) return WKV_ERR_INVALID_ARG;
   Plan pl;
-  if (!make_plan(B, T, C, opts, &pl)) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, opts, &pl, kv_dtype == WKV_F32 ? 4 : 2)) return WKV_ERR_INVALID_ARG;
   if (!workspace) return WKV_ERR_INVALID_ARG;
   if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
@@ -346,7 +439,7 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   p.hdr = reinterpret_cast<WsHeader*>(ws);
   p.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? (uint64_t)opts->wait_timeout_ns : kDefaultTimeoutNs;
   p.inject_tile = (opts && opts->inject_enable) ? (int)std::min<int64_t>(opts->inject_unpublished_tile, INT32_MAX) : -1;
-  if (pl.kernel == 2) {
+  if (pl.kernel >= 2) {
     p.NG = pl.NG;
     p.nch = pl.nch;
     p.G = pl.G;
@@ -355,6 +448,10 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
     p.flags_p = reinterpret_cast<uint32_t*>(ws + pl.off_flags_p);
     p.agg_a = reinterpret_cast<float4*>(ws + pl.off_agg_a);
     p.agg_p = reinterpret_cast<float4*>(ws + pl.off_agg_p);
+    if (pl.kernel == 3) {
+      p.flags_a = p.flags_p = nullptr;
+      p.x0 = reinterpret_cast<float4*>(ws + pl.off_x0);
+    }
   }
   const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
   const size_t oes = out_dtype == WKV_F32 ? 4 : 2;
@@ -364,6 +461,8 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   const int vec = pl.kernel == 1 ? (tma ? (kv_dtype == WKV_F32 ? kSeqVecF32 : kSeqVecBf16) : kSeqFallbackVec)
                                  : kChunkVec;
   p.vec_store = aligned(out, oes * vec) && (C % vec) == 0;
+  if (pl.kernel >= 2)  // the chunked kernels also load k and v VEC-wide
+    p.vec_store = p.vec_store && aligned(k, kes * vec) && aligned(v, kes * vec);
 
   if (kv_dtype == WKV_F32) return dispatch_forward<float, float>(pl, p, tma, kv_dtype, st, dev, di.sms);
   if (out_dtype == WKV_BF16)
@@ -472,7 +571,7 @@ wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, c
                                const wkv_cstate* state_in, const wkv_state* state_out, void* stream) {
   if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
   Plan pl;
-  if (!make_plan(B, T, C, nullptr, &pl)) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, nullptr, &pl, kv_dtype == WKV_BF16 ? 2 : 4)) return WKV_ERR_INVALID_ARG;
   if (pl.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (B * C == 0) {
     // nothing to compute: wkv_forward checks the other arguments and returns

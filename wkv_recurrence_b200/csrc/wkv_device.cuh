@@ -238,6 +238,78 @@ __device__ __forceinline__ void store_vec<__nv_bfloat16, 8>(__nv_bfloat16* p, co
                                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
 }
 
+// Streaming global loads straight into registers (read once: no L1
+// allocation) and streaming stores (evict-first in L2). `p` is aligned to VEC
+// elements.
+template <typename T, int VEC>
+__device__ __forceinline__ void ldg_stream(const T* p, float (&x)[VEC]);
+
+template <>
+__device__ __forceinline__ void ldg_stream<float, 1>(const float* p, float (&x)[1]) {
+  asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(x[0]) : "l"(p));
+}
+template <>
+__device__ __forceinline__ void ldg_stream<float, 2>(const float* p, float (&x)[2]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v2.f32 {%0, %1}, [%2];" : "=f"(x[0]), "=f"(x[1]) : "l"(p));
+}
+template <>
+__device__ __forceinline__ void ldg_stream<float, 4>(const float* p, float (&x)[4]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3])
+               : "l"(p));
+}
+template <>
+__device__ __forceinline__ void ldg_stream<__nv_bfloat16, 1>(const __nv_bfloat16* p, float (&x)[1]) {
+  unsigned short h;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(h) : "l"(p));
+  x[0] = __uint_as_float(((uint32_t)h) << 16);
+}
+template <>
+__device__ __forceinline__ void ldg_stream<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&x)[2]) {
+  uint32_t u;
+  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(u) : "l"(p));
+  unpack_bf16x2(u, x[0], x[1]);
+}
+template <>
+__device__ __forceinline__ void ldg_stream<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&x)[4]) {
+  uint32_t a, b;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "l"(p));
+  unpack_bf16x2(a, x[0], x[1]);
+  unpack_bf16x2(b, x[2], x[3]);
+}
+
+template <typename T, int VEC>
+__device__ __forceinline__ void stg_stream(T* p, const float (&x)[VEC]);
+
+template <>
+__device__ __forceinline__ void stg_stream<float, 1>(float* p, const float (&x)[1]) {
+  asm volatile("st.global.cs.f32 [%0], %1;" ::"l"(p), "f"(x[0]) : "memory");
+}
+template <>
+__device__ __forceinline__ void stg_stream<float, 2>(float* p, const float (&x)[2]) {
+  asm volatile("st.global.cs.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(x[0]), "f"(x[1]) : "memory");
+}
+template <>
+__device__ __forceinline__ void stg_stream<float, 4>(float* p, const float (&x)[4]) {
+  asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(x[0]), "f"(x[1]), "f"(x[2]),
+               "f"(x[3])
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void stg_stream<__nv_bfloat16, 1>(__nv_bfloat16* p, const float (&x)[1]) {
+  *p = __float2bfloat16_rn(x[0]);
+}
+template <>
+__device__ __forceinline__ void stg_stream<__nv_bfloat16, 2>(__nv_bfloat16* p, const float (&x)[2]) {
+  asm volatile("st.global.cs.b32 [%0], %1;" ::"l"(p), "r"(pack_bf16x2(x[0], x[1])) : "memory");
+}
+template <>
+__device__ __forceinline__ void stg_stream<__nv_bfloat16, 4>(__nv_bfloat16* p, const float (&x)[4]) {
+  asm volatile("st.global.cs.v2.b32 [%0], {%1, %2};" ::"l"(p), "r"(pack_bf16x2(x[0], x[1])),
+               "r"(pack_bf16x2(x[2], x[3]))
+               : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // The recurrence in anchored form
 // ---------------------------------------------------------------------------
@@ -291,6 +363,41 @@ __device__ __forceinline__ void add_token(Acc& s, float k, float v, float w) {
   s.den = fmaf(a, s.den, b);
   s.ma = reset ? k : s.ma;
   s.nf = reset ? 0.f : nf1;
+}
+
+// Output and state advance for one token, with one exponential.
+//
+// Let Md be the state's max exponent after this token's decay and D2 = k - Md.
+// The update needs e^{-|D2|} (the smaller of the two weights; the other is 1).
+// The output compares the undecayed state (exponent Md + w) with the current
+// token with its bonus (exponent k + u); dividing both weights by e^{w} makes
+// them the update's weights, with the current token's multiplied by the
+// per-channel constant c = e^{u-w}. So one ex2 serves both halves.
+// Valid while c and 1/c stay far inside the fp32 range; callers take this
+// path only when |u - w| <= kFastUW (else out_token + add_token).
+constexpr float kFastUW = 40.0f;
+
+__device__ __forceinline__ float step_token(Acc& s, float k, float v, float w, float c) {
+  const float nf1 = s.nf + 1.f;
+  const float Md = fmaf(-nf1, w, s.ma);
+  const float D2 = k - Md;
+  const float x = ex2(-fabsf(D2) * kLog2e);
+  const bool reset = D2 > 0.f;          // the key is the new maximum (and anchor)
+  const float a = reset ? x : 1.f;      // weight of the carried state
+  const float b = reset ? 1.f : x;      // weight of the current token (no bonus)
+  const float bc = b * c;               // ... and with the bonus
+  const float out = fmaf(bc, v, a * s.num) * rcp(fmaf(a, s.den, bc));
+  s.num = fmaf(a, s.num, b * v);
+  s.den = fmaf(a, s.den, b);
+  s.ma = reset ? k : s.ma;
+  s.nf = reset ? 0.f : nf1;
+  return out;
+}
+
+__device__ __forceinline__ bool fast_uw(float u, float w) { return fabsf(u - w) <= kFastUW; }
+
+__device__ __forceinline__ float bonus_factor(float u, float w) {
+  return ex2((u - w) * kLog2e);
 }
 
 // Associative combine: `a` covers the tokens before `b`, and `b` spans len_b

@@ -1,26 +1,27 @@
 // Forward kernels of the WKV operator over [B, T, C] sequences.
 //
-// Both kernels stream k and v through shared memory with TMA (3-D tiled bulk
-// copies of a [tokens x channel-group] box, completion on an mbarrier) and run
-// the recurrence of "Linear attention without writing a CUDA kernel", section
-// "The recurrence", in the anchored form of wkv_device.cuh, one channel per
-// register lane, VEC adjacent channels per thread.
+// Both kernels run the recurrence of "Linear attention without writing a CUDA
+// kernel", section "The recurrence", in the anchored form of wkv_device.cuh,
+// one channel per register lane, VEC adjacent channels per thread. The
+// sequential kernel streams k and v through shared memory with TMA (3-D tiled
+// bulk copies of a [tokens x channel-group] box, completion on an mbarrier);
+// the chunked kernel loads its short spans straight into registers.
 //
 // * wkv_fwd_seq: one CTA per (batch row, channel group), walking all T tokens
 //   through a STAGES-deep ring of [LT x CG] tiles. For many channels (B*C
 //   large): the state never leaves registers.
 //
 // * wkv_fwd_chunk: for few channels and long T. T is cut into chunks of
-//   L = P*J tokens; a tile is (chunk, batch row, channel group). Persistent
-//   CTAs take tiles in order from a ticket counter, so every tile a CTA waits
-//   for was handed out earlier to a running CTA. Per tile:
-//     1. P sub-chunks of J tokens each (one warp-row of threads per sub-chunk)
-//        fold their tokens from the empty state into an aggregate;
-//     2. one row of threads combines the P aggregates into the tile total,
-//        publishes it, and forms the tile's incoming state from the chunks
-//        before it (look-back, below);
-//     3. every sub-chunk replays its tokens from its incoming state, still in
-//        shared memory, and writes the outputs.
+//   L = NW*J tokens; a tile is (chunk, batch row, 64-channel group) and one
+//   CTA of NW warps. Tiles are handed out in order by a ticket counter, so
+//   every tile a CTA waits for belongs to a CTA that is already running. Per
+//   tile, each warp loads its J tokens straight into registers and
+//     1. folds them from the empty state into an aggregate (two passes: the
+//        largest end-of-span exponent, then the weighted sums);
+//     2. combines the aggregates of the warps before it (its in-tile prefix);
+//        the last warp forms the tile total, publishes it and gathers the
+//        tile's incoming state by look-back;
+//     3. replays its tokens from registers, from (incoming state + prefix).
 //   The associative combine of two spans (a, then b of len_b tokens) decays a
 //   across b and adds the two relative to the larger exponent
 //   (wkv::combine). The pages only say the recurrence has a parallel
@@ -68,8 +69,16 @@ struct FwdParams {
   uint32_t* flags_a;   // [n_tiles]
   uint32_t* flags_p;   // [nblk * B * NG]
   float4* agg_a;       // [n_tiles][CG]
-  float4* agg_p;       // [nblk * B * NG][CG]
+  float4* agg_p;       // [nblk * B * NG][CG] (single launch) or [n_tiles][NW][CG] (two launches)
+  float4* x0;          // [B * NG][CG]: state in, anchored (two launches)
 };
+
+// State in for one channel, anchored; empty when no state is passed.
+__device__ __forceinline__ Acc state_in_acc(const FwdParams& p, int b, int c) {
+  if (!p.s_num || c >= p.C) return acc_empty();
+  const size_t i = (size_t)b * p.C + c;
+  return acc_from_state(p.s_num[i], p.s_den[i], p.s_max[i]);
+}
 
 template <typename OUT, int VEC>
 __device__ __forceinline__ void store_out(OUT* row, int c0, int C, bool vec_ok, const float (&o)[VEC]) {
@@ -128,20 +137,24 @@ __global__ void __launch_bounds__(THREADS)
     }
   }
 
-  float w[VEC], u[VEC];
+  float w[VEC], u[VEC], cb[VEC];
   Acc st[VEC];
+  bool fast = true;
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
     const int c = c0 + e;
     const bool ok = c < C;
     w[e] = ok ? p.w[c] : 0.f;
     u[e] = ok ? p.u[c] : 0.f;
+    fast &= fast_uw(u[e], w[e]);
+    cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
     st[e] = acc_empty();
     if (ok && p.s_num) {
       const size_t i = (size_t)b * C + c;
       st[e] = acc_from_state(p.s_num[i], p.s_den[i], p.s_max[i]);
     }
   }
+  fast = __all_sync(0xffffffffu, fast);  // one path per warp
   __syncthreads();
 
   OUT* out = reinterpret_cast<OUT*>(p.out);
@@ -167,7 +180,17 @@ __global__ void __launch_bounds__(THREADS)
     const int nv = min(LT, T - t0);
     OUT* orow = out + ((size_t)b * T + t0) * C;
     if (c0 < C) {
-      if (nv == LT) {
+      if (nv == LT && fast) {
+#pragma unroll 4
+        for (int j = 0; j < LT; ++j) {
+          float kx[VEC], vx[VEC], o[VEC];
+          load_vec<KV, VEC>(ks + j * CG, kx);
+          load_vec<KV, VEC>(vs + j * CG, vx);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+          store_out<OUT, VEC>(orow + (size_t)j * C, c0, C, vec_ok, o);
+        }
+      } else if (nv == LT) {
 #pragma unroll 4
         for (int j = 0; j < LT; ++j) {
           float kx[VEC], vx[VEC], o[VEC];
@@ -242,297 +265,580 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* q) {
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 template <int N>
-__device__ __forceinline__ void row_sync() {
-  // barrier among the first N threads of the CTA (whole warps)
-  if (N == 32) {
-    __syncwarp();
-  } else {
-    asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void named_sync(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(N) : "memory");
+}
+
+// Aggregate of one warp's span of n <= J tokens from the empty state, read
+// from a shared-memory tile in two passes: first the largest exponent M that
+// any token has at the end of the span (s_i = k_i - (n-1-i) w, one fma each),
+// then the sums of e^{s_i - M} v_i and e^{s_i - M}. No per-token
+// compare-and-select is needed. The result is anchored at M with count 0.
+// `ks`, `vs` point at this lane's channels in the span's first row; rows are
+// CG elements apart.
+template <typename KV, int J, int VEC, int CG>
+__device__ __forceinline__ void aggregate_tile_span(const KV* ks, const KV* vs, int n, const float (&w)[VEC],
+                                                    Acc (&agg)[VEC]) {
+  float M[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) M[e] = kNegBig;
+  const float last = (float)(n - 1);
+#pragma unroll
+  for (int i = 0; i < J; ++i) {
+    if (i < n) {
+      float kx[VEC];
+      load_vec<KV, VEC>(ks + i * CG, kx);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) M[e] = fmaxf(M[e], fmaf((float)i - last, w[e], kx[e]));
+    }
+  }
+  float ML[VEC], num[VEC], den[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    ML[e] = M[e] * kLog2e;
+    num[e] = den[e] = 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < J; ++i) {
+    if (i < n) {
+      float kx[VEC], vx[VEC];
+      load_vec<KV, VEC>(ks + i * CG, kx);
+      load_vec<KV, VEC>(vs + i * CG, vx);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float x = ex2(fmaf(fmaf((float)i - last, w[e], kx[e]), kLog2e, -ML[e]));
+        num[e] = fmaf(x, vx[e], num[e]);
+        den[e] += x;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    if (n <= 0) {
+      agg[e] = acc_empty();
+    } else {
+      // all weights share the factor 2^{M log2e - ML} from rounding ML
+      const float corr = fmaf(M[e], kLog2e, -ML[e]);
+      const float fix = fmaf(-corr, 0.6931471805599453f, 1.f);
+      agg[e] = Acc{num[e] * fix, den[e] * fix, M[e], 0.f};
+    }
   }
 }
 
-template <typename KV, typename OUT, int VEC, int RW, int P, int J, bool kTMA>
-__global__ void __launch_bounds__(RW * P)
+// Tile = 64 channels (32 lanes x 2) by L = NW * J tokens of one batch row, one
+// CTA of NW compute warps plus one scan warp. Thread 0 takes the tile's ticket
+// and starts its TMA copy (k and v boxes into shared memory); meanwhile the
+// scan warp gathers the tile's incoming state from earlier chunks (look-back),
+// which needs nothing from this tile. Compute warp wp owns tokens
+// [t0 + wp*J, t0 + (wp+1)*J): it folds them into an aggregate, takes the
+// aggregates of the compute warps before it as its in-tile prefix, and the last
+// compute warp publishes the tile total -- before waiting for the scan warp,
+// so that no tile's total waits on another tile's look-back. Then every
+// compute warp replays its tokens from shared memory.
+template <typename KV, typename OUT, int NW, int J, bool kTMA>
+__global__ void __launch_bounds__((NW + 1) * 32)
     wkv_fwd_chunk(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-  static_assert(RW % 32 == 0, "a row of threads is whole warps");
-  constexpr int CG = RW * VEC;  // channels per tile
-  constexpr int L = P * J;      // tokens per tile
+  constexpr int VEC = 2;
+  constexpr int CG = 32 * VEC;
+  constexpr int L = NW * J;
   constexpr int kTile = L * CG;
-  constexpr uint32_t kStageBytes = 2u * kTile * sizeof(KV);
+  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
   extern __shared__ __align__(1024) unsigned char smem[];
-  KV* tiles = reinterpret_cast<KV*>(smem);                                 // [2 stages][k,v][L][CG]
-  float4* buf = reinterpret_cast<float4*>(smem + 2 * kStageBytes);          // [P][CG]
-  uint64_t* full = reinterpret_cast<uint64_t*>(buf + P * CG);               // [2]
-  int* tile_id = reinterpret_cast<int*>(full + 2);                          // [2]
+  KV* ktile = reinterpret_cast<KV*>(smem);
+  KV* vtile = ktile + kTile;
+  float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
+  float4* sh_x = sh_agg + NW * CG;                             // [CG]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_x + CG);
+  int* sh_tile = reinterpret_cast<int*>(bar + 1);
 
-  const int tid = threadIdx.x;
-  const int pr = tid / RW;  // sub-chunk of this thread
-  const int rr = tid % RW;  // position in the row
+  const int lane = threadIdx.x & 31;
+  const int wp = threadIdx.x >> 5;
+  const bool scan = (wp == NW);
   const int T = p.T, C = p.C;
   const int BNG = p.B * p.NG;
   const uint32_t target = *reinterpret_cast<volatile uint32_t*>(&p.hdr->epoch) + 1u;
-  OUT* out = reinterpret_cast<OUT*>(p.out);
-  const bool vec_ok = p.vec_store != 0;
 
-  if (tid == 0) {
-    if (kTMA) {
-      prefetch_tmap(&tmk);
-      prefetch_tmap(&tmv);
-      mbar_init(&full[0], 1);
-      mbar_init(&full[1], 1);
-      fence_mbar_init();
-    }
+  if (threadIdx.x == 0) {
     const int t = (int)atomicAdd(&p.hdr->ticket, 1u);
-    tile_id[0] = t;
-    if (kTMA && t < p.n_tiles) {
-      const int j = t / BNG, bg = t % BNG;
-      mbar_arrive_expect_tx(&full[0], kStageBytes);
-      tma_load_3d(tiles, &tmk, &full[0], (bg % p.NG) * CG, j * L, bg / p.NG);
-      tma_load_3d(tiles + kTile, &tmv, &full[0], (bg % p.NG) * CG, j * L, bg / p.NG);
+    *sh_tile = t;
+    if (kTMA) {
+      const int jj = t / BNG, bgg = t % BNG;
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(bar, kBytes);
+      tma_load_3d(ktile, &tmk, bar, (bgg % p.NG) * CG, jj * L, bgg / p.NG);
+      tma_load_3d(vtile, &tmv, bar, (bgg % p.NG) * CG, jj * L, bgg / p.NG);
     }
   }
   __syncthreads();
-
-  bool timed_out = false;
-  int stuck_it = -1;  // iteration whose copy did not arrive in time, if any
-  for (int it = 0;; ++it) {
-    const int slot = it & 1;             // ticket slot (and stage, with TMA)
-    const int s = kTMA ? slot : 0;       // shared-memory stage
-    const int tile = tile_id[slot];
-    if (tile >= p.n_tiles) break;
-    const int j = tile / BNG;
-    const int bg = tile % BNG;
-    const int b = bg / p.NG, g = bg % p.NG;
-    const int t0 = j * L;
-    const int cbase = g * CG;
-
-    if (tid == 0) {  // hand out and prefetch the next tile
-      const int tn = (int)atomicAdd(&p.hdr->ticket, 1u);
-      tile_id[slot ^ 1] = tn;
-      if (kTMA && tn < p.n_tiles) {
-        const int jn = tn / BNG, bgn = tn % BNG;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&full[s ^ 1], kStageBytes);
-        tma_load_3d(tiles + (2 * (s ^ 1)) * kTile, &tmk, &full[s ^ 1], (bgn % p.NG) * CG, jn * L, bgn / p.NG);
-        tma_load_3d(tiles + (2 * (s ^ 1) + 1) * kTile, &tmv, &full[s ^ 1], (bgn % p.NG) * CG, jn * L,
-                    bgn / p.NG);
-      }
-    }
-
-    if (kTMA) {
-      const bool ok = mbar_wait(&full[s], (it >> 1) & 1, p.timeout_ns);
-      if (__syncthreads_or(!ok)) {
-        timed_out = true;
-        stuck_it = it;
-        break;
-      }
-    } else {
-      coop_load_tile<KV>(tiles, reinterpret_cast<const KV*>(p.k), b, t0, L, cbase, CG, T, C);
-      coop_load_tile<KV>(tiles + kTile, reinterpret_cast<const KV*>(p.v), b, t0, L, cbase, CG, T, C);
-      __syncthreads();
-    }
-
-    const KV* ks = tiles + (2 * s) * kTile + rr * VEC;
-    const KV* vs = ks + kTile;
-    const int cl = rr * VEC;       // channel offset inside the group
-    const int c0 = cbase + cl;     // first channel of this thread
-    float w[VEC], u[VEC];
+  const int tile = *sh_tile;
+  const int j = tile / BNG;
+  const int bg = tile % BNG;
+  const int b = bg / p.NG, g = bg % p.NG;
+  const int t0 = j * L;
+  const int cl = lane * VEC;
+  const int c0 = g * CG + cl;
+  const bool last_chunk = (j == p.nch - 1);
+  const bool inject = (tile == p.inject_tile);
+  float w[VEC], u[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const bool ok = c0 + e < C;
-      w[e] = ok ? __ldg(p.w + c0 + e) : 0.f;
-      u[e] = ok ? __ldg(p.u + c0 + e) : 0.f;
-    }
-    const bool last_chunk = (j == p.nch - 1);
-    const int ts = t0 + pr * J;                       // first token of this sub-chunk
-    const int nv = max(0, min(J, T - ts));            // its tokens
-    const int p_last = last_chunk ? (T - 1 - t0) / J : P - 1;
+  for (int e = 0; e < VEC; ++e) {
+    const bool ok = c0 + e < C;
+    w[e] = ok ? __ldg(p.w + c0 + e) : 0.f;
+    u[e] = ok ? __ldg(p.u + c0 + e) : 0.f;
+  }
 
-    // 1. sub-chunk aggregates from the empty state
-    {
-      Acc a[VEC];
+  if (scan) {
+    // ---- look-back: incoming state of the tile (overlaps the TMA copy)
+    Acc x[VEC];
+    const int qb = j / p.G;
+    const int first = qb * p.G;
+    // Only chunk 0 reads the state in; its published total already contains
+    // it, so no later tile reads the caller's state (which state_out may alias).
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) a[e] = acc_empty();
-      if (!(last_chunk && pr >= p_last)) {
-        if (nv == J) {
-#pragma unroll 4
-          for (int jj = 0; jj < J; ++jj) {
-            float kx[VEC], vx[VEC];
-            load_vec<KV, VEC>(ks + (pr * J + jj) * CG, kx);
-            load_vec<KV, VEC>(vs + (pr * J + jj) * CG, vx);
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) add_token(a[e], kx[e], vx[e], w[e]);
-          }
-        } else {
-          for (int jj = 0; jj < nv; ++jj) {
-            float kx[VEC], vx[VEC];
-            load_vec<KV, VEC>(ks + (pr * J + jj) * CG, kx);
-            load_vec<KV, VEC>(vs + (pr * J + jj) * CG, vx);
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) add_token(a[e], kx[e], vx[e], w[e]);
-          }
+    for (int e = 0; e < VEC; ++e) x[e] = (j == 0) ? state_in_acc(p, b, c0 + e) : acc_empty();
+    if (j > 0) {
+      const uint32_t* fp = p.flags_p + (size_t)(qb - 1) * BNG + bg;
+      bool ready = false;
+      uint64_t tstart = 0;
+      while (true) {
+        bool all = (qb == 0) || ld_relaxed_u32(fp) == target;
+        for (int jj = first + lane; jj < j; jj += 32)
+          all &= ld_relaxed_u32(p.flags_a + (size_t)jj * BNG + bg) == target;
+        all = __all_sync(0xffffffffu, all);
+        if (all) {
+          ready = true;
+          break;
         }
+        if (tstart == 0) {
+          tstart = global_ns();
+        } else if (global_ns() - tstart > p.timeout_ns) {
+          break;
+        }
+        __nanosleep(32);
       }
+      if (!ready && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+      fence_acq_rel_gpu();
+      if (qb > 0) {
+        const float4* src = p.agg_p + ((size_t)(qb - 1) * BNG + bg) * CG + cl;
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) buf[pr * CG + cl + e] = acc_pack(a[e]);
+        for (int e = 0; e < VEC; ++e) x[e] = acc_unpack(ld_relaxed_f4(src + e));
+      }
+      for (int jj = first; jj < j; ++jj) {
+        const float4* src = p.agg_a + ((size_t)jj * BNG + bg) * CG + cl;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) x[e] = combine(x[e], acc_unpack(ld_relaxed_f4(src + e)), (float)L, w[e]);
+      }
     }
-    __syncthreads();
-
-    // 2. tile total, publication, look-back, sub-chunk prefixes (row 0 only)
-    if (pr == 0) {
-      Acc tot[VEC], x[VEC];
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) tot[e] = acc_unpack(buf[cl + e]);
-      for (int q = 1; q < P; ++q) {
-        const float len = (float)max(0, min(J, T - (t0 + q * J)));
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) tot[e] = combine(tot[e], acc_unpack(buf[q * CG + cl + e]), len, w[e]);
+    for (int e = 0; e < VEC; ++e) sh_x[cl + e] = acc_pack(x[e]);
+    named_sync<(NW + 1) * 32>(2);  // (A) incoming state ready; totals published
+  } else {
+    // ---- compute warps
+    const int ts = t0 + wp * J;
+    const int nv = max(0, min(J, T - ts));
+    const int p_last = last_chunk ? (T - 1 - t0) / J : NW - 1;
+    bool copy_ok = true;
+    if (kTMA) {
+      copy_ok = mbar_wait(bar, 0, p.timeout_ns);
+      if (!copy_ok && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+    } else {
+      for (int i = threadIdx.x; i < kTile; i += NW * 32) {
+        const int r = i / CG, cc = i % CG;
+        const int t = t0 + r, c = g * CG + cc;
+        KV kk = Elem<KV>::from_f32(0.f), vv = Elem<KV>::from_f32(0.f);
+        if (t < T && c < C) {
+          kk = reinterpret_cast<const KV*>(p.k)[((size_t)b * T + t) * C + c];
+          vv = reinterpret_cast<const KV*>(p.v)[((size_t)b * T + t) * C + c];
+        }
+        ktile[i] = kk;
+        vtile[i] = vv;
       }
-      const bool inject = (tile == p.inject_tile);
+      named_sync<NW * 32>(1);
+    }
+    const KV* ks = ktile + (wp * J) * CG + cl;
+    const KV* vs = vtile + (wp * J) * CG + cl;
+    // 1. aggregate of this warp's span
+    {
+      Acc agg[VEC];
+      if (last_chunk && wp >= p_last) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) agg[e] = acc_empty();
+      } else {
+        aggregate_tile_span<KV, J, VEC, CG>(ks, vs, nv, w, agg);
+      }
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(agg[e]);
+    }
+    named_sync<NW * 32>(1);
+    // 2. in-tile prefix; the last compute warp publishes the tile total
+    Acc pre[VEC], tot[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) pre[e] = acc_empty();
+    for (int q = 0; q < wp; ++q) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) pre[e] = combine(pre[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+    }
+    if (wp == NW - 1) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) tot[e] = combine(pre[e], acc_unpack(sh_agg[wp * CG + cl + e]), (float)nv, w[e]);
       if (!last_chunk) {
         float4* dst = p.agg_a + (size_t)tile * CG + cl;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(tot[e]);
+        for (int e = 0; e < VEC; ++e)
+          dst[e] = acc_pack(j == 0 ? combine(state_in_acc(p, b, c0 + e), tot[e], (float)L, w[e]) : tot[e]);
         __threadfence();
-        row_sync<RW>();
-        if (rr == 0 && !inject) st_release_u32(p.flags_a + tile, target);
-      }
-
-      // incoming state of the tile
-      const int qb = j / p.G;
-      const int first = qb * p.G;  // first chunk of this look-back group
-      if (qb == 0) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          x[e] = acc_empty();
-          if (p.s_num && c0 + e < C) {
-            const size_t i = (size_t)b * C + c0 + e;
-            x[e] = acc_from_state(p.s_num[i], p.s_den[i], p.s_max[i]);
-          }
-        }
-      }
-      if (j > 0) {
-        // wait until every flag this tile needs is set
-        const uint32_t* fp = p.flags_p + (size_t)(qb - 1) * BNG + bg;
-        bool ready = false;
-        uint64_t tstart = 0;
-        while (true) {
-          bool all = (qb == 0) || ld_relaxed_u32(fp) == target;
-          for (int jj = first; jj < j; ++jj) all &= ld_relaxed_u32(p.flags_a + (size_t)jj * BNG + bg) == target;
-          if (all) {
-            ready = true;
-            break;
-          }
-          if (tstart == 0) {
-            tstart = global_ns();
-          } else if (global_ns() - tstart > p.timeout_ns) {
-            break;
-          }
-          __nanosleep(64);
-        }
-        if (!ready) timed_out = true;
-        fence_acq_rel_gpu();
-        if (qb > 0) {
-          const float4* src = p.agg_p + ((size_t)(qb - 1) * BNG + bg) * CG + cl;
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) x[e] = acc_unpack(ld_relaxed_f4(src + e));
-        }
-        for (int jj = first; jj < j; ++jj) {
-          const float4* src = p.agg_a + ((size_t)jj * BNG + bg) * CG + cl;
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) x[e] = combine(x[e], acc_unpack(ld_relaxed_f4(src + e)), (float)L, w[e]);
-        }
-      }
-      // the last chunk of a group publishes its inclusive prefix
-      if (!last_chunk && (j % p.G) == p.G - 1) {
-        float4* dst = p.agg_p + ((size_t)qb * BNG + bg) * CG + cl;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(combine(x[e], tot[e], (float)L, w[e]));
-        __threadfence();
-        row_sync<RW>();
-        if (rr == 0 && !inject) st_release_u32(p.flags_p + (size_t)qb * BNG + bg, target);
-      }
-      // incoming state of every sub-chunk
-      for (int q = 0; q < P; ++q) {
-        const float len = (float)max(0, min(J, T - (t0 + q * J)));
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const Acc a = acc_unpack(buf[q * CG + cl + e]);
-          buf[q * CG + cl + e] = acc_pack(x[e]);
-          x[e] = combine(x[e], a, len, w[e]);
-        }
+        __syncwarp();
+        if (lane == 0 && !inject) st_release_u32(p.flags_a + tile, target);
       }
     }
-    __syncthreads();
-
-    // 3. replay each sub-chunk from its incoming state and write the outputs
-    {
+    named_sync<(NW + 1) * 32>(2);  // (A) incoming state ready
+    if (wp == NW - 1 && !last_chunk && (j % p.G) == p.G - 1) {
+      // the last chunk of a look-back group publishes its inclusive prefix
+      const int qb = j / p.G;
+      float4* dst = p.agg_p + ((size_t)qb * BNG + bg) * CG + cl;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(combine(acc_unpack(sh_x[cl + e]), tot[e], (float)L, w[e]));
+      __threadfence();
+      __syncwarp();
+      if (lane == 0 && !inject) st_release_u32(p.flags_p + (size_t)qb * BNG + bg, target);
+    }
+    // 3. replay this warp's tokens from shared memory
+    if (nv > 0 && copy_ok) {
+      float cb[VEC];
+      bool fast = true;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        fast &= fast_uw(u[e], w[e]);
+        cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+      }
+      fast = __all_sync(0xffffffffu, fast);
       Acc st[VEC];
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) st[e] = acc_unpack(buf[pr * CG + cl + e]);
-      OUT* orow = out + ((size_t)b * T + ts) * C;
-      if (c0 < C) {
-        if (nv == J) {
-#pragma unroll 4
-          for (int jj = 0; jj < J; ++jj) {
-            float kx[VEC], vx[VEC], o[VEC];
-            load_vec<KV, VEC>(ks + (pr * J + jj) * CG, kx);
-            load_vec<KV, VEC>(vs + (pr * J + jj) * CG, vx);
+      for (int e = 0; e < VEC; ++e) st[e] = combine(acc_unpack(sh_x[cl + e]), pre[e], (float)(wp * J), w[e]);
+      OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
+      const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
+      if (fast) {
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-              o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
-              add_token(st[e], kx[e], vx[e], w[e]);
-            }
-            store_out<OUT, VEC>(orow + (size_t)jj * C, c0, C, vec_ok, o);
-          }
-        } else {
-          for (int jj = 0; jj < nv; ++jj) {
+        for (int i = 0; i < J; ++i) {
+          if (i < nv) {
             float kx[VEC], vx[VEC], o[VEC];
-            load_vec<KV, VEC>(ks + (pr * J + jj) * CG, kx);
-            load_vec<KV, VEC>(vs + (pr * J + jj) * CG, vx);
+            load_vec<KV, VEC>(ks + i * CG, kx);
+            load_vec<KV, VEC>(vs + i * CG, vx);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-              o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
-              add_token(st[e], kx[e], vx[e], w[e]);
+            for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+            if (lane_vec) {
+              stg_stream<OUT, VEC>(orow + (size_t)i * C, o);
+            } else {
+#pragma unroll
+              for (int e = 0; e < VEC; ++e)
+                if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
             }
-            store_out<OUT, VEC>(orow + (size_t)jj * C, c0, C, vec_ok, o);
           }
         }
-        if (last_chunk && pr == p_last && p.o_num) {
+      } else {
+        for (int i = 0; i < nv; ++i) {
+          float kx[VEC], vx[VEC], o[VEC];
+          load_vec<KV, VEC>(ks + i * CG, kx);
+          load_vec<KV, VEC>(vs + i * CG, vx);
 #pragma unroll
           for (int e = 0; e < VEC; ++e) {
-            if (c0 + e < C) {
-              const size_t i = (size_t)b * C + c0 + e;
-              p.o_num[i] = st[e].num;
-              p.o_den[i] = st[e].den;
-              p.o_max[i] = acc_max_e(st[e], w[e]);
-            }
+            o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
+            add_token(st[e], kx[e], vx[e], w[e]);
+          }
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
+        }
+      }
+      if (last_chunk && wp == p_last && p.o_num) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          if (c0 + e < C) {
+            const size_t i = (size_t)b * C + c0 + e;
+            p.o_num[i] = st[e].num;
+            p.o_den[i] = st[e].den;
+            p.o_max[i] = acc_max_e(st[e], w[e]);
           }
         }
       }
     }
-    __syncthreads();  // stage s and buf are free again
+    if (kTMA && !copy_ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
   }
 
-  // leave: report, drain a copy still in flight (bounded), hand the workspace
-  // back for the next launch
-  if (timed_out) atomicOr(&p.hdr->status, kStatusWaitTimeout);
-  if (kTMA && tid == 0 && stuck_it >= 0) {
-    // the late copy, and the prefetch issued in the same iteration: bounded
-    (void)mbar_wait(&full[stuck_it & 1], (stuck_it >> 1) & 1, p.timeout_ns);
-    const int nx = stuck_it + 1;
-    if (tile_id[nx & 1] < p.n_tiles) (void)mbar_wait(&full[nx & 1], (nx >> 1) & 1, p.timeout_ns);
-  }
+  // ---- hand the workspace back for the next launch once every tile is done
   __syncthreads();
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     __threadfence();
     const uint32_t prev = atomicAdd(&p.hdr->done, 1u);
-    if (prev == gridDim.x - 1) {
+    if (prev == (uint32_t)p.n_tiles - 1u) {
       p.hdr->ticket = 0;
       p.hdr->done = 0;
       __threadfence();
       atomicExch(&p.hdr->epoch, target);
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// two-launch chunked scan for inputs that fit in L2
+// ---------------------------------------------------------------------------
+//
+// When k and v together fit comfortably in the 126 MB L2, the scan runs as two
+// launches with no waiting between CTAs at all:
+//   A (wkv_chunk_totals): every tile streams its k, v box from HBM once, folds
+//     each warp's span into an aggregate, and writes the tile total and the
+//     in-tile prefix of every warp to the workspace;
+//   B (wkv_chunk_replay): every tile loads its box again -- from L2 -- while
+//     its scan warp combines the state in with the totals of the tile's
+//     earlier chunks; every compute warp then replays its span from
+//     (incoming state + its in-tile prefix).
+// B is launched with programmatic stream serialization: its CTAs start their
+// TMA copies (inputs only) as A drains, and wait (griddepcontrol.wait) before
+// reading anything A wrote.
+
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename KV, int NW, int J, bool kTMA>
+__global__ void __launch_bounds__(NW * 32)
+    wkv_chunk_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  constexpr int VEC = 2;
+  constexpr int CG = 32 * VEC;
+  constexpr int L = NW * J;
+  constexpr int kTile = L * CG;
+  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
+  extern __shared__ __align__(1024) unsigned char smem[];
+  KV* ktile = reinterpret_cast<KV*>(smem);
+  KV* vtile = ktile + kTile;
+  float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_agg + NW * CG);
+
+  const int lane = threadIdx.x & 31;
+  const int wp = threadIdx.x >> 5;
+  const int T = p.T, C = p.C;
+  const int BNG = p.B * p.NG;
+  const int tile = blockIdx.x;
+  const int j = tile / BNG;
+  const int bg = tile % BNG;
+  const int b = bg / p.NG, g = bg % p.NG;
+  const int t0 = j * L;
+  if (kTMA && threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, kBytes);
+    tma_load_3d(ktile, &tmk, bar, g * CG, t0, b);
+    tma_load_3d(vtile, &tmv, bar, g * CG, t0, b);
+  }
+  __syncthreads();
+  // the replay launch may start its own copies now
+  grid_launch_dependents();
+  const int cl = lane * VEC;
+  const int c0 = g * CG + cl;
+  float w[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < C) ? __ldg(p.w + c0 + e) : 0.f;
+  const int ts = t0 + wp * J;
+  const int nv = max(0, min(J, T - ts));
+  if (kTMA) {
+    if (!mbar_wait(bar, 0, p.timeout_ns)) {
+      if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+    }
+  } else {
+    for (int i = threadIdx.x; i < kTile; i += NW * 32) {
+      const int r = i / CG, cc = i % CG;
+      const int t = t0 + r, c = g * CG + cc;
+      KV kk = Elem<KV>::from_f32(0.f), vv = Elem<KV>::from_f32(0.f);
+      if (t < T && c < C) {
+        kk = reinterpret_cast<const KV*>(p.k)[((size_t)b * T + t) * C + c];
+        vv = reinterpret_cast<const KV*>(p.v)[((size_t)b * T + t) * C + c];
+      }
+      ktile[i] = kk;
+      vtile[i] = vv;
+    }
+    __syncthreads();
+  }
+  Acc agg[VEC];
+  aggregate_tile_span<KV, J, VEC, CG>(ktile + (wp * J) * CG + cl, vtile + (wp * J) * CG + cl, nv, w, agg);
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(agg[e]);
+  __syncthreads();
+  Acc pre[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) pre[e] = acc_empty();
+  for (int q = 0; q < wp; ++q) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) pre[e] = combine(pre[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+  }
+  float4* dpre = p.agg_p + ((size_t)tile * NW + wp) * CG + cl;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) dpre[e] = acc_pack(pre[e]);
+  if (wp == NW - 1) {
+    // chunk 0 reads the state in once, keeps a copy for its replay, and folds
+    // it into its total; the replay launch never reads the caller's state
+    // (which state_out may alias)
+    float4* dtot = p.agg_a + (size_t)tile * CG + cl;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const Acc tot = combine(pre[e], agg[e], (float)nv, w[e]);
+      if (j == 0) {
+        const Acc x = state_in_acc(p, b, c0 + e);
+        p.x0[(size_t)bg * CG + cl + e] = acc_pack(x);
+        dtot[e] = acc_pack(combine(x, tot, (float)min(L, T - t0), w[e]));
+      } else {
+        dtot[e] = acc_pack(tot);
+      }
+    }
+  }
+}
+
+template <typename KV, typename OUT, int NW, int J, bool kTMA>
+__global__ void __launch_bounds__((NW + 1) * 32)
+    wkv_chunk_replay(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  constexpr int VEC = 2;
+  constexpr int CG = 32 * VEC;
+  constexpr int L = NW * J;
+  constexpr int kTile = L * CG;
+  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
+  extern __shared__ __align__(1024) unsigned char smem[];
+  KV* ktile = reinterpret_cast<KV*>(smem);
+  KV* vtile = ktile + kTile;
+  float4* sh_x = reinterpret_cast<float4*>(smem + kBytes);  // [CG]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_x + CG);
+
+  const int lane = threadIdx.x & 31;
+  const int wp = threadIdx.x >> 5;
+  const bool scan = (wp == NW);
+  const int T = p.T, C = p.C;
+  const int BNG = p.B * p.NG;
+  const int tile = blockIdx.x;
+  const int j = tile / BNG;
+  const int bg = tile % BNG;
+  const int b = bg / p.NG, g = bg % p.NG;
+  const int t0 = j * L;
+  // the inputs are not written by the totals launch: copy them right away
+  if (kTMA && threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, kBytes);
+    tma_load_3d(ktile, &tmk, bar, g * CG, t0, b);
+    tma_load_3d(vtile, &tmv, bar, g * CG, t0, b);
+  }
+  __syncthreads();
+  const int cl = lane * VEC;
+  const int c0 = g * CG + cl;
+  float w[VEC], u[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    const bool ok = c0 + e < C;
+    w[e] = ok ? __ldg(p.w + c0 + e) : 0.f;
+    u[e] = ok ? __ldg(p.u + c0 + e) : 0.f;
+  }
+  // everything below reads what the totals launch wrote
+  grid_wait_prerequisites();
+  if (scan) {
+    Acc x[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) x[e] = (j == 0) ? acc_unpack(p.x0[(size_t)bg * CG + cl + e]) : acc_empty();
+    for (int jj = 0; jj < j; ++jj) {
+      const float4* src = p.agg_a + ((size_t)jj * BNG + bg) * CG + cl;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) x[e] = combine(x[e], acc_unpack(src[e]), (float)L, w[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) sh_x[cl + e] = acc_pack(x[e]);
+    named_sync<(NW + 1) * 32>(2);
+  } else {
+    const int ts = t0 + wp * J;
+    const int nv = max(0, min(J, T - ts));
+    const bool last_chunk = (j == p.nch - 1);
+    const int p_last = last_chunk ? (T - 1 - t0) / J : NW - 1;
+    Acc pre[VEC];
+    const float4* spre = p.agg_p + ((size_t)tile * NW + wp) * CG + cl;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) pre[e] = acc_unpack(spre[e]);
+    bool copy_ok = true;
+    if (kTMA) {
+      copy_ok = mbar_wait(bar, 0, p.timeout_ns);
+      if (!copy_ok && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+    } else {
+      for (int i = threadIdx.x; i < kTile; i += NW * 32) {
+        const int r = i / CG, cc = i % CG;
+        const int t = t0 + r, c = g * CG + cc;
+        KV kk = Elem<KV>::from_f32(0.f), vv = Elem<KV>::from_f32(0.f);
+        if (t < T && c < C) {
+          kk = reinterpret_cast<const KV*>(p.k)[((size_t)b * T + t) * C + c];
+          vv = reinterpret_cast<const KV*>(p.v)[((size_t)b * T + t) * C + c];
+        }
+        ktile[i] = kk;
+        vtile[i] = vv;
+      }
+    }
+    named_sync<(NW + 1) * 32>(2);  // incoming state (and, without TMA, the tile) ready
+    if (nv > 0 && copy_ok) {
+      float cb[VEC];
+      bool fast = true;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        fast &= fast_uw(u[e], w[e]);
+        cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+      }
+      fast = __all_sync(0xffffffffu, fast);
+      Acc st[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) st[e] = combine(acc_unpack(sh_x[cl + e]), pre[e], (float)(wp * J), w[e]);
+      const KV* ks = ktile + (wp * J) * CG + cl;
+      const KV* vs = vtile + (wp * J) * CG + cl;
+      OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
+      const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
+      if (fast) {
+#pragma unroll
+        for (int i = 0; i < J; ++i) {
+          if (i < nv) {
+            float kx[VEC], vx[VEC], o[VEC];
+            load_vec<KV, VEC>(ks + i * CG, kx);
+            load_vec<KV, VEC>(vs + i * CG, vx);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+            if (lane_vec) {
+              stg_stream<OUT, VEC>(orow + (size_t)i * C, o);
+            } else {
+#pragma unroll
+              for (int e = 0; e < VEC; ++e)
+                if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
+            }
+          }
+        }
+      } else {
+        for (int i = 0; i < nv; ++i) {
+          float kx[VEC], vx[VEC], o[VEC];
+          load_vec<KV, VEC>(ks + i * CG, kx);
+          load_vec<KV, VEC>(vs + i * CG, vx);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
+            add_token(st[e], kx[e], vx[e], w[e]);
+          }
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
+        }
+      }
+      if (last_chunk && wp == p_last && p.o_num) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          if (c0 + e < C) {
+            const size_t i = (size_t)b * C + c0 + e;
+            p.o_num[i] = st[e].num;
+            p.o_den[i] = st[e].den;
+            p.o_max[i] = acc_max_e(st[e], w[e]);
+          }
+        }
+      }
+    }
+    if (kTMA && !copy_ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
   }
 }
 
