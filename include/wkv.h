@@ -94,6 +94,10 @@ typedef struct {
  *                   chunk_len / span warps share a tile
  *   seq_threads     threads per CTA of the sequential kernel: 32, 64 or 128
  *                   (0 = choose); each thread carries 2 channels
+ *   replay          how the span-streaming scan (kernel 3) replays its spans:
+ *                   0 = choose, 1 = through per-warp TMA rings in shared
+ *                   memory, 2 = with loads straight into registers
+ *   reserved        must be 0
  *   inject_enable, inject_unpublished_tile
  *                   tests of the bounded waits only: with inject_enable = 1,
  *                   chunk-scan tile number inject_unpublished_tile computes
@@ -110,6 +114,8 @@ typedef struct {
     int64_t inject_unpublished_tile;
     int32_t span;
     int32_t seq_threads;
+    int32_t replay;
+    int32_t reserved;
 } wkv_options;
 
 /*

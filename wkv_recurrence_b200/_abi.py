@@ -42,7 +42,8 @@ class wkv_options(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
                 ("lookback_group", ctypes.c_int32), ("inject_enable", ctypes.c_int32),
                 ("wait_timeout_ns", ctypes.c_int64), ("inject_unpublished_tile", ctypes.c_int64),
-                ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32)]
+                ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32),
+                ("replay", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class WkvError(RuntimeError):

@@ -38,6 +38,7 @@ constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 struct Plan {
   int kernel;  // 1 seq, 2 chunked single launch, 3 chunked two launches (L2-resident inputs)
   int seq_threads;  // CTA width of the sequential kernel
+  int replay;       // span-streaming replay: 1 TMA rings, 2 loads into registers
   int L;       // chunk length (chunk kernel)
   int J;       // tokens per warp (chunk kernel)
   int G;       // look-back group
@@ -48,14 +49,18 @@ struct Plan {
   size_t off_flags_a, off_flags_p, off_agg_a, off_agg_p, off_x0, bytes;
 };
 
-// Inputs up to this size take the two-launch scan (they stay in L2 between
-// the launches; B200 has 126 MB of L2).
-constexpr int64_t kL2ResidentBytes = 64ll << 20;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, int kv_bytes = 4) {
+// The plan for a call: which kernel, tile sizes, and the workspace layout.
+// tma_ok = false (inputs that TMA cannot address: misaligned base, row pitch
+// not a multiple of 16 bytes) turns the three-launch scan, which needs TMA,
+// into the single-launch one. A three-launch plan reserves enough workspace
+// for either, so a workspace sized by wkv_forward_workspace_size always fits.
+bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, int kv_bytes = 4,
+               bool tma_ok = true) {
   std::memset(pl, 0, sizeof *pl);
+  (void)kv_bytes;
   const int want = o ? o->kernel : 0;
   if (want < 0 || want > 3) return false;
   const int64_t lanes = B * C;
@@ -64,15 +69,17 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     if (lanes >= 65536 || T <= 64) {
       kernel = 1;
     } else {
-      const int Ld = (o && o->chunk_len) ? o->chunk_len : 128;
-      const int64_t nch = (T + Ld - 1) / Ld;
-      kernel = (2 * B * T * C * kv_bytes <= kL2ResidentBytes && nch <= 64) ? 3 : 2;
+      kernel = 2;
     }
   }
+  const bool three_requested = (kernel == 3);
+  if (kernel == 3 && !tma_ok) kernel = 2;
   pl->kernel = kernel;
   pl->bytes = sizeof(WsHeader);
+  if (o && (o->reserved != 0 || o->replay < 0 || o->replay > 2)) return false;
+  pl->replay = (o && o->replay) ? o->replay : 2;
   int sth = o ? o->seq_threads : 0;
-  if (sth == 0) sth = 128;
+  if (sth == 0) sth = 32;  // many small CTAs: more resident warps per SM
   if (sth != 32 && sth != 64 && sth != 128) return false;
   pl->seq_threads = sth;
   if (kernel == 1) return true;
@@ -95,17 +102,15 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   pl->n_tiles = (long long)pl->nch * BNG;
   if (pl->n_tiles >= (1ll << 31)) return false;
   pl->nblk = (pl->nch + G - 1) / G;
-  if (kernel == 3) {
-    size_t off = sizeof(WsHeader);
-    pl->off_agg_a = off;
-    off = round_up(off + sizeof(float4) * (size_t)pl->n_tiles * kChunkCG, 256);
-    pl->off_agg_p = off;
-    off = round_up(off + sizeof(float4) * (size_t)pl->n_tiles * (L / J) * kChunkCG, 256);
-    pl->off_x0 = off;
-    off = round_up(off + sizeof(float4) * (size_t)BNG * kChunkCG, 256);
-    pl->bytes = off;
-    return true;
-  }
+  // span-streaming layout: span aggregates, span incoming states
+  const long long n_spans = (long long)((T + J - 1) / J) * BNG;
+  if (n_spans >= (1ll << 31)) return false;
+  size_t off3 = sizeof(WsHeader);
+  const size_t t_agg_a = off3;
+  off3 = round_up(off3 + sizeof(float4) * (size_t)n_spans * kChunkCG, 256);
+  const size_t t_x0 = off3;
+  off3 = round_up(off3 + sizeof(float4) * (size_t)n_spans * kChunkCG, 256);
+  // single-launch layout: flags, chunk totals, group prefixes
   size_t off = sizeof(WsHeader);
   pl->off_flags_a = off;
   off = round_up(off + sizeof(uint32_t) * (size_t)pl->n_tiles, 256);
@@ -115,8 +120,21 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   off = round_up(off + sizeof(float4) * (size_t)pl->n_tiles * kChunkCG, 256);
   pl->off_agg_p = off;
   off = round_up(off + sizeof(float4) * (size_t)(pl->nblk * BNG) * kChunkCG, 256);
-  pl->bytes = off;
+  if (kernel == 3) {
+    pl->off_flags_a = pl->off_flags_p = pl->off_agg_p = 0;
+    pl->off_agg_a = t_agg_a;
+    pl->off_x0 = t_x0;
+    pl->n_tiles = n_spans;
+    pl->bytes = std::max(off3, off);
+  } else {
+    pl->bytes = three_requested ? std::max(off3, off) : off;
+  }
   return true;
+}
+
+bool tma_usable(const void* k, const void* v, int64_t C, size_t es) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(k), b = reinterpret_cast<uintptr_t>(v);
+  return a % 16 == 0 && b % 16 == 0 && (C * (int64_t)es) % 16 == 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -230,6 +248,7 @@ wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorM
 
 template <typename KV, typename OUT, int NW, int J, bool kTMA>
 wkv_status launch_chunk(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
+  if (!p.flags_a || !p.flags_p || !p.agg_a || !p.agg_p || !p.hdr) return WKV_ERR_INVALID_ARG;
   constexpr int L = NW * J;
   const size_t smem = 2ull * L * kChunkCG * sizeof(KV) + sizeof(float4) * (NW + 1) * kChunkCG + 64;
   auto fn = wkv_fwd_chunk<KV, OUT, NW, J, kTMA>;
@@ -239,50 +258,59 @@ wkv_status launch_chunk(const FwdParams& p, const CUtensorMap& tk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
-template <typename KV, typename OUT, int NW, int J, bool kTMA>
-wkv_status launch_two(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
-  constexpr int L = NW * J;
-  const size_t tile = 2ull * L * kChunkCG * sizeof(KV);
-  const size_t smem_a = tile + sizeof(float4) * NW * kChunkCG + 64;
-  const size_t smem_b = tile + sizeof(float4) * kChunkCG + 64;
-  auto fa = wkv_chunk_totals<KV, NW, J, kTMA>;
-  auto fb = wkv_chunk_replay<KV, OUT, NW, J, kTMA>;
-  int occ = 0;
-  if (!kernel_setup(fa, dev, NW * 32, smem_a, &occ) || occ < 1) return WKV_ERR_CUDA;
-  if (!kernel_setup(fb, dev, (NW + 1) * 32, smem_b, &occ) || occ < 1) return WKV_ERR_CUDA;
-  fa<<<(unsigned)p.n_tiles, NW * 32, smem_a, st>>>(p, tk, tv);
-  if (cudaGetLastError() != cudaSuccess) return WKV_ERR_CUDA;
-  // the replay launch may begin while the totals launch drains: it copies its
-  // inputs first and waits (griddepcontrol.wait) before reading any total
+// Launch configuration with programmatic stream serialization: the launch may
+// begin while the previous one on the stream drains; the kernel orders itself
+// with griddepcontrol.
+struct PdlConfig {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.n_tiles);
-  cfg.blockDim = dim3((NW + 1) * 32);
-  cfg.dynamicSmemBytes = smem_b;
-  cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, fb, p, tk, tv) != cudaSuccess) return WKV_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
-}
+  PdlConfig(dim3 grid, dim3 block, size_t smem, cudaStream_t st) {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
 
-template <typename KV, typename OUT, bool kTMA>
-wkv_status launch_two_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                            cudaStream_t st, int dev) {
-  if (pl.J == 8) {
-    switch (pl.L) {
-      case 32: return launch_two<KV, OUT, 4, 8, kTMA>(p, tk, tv, st, dev);
-      case 64: return launch_two<KV, OUT, 8, 8, kTMA>(p, tk, tv, st, dev);
-      default: return launch_two<KV, OUT, 16, 8, kTMA>(p, tk, tv, st, dev);
-    }
+template <typename KV, typename OUT, int J>
+wkv_status launch_spans(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev,
+                        int sms) {
+  if (!p.agg_a || !p.x0 || !p.hdr) return WKV_ERR_INVALID_ARG;
+  // per-warp rings of 3 span stages; about 192 KB of shared memory per SM
+  constexpr int STAGES = 3;
+  constexpr int kSpanBytes = 2 * J * 64 * (int)sizeof(KV);
+  constexpr int WARPS = (192 * 1024 / (STAGES * kSpanBytes)) > 16 ? 16 : (192 * 1024 / (STAGES * kSpanBytes));
+  const size_t smem = (size_t)WARPS * STAGES * (kSpanBytes + 8);
+  auto fa = wkv_span_totals<KV, J, STAGES, WARPS>;
+  auto fb = wkv_span_replay<KV, OUT, J, STAGES, WARPS>;
+  auto fs = wkv_span_scan<8>;
+  int occ_a = 0, occ_b = 0;
+  if (!kernel_setup(fa, dev, WARPS * 32, smem, &occ_a) || occ_a < 1) return WKV_ERR_CUDA;
+  if (!kernel_setup(fb, dev, WARPS * 32, smem, &occ_b) || occ_b < 1) return WKV_ERR_CUDA;
+  const long long blocks_needed = (p.n_tiles + WARPS - 1) / WARPS;
+  const unsigned ga = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_a * sms, blocks_needed));
+  const unsigned gb = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_b * sms, blocks_needed));
+  fa<<<ga, WARPS * 32, smem, st>>>(p, tk, tv);
+  if (cudaGetLastError() != cudaSuccess) return WKV_ERR_CUDA;
+  PdlConfig cs(dim3((unsigned)((long long)p.B * p.NG)), dim3(64 * 8), 0, st);
+  if (cudaLaunchKernelEx(&cs.cfg, fs, p, (int)J) != cudaSuccess) return WKV_ERR_CUDA;
+  if (p.replay_mode == 1) {
+    // replay straight from L2 into registers
+    auto fr = wkv_span_replay_ldg<KV, OUT, J>;
+    int occ_r = 0;
+    if (!kernel_setup(fr, dev, 256, 0, &occ_r) || occ_r < 1) return WKV_ERR_CUDA;
+    const unsigned gr = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_r * sms, (p.n_tiles + 7) / 8));
+    PdlConfig cr(dim3(gr), dim3(256), 0, st);
+    if (cudaLaunchKernelEx(&cr.cfg, fr, p) != cudaSuccess) return WKV_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   }
-  switch (pl.L) {
-    case 32: return launch_two<KV, OUT, 2, 16, kTMA>(p, tk, tv, st, dev);
-    case 64: return launch_two<KV, OUT, 4, 16, kTMA>(p, tk, tv, st, dev);
-    default: return launch_two<KV, OUT, 8, 16, kTMA>(p, tk, tv, st, dev);
-  }
+  PdlConfig cb(dim3(gb), dim3(WARPS * 32), smem, st);
+  if (cudaLaunchKernelEx(&cb.cfg, fb, p, tk, tv) != cudaSuccess) return WKV_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
 template <typename KV, typename OUT, bool kTMA>
@@ -325,15 +353,19 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
     }
     return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
   }
-  (void)sms;
+  if (pl.kernel == 3) {  // span streaming (make_plan only chooses it when TMA works)
+    if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.J, kChunkCG) ||
+        !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.J, kChunkCG))
+      return WKV_ERR_CUDA;
+    if (pl.J == 8) return launch_spans<KV, OUT, 8>(p, tk, tv, st, dev, sms);
+    return launch_spans<KV, OUT, 16>(p, tk, tv, st, dev, sms);
+  }
   if (tma) {
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
         !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
       return WKV_ERR_CUDA;
-    if (pl.kernel == 3) return launch_two_shape<KV, OUT, true>(pl, p, tk, tv, st, dev);
     return launch_chunk_shape<KV, OUT, true>(pl, p, tk, tv, st, dev);
   }
-  if (pl.kernel == 3) return launch_two_shape<KV, OUT, false>(pl, p, tk, tv, st, dev);
   return launch_chunk_shape<KV, OUT, false>(pl, p, tk, tv, st, dev);
 }
 
@@ -382,8 +414,12 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   if (state_out && (!state_out->num || !state_out->den || !state_out->max_e)) return WKV_ERR_INVALID_ARG;
   if (opts && opts->wait_timeout_ns < 0) return WKV_ERR_INVALID_ARG;
   if (opts && (opts->inject_enable != 0 && opts->inject_enable != 1)) return WKV_ERR_INVALID_ARG;
+  const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
+  // TMA needs 16-byte aligned bases and row pitches; otherwise the kernels
+  // fill their tiles with plain loads
+  const bool tma = tma_usable(k, v, C, kes);
   Plan pl;
-  if (!make_plan(B, T, C, opts, &pl, kv_dtype == WKV_F32 ? 4 : 2)) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, opts, &pl, (int)kes, tma)) return WKV_ERR_INVALID_ARG;
   if (!workspace) return WKV_ERR_INVALID_ARG;
   if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
@@ -451,13 +487,10 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
     if (pl.kernel == 3) {
       p.flags_a = p.flags_p = nullptr;
       p.x0 = reinterpret_cast<float4*>(ws + pl.off_x0);
+      p.replay_mode = pl.replay == 2 ? 1 : 0;
     }
   }
-  const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
   const size_t oes = out_dtype == WKV_F32 ? 4 : 2;
-  // TMA needs 16-byte aligned bases and row pitches; otherwise the same
-  // kernels fill their tiles with plain loads
-  const bool tma = aligned(k, 16) && aligned(v, 16) && (C * kes) % 16 == 0;
   const int vec = pl.kernel == 1 ? (tma ? (kv_dtype == WKV_F32 ? kSeqVecF32 : kSeqVecBf16) : kSeqFallbackVec)
                                  : kChunkVec;
   p.vec_store = aligned(out, oes * vec) && (C % vec) == 0;
@@ -571,7 +604,8 @@ wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, c
                                const wkv_cstate* state_in, const wkv_state* state_out, void* stream) {
   if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
   Plan pl;
-  if (!make_plan(B, T, C, nullptr, &pl, kv_dtype == WKV_BF16 ? 2 : 4)) return WKV_ERR_INVALID_ARG;
+  const size_t kes = kv_dtype == WKV_BF16 ? 2 : 4;
+  if (!make_plan(B, T, C, nullptr, &pl, (int)kes, tma_usable(k, v, C, kes))) return WKV_ERR_INVALID_ARG;
   if (pl.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (B * C == 0) {
     // nothing to compute: wkv_forward checks the other arguments and returns

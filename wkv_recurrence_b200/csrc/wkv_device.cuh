@@ -396,6 +396,46 @@ __device__ __forceinline__ float step_token(Acc& s, float k, float v, float w, f
 
 __device__ __forceinline__ bool fast_uw(float u, float w) { return fabsf(u - w) <= kFastUW; }
 
+// step_token over N consecutive tokens of VEC channels, reorganised for
+// instruction-level parallelism. Only the anchor and count are carried from
+// token to token through a short chain (fma, subtract, compare, select), and
+// only it runs first, for all N tokens; the exponentials, the num/den updates
+// and the outputs of the N tokens then have no dependency on each other
+// beyond one fma per token, so their latencies overlap. Every token goes
+// through exactly the operations of step_token, in the same order, so the
+// results are bitwise the same.
+template <int N, int VEC>
+__device__ __forceinline__ void step_tokens(Acc (&s)[VEC], const float (&k)[N][VEC], const float (&v)[N][VEC],
+                                            const float (&w)[VEC], const float (&c)[VEC], float (&out)[N][VEC]) {
+  float d2[N][VEC];
+  bool rs[N][VEC];
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const float nf1 = s[e].nf + 1.f;
+      const float Md = fmaf(-nf1, w[e], s[e].ma);
+      d2[i][e] = k[i][e] - Md;
+      rs[i][e] = d2[i][e] > 0.f;
+      s[e].ma = rs[i][e] ? k[i][e] : s[e].ma;
+      s[e].nf = rs[i][e] ? 0.f : nf1;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const float x = ex2(-fabsf(d2[i][e]) * kLog2e);
+      const float a = rs[i][e] ? x : 1.f;
+      const float b = rs[i][e] ? 1.f : x;
+      const float bc = b * c[e];
+      out[i][e] = fmaf(bc, v[i][e], a * s[e].num) * rcp(fmaf(a, s[e].den, bc));
+      s[e].num = fmaf(a, s[e].num, b * v[i][e]);
+      s[e].den = fmaf(a, s[e].den, b);
+    }
+  }
+}
+
 __device__ __forceinline__ float bonus_factor(float u, float w) {
   return ex2((u - w) * kLog2e);
 }

@@ -70,7 +70,8 @@ struct FwdParams {
   uint32_t* flags_p;   // [nblk * B * NG]
   float4* agg_a;       // [n_tiles][CG]
   float4* agg_p;       // [nblk * B * NG][CG] (single launch) or [n_tiles][NW][CG] (two launches)
-  float4* x0;          // [B * NG][CG]: state in, anchored (two launches)
+  float4* x0;          // incoming states of spans (span-streaming scan)
+  int replay_mode;     // span-streaming replay: 0 = TMA rings, 1 = loads into registers
 };
 
 // State in for one channel, anchored; empty when no state is passed.
@@ -181,14 +182,18 @@ __global__ void __launch_bounds__(THREADS)
     OUT* orow = out + ((size_t)b * T + t0) * C;
     if (c0 < C) {
       if (nv == LT && fast) {
-#pragma unroll 4
-        for (int j = 0; j < LT; ++j) {
-          float kx[VEC], vx[VEC], o[VEC];
-          load_vec<KV, VEC>(ks + j * CG, kx);
-          load_vec<KV, VEC>(vs + j * CG, vx);
+        constexpr int NB = LT < 8 ? LT : 8;  // tokens per block of step_tokens
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
-          store_out<OUT, VEC>(orow + (size_t)j * C, c0, C, vec_ok, o);
+        for (int j0 = 0; j0 < LT; j0 += NB) {
+          float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
+#pragma unroll
+          for (int jj = 0; jj < NB; ++jj) {
+            load_vec<KV, VEC>(ks + (j0 + jj) * CG, kb[jj]);
+            load_vec<KV, VEC>(vs + (j0 + jj) * CG, vb[jj]);
+          }
+          step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
+#pragma unroll
+          for (int jj = 0; jj < NB; ++jj) store_out<OUT, VEC>(orow + (size_t)(j0 + jj) * C, c0, C, vec_ok, ob[jj]);
         }
       } else if (nv == LT) {
 #pragma unroll 4
@@ -267,6 +272,21 @@ __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_re
 template <int N>
 __device__ __forceinline__ void named_sync(int id) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(N) : "memory");
+}
+
+// Named barrier that also ORs a predicate over the N participating threads.
+template <int N>
+__device__ __forceinline__ bool named_sync_or(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "n"(N)
+      : "memory");
+  return r != 0;
 }
 
 // Aggregate of one warp's span of n <= J tokens from the empty state, read
@@ -518,23 +538,38 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       for (int e = 0; e < VEC; ++e) st[e] = combine(acc_unpack(sh_x[cl + e]), pre[e], (float)(wp * J), w[e]);
       OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
       const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
-      if (fast) {
+      if (fast && nv == J) {
+        constexpr int NB = J < 8 ? J : 8;  // tokens per block of step_tokens
 #pragma unroll
-        for (int i = 0; i < J; ++i) {
-          if (i < nv) {
-            float kx[VEC], vx[VEC], o[VEC];
-            load_vec<KV, VEC>(ks + i * CG, kx);
-            load_vec<KV, VEC>(vs + i * CG, vx);
+        for (int i0 = 0; i0 < J; i0 += NB) {
+          float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+          for (int ii = 0; ii < NB; ++ii) {
+            load_vec<KV, VEC>(ks + (i0 + ii) * CG, kb[ii]);
+            load_vec<KV, VEC>(vs + (i0 + ii) * CG, vb[ii]);
+          }
+          step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
+#pragma unroll
+          for (int ii = 0; ii < NB; ++ii) {
             if (lane_vec) {
-              stg_stream<OUT, VEC>(orow + (size_t)i * C, o);
+              stg_stream<OUT, VEC>(orow + (size_t)(i0 + ii) * C, ob[ii]);
             } else {
 #pragma unroll
               for (int e = 0; e < VEC; ++e)
-                if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
+                if (c0 + e < C) orow[(size_t)(i0 + ii) * C + e] = Elem<OUT>::from_f32(ob[ii][e]);
             }
           }
+        }
+      } else if (fast) {
+        for (int i = 0; i < nv; ++i) {
+          float kx[VEC], vx[VEC], o[VEC];
+          load_vec<KV, VEC>(ks + i * CG, kx);
+          load_vec<KV, VEC>(vs + i * CG, vx);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
         }
       } else {
         for (int i = 0; i < nv; ++i) {
@@ -581,264 +616,464 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 }
 
 // ---------------------------------------------------------------------------
-// two-launch chunked scan for inputs that fit in L2
+// span-streaming scan in three launches, for inputs that fit in L2
 // ---------------------------------------------------------------------------
 //
-// When k and v together fit comfortably in the 126 MB L2, the scan runs as two
-// launches with no waiting between CTAs at all:
-//   A (wkv_chunk_totals): every tile streams its k, v box from HBM once, folds
-//     each warp's span into an aggregate, and writes the tile total and the
-//     in-tile prefix of every warp to the workspace;
-//   B (wkv_chunk_replay): every tile loads its box again -- from L2 -- while
-//     its scan warp combines the state in with the totals of the tile's
-//     earlier chunks; every compute warp then replays its span from
-//     (incoming state + its in-tile prefix).
-// B is launched with programmatic stream serialization: its CTAs start their
-// TMA copies (inputs only) as A drains, and wait (griddepcontrol.wait) before
-// reading anything A wrote.
+// A span is 64 channels of one batch row by J consecutive tokens. When k and v
+// together fit comfortably in the 126 MB L2:
+//   A (wkv_span_totals): every warp streams spans from HBM through its own
+//     ring of TMA stages and writes each span's aggregate (from the empty
+//     state) to the workspace;
+//   S (wkv_span_scan): for each (batch row, channel), the incoming state of
+//     every span: the state in combined with the aggregates of all earlier
+//     spans, as a two-level scan (segments of spans, then within segments);
+//   B (wkv_span_replay): every warp streams spans again -- from L2 -- and
+//     replays each from its incoming state, writing the outputs.
+// No warp ever waits for another warp or CTA inside a launch. S and B are
+// launched with programmatic stream serialization: B's warps start copying
+// their first spans (inputs only) while S runs, and wait (griddepcontrol.wait)
+// before reading any incoming state. Only S reads the caller's state in, and
+// it completes before B writes the state out, so the two may alias.
 
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void grid_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-template <typename KV, int NW, int J, bool kTMA>
-__global__ void __launch_bounds__(NW * 32)
-    wkv_chunk_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-  constexpr int VEC = 2;
-  constexpr int CG = 32 * VEC;
-  constexpr int L = NW * J;
-  constexpr int kTile = L * CG;
-  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
-  extern __shared__ __align__(1024) unsigned char smem[];
-  KV* ktile = reinterpret_cast<KV*>(smem);
-  KV* vtile = ktile + kTile;
-  float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_agg + NW * CG);
+__device__ __forceinline__ float4 ldg_f4(const float4* q) {
+  float4 r;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(q));
+  return r;
+}
 
-  const int lane = threadIdx.x & 31;
-  const int wp = threadIdx.x >> 5;
-  const int T = p.T, C = p.C;
+// Per-warp ring of STAGES span buffers (k box then v box, [J][64] each).
+template <typename KV, int J>
+struct SpanRing {
+  static constexpr int CG = 64;
+  static constexpr int kBox = J * CG;                                     // elements per tensor
+  static constexpr uint32_t kBytes = 2u * kBox * (uint32_t)sizeof(KV);   // per stage
+};
+
+// Span number sp (0 <= sp < n_spans) in time-major order: sp = q * BNG + bg,
+// so consecutive spans cover neighbouring channel groups of the same rows.
+__device__ __forceinline__ void span_coords(const FwdParams& p, int sp, int& q, int& b, int& g, int& bg) {
   const int BNG = p.B * p.NG;
-  const int tile = blockIdx.x;
-  const int j = tile / BNG;
-  const int bg = tile % BNG;
-  const int b = bg / p.NG, g = bg % p.NG;
-  const int t0 = j * L;
-  if (kTMA && threadIdx.x == 0) {
-    mbar_init(bar, 1);
+  q = sp / BNG;
+  bg = sp % BNG;
+  b = bg / p.NG;
+  g = bg % p.NG;
+}
+
+// Walks a warp's spans sp, sp + GW, sp + 2 GW, ... keeping (q, b, g) up to
+// date with additions only (the divisions happen once, at the start).
+struct SpanWalk {
+  int sp, q, b, g;
+  int step, dq, db, dg, B, NG;
+  __device__ __forceinline__ SpanWalk(const FwdParams& p, int first, int stride) {
+    int bg;
+    sp = first;
+    step = stride;
+    span_coords(p, first, q, b, g, bg);
+    B = p.B;
+    NG = p.NG;
+    const int BNG = p.B * p.NG;
+    dq = stride / BNG;
+    const int rb = stride % BNG;
+    db = rb / p.NG;
+    dg = rb % p.NG;
+  }
+  __device__ __forceinline__ void next() {
+    sp += step;
+    g += dg;
+    int carry = g >= NG;
+    g -= carry ? NG : 0;
+    b += db + carry;
+    carry = b >= B;
+    b -= carry ? B : 0;
+    q += dq + carry;
+  }
+};
+
+template <typename KV, int J>
+__device__ __forceinline__ void span_issue(const FwdParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv, KV* buf,
+                                           uint64_t* bar, int sp) {
+  using R = SpanRing<KV, J>;
+  int q, b, g, bg;
+  span_coords(p, sp, q, b, g, bg);
+  mbar_arrive_expect_tx(bar, R::kBytes);
+  tma_load_3d(buf, tmk, bar, g * R::CG, q * J, b);
+  tma_load_3d(buf + R::kBox, tmv, bar, g * R::CG, q * J, b);
+}
+
+// After a warp stopped on a timeout at its i-th span: give the copies it had
+// in flight (its next STAGES spans) a bounded chance to land before it exits.
+template <int STAGES>
+__device__ __forceinline__ void span_ring_drain(const FwdParams& p, uint64_t* full, int i, int gw, int GW) {
+  if ((threadIdx.x & 31) != 0) return;
+  for (int k = i; k < i + STAGES; ++k)
+    if (gw + k * GW < p.n_tiles) (void)mbar_wait(&full[k % STAGES], (k / STAGES) & 1, p.timeout_ns);
+}
+
+// Common prologue of the streaming kernels: per-warp barriers and the first
+// STAGES copies of this warp's spans. Spans of warp gw: gw, gw + GW, ...
+template <typename KV, int J, int STAGES>
+__device__ __forceinline__ void span_ring_start(const FwdParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                                                KV* ring, uint64_t* full, int gw, int GW) {
+  using R = SpanRing<KV, J>;
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar, kBytes);
-    tma_load_3d(ktile, &tmk, bar, g * CG, t0, b);
-    tma_load_3d(vtile, &tmv, bar, g * CG, t0, b);
+    for (int s = 0; s < STAGES; ++s) {
+      const int sp = gw + s * GW;
+      if (sp < p.n_tiles) span_issue<KV, J>(p, tmk, tmv, ring + (size_t)s * 2 * R::kBox, &full[s], sp);
+    }
   }
-  __syncthreads();
-  // the replay launch may start its own copies now
-  grid_launch_dependents();
-  const int cl = lane * VEC;
-  const int c0 = g * CG + cl;
-  float w[VEC];
+  __syncwarp();
+}
+
+template <typename KV, int J, int STAGES, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32)
+    wkv_span_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  using R = SpanRing<KV, J>;
+  constexpr int VEC = 2, CG = R::CG;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  KV* ring = reinterpret_cast<KV*>(smem) + (size_t)wp * STAGES * 2 * R::kBox;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)WARPS * STAGES * R::kBytes) + wp * STAGES;
+  const int GW = gridDim.x * WARPS;
+  const int gw = blockIdx.x * WARPS + wp;
+  if (lane == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  span_ring_start<KV, J, STAGES>(p, &tmk, &tmv, ring, full, gw, GW);
+  const int T = p.T, C = p.C, cl = lane * VEC;
+  int i = 0;
+  SpanWalk it(p, gw, GW);
+  for (; it.sp < p.n_tiles; it.next(), ++i) {
+    const int s = i % STAGES;
+    const int sp = it.sp, q = it.q;
+    const int c0 = it.g * CG + cl;
+    float w[VEC];
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < C) ? __ldg(p.w + c0 + e) : 0.f;
-  const int ts = t0 + wp * J;
-  const int nv = max(0, min(J, T - ts));
-  if (kTMA) {
-    if (!mbar_wait(bar, 0, p.timeout_ns)) {
+    for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < C) ? __ldg(p.w + c0 + e) : 0.f;
+    const int nv = min(J, T - q * J);
+    if (!mbar_wait(&full[s], (i / STAGES) & 1, p.timeout_ns)) {
       if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+      span_ring_drain<STAGES>(p, full, i, gw, GW);
+      break;
     }
-  } else {
-    for (int i = threadIdx.x; i < kTile; i += NW * 32) {
-      const int r = i / CG, cc = i % CG;
-      const int t = t0 + r, c = g * CG + cc;
-      KV kk = Elem<KV>::from_f32(0.f), vv = Elem<KV>::from_f32(0.f);
-      if (t < T && c < C) {
-        kk = reinterpret_cast<const KV*>(p.k)[((size_t)b * T + t) * C + c];
-        vv = reinterpret_cast<const KV*>(p.v)[((size_t)b * T + t) * C + c];
-      }
-      ktile[i] = kk;
-      vtile[i] = vv;
-    }
-    __syncthreads();
-  }
-  Acc agg[VEC];
-  aggregate_tile_span<KV, J, VEC, CG>(ktile + (wp * J) * CG + cl, vtile + (wp * J) * CG + cl, nv, w, agg);
+    KV* buf = ring + (size_t)s * 2 * R::kBox;
+    Acc agg[VEC];
+    aggregate_tile_span<KV, J, VEC, CG>(buf + cl, buf + R::kBox + cl, nv, w, agg);
+    float4* dst = p.agg_a + (size_t)sp * CG + cl;
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(agg[e]);
+    for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(agg[e]);
+    __syncwarp();  // every lane is done with the stage
+    const int nxt = sp + STAGES * GW;
+    if (lane == 0 && nxt < p.n_tiles) {
+      fence_proxy_async_smem();
+      span_issue<KV, J>(p, &tmk, &tmv, buf, &full[s], nxt);
+    }
+  }
+  grid_launch_dependents();
+}
+
+// Two-level scan over the spans of one (batch row, channel): SEG threads per
+// channel each own a contiguous segment of spans. The span aggregates are
+// read-only here (written by the previous launch), so they are loaded through
+// the non-coherent path, eight at a time.
+template <int SEG>
+__global__ void __launch_bounds__(64 * SEG) wkv_span_scan(const FwdParams p, int J) {
+  constexpr int CG = 64;
+  __shared__ float4 seg_tot[SEG][CG];
+  grid_wait_prerequisites();
+  grid_launch_dependents();
+  const int BNG = p.B * p.NG;
+  const int bg = blockIdx.x;
+  const int cl = threadIdx.x % CG;
+  const int sg = threadIdx.x / CG;
+  const int b = bg / p.NG, c = (bg % p.NG) * CG + cl;
+  const float w = c < p.C ? __ldg(p.w + c) : 0.f;
+  const int nsp = (p.T + J - 1) / J;
+  const int per = (nsp + SEG - 1) / SEG;
+  const int q0 = min(nsp, sg * per), q1 = min(nsp, q0 + per);
+  const float fJ = (float)J;
+  // 1. this segment's total (the spans before the last one are full J tokens)
+  Acc tot = acc_empty();
+  for (int qq = q0; qq < q1; qq += 8) {
+    float4 a[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (qq + r < q1) a[r] = ldg_f4(p.agg_a + ((size_t)(qq + r) * BNG + bg) * CG + cl);
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), (float)min(J, p.T - (qq + r) * J), w);
+  }
+  seg_tot[sg][cl] = acc_pack(tot);
   __syncthreads();
-  Acc pre[VEC];
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) pre[e] = acc_empty();
-  for (int q = 0; q < wp; ++q) {
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) pre[e] = combine(pre[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+  // 2. incoming state of the segment, then of every span in it
+  Acc x = state_in_acc(p, b, c);
+  for (int k = 0; k < sg; ++k) {
+    const int kq0 = min(nsp, k * per), kq1 = min(nsp, kq0 + per);
+    x = combine(x, acc_unpack(seg_tot[k][cl]), (float)max(0, min(p.T, kq1 * J) - kq0 * J), w);
   }
-  float4* dpre = p.agg_p + ((size_t)tile * NW + wp) * CG + cl;
+  for (int qq = q0; qq < q1; qq += 8) {
+    float4 a[8];
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) dpre[e] = acc_pack(pre[e]);
-  if (wp == NW - 1) {
-    // chunk 0 reads the state in once, keeps a copy for its replay, and folds
-    // it into its total; the replay launch never reads the caller's state
-    // (which state_out may alias)
-    float4* dtot = p.agg_a + (size_t)tile * CG + cl;
+    for (int r = 0; r < 8; ++r)
+      if (qq + r < q1) a[r] = ldg_f4(p.agg_a + ((size_t)(qq + r) * BNG + bg) * CG + cl);
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const Acc tot = combine(pre[e], agg[e], (float)nv, w[e]);
-      if (j == 0) {
-        const Acc x = state_in_acc(p, b, c0 + e);
-        p.x0[(size_t)bg * CG + cl + e] = acc_pack(x);
-        dtot[e] = acc_pack(combine(x, tot, (float)min(L, T - t0), w[e]));
-      } else {
-        dtot[e] = acc_pack(tot);
+    for (int r = 0; r < 8; ++r) {
+      if (qq + r < q1) {
+        p.x0[((size_t)(qq + r) * BNG + bg) * CG + cl] = acc_pack(x);
+        x = combine(x, acc_unpack(a[r]), fJ, w);
       }
     }
   }
 }
 
-template <typename KV, typename OUT, int NW, int J, bool kTMA>
-__global__ void __launch_bounds__((NW + 1) * 32)
-    wkv_chunk_replay(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-  constexpr int VEC = 2;
-  constexpr int CG = 32 * VEC;
-  constexpr int L = NW * J;
-  constexpr int kTile = L * CG;
-  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
+template <typename KV, typename OUT, int J, int STAGES, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32)
+    wkv_span_replay(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  using R = SpanRing<KV, J>;
+  constexpr int VEC = 2, CG = R::CG;
   extern __shared__ __align__(1024) unsigned char smem[];
-  KV* ktile = reinterpret_cast<KV*>(smem);
-  KV* vtile = ktile + kTile;
-  float4* sh_x = reinterpret_cast<float4*>(smem + kBytes);  // [CG]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_x + CG);
-
-  const int lane = threadIdx.x & 31;
-  const int wp = threadIdx.x >> 5;
-  const bool scan = (wp == NW);
-  const int T = p.T, C = p.C;
-  const int BNG = p.B * p.NG;
-  const int tile = blockIdx.x;
-  const int j = tile / BNG;
-  const int bg = tile % BNG;
-  const int b = bg / p.NG, g = bg % p.NG;
-  const int t0 = j * L;
-  // the inputs are not written by the totals launch: copy them right away
-  if (kTMA && threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(bar, kBytes);
-    tma_load_3d(ktile, &tmk, bar, g * CG, t0, b);
-    tma_load_3d(vtile, &tmv, bar, g * CG, t0, b);
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  KV* ring = reinterpret_cast<KV*>(smem) + (size_t)wp * STAGES * 2 * R::kBox;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)WARPS * STAGES * R::kBytes) + wp * STAGES;
+  const int GW = gridDim.x * WARPS;
+  const int gw = blockIdx.x * WARPS + wp;
+  if (lane == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
   }
-  __syncthreads();
-  const int cl = lane * VEC;
-  const int c0 = g * CG + cl;
-  float w[VEC], u[VEC];
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    const bool ok = c0 + e < C;
-    w[e] = ok ? __ldg(p.w + c0 + e) : 0.f;
-    u[e] = ok ? __ldg(p.u + c0 + e) : 0.f;
-  }
-  // everything below reads what the totals launch wrote
-  grid_wait_prerequisites();
-  if (scan) {
-    Acc x[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) x[e] = (j == 0) ? acc_unpack(p.x0[(size_t)bg * CG + cl + e]) : acc_empty();
-    for (int jj = 0; jj < j; ++jj) {
-      const float4* src = p.agg_a + ((size_t)jj * BNG + bg) * CG + cl;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) x[e] = combine(x[e], acc_unpack(src[e]), (float)L, w[e]);
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) sh_x[cl + e] = acc_pack(x[e]);
-    named_sync<(NW + 1) * 32>(2);
-  } else {
-    const int ts = t0 + wp * J;
-    const int nv = max(0, min(J, T - ts));
-    const bool last_chunk = (j == p.nch - 1);
-    const int p_last = last_chunk ? (T - 1 - t0) / J : NW - 1;
-    Acc pre[VEC];
-    const float4* spre = p.agg_p + ((size_t)tile * NW + wp) * CG + cl;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) pre[e] = acc_unpack(spre[e]);
-    bool copy_ok = true;
-    if (kTMA) {
-      copy_ok = mbar_wait(bar, 0, p.timeout_ns);
-      if (!copy_ok && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
-    } else {
-      for (int i = threadIdx.x; i < kTile; i += NW * 32) {
-        const int r = i / CG, cc = i % CG;
-        const int t = t0 + r, c = g * CG + cc;
-        KV kk = Elem<KV>::from_f32(0.f), vv = Elem<KV>::from_f32(0.f);
-        if (t < T && c < C) {
-          kk = reinterpret_cast<const KV*>(p.k)[((size_t)b * T + t) * C + c];
-          vv = reinterpret_cast<const KV*>(p.v)[((size_t)b * T + t) * C + c];
-        }
-        ktile[i] = kk;
-        vtile[i] = vv;
-      }
-    }
-    named_sync<(NW + 1) * 32>(2);  // incoming state (and, without TMA, the tile) ready
-    if (nv > 0 && copy_ok) {
-      float cb[VEC];
-      bool fast = true;
+  // the inputs are not written by the earlier launches: start copying now
+  span_ring_start<KV, J, STAGES>(p, &tmk, &tmv, ring, full, gw, GW);
+  grid_wait_prerequisites();  // incoming states are ready
+  const int T = p.T, C = p.C, cl = lane * VEC;
+  const int nsp = (T + J - 1) / J;
+  int i = 0;
+  SpanWalk it(p, gw, GW);
+  // the incoming state and parameters of a span are loaded one span ahead,
+  // so that their latency hides behind the previous span's replay
+  float4 nx[VEC];
+  float nw[VEC], nu[VEC];
+  auto fetch = [&](const SpanWalk& sw) {
+    if (sw.sp < p.n_tiles) {
+      const int cc = sw.g * CG + cl;
+      const float4* px = p.x0 + (size_t)sw.sp * CG + cl;
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
-        fast &= fast_uw(u[e], w[e]);
-        cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+        const bool ok = cc + e < C;
+        nw[e] = ok ? __ldg(p.w + cc + e) : 0.f;
+        nu[e] = ok ? __ldg(p.u + cc + e) : 0.f;
+        nx[e] = px[e];
       }
-      fast = __all_sync(0xffffffffu, fast);
-      Acc st[VEC];
+    }
+  };
+  fetch(it);
+  for (; it.sp < p.n_tiles; ++i) {
+    const int s = i % STAGES;
+    const int sp = it.sp, q = it.q, b = it.b;
+    const int c0 = it.g * CG + cl;
+    const int ts = q * J;
+    const int nv = min(J, T - ts);
+    float w[VEC], u[VEC], cb[VEC];
+    bool fast = true;
+    Acc st[VEC];
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) st[e] = combine(acc_unpack(sh_x[cl + e]), pre[e], (float)(wp * J), w[e]);
-      const KV* ks = ktile + (wp * J) * CG + cl;
-      const KV* vs = vtile + (wp * J) * CG + cl;
-      OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
-      const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
-      if (fast) {
+    for (int e = 0; e < VEC; ++e) {
+      w[e] = nw[e];
+      u[e] = nu[e];
+      st[e] = acc_unpack(nx[e]);
+      fast &= fast_uw(u[e], w[e]);
+      cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+    }
+    fast = __all_sync(0xffffffffu, fast);
+    it.next();
+    fetch(it);
+    if (!mbar_wait(&full[s], (i / STAGES) & 1, p.timeout_ns)) {
+      if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+      span_ring_drain<STAGES>(p, full, i, gw, GW);
+      break;
+    }
+    const KV* ks = ring + (size_t)s * 2 * R::kBox + cl;
+    const KV* vs = ks + R::kBox;
+    OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
+    const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
+    if (fast && nv == J) {
 #pragma unroll
-        for (int i = 0; i < J; ++i) {
-          if (i < nv) {
-            float kx[VEC], vx[VEC], o[VEC];
-            load_vec<KV, VEC>(ks + i * CG, kx);
-            load_vec<KV, VEC>(vs + i * CG, vx);
+      for (int ii = 0; ii < J; ++ii) {
+        float kx[VEC], vx[VEC], o[VEC];
+        load_vec<KV, VEC>(ks + ii * CG, kx);
+        load_vec<KV, VEC>(vs + ii * CG, vx);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
-            if (lane_vec) {
-              stg_stream<OUT, VEC>(orow + (size_t)i * C, o);
-            } else {
+        for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+        if (lane_vec) {
+          stg_stream<OUT, VEC>(orow + (size_t)ii * C, o);
+        } else {
 #pragma unroll
-              for (int e = 0; e < VEC; ++e)
-                if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
-            }
-          }
+          for (int e = 0; e < VEC; ++e)
+            if (c0 + e < C) orow[(size_t)ii * C + e] = Elem<OUT>::from_f32(o[e]);
         }
-      } else {
-        for (int i = 0; i < nv; ++i) {
-          float kx[VEC], vx[VEC], o[VEC];
-          load_vec<KV, VEC>(ks + i * CG, kx);
-          load_vec<KV, VEC>(vs + i * CG, vx);
+      }
+    } else {
+      for (int ii = 0; ii < nv; ++ii) {
+        float kx[VEC], vx[VEC], o[VEC];
+        load_vec<KV, VEC>(ks + ii * CG, kx);
+        load_vec<KV, VEC>(vs + ii * CG, vx);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) {
+        for (int e = 0; e < VEC; ++e) {
+          if (fast) {
+            o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+          } else {
             o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
             add_token(st[e], kx[e], vx[e], w[e]);
           }
+        }
 #pragma unroll
-          for (int e = 0; e < VEC; ++e)
-            if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
+        for (int e = 0; e < VEC; ++e)
+          if (c0 + e < C) orow[(size_t)ii * C + e] = Elem<OUT>::from_f32(o[e]);
+      }
+    }
+    if (q == nsp - 1 && p.o_num) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        if (c0 + e < C) {
+          const size_t ii = (size_t)b * C + c0 + e;
+          p.o_num[ii] = st[e].num;
+          p.o_den[ii] = st[e].den;
+          p.o_max[ii] = acc_max_e(st[e], w[e]);
         }
       }
-      if (last_chunk && wp == p_last && p.o_num) {
+    }
+    __syncwarp();
+    const int nxt = sp + STAGES * GW;
+    if (lane == 0 && nxt < p.n_tiles) {
+      fence_proxy_async_smem();
+      span_issue<KV, J>(p, &tmk, &tmv, ring + (size_t)s * 2 * R::kBox, &full[s], nxt);
+    }
+  }
+}
+
+// Replay of the span-streaming scan that reads k and v straight from global
+// memory (they are L2-resident after the totals launch) into registers: no
+// shared memory, so occupancy is bounded by registers, not by staging
+// buffers, and each warp's 16-token span is one batch of coalesced loads.
+template <typename KV, typename OUT, int J>
+__global__ void __launch_bounds__(256) wkv_span_replay_ldg(const FwdParams p) {
+  constexpr int VEC = 2, CG = 64;
+  const int lane = threadIdx.x & 31;
+  const int GW = gridDim.x * (blockDim.x >> 5);
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  grid_wait_prerequisites();  // incoming states are ready
+  const int T = p.T, C = p.C, cl = lane * VEC;
+  const int nsp = (T + J - 1) / J;
+  const bool vec_in = p.vec_store != 0;
+  for (SpanWalk it(p, gw, GW); it.sp < p.n_tiles; it.next()) {
+    const int sp = it.sp, q = it.q, b = it.b;
+    const int c0 = it.g * CG + cl;
+    const int ts = q * J;
+    const int nv = min(J, T - ts);
+    const bool lane_vec = vec_in && c0 + VEC <= C;
+    // this span's tokens, all requested at once
+    float kx[J][VEC], vx[J][VEC];
+    const KV* kp = reinterpret_cast<const KV*>(p.k) + ((size_t)b * T + ts) * C + c0;
+    const KV* vp = reinterpret_cast<const KV*>(p.v) + ((size_t)b * T + ts) * C + c0;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          if (c0 + e < C) {
-            const size_t i = (size_t)b * C + c0 + e;
-            p.o_num[i] = st[e].num;
-            p.o_den[i] = st[e].den;
-            p.o_max[i] = acc_max_e(st[e], w[e]);
+    for (int ii = 0; ii < J; ++ii) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) kx[ii][e] = vx[ii][e] = 0.f;
+      if (ii < nv) {
+        if (lane_vec) {
+          ldg_stream<KV, VEC>(kp + (size_t)ii * C, kx[ii]);
+          ldg_stream<KV, VEC>(vp + (size_t)ii * C, vx[ii]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            if (c0 + e < C) {
+              kx[ii][e] = Elem<KV>::to_f32(kp[(size_t)ii * C + e]);
+              vx[ii][e] = Elem<KV>::to_f32(vp[(size_t)ii * C + e]);
+            }
           }
         }
       }
     }
-    if (kTMA && !copy_ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
+    float w[VEC], u[VEC], cb[VEC];
+    bool fast = true;
+    Acc st[VEC];
+    {
+      const float4* px = p.x0 + (size_t)sp * CG + cl;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const bool ok = c0 + e < C;
+        w[e] = ok ? __ldg(p.w + c0 + e) : 0.f;
+        u[e] = ok ? __ldg(p.u + c0 + e) : 0.f;
+        fast &= fast_uw(u[e], w[e]);
+        cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+        st[e] = acc_unpack(ldg_f4(px + e));
+      }
+    }
+    fast = __all_sync(0xffffffffu, fast);
+    OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
+    if (fast && nv == J) {
+      constexpr int NB = 8;  // tokens per block of step_tokens
+#pragma unroll
+      for (int i0 = 0; i0 < J; i0 += NB) {
+        float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
+#pragma unroll
+        for (int ii = 0; ii < NB; ++ii) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            kb[ii][e] = kx[i0 + ii][e];
+            vb[ii][e] = vx[i0 + ii][e];
+          }
+        }
+        step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
+#pragma unroll
+        for (int ii = 0; ii < NB; ++ii) {
+          if (lane_vec) {
+            stg_stream<OUT, VEC>(orow + (size_t)(i0 + ii) * C, ob[ii]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+              if (c0 + e < C) orow[(size_t)(i0 + ii) * C + e] = Elem<OUT>::from_f32(ob[ii][e]);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ii = 0; ii < J; ++ii) {
+        if (ii < nv) {
+          float o[VEC];
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            if (fast) {
+              o[e] = step_token(st[e], kx[ii][e], vx[ii][e], w[e], cb[e]);
+            } else {
+              o[e] = out_token(st[e], kx[ii][e], vx[ii][e], w[e], u[e]);
+              add_token(st[e], kx[ii][e], vx[ii][e], w[e]);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if (c0 + e < C) orow[(size_t)ii * C + e] = Elem<OUT>::from_f32(o[e]);
+        }
+      }
+    }
+    if (q == nsp - 1 && p.o_num) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        if (c0 + e < C) {
+          const size_t ii = (size_t)b * C + c0 + e;
+          p.o_num[ii] = st[e].num;
+          p.o_den[ii] = st[e].den;
+          p.o_max[ii] = acc_max_e(st[e], w[e]);
+        }
+      }
+    }
   }
 }
 
