@@ -139,14 +139,16 @@ def step_bytes(wl) -> int:
     return 36 * wl.B * wl.C + 8 * wl.C
 
 
+KERNEL_NAMES = {1: "wkv_fwd_seq", 2: "wkv_fwd_chunk", 3: "wkv_span_totals+scan+replay", 4: "wkv_fwd_pipe"}
+
+
 def forward_kernel_name(wl, options) -> str:
-    """The kernel that wkv_forward dispatches to for this workload (mirrors
-    the library's choice: the sequential kernel for many channels or short
-    sequences, the single-launch chunked scan otherwise)."""
-    kernel = (options or {}).get("kernel", 0)
-    if kernel == 0:
-        kernel = 1 if (wl.B * wl.C >= 65536 or wl.T <= 64) else 2
-    return {1: "wkv_fwd_seq", 2: "wkv_fwd_chunk", 3: "wkv_span_totals+scan+replay"}[kernel]
+    """The kernel that wkv_forward launches for this workload, as the library
+    itself reports it."""
+    import torch
+    import wkv_recurrence_b200 as W
+    kv = torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32
+    return KERNEL_NAMES[W.forward_kernel(wl.B, wl.T, wl.C, kv, options)]
 
 
 def launches_per_step(wl, options) -> int:

@@ -82,8 +82,12 @@ typedef struct {
  * zero-filled struct also means "defaults".
  *   kernel          0 = choose by shape, 1 = sequential-over-T kernel,
  *                   2 = chunked scan in one launch (look-back between CTAs),
- *                   3 = chunked scan in two launches (chunk totals, then
- *                   replay; for inputs that stay in L2 between them)
+ *                   3 = span-streaming scan in three launches (span totals,
+ *                   their scan, then the replay; for inputs that stay in L2
+ *                   between the launches),
+ *                   4 = chunked scan in one launch of persistent CTAs that
+ *                   pipeline their tiles (look-back of one tile overlapped
+ *                   with the next tile's fold and later tiles' copies)
  *   chunk_len       tokens per chunk for the chunked kernels (0 = choose;
  *                   otherwise 32, 64 or 128)
  *   lookback_group  G: the chunked kernel publishes a running prefix every G
@@ -91,13 +95,16 @@ typedef struct {
  *                   after the last one (0 = choose; otherwise 1..1024)
  *   wait_timeout_ns limit of every device-side wait (0 = 1 second)
  *   span            tokens per warp in a chunk-scan tile, 8 or 16 (0 = choose);
- *                   chunk_len / span warps share a tile
+ *                   chunk_len / span warps share a tile (at most 8 for the
+ *                   pipelined scan, so chunk_len 128 needs span 16 there)
  *   seq_threads     threads per CTA of the sequential kernel: 32, 64 or 128
  *                   (0 = choose); each thread carries 2 channels
  *   replay          how the span-streaming scan (kernel 3) replays its spans:
  *                   0 = choose, 1 = through per-warp TMA rings in shared
  *                   memory, 2 = with loads straight into registers
- *   reserved        must be 0
+ *   stages          shared-memory ring stages of the pipelined scan
+ *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
+ *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)
  *   inject_enable, inject_unpublished_tile
  *                   tests of the bounded waits only: with inject_enable = 1,
  *                   chunk-scan tile number inject_unpublished_tile computes
@@ -115,7 +122,7 @@ typedef struct {
     int32_t span;
     int32_t seq_threads;
     int32_t replay;
-    int32_t reserved;
+    int32_t stages;
 } wkv_options;
 
 /*
@@ -125,6 +132,13 @@ typedef struct {
  * not be used by two calls that may run at the same time.
  */
 WKV_API size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const wkv_options *opts);
+
+/*
+ * The kernel (1..4, numbered as wkv_options.kernel) that wkv_forward launches
+ * for these sizes, input dtype and options, for k and v whose base addresses
+ * are 16-byte aligned; 0 for invalid arguments. Host-only; touches no device.
+ */
+WKV_API int32_t wkv_forward_kernel(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype, const wkv_options *opts);
 
 /*
  * Sequence forward: for every (b, c), run the recurrence over t = 0..T-1,
@@ -222,6 +236,13 @@ WKV_API const char *wkv_status_string(wkv_status status);
 
 /* Library version as 10000*major + 100*minor + patch. Host-only. */
 WKV_API int32_t wkv_version(void);
+
+/*
+ * Name of the last CUDA runtime error that made a call of this library in the
+ * calling thread return WKV_ERR_CUDA ("cudaSuccess" if none has). Static
+ * text; host-only; the record is not cleared by reading it.
+ */
+WKV_API const char *wkv_last_cuda_error(void);
 
 #ifdef __cplusplus
 }

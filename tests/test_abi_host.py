@@ -39,6 +39,7 @@ def test_status_strings(L):
         assert s and s != "unknown status"
     assert _abi.status_string(99) == "unknown status"
     assert L.wkv_version() >= 100
+    assert L.wkv_last_cuda_error().decode().startswith("cuda")
 
 
 def test_workspace_size(L):
@@ -53,6 +54,25 @@ def test_workspace_size(L):
     assert L.wkv_forward_workspace_size(1, 64, 64, ctypes.byref(o)) == 0
     o = _abi.wkv_options(kernel=2, chunk_len=32, lookback_group=4)
     assert L.wkv_forward_workspace_size(1, 64, 64, ctypes.byref(o)) > 256
+
+
+def test_forward_kernel_choice(L):
+    F32, BF16 = _abi.WKV_F32, _abi.WKV_BF16
+    # many channels or short sequences: the sequential kernel; otherwise a chunked scan
+    assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
+    assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
+    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) in (2, 4)
+    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) in (2, 4)
+    # an explicit choice stands, except that the TMA-only scans fall back to the
+    # single-launch scan when a row pitch is not a multiple of 16 bytes
+    for kernel in (1, 2, 3, 4):
+        o = _abi.wkv_options(kernel=kernel)
+        assert L.wkv_forward_kernel(2, 500, 64, F32, ctypes.byref(o)) == kernel
+        assert L.wkv_forward_kernel(2, 500, 65, F32, ctypes.byref(o)) == (2 if kernel in (3, 4) else kernel)
+    assert L.wkv_forward_kernel(-1, 4, 4, F32, None) == 0
+    assert L.wkv_forward_kernel(1, 4, 4, 9, None) == 0
+    o = _abi.wkv_options(kernel=4, stages=1)
+    assert L.wkv_forward_kernel(1, 4, 4, F32, ctypes.byref(o)) == 0
 
 
 FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails its checks first
@@ -79,8 +99,13 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, sin=ctypes.byref(bad_state)) == _abi.WKV_ERR_INVALID_ARG
     bad_out = _abi.wkv_state(0x1000, 0x1000, None)
     assert fwd(L, sout=ctypes.byref(bad_out)) == _abi.WKV_ERR_INVALID_ARG
-    o = _abi.wkv_options(kernel=4)
+    o = _abi.wkv_options(kernel=5)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(kernel=4, chunk_len=128, span=8)  # 16 warps per role: too many
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    for bad_stages in (1, 9, -1):
+        o = _abi.wkv_options(kernel=4, stages=bad_stages)
+        assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(kernel=2, chunk_len=100)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(wait_timeout_ns=-5)

@@ -21,8 +21,9 @@ pytestmark = pytest.mark.gpu
 SEQ = {"kernel": 1}
 CHUNK = {"kernel": 2}
 TWO = {"kernel": 3}
-KERNELS = [SEQ, CHUNK, TWO]
-KIDS = ["seq", "chunk", "two"]
+PIPE = {"kernel": 4}
+KERNELS = [SEQ, CHUNK, TWO, PIPE]
+KIDS = ["seq", "chunk", "two", "pipe"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -64,9 +65,14 @@ def compare(oracle, k, v, w, u, state=None, kv="f32", out_dtype=None, options=No
                                   {"kernel": 2, "chunk_len": 32, "lookback_group": 5, "span": 8},
                                   {"kernel": 2, "chunk_len": 64, "span": 8},
                                   TWO, {"kernel": 3, "chunk_len": 32, "span": 8},
-                                  {"kernel": 3, "chunk_len": 64}],
+                                  {"kernel": 3, "chunk_len": 64},
+                                  PIPE, {"kernel": 4, "chunk_len": 32, "lookback_group": 1},
+                                  {"kernel": 4, "chunk_len": 64, "span": 8, "stages": 2},
+                                  {"kernel": 4, "chunk_len": 64, "span": 8, "lookback_group": 3, "stages": 5},
+                                  {"kernel": 4, "chunk_len": 32, "span": 8, "lookback_group": 5, "stages": 8}],
                          ids=["auto", "seq", "chunk128", "chunk32g1", "chunk128g3", "chunk32g5s8", "chunk64s8",
-                              "two128", "two32s8", "two64"])
+                              "two128", "two32s8", "two64", "pipe128", "pipe32g1", "pipe64s8st2",
+                              "pipe64s8g3st5", "pipe32s8g5st8"])
 @pytest.mark.parametrize("shape", [(1, 1, 64), (2, 33, 64), (3, 1000, 128), (2, 517, 200), (1, 2048, 64)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_random_f32(oracle, opts, shape):
@@ -184,8 +190,8 @@ def test_split_and_resume(oracle, opts):
     assert_state(s2, rst, sst[0], RTOL_F32)
 
 
-@pytest.mark.parametrize("opts", [SEQ, {"kernel": 2, "chunk_len": 32}, {"kernel": 3, "chunk_len": 32}],
-                         ids=KIDS)
+@pytest.mark.parametrize("opts", [SEQ, {"kernel": 2, "chunk_len": 32}, {"kernel": 3, "chunk_len": 32},
+                                  {"kernel": 4, "chunk_len": 32}], ids=KIDS)
 def test_in_place_state(oracle, opts):
     """state_out aliases state_in; the chunked kernels use many chunks here."""
     k, v, w, u, st = I.random_case(2, 1000, 128, seed=19, state=True)
@@ -261,7 +267,7 @@ def test_kernels_agree_and_are_deterministic(oracle):
         assert np.all(np.abs(a1 - r1) <= 2 * RTOL_F32 * sc), opts
 
 
-@pytest.mark.parametrize("opts", [CHUNK, TWO], ids=["chunk", "two"])
+@pytest.mark.parametrize("opts", [CHUNK, TWO, PIPE], ids=["chunk", "two", "pipe"])
 def test_workspace_reuse_across_shapes(oracle, opts):
     """One workspace serves successive calls of different shapes (the epoch scheme)."""
     ws = W.make_workspace(4, 4096, 256, options=opts)
@@ -274,13 +280,14 @@ def test_workspace_reuse_across_shapes(oracle, opts):
         assert_out(host(out), ref, sc, RTOL_F32)
 
 
-def test_bounded_wait_reports_timeout_and_recovers(oracle):
+@pytest.mark.parametrize("kernel", [2, 4], ids=["chunk", "pipe"])
+def test_bounded_wait_reports_timeout_and_recovers(oracle, kernel):
     """A chunk tile that never publishes: waiters give up after the limit,
     report WKV_ERR_WAIT_TIMEOUT, and the next call on the same workspace is
     correct again."""
     B, T, C = 2, 4096, 128
     k, v, w, u, _ = I.random_case(B, T, C, seed=41)
-    opts = {"kernel": 2, "chunk_len": 64, "lookback_group": 4, "wait_timeout_ns": 20_000_000,
+    opts = {"kernel": kernel, "chunk_len": 64, "lookback_group": 4, "wait_timeout_ns": 20_000_000,
             "inject_enable": 1, "inject_unpublished_tile": 9}
     ws = W.make_workspace(B, T, C, options=opts)
     K, V, Wt, U = dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u)
@@ -295,6 +302,42 @@ def test_bounded_wait_reports_timeout_and_recovers(oracle):
     ref, _ = oracle.recurrence_forward(k, v, w, u)
     sc, _ = oracle.abs_scale_forward(k, v, w, u)
     assert_out(host(out), ref, sc, RTOL_F32)
+
+
+def test_stage_counts_in_any_order(oracle):
+    """Launches of one kernel with more, fewer, then more shared-memory stages
+    again (the kernel's shared-memory limit must not shrink under a later call)."""
+    B, T, C = 2, 1500, 128
+    k, v, w, u, _ = I.random_case(B, T, C, seed=47)
+    ref, _ = oracle.recurrence_forward(k, v, w, u)
+    sc, _ = oracle.abs_scale_forward(k, v, w, u)
+    for stages in (3, 2, 3, 0, 2):
+        out, _ = run_forward(k, v, w, u, options={"kernel": 4, "chunk_len": 128, "stages": stages})
+        assert_out(out, ref, sc, RTOL_F32)
+    # a ring that does not fit in one CTA's shared memory is refused, not launched
+    with pytest.raises(W.WkvError) as e:
+        run_forward(k, v, w, u, options={"kernel": 4, "chunk_len": 128, "span": 16, "stages": 8})
+    assert e.value.code == 1  # WKV_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("opts", KERNELS, ids=KIDS)
+def test_no_wait_reaches_its_limit(oracle, opts):
+    """With a 0.2 s wait limit, correct calls finish far below it: no wait in
+    any kernel runs to its limit on a normal run (such a wait would give
+    correct results but cost the whole limit)."""
+    B, T, C = 2, 3000, 128
+    k, v, w, u, _ = I.random_case(B, T, C, seed=43)
+    o = dict(opts, wait_timeout_ns=200_000_000)
+    ws = W.make_workspace(B, T, C, options=o)
+    K, V, Wt, U = dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u)
+    W.forward(K, V, Wt, U, workspace=ws, options=o)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        t0 = time.perf_counter()
+        W.forward(K, V, Wt, U, workspace=ws, options=o)
+        torch.cuda.synchronize()
+        assert time.perf_counter() - t0 < 0.1
+    assert W.query_status(ws) == 0
 
 
 # ---------------------------------------------------------------------------
@@ -327,10 +370,22 @@ def test_workload_full_size(oracle, name):
     print(f"{name}: max normalised out error {eo:.2e}, state errors {es}")
 
 
+@pytest.mark.parametrize("name", ["layer", "long", "mixed"])
+def test_workload_full_size_pipelined(oracle, name):
+    """The pipelined chunked scan on the benchmark shapes, whatever the
+    automatic choice of kernel is."""
+    wl = I.WORKLOADS[name]
+    k, v = I.draw_kv(wl)
+    w, u = I.draw_w(wl), I.draw_u(wl)
+    st = I.draw_state(wl)
+    _, _, eo, es = compare(oracle, k, v, w, u, st, kv=wl.kv_dtype, out_dtype=wl.out_dtype, options=PIPE)
+    print(f"{name} (pipelined): max normalised out error {eo:.2e}, state errors {es}")
+
+
 def test_tiny_against_decimal_golden():
     from test_oracle_pins import load_golden
     k, v, w, u, ref = load_golden()
-    for opts in (None, SEQ, CHUNK, TWO):
+    for opts in (None, SEQ, CHUNK, TWO, PIPE):
         out, _ = run_forward(k, v, w, u, options=opts)
         assert np.allclose(out, ref, rtol=RTOL_F32, atol=RTOL_F32 * np.abs(v).max())
 

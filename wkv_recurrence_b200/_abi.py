@@ -23,8 +23,8 @@ WKV_F32 = 0
 WKV_BF16 = 1
 
 # entry points declared in include/wkv.h
-EXPORTS = ("wkv_forward_workspace_size", "wkv_forward", "wkv_step", "wkv_query_status",
-           "wkv_status_string", "wkv_version", "wkv_forward_noalloc")
+EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward", "wkv_step", "wkv_query_status",
+           "wkv_status_string", "wkv_version", "wkv_forward_noalloc", "wkv_last_cuda_error")
 
 # size of the library's built-in scratch array used by wkv_forward_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -43,13 +43,16 @@ class wkv_options(ctypes.Structure):
                 ("lookback_group", ctypes.c_int32), ("inject_enable", ctypes.c_int32),
                 ("wait_timeout_ns", ctypes.c_int64), ("inject_unpublished_tile", ctypes.c_int64),
                 ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32),
-                ("replay", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("replay", ctypes.c_int32), ("stages", ctypes.c_int32)]
 
 
 class WkvError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_string(code)} (status {code})")
+        msg = f"{where}: {status_string(code)} (status {code})"
+        if code == WKV_ERR_CUDA:
+            msg += f", last CUDA error {lib().wkv_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 _lib = None
@@ -65,6 +68,8 @@ def lib() -> ctypes.CDLL:
         P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
         L.wkv_forward_workspace_size.argtypes = [I64, I64, I64, ctypes.POINTER(wkv_options)]
         L.wkv_forward_workspace_size.restype = SZ
+        L.wkv_forward_kernel.argtypes = [I64, I64, I64, I, ctypes.POINTER(wkv_options)]
+        L.wkv_forward_kernel.restype = ctypes.c_int32
         L.wkv_forward.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
                                   ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state),
                                   P, SZ, P, ctypes.POINTER(wkv_options)]
@@ -81,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.wkv_status_string.restype = ctypes.c_char_p
         L.wkv_version.argtypes = []
         L.wkv_version.restype = ctypes.c_int32
+        L.wkv_last_cuda_error.argtypes = []
+        L.wkv_last_cuda_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
 

@@ -68,6 +68,18 @@ def workspace_size(B: int, T: int, C: int, options: Optional[dict] = None) -> in
     return int(n)
 
 
+def forward_kernel(B: int, T: int, C: int, kv_dtype: torch.dtype = torch.float32,
+                   options: Optional[dict] = None) -> int:
+    """The kernel number (as in ``options["kernel"]``) ``forward`` launches for
+    this shape with 16-byte aligned inputs (host-only)."""
+    if kv_dtype not in _DT:
+        raise TypeError(f"dtype {kv_dtype} is not supported (float32 or bfloat16)")
+    n = _abi.lib().wkv_forward_kernel(int(B), int(T), int(C), _DT[kv_dtype], _options(options))
+    if n == 0:
+        raise ValueError("invalid sizes or options")
+    return int(n)
+
+
 def make_workspace(B: int, T: int, C: int, options: Optional[dict] = None, device=None) -> torch.Tensor:
     """A zero-filled workspace for ``forward`` (zero once; the library keeps it ready)."""
     return torch.zeros(workspace_size(B, T, C, options), dtype=torch.uint8,

@@ -36,9 +36,10 @@ constexpr int kSeqFallbackVec = 1, kSeqFallbackLt = 16;
 constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 
 struct Plan {
-  int kernel;  // 1 seq, 2 chunked single launch, 3 chunked two launches (L2-resident inputs)
+  int kernel;  // 1 seq, 2 chunked single launch, 3 span streaming (three launches), 4 pipelined chunked
   int seq_threads;  // CTA width of the sequential kernel
   int replay;       // span-streaming replay: 1 TMA rings, 2 loads into registers
+  int stages;       // pipelined chunked scan: ring stages (0 = choose at launch)
   int L;       // chunk length (chunk kernel)
   int J;       // tokens per warp (chunk kernel)
   int G;       // look-back group
@@ -50,19 +51,34 @@ struct Plan {
 };
 
 
+// The last CUDA error this library met in the calling thread (for
+// wkv_last_cuda_error), recorded wherever a call returns WKV_ERR_CUDA because
+// of one.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+bool cuda_ok(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error = e;
+  return e == cudaSuccess;
+}
+
+// Status of the launch just made (<<<>>> launches report only through
+// cudaGetLastError).
+wkv_status launch_result() { return cuda_ok(cudaGetLastError()) ? WKV_OK : WKV_ERR_CUDA; }
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // The plan for a call: which kernel, tile sizes, and the workspace layout.
 // tma_ok = false (inputs that TMA cannot address: misaligned base, row pitch
-// not a multiple of 16 bytes) turns the three-launch scan, which needs TMA,
-// into the single-launch one. A three-launch plan reserves enough workspace
+// not a multiple of 16 bytes) turns the three-launch and the pipelined scans,
+// which need TMA, into the single-launch one (the pipelined scan uses the same
+// workspace layout as the single-launch one). A three-launch plan reserves enough workspace
 // for either, so a workspace sized by wkv_forward_workspace_size always fits.
 bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, int kv_bytes = 4,
                bool tma_ok = true) {
   std::memset(pl, 0, sizeof *pl);
   (void)kv_bytes;
   const int want = o ? o->kernel : 0;
-  if (want < 0 || want > 3) return false;
+  if (want < 0 || want > 4) return false;
   const int64_t lanes = B * C;
   int kernel = want;
   if (kernel == 0) {
@@ -73,10 +89,12 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     }
   }
   const bool three_requested = (kernel == 3);
-  if (kernel == 3 && !tma_ok) kernel = 2;
+  if ((kernel == 3 || kernel == 4) && !tma_ok) kernel = 2;
   pl->kernel = kernel;
   pl->bytes = sizeof(WsHeader);
-  if (o && (o->reserved != 0 || o->replay < 0 || o->replay > 2)) return false;
+  if (o && (o->replay < 0 || o->replay > 2)) return false;
+  if (o && (o->stages < 0 || o->stages == 1 || o->stages > 8)) return false;
+  pl->stages = o ? o->stages : 0;
   pl->replay = (o && o->replay) ? o->replay : 2;
   int sth = o ? o->seq_threads : 0;
   if (sth == 0) sth = 32;  // many small CTAs: more resident warps per SM
@@ -90,6 +108,9 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   int J = o ? o->span : 0;
   if (J == 0) J = 16;
   if (J != 8 && J != 16) return false;
+  // the pipelined scan runs L/J fold and L/J replay warps plus two: at most 8
+  // of each keeps the CTA within 1024 threads
+  if (kernel == 4 && L / J > 8) return false;
   int G = o ? o->lookback_group : 0;
   if (G == 0) G = 16;
   if (G < 1 || G > 1024) return false;
@@ -163,29 +184,48 @@ bool dev_info(int dev, DevInfo* out) {
   return true;
 }
 
-// Sets the dynamic shared memory limit of kernel `fn` once per device and
-// returns how many CTAs of it fit on one SM (cached per kernel and device).
+// Raises the dynamic shared memory limit of kernel `fn` on device `dev` to at
+// least `smem` and returns how many CTAs of it fit on one SM with that much
+// shared memory. The limit is an attribute of the kernel, shared by every
+// launch of it, so it only ever grows (a launch with less shared memory must
+// not lower it under a later, larger one); occupancies are cached per size.
 struct KernelSetup {
   const void* fn;
   int dev;
   size_t smem;
   int occ;
 };
+struct KernelLimit {
+  const void* fn;
+  int dev;
+  size_t smem;
+};
 std::vector<KernelSetup> g_setups;
+std::vector<KernelLimit> g_limits;
 
 template <typename F>
 bool kernel_setup(F fn, int dev, int threads, size_t smem, int* blocks_per_sm) {
   const void* key = reinterpret_cast<const void*>(fn);
   std::lock_guard<std::mutex> lk(g_mu);
+  KernelLimit* lim = nullptr;
+  for (KernelLimit& l : g_limits)
+    if (l.fn == key && l.dev == dev) lim = &l;
+  if (!lim || lim->smem < smem) {
+    if (!cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return false;
+    if (lim) {
+      lim->smem = smem;
+    } else {
+      g_limits.push_back(KernelLimit{key, dev, smem});
+    }
+  }
   for (const KernelSetup& s : g_setups) {
     if (s.fn == key && s.dev == dev && s.smem == smem) {
       *blocks_per_sm = s.occ;
       return true;
     }
   }
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return false;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess) return false;
+  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem))) return false;
   g_setups.push_back(KernelSetup{key, dev, smem, n});
   *blocks_per_sm = n;
   return true;
@@ -243,7 +283,7 @@ wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorM
   const long long grid = (long long)p.B * q.NG;
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
   fn<<<(unsigned)grid, THREADS, smem, st>>>(q, tk, tv);
-  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  return launch_result();
 }
 
 template <typename KV, typename OUT, int NW, int J, bool kTMA>
@@ -255,7 +295,46 @@ wkv_status launch_chunk(const FwdParams& p, const CUtensorMap& tk, const CUtenso
   int occ = 0;
   if (!kernel_setup(fn, dev, (NW + 1) * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
   fn<<<(unsigned)p.n_tiles, (NW + 1) * 32, smem, st>>>(p, tk, tv);
-  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  return launch_result();
+}
+
+// Persistent launch of the pipelined chunked scan: as many CTAs as fit on the
+// device at once (never more than there are tiles). `stages` = 0 chooses the
+// deepest ring of up to 8 stages that fits in one CTA's shared memory.
+template <typename KV, typename OUT, int NC, int J>
+wkv_status launch_pipe(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev,
+                       const DevInfo& di, int stages) {
+  if (!p.flags_a || !p.flags_p || !p.agg_a || !p.agg_p || !p.hdr) return WKV_ERR_INVALID_ARG;
+  constexpr size_t kStage = 2ull * NC * J * kChunkCG * sizeof(KV);
+  auto bytes = [](int s) { return (size_t)s * kStage + pipe_aux_bytes<NC>(s); };
+  if (stages == 0) {
+    stages = 8;
+    while (stages > 2 && bytes(stages) > (size_t)di.smem_optin) --stages;
+  }
+  const size_t smem = bytes(stages);
+  if (smem > (size_t)di.smem_optin) return WKV_ERR_INVALID_ARG;
+  auto fn = wkv_fwd_pipe<KV, OUT, NC, J>;
+  int occ = 0;
+  if (!kernel_setup(fn, dev, (2 * NC + 2) * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  FwdParams q = p;
+  q.stages = stages;
+  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ * di.sms, p.n_tiles));
+  fn<<<grid, (2 * NC + 2) * 32, smem, st>>>(q, tk, tv);
+  return launch_result();
+}
+
+template <typename KV, typename OUT>
+wkv_status launch_pipe_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                             cudaStream_t st, int dev, const DevInfo& di) {
+  if (pl.J == 8) {  // make_plan refuses L = 128 with J = 8 for this kernel
+    if (pl.L == 32) return launch_pipe<KV, OUT, 4, 8>(p, tk, tv, st, dev, di, pl.stages);
+    return launch_pipe<KV, OUT, 8, 8>(p, tk, tv, st, dev, di, pl.stages);
+  }
+  switch (pl.L) {
+    case 32: return launch_pipe<KV, OUT, 2, 16>(p, tk, tv, st, dev, di, pl.stages);
+    case 64: return launch_pipe<KV, OUT, 4, 16>(p, tk, tv, st, dev, di, pl.stages);
+    default: return launch_pipe<KV, OUT, 8, 16>(p, tk, tv, st, dev, di, pl.stages);
+  }
 }
 
 // Launch configuration with programmatic stream serialization: the launch may
@@ -295,9 +374,9 @@ wkv_status launch_spans(const FwdParams& p, const CUtensorMap& tk, const CUtenso
   const unsigned ga = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_a * sms, blocks_needed));
   const unsigned gb = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_b * sms, blocks_needed));
   fa<<<ga, WARPS * 32, smem, st>>>(p, tk, tv);
-  if (cudaGetLastError() != cudaSuccess) return WKV_ERR_CUDA;
+  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   PdlConfig cs(dim3((unsigned)((long long)p.B * p.NG)), dim3(64 * 8), 0, st);
-  if (cudaLaunchKernelEx(&cs.cfg, fs, p, (int)J) != cudaSuccess) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaLaunchKernelEx(&cs.cfg, fs, p, (int)J))) return WKV_ERR_CUDA;
   if (p.replay_mode == 1) {
     // replay straight from L2 into registers
     auto fr = wkv_span_replay_ldg<KV, OUT, J>;
@@ -305,12 +384,12 @@ wkv_status launch_spans(const FwdParams& p, const CUtensorMap& tk, const CUtenso
     if (!kernel_setup(fr, dev, 256, 0, &occ_r) || occ_r < 1) return WKV_ERR_CUDA;
     const unsigned gr = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_r * sms, (p.n_tiles + 7) / 8));
     PdlConfig cr(dim3(gr), dim3(256), 0, st);
-    if (cudaLaunchKernelEx(&cr.cfg, fr, p) != cudaSuccess) return WKV_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    if (!cuda_ok(cudaLaunchKernelEx(&cr.cfg, fr, p))) return WKV_ERR_CUDA;
+    return launch_result();
   }
   PdlConfig cb(dim3(gb), dim3(WARPS * 32), smem, st);
-  if (cudaLaunchKernelEx(&cb.cfg, fb, p, tk, tv) != cudaSuccess) return WKV_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, tk, tv))) return WKV_ERR_CUDA;
+  return launch_result();
 }
 
 template <typename KV, typename OUT, bool kTMA>
@@ -332,7 +411,8 @@ wkv_status launch_chunk_shape(const Plan& pl, const FwdParams& p, const CUtensor
 
 template <typename KV, typename OUT>
 wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kvdt, cudaStream_t st, int dev,
-                            int sms) {
+                            const DevInfo& di) {
+  const int sms = di.sms;
   CUtensorMap tk, tv;
   std::memset(&tk, 0, sizeof tk);
   std::memset(&tv, 0, sizeof tv);
@@ -360,6 +440,12 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
     if (pl.J == 8) return launch_spans<KV, OUT, 8>(p, tk, tv, st, dev, sms);
     return launch_spans<KV, OUT, 16>(p, tk, tv, st, dev, sms);
   }
+  if (pl.kernel == 4) {  // pipelined (make_plan only chooses it when TMA works)
+    if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
+        !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
+      return WKV_ERR_CUDA;
+    return launch_pipe_shape<KV, OUT>(pl, p, tk, tv, st, dev, di);
+  }
   if (tma) {
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
         !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
@@ -377,6 +463,8 @@ using namespace wkv;
 extern "C" {
 
 int32_t wkv_version(void) { return 100; }
+
+const char* wkv_last_cuda_error(void) { return cudaGetErrorName(g_last_cuda_error); }
 
 const char* wkv_status_string(wkv_status s) {
   switch (s) {
@@ -397,6 +485,15 @@ size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const wkv_opt
   Plan a, b;
   if (B < 0 || T < 0 || C < 0 || !make_plan(B, T, C, opts, &a, 4) || !make_plan(B, T, C, opts, &b, 2)) return 0;
   return std::max(a.bytes, b.bytes);
+}
+
+int32_t wkv_forward_kernel(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype, const wkv_options* opts) {
+  if (B < 0 || T < 0 || C < 0) return 0;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return 0;
+  const size_t es = kv_dtype == WKV_F32 ? 4 : 2;
+  Plan pl;
+  if (!make_plan(B, T, C, opts, &pl, (int)es, (C * (int64_t)es) % 16 == 0)) return 0;
+  return pl.kernel;
 }
 
 wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
@@ -432,7 +529,7 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaGetDevice(&dev))) return WKV_ERR_CUDA;
   DevInfo di;
   if (!dev_info(dev, &di)) return WKV_ERR_CUDA;
   if (T == 0) {  // the state passes through unchanged
@@ -442,13 +539,13 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
       float* dst[3] = {state_out->num, state_out->den, state_out->max_e};
       for (int i = 0; i < 3; ++i)
         if (src[i] != dst[i] &&
-            cudaMemcpyAsync(dst[i], src[i], sizeof(float) * BC, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            !cuda_ok(cudaMemcpyAsync(dst[i], src[i], sizeof(float) * BC, cudaMemcpyDeviceToDevice, st)))
           return WKV_ERR_CUDA;
       return WKV_OK;
     }
     wkv_fill_empty_state<<<(unsigned)((BC + 255) / 256), 256, 0, st>>>(BC, state_out->num, state_out->den,
                                                                       state_out->max_e);
-    return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return launch_result();
   }
 
   FwdParams p;
@@ -497,10 +594,10 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   if (pl.kernel >= 2)  // the chunked kernels also load k and v VEC-wide
     p.vec_store = p.vec_store && aligned(k, kes * vec) && aligned(v, kes * vec);
 
-  if (kv_dtype == WKV_F32) return dispatch_forward<float, float>(pl, p, tma, kv_dtype, st, dev, di.sms);
+  if (kv_dtype == WKV_F32) return dispatch_forward<float, float>(pl, p, tma, kv_dtype, st, dev, di);
   if (out_dtype == WKV_BF16)
-    return dispatch_forward<__nv_bfloat16, __nv_bfloat16>(pl, p, tma, kv_dtype, st, dev, di.sms);
-  return dispatch_forward<__nv_bfloat16, float>(pl, p, tma, kv_dtype, st, dev, di.sms);
+    return dispatch_forward<__nv_bfloat16, __nv_bfloat16>(pl, p, tma, kv_dtype, st, dev, di);
+  return dispatch_forward<__nv_bfloat16, float>(pl, p, tma, kv_dtype, st, dev, di);
 }
 
 wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype, const float* w,
@@ -552,19 +649,19 @@ wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtyp
     if (vec) wkv_step_kernel<__nv_bfloat16, float, VEC><<<blocks, 256, 0, st>>>(p);
     else wkv_step_kernel<__nv_bfloat16, float, 1><<<blocks, 256, 0, st>>>(p);
   }
-  return cudaGetLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  return launch_result();
 }
 
 wkv_status wkv_query_status(void* workspace, void* stream) {
   if (!workspace) return WKV_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize(st))) return WKV_ERR_CUDA;
   WsHeader* h = static_cast<WsHeader*>(workspace);
   uint32_t bits = 0;
-  if (cudaMemcpy(&bits, &h->status, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpy(&bits, &h->status, sizeof bits, cudaMemcpyDeviceToHost))) return WKV_ERR_CUDA;
   if (bits) {
     const uint32_t zero = 0;
-    if (cudaMemcpy(&h->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return WKV_ERR_CUDA;
+    if (!cuda_ok(cudaMemcpy(&h->status, &zero, sizeof zero, cudaMemcpyHostToDevice))) return WKV_ERR_CUDA;
   }
   return (bits & kStatusWaitTimeout) ? WKV_ERR_WAIT_TIMEOUT : WKV_OK;
 }
@@ -591,7 +688,7 @@ bool noalloc_scratch(int dev, void** ptr) {
   std::lock_guard<std::mutex> lk(wkv::g_mu);
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return false;
+    if (!cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_scratch)) || !p) return false;
     g_noalloc_ptr[dev] = p;
   }
   *ptr = g_noalloc_ptr[dev];
@@ -615,12 +712,12 @@ wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, c
                        reinterpret_cast<void*>(uintptr_t(256)), WKV_NOALLOC_SCRATCH_BYTES, stream, nullptr);
   }
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaGetDevice(&dev))) return WKV_ERR_CUDA;
   void* scratch = nullptr;
   if (!noalloc_scratch(dev, &scratch)) return WKV_ERR_CUDA;
   // counters, epoch, status and flags start at zero for this call
-  const size_t clear = pl.kernel == 2 ? pl.off_agg_a : sizeof(WsHeader);
-  if (cudaMemsetAsync(scratch, 0, clear, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  const size_t clear = (pl.kernel == 2 || pl.kernel == 4) ? pl.off_agg_a : sizeof(WsHeader);
+  if (!cuda_ok(cudaMemsetAsync(scratch, 0, clear, reinterpret_cast<cudaStream_t>(stream))))
     return WKV_ERR_CUDA;
   return wkv_forward(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, scratch,
                      WKV_NOALLOC_SCRATCH_BYTES, stream, nullptr);

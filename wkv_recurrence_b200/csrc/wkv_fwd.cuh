@@ -72,6 +72,7 @@ struct FwdParams {
   float4* agg_p;       // [nblk * B * NG][CG] (single launch) or [n_tiles][NW][CG] (two launches)
   float4* x0;          // incoming states of spans (span-streaming scan)
   int replay_mode;     // span-streaming replay: 0 = TMA rings, 1 = loads into registers
+  int stages;          // pipelined chunk scan: shared-memory stages in the ring
 };
 
 // State in for one channel, anchored; empty when no state is passed.
@@ -345,6 +346,42 @@ __device__ __forceinline__ void aggregate_tile_span(const KV* ks, const KV* vs, 
   }
 }
 
+// Incoming state of chunk j from the published values of its look-back group
+// (chunks first .. j-1) and, when given, the previous group's inclusive prefix:
+// x = prefix, then combined with each chunk total in chunk order (the order
+// of combines is fixed, so results do not depend on timing). Loading several
+// totals before combining them (kBatch > 1) was measured: it costs registers
+// (and so resident CTAs) and gained nothing, so they are loaded one by one.
+template <int VEC, int CG, int L>
+__device__ __forceinline__ void gather_group(const FwdParams& p, Acc (&x)[VEC], int first, int j, int bg, int cl,
+                                             const float (&w)[VEC], bool has_prefix, int qb) {
+  constexpr int kBatch = 1;
+  const int BNG = p.B * p.NG;
+  if (has_prefix) {
+    const float4* src = p.agg_p + ((size_t)(qb - 1) * BNG + bg) * CG + cl;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) x[e] = acc_unpack(ld_relaxed_f4(src + e));
+  }
+  for (int j0 = first; j0 < j; j0 += kBatch) {
+    float4 t[kBatch][VEC];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (j0 + i < j) {
+        const float4* src = p.agg_a + ((size_t)(j0 + i) * BNG + bg) * CG + cl;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) t[i][e] = ld_relaxed_f4(src + e);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (j0 + i < j) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) x[e] = combine(x[e], acc_unpack(t[i][e]), (float)L, w[e]);
+      }
+    }
+  }
+}
+
 // Tile = 64 channels (32 lanes x 2) by L = NW * J tokens of one batch row, one
 // CTA of NW compute warps plus one scan warp. Thread 0 takes the tile's ticket
 // and starts its TMA copy (k and v boxes into shared memory); meanwhile the
@@ -439,16 +476,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       }
       if (!ready && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
       fence_acq_rel_gpu();
-      if (qb > 0) {
-        const float4* src = p.agg_p + ((size_t)(qb - 1) * BNG + bg) * CG + cl;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) x[e] = acc_unpack(ld_relaxed_f4(src + e));
-      }
-      for (int jj = first; jj < j; ++jj) {
-        const float4* src = p.agg_a + ((size_t)jj * BNG + bg) * CG + cl;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) x[e] = combine(x[e], acc_unpack(ld_relaxed_f4(src + e)), (float)L, w[e]);
-      }
+      gather_group<VEC, CG, L>(p, x, first, j, bg, cl, w, qb > 0, qb);
     }
 #pragma unroll
     for (int e = 0; e < VEC; ++e) sh_x[cl + e] = acc_pack(x[e]);
@@ -1073,6 +1101,355 @@ __global__ void __launch_bounds__(256) wkv_span_replay_ldg(const FwdParams p) {
           p.o_max[ii] = acc_max_e(st[e], w[e]);
         }
       }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// pipelined single-launch chunked scan (persistent, warp-specialised)
+// ---------------------------------------------------------------------------
+//
+// The same tiles, look-back and arithmetic as wkv_fwd_chunk, but CTAs are
+// persistent (one or a few per SM) and take tiles in ticket order, streaming
+// them through a ring of p.stages shared-memory stages. Four warp roles, each
+// walking the tiles of its CTA in order:
+//   producer warp   takes the next ticket and copies the tile's k and v boxes
+//                   into the next free stage (TMA, mbarriers);
+//   fold warps      (NC, J tokens each) fold the tile into span aggregates as
+//                   soon as it has landed; the last of them forms the tile
+//                   total and publishes it at once;
+//   look-back warp  gathers the tile's incoming state from earlier chunks,
+//                   publishes the group prefix where due, and marks the stage
+//                   ready for replay;
+//   replay warps    (NC, J tokens each) replay the tile from (incoming state +
+//                   in-tile prefix), write the outputs and free the stage.
+// Folding never waits for a replay, so the totals that every look-back needs
+// appear at the speed the data arrives, and the ring's depth bounds how far
+// the folds run ahead. Every dependency of a tile is on tiles with smaller
+// tickets, so the tile with the smallest unfinished ticket can always proceed.
+// Every wait is bounded; a wait that gives up sets the status word and the
+// CTA stops taking tiles.
+//
+// Shared memory: [stages][k | v][L][64] tiles, then float4 agg[stages][NC][64],
+// tot[stages][64], xin[stages][64], then four mbarriers per stage, the stage
+// tile numbers and an abort flag.
+template <int NC>
+__host__ __device__ constexpr size_t pipe_aux_bytes(int stages) {
+  return sizeof(float4) * 64 * (size_t)stages * (NC + 2) + sizeof(uint64_t) * 4 * stages + sizeof(int) * (stages + 1);
+}
+
+__device__ __forceinline__ void pipe_fail(const FwdParams& p, volatile int* abort_flag, int lane) {
+  if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+  *abort_flag = 1;
+}
+
+template <typename KV, typename OUT, int NC, int J>
+__global__ void __launch_bounds__((2 * NC + 2) * 32)
+    wkv_fwd_pipe(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  constexpr int VEC = 2;
+  constexpr int CG = 64;
+  constexpr int L = NC * J;
+  constexpr int kTile = L * CG;
+  constexpr uint32_t kStage = 2u * kTile * (uint32_t)sizeof(KV);
+  constexpr int kReplay0 = NC, kLookback = 2 * NC, kProducer = 2 * NC + 1;  // fold warps: 0 .. NC-1
+  const int S = p.stages;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  KV* tiles = reinterpret_cast<KV*>(smem);                            // [S][k|v][L][CG]
+  float4* agg = reinterpret_cast<float4*>(smem + (size_t)S * kStage);  // [S][NC][CG]
+  float4* tot = agg + (size_t)S * NC * CG;                             // [S][CG]
+  float4* xin = tot + (size_t)S * CG;                                  // [S][CG]
+  uint64_t* full = reinterpret_cast<uint64_t*>(xin + (size_t)S * CG);  // [S] copy landed
+  uint64_t* folded = full + S;                                         // [S] aggregates and total ready
+  uint64_t* ready = folded + S;                                        // [S] incoming state ready
+  uint64_t* empty = ready + S;                                         // [S] replayed, stage free
+  int* tile_id = reinterpret_cast<int*>(empty + S);                    // [S]
+  volatile int* abort_flag = tile_id + S;
+
+  const int lane = threadIdx.x & 31;
+  const int wp = threadIdx.x >> 5;
+  const int T = p.T, C = p.C;
+  const int BNG = p.B * p.NG;
+  const int cl = lane * VEC;
+  const uint32_t target = *reinterpret_cast<volatile uint32_t*>(&p.hdr->epoch) + 1u;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&folded[i], 1);
+      mbar_init(&ready[i], 1);
+      mbar_init(&empty[i], NC);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (wp == kProducer) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int n = 0;
+      for (;; ++n) {
+        const int s = n % S;
+        if (n >= S && !mbar_wait(&empty[s], ((n / S) - 1) & 1, p.timeout_ns)) pipe_fail(p, abort_flag, 0);
+        const int t = *abort_flag ? p.n_tiles : (int)atomicAdd(&p.hdr->ticket, 1u);
+        if (t >= p.n_tiles) {
+          // the previous copy into this stage must have landed before the
+          // stage's next phase marks the end of the stream
+          if (n >= S && !mbar_wait(&full[s], ((n / S) - 1) & 1, p.timeout_ns))
+            atomicOr(&p.hdr->status, kStatusWaitTimeout);
+          tile_id[s] = t;
+          mbar_arrive(&full[s]);  // end of the stream for the other warps
+          break;
+        }
+        tile_id[s] = t;
+        const int j = t / BNG, bg = t % BNG;
+        mbar_arrive_expect_tx(&full[s], kStage);
+        tma_load_3d(tiles + (size_t)s * 2 * kTile, &tmk, &full[s], (bg % p.NG) * CG, j * L, bg / p.NG);
+        tma_load_3d(tiles + (size_t)s * 2 * kTile + kTile, &tmv, &full[s], (bg % p.NG) * CG, j * L, bg / p.NG);
+      }
+      // no copy may still be writing into shared memory when the CTA exits
+      // (the stage of the end marker was drained above)
+      for (int m = max(0, n - S + 1); m < n; ++m)
+        if (!mbar_wait(&full[m % S], (m / S) & 1, p.timeout_ns)) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+    }
+  } else if (wp == kLookback) {
+    // ----------------------------------------------------------- look-back
+    for (int n = 0;; ++n) {
+      const int s = n % S;
+      const uint32_t ph = (n / S) & 1;
+      if (!mbar_wait(&full[s], ph, p.timeout_ns)) {
+        pipe_fail(p, abort_flag, lane);
+        break;
+      }
+      const int tile = tile_id[s];
+      if (tile >= p.n_tiles) {  // end of the stream: pass it on to the replay warps
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ready[s]);
+        break;
+      }
+      const int j = tile / BNG, bg = tile % BNG;
+      const int b = bg / p.NG, c0 = (bg % p.NG) * CG + cl;
+      float w[VEC];
+      Acc x[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < C) ? __ldg(p.w + c0 + e) : 0.f;
+      // The incoming state needs nothing from this tile. Only chunk 0 reads
+      // the state in; its published total already contains it, so no later
+      // tile reads the caller's state (which state_out may alias).
+      const int qb = j / p.G;
+      const int first = qb * p.G;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) x[e] = (j == 0) ? state_in_acc(p, b, c0 + e) : acc_empty();
+      if (j > 0) {
+        const uint32_t* fp = p.flags_p + (size_t)(qb - 1) * BNG + bg;
+        bool got = false;
+        uint64_t tstart = 0;
+        while (true) {
+          bool all = (qb == 0) || ld_relaxed_u32(fp) == target;
+          for (int jj = first + lane; jj < j; jj += 32)
+            all &= ld_relaxed_u32(p.flags_a + (size_t)jj * BNG + bg) == target;
+          all = __all_sync(0xffffffffu, all);
+          if (all) {
+            got = true;
+            break;
+          }
+          if (tstart == 0) {
+            tstart = global_ns();
+          } else if (global_ns() - tstart > p.timeout_ns) {
+            break;
+          }
+          __nanosleep(32);
+        }
+        if (!got && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+        fence_acq_rel_gpu();
+        gather_group<VEC, CG, L>(p, x, first, j, bg, cl, w, qb > 0, qb);
+      }
+      // the replay also needs this tile's aggregates: wait for its fold
+      if (!mbar_wait(&folded[s], ph, p.timeout_ns)) {
+        pipe_fail(p, abort_flag, lane);
+        break;
+      }
+      if (j != p.nch - 1 && (j % p.G) == p.G - 1) {
+        // the last chunk of a look-back group publishes its inclusive prefix
+        float4* dst = p.agg_p + ((size_t)qb * BNG + bg) * CG + cl;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e)
+          dst[e] = acc_pack(combine(x[e], acc_unpack(tot[(size_t)s * CG + cl + e]), (float)L, w[e]));
+        __threadfence();
+        __syncwarp();
+        if (lane == 0 && tile != p.inject_tile) st_release_u32(p.flags_p + (size_t)qb * BNG + bg, target);
+      }
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) xin[(size_t)s * CG + cl + e] = acc_pack(x[e]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[s]);
+    }
+  } else if (wp < kReplay0) {
+    // --------------------------------------------------------------- fold
+    for (int n = 0;; ++n) {
+      const int s = n % S;
+      const bool got = mbar_wait(&full[s], (n / S) & 1, p.timeout_ns);
+      const int tile = got ? tile_id[s] : p.n_tiles;
+      if (named_sync_or<NC * 32>(1, !got || *abort_flag != 0)) {
+        pipe_fail(p, abort_flag, lane);
+        break;
+      }
+      if (tile >= p.n_tiles) break;
+      const int j = tile / BNG, bg = tile % BNG;
+      const int c0 = (bg % p.NG) * CG + cl;
+      const int nv = max(0, min(J, T - (j * L + wp * J)));
+      float w[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < C) ? __ldg(p.w + c0 + e) : 0.f;
+      const KV* ks = tiles + (size_t)s * 2 * kTile + (wp * J) * CG + cl;
+      Acc a[VEC];
+      aggregate_tile_span<KV, J, VEC, CG>(ks, ks + kTile, nv, w, a);
+      float4* ag = agg + (size_t)s * NC * CG;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) ag[wp * CG + cl + e] = acc_pack(a[e]);
+      named_sync<NC * 32>(1);
+      if (wp == NC - 1) {
+        // the tile total: published at once, and kept for the group prefix
+        Acc tt[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) tt[e] = acc_empty();
+        for (int qq = 0; qq < NC - 1; ++qq) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) tt[e] = combine(tt[e], acc_unpack(ag[qq * CG + cl + e]), (float)J, w[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          tt[e] = combine(tt[e], a[e], (float)nv, w[e]);
+          tot[(size_t)s * CG + cl + e] = acc_pack(tt[e]);
+        }
+        if (j != p.nch - 1) {
+          const int b = bg / p.NG;
+          float4* dst = p.agg_a + (size_t)tile * CG + cl;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            dst[e] = acc_pack(j == 0 ? combine(state_in_acc(p, b, c0 + e), tt[e], (float)L, w[e]) : tt[e]);
+          __threadfence();
+          __syncwarp();
+          if (lane == 0 && tile != p.inject_tile) st_release_u32(p.flags_a + tile, target);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&folded[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- replay
+    const int r = wp - kReplay0;  // this warp's span of every tile
+    for (int n = 0;; ++n) {
+      const int s = n % S;
+      if (!mbar_wait(&ready[s], (n / S) & 1, p.timeout_ns)) {
+        pipe_fail(p, abort_flag, lane);
+        break;
+      }
+      const int tile = tile_id[s];
+      if (tile >= p.n_tiles || *abort_flag) break;
+      const int j = tile / BNG, bg = tile % BNG;
+      const int b = bg / p.NG, c0 = (bg % p.NG) * CG + cl;
+      const int ts = j * L + r * J;
+      const int nv = max(0, min(J, T - ts));
+      const bool last_chunk = (j == p.nch - 1);
+      const int p_last = last_chunk ? (T - 1 - j * L) / J : NC - 1;
+      if (nv > 0) {
+        float w[VEC], u[VEC], cb[VEC];
+        bool fast = true;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const bool okc = c0 + e < C;
+          w[e] = okc ? __ldg(p.w + c0 + e) : 0.f;
+          u[e] = okc ? __ldg(p.u + c0 + e) : 0.f;
+          fast &= fast_uw(u[e], w[e]);
+          cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+        }
+        fast = __all_sync(0xffffffffu, fast);
+        // state at the start of the span: incoming state, then the spans before it
+        const float4* ag = agg + (size_t)s * NC * CG;
+        Acc st[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) st[e] = acc_empty();
+        for (int qq = 0; qq < r; ++qq) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) st[e] = combine(st[e], acc_unpack(ag[qq * CG + cl + e]), (float)J, w[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e)
+          st[e] = combine(acc_unpack(xin[(size_t)s * CG + cl + e]), st[e], (float)(r * J), w[e]);
+        const KV* ks = tiles + (size_t)s * 2 * kTile + (r * J) * CG + cl;
+        const KV* vs = ks + kTile;
+        OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
+        const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
+        if (fast && nv == J) {
+          constexpr int NB = J < 8 ? J : 8;  // tokens per block of step_tokens
+#pragma unroll
+          for (int i0 = 0; i0 < J; i0 += NB) {
+            float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
+#pragma unroll
+            for (int ii = 0; ii < NB; ++ii) {
+              load_vec<KV, VEC>(ks + (i0 + ii) * CG, kb[ii]);
+              load_vec<KV, VEC>(vs + (i0 + ii) * CG, vb[ii]);
+            }
+            step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
+#pragma unroll
+            for (int ii = 0; ii < NB; ++ii) {
+              if (lane_vec) {
+                stg_stream<OUT, VEC>(orow + (size_t)(i0 + ii) * C, ob[ii]);
+              } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                  if (c0 + e < C) orow[(size_t)(i0 + ii) * C + e] = Elem<OUT>::from_f32(ob[ii][e]);
+              }
+            }
+          }
+        } else {
+          for (int i = 0; i < nv; ++i) {
+            float kx[VEC], vx[VEC], o[VEC];
+            load_vec<KV, VEC>(ks + i * CG, kx);
+            load_vec<KV, VEC>(vs + i * CG, vx);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+              if (fast) {
+                o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+              } else {
+                o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
+                add_token(st[e], kx[e], vx[e], w[e]);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+              if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
+          }
+        }
+        if (last_chunk && r == p_last && p.o_num) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            if (c0 + e < C) {
+              const size_t i = (size_t)b * C + c0 + e;
+              p.o_num[i] = st[e].num;
+              p.o_den[i] = st[e].den;
+              p.o_max[i] = acc_max_e(st[e], w[e]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // the stage may be refilled
+    }
+  }
+
+  // ---- hand the workspace back for the next launch once every CTA is done
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(&p.hdr->done, 1u);
+    if (prev == gridDim.x - 1) {
+      p.hdr->ticket = 0;
+      p.hdr->done = 0;
+      __threadfence();
+      atomicExch(&p.hdr->epoch, target);
     }
   }
 }
