@@ -80,7 +80,10 @@ typedef struct {
 /*
  * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
  * zero-filled struct also means "defaults".
- *   kernel          0 = choose by shape, 1 = sequential-over-T kernel,
+ *   kernel          0 = choose by shape (sequential for many channels or short
+ *                   sequences; otherwise a chunked scan, pipelined from 4096
+ *                   tiles of 64 channels x chunk_len tokens on),
+ *                   1 = sequential-over-T kernel,
  *                   2 = chunked scan in one launch (look-back between CTAs),
  *                   3 = span-streaming scan in three launches (span totals,
  *                   their scan, then the replay; for inputs that stay in L2

@@ -62,7 +62,8 @@ def test_forward_kernel_choice(L):
     assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
     assert L.wkv_forward_kernel(8, 1024, 768, F32, None) in (2, 4)
-    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) in (2, 4)
+    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 4
+    assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 2  # rows TMA cannot address
     # an explicit choice stands, except that the TMA-only scans fall back to the
     # single-launch scan when a row pitch is not a multiple of 16 bytes
     for kernel in (1, 2, 3, 4):
