@@ -105,6 +105,9 @@ typedef struct {
  *   replay          how the span-streaming scan (kernel 3) replays its spans:
  *                   0 = choose, 1 = through per-warp TMA rings in shared
  *                   memory, 2 = with loads straight into registers
+ *   seq_vec         channels per thread of the sequential kernel: 1 or 2
+ *                   (0 = choose: 1 below 151552 channels B*C, else 2)
+ *   reserved        must be 0
  *   stages          shared-memory ring stages of the pipelined scan
  *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
  *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)
@@ -126,6 +129,8 @@ typedef struct {
     int32_t seq_threads;
     int32_t replay;
     int32_t stages;
+    int32_t seq_vec;
+    int32_t reserved;
 } wkv_options;
 
 /*

@@ -113,6 +113,22 @@ def test_bf16_inputs(oracle, out_dtype, opts):
     compare(oracle, kb, vb, w, u, st, kv="bf16", out_dtype=out_dtype, options=opts, rtol=rtol)
 
 
+SEQ1 = [{"kernel": 1, "seq_vec": 1}, {"kernel": 1, "seq_vec": 1, "seq_threads": 64},
+        {"kernel": 1, "seq_vec": 1, "seq_threads": 128}]
+
+
+@pytest.mark.parametrize("opts", SEQ1, ids=["t32", "t64", "t128"])
+@pytest.mark.parametrize("shape", [(2, 33, 64), (3, 1000, 128), (2, 517, 200), (1, 70, 36)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_sequential_one_channel_per_thread(oracle, opts, shape):
+    """The sequential kernel with one channel per thread (ragged channel groups and token tails)."""
+    B, T, C = shape
+    k, v, w, u, st = I.random_case(B, T, C, seed=B + T + C, k_scale=2.0, k_spike=30.0, state=True)
+    compare(oracle, k, v, w, u, st, options=opts)
+    kb, vb = I.f32_to_bf16_bits(2.0 * k), I.f32_to_bf16_bits(v)
+    compare(oracle, kb, vb, w, u, st, kv="bf16", out_dtype="bf16", options=opts)
+
+
 # ---------------------------------------------------------------------------
 # special cases with closed forms
 # ---------------------------------------------------------------------------

@@ -28,18 +28,23 @@ constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s
 // kernel configurations
 // ---------------------------------------------------------------------------
 // sequential kernel: CTA = 32, 64 or 128 threads x VEC channels, LT-token tiles
-constexpr int kSeqVecF32 = 2, kSeqLtF32 = 8, kSeqStagesF32 = 4;    // 4 stages of 64 B x CG
-constexpr int kSeqVecBf16 = 2, kSeqLtBf16 = 16, kSeqStagesBf16 = 4;  // 4 stages of 64 B x CG
+// (tokens per stage for 2 channels per thread; twice as many for 1)
+constexpr int kSeqLtF32 = 8, kSeqStagesF32 = 4;    // 4 stages of 64 B x CG
+constexpr int kSeqLtBf16 = 16, kSeqStagesBf16 = 4;  // 4 stages of 64 B x CG
 constexpr int kSeqFallbackVec = 1, kSeqFallbackLt = 16;
 
 // chunked kernel: a tile is 64 channels (32 lanes x 2) by L = NW x 16 tokens
 constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
+// the automatic choice gives the sequential kernel one channel per thread below
+// this many channels (148 SMs x 16 warps x 64 channels)
+constexpr long long kSeqVec1MaxLanes = 148ll * 16 * 64;
 // the automatic choice takes the pipelined chunked scan from this many tiles on
 constexpr long long kPipeMinTiles = 4096;
 
 struct Plan {
   int kernel;  // 1 seq, 2 chunked single launch, 3 span streaming (three launches), 4 pipelined chunked
   int seq_threads;  // CTA width of the sequential kernel
+  int seq_vec;      // channels per thread of the sequential kernel
   int replay;       // span-streaming replay: 1 TMA rings, 2 loads into registers
   int stages;       // pipelined chunked scan: ring stages (0 = choose at launch)
   int L;       // chunk length (chunk kernel)
@@ -96,6 +101,11 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   pl->bytes = sizeof(WsHeader);
   if (o && (o->replay < 0 || o->replay > 2)) return false;
   if (o && (o->stages < 0 || o->stages == 1 || o->stages > 8)) return false;
+  if (o && (o->seq_vec < 0 || o->seq_vec > 2 || o->reserved != 0)) return false;
+  // one channel per thread doubles the warps of the sequential kernel; worth
+  // it while two per thread would leave fewer than ~16 warps per SM (measured,
+  // 65536 channels: 377 vs 424 us)
+  pl->seq_vec = (o && o->seq_vec) ? o->seq_vec : (lanes < kSeqVec1MaxLanes ? 1 : 2);
   pl->stages = o ? o->stages : 0;
   pl->replay = (o && o->replay) ? o->replay : 2;
   int sth = o ? o->seq_threads : 0;
@@ -418,6 +428,25 @@ wkv_status launch_chunk_shape(const Plan& pl, const FwdParams& p, const CUtensor
   }
 }
 
+// The sequential kernel with TMA-fed stages of VEC channels per thread. A
+// stage holds about 4 KB of k and v whatever VEC is (fewer channels, more
+// tokens).
+template <typename KV, typename OUT, int VEC>
+wkv_status launch_seq_tma(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
+  constexpr bool kF32 = sizeof(KV) == 4;
+  constexpr int LT = (kF32 ? kSeqLtF32 : kSeqLtBf16) * (2 / VEC);
+  constexpr int STG = kF32 ? kSeqStagesF32 : kSeqStagesBf16;
+  CUtensorMap tk, tv;
+  const int cg = pl.seq_threads * VEC;
+  if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, cg) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, cg))
+    return WKV_ERR_CUDA;
+  switch (pl.seq_threads) {
+    case 32: return launch_seq<KV, OUT, 32, VEC, LT, STG, true>(p, tk, tv, st, dev);
+    case 64: return launch_seq<KV, OUT, 64, VEC, LT, STG, true>(p, tk, tv, st, dev);
+    default: return launch_seq<KV, OUT, 128, VEC, LT, STG, true>(p, tk, tv, st, dev);
+  }
+}
+
 template <typename KV, typename OUT>
 wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kvdt, cudaStream_t st, int dev,
                             const DevInfo& di) {
@@ -426,19 +455,9 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
   std::memset(&tk, 0, sizeof tk);
   std::memset(&tv, 0, sizeof tv);
   if (pl.kernel == 1) {
-    constexpr bool kF32 = sizeof(KV) == 4;
-    constexpr int VEC = kF32 ? kSeqVecF32 : kSeqVecBf16;
-    constexpr int LT = kF32 ? kSeqLtF32 : kSeqLtBf16;
-    constexpr int STG = kF32 ? kSeqStagesF32 : kSeqStagesBf16;
     if (tma) {
-      const int cg = pl.seq_threads * VEC;
-      if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, cg) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, cg))
-        return WKV_ERR_CUDA;
-      switch (pl.seq_threads) {
-        case 32: return launch_seq<KV, OUT, 32, VEC, LT, STG, true>(p, tk, tv, st, dev);
-        case 64: return launch_seq<KV, OUT, 64, VEC, LT, STG, true>(p, tk, tv, st, dev);
-        default: return launch_seq<KV, OUT, 128, VEC, LT, STG, true>(p, tk, tv, st, dev);
-      }
+      if (pl.seq_vec == 1) return launch_seq_tma<KV, OUT, 1>(pl, p, kvdt, st, dev);
+      return launch_seq_tma<KV, OUT, 2>(pl, p, kvdt, st, dev);
     }
     return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
   }
@@ -597,7 +616,7 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
     }
   }
   const size_t oes = out_dtype == WKV_F32 ? 4 : 2;
-  const int vec = pl.kernel == 1 ? (tma ? (kv_dtype == WKV_F32 ? kSeqVecF32 : kSeqVecBf16) : kSeqFallbackVec)
+  const int vec = pl.kernel == 1 ? (tma ? pl.seq_vec : kSeqFallbackVec)
                                  : kChunkVec;
   p.vec_store = aligned(out, oes * vec) && (C % vec) == 0;
   if (pl.kernel >= 2)  // the chunked kernels also load k and v VEC-wide
