@@ -435,7 +435,9 @@ template <typename KV, typename OUT, int VEC>
 wkv_status launch_seq_tma(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
   constexpr bool kF32 = sizeof(KV) == 4;
   constexpr int LT = (kF32 ? kSeqLtF32 : kSeqLtBf16) * (2 / VEC);
-  constexpr int STG = kF32 ? kSeqStagesF32 : kSeqStagesBf16;
+  // one channel per thread: 3 stages (12 KB), so that the many one-warp CTAs
+  // this variant is for all fit on the device at once
+  constexpr int STG = VEC == 1 ? 3 : (kF32 ? kSeqStagesF32 : kSeqStagesBf16);
   CUtensorMap tk, tv;
   const int cg = pl.seq_threads * VEC;
   if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, cg) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, cg))
