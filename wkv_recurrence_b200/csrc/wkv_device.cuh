@@ -365,7 +365,7 @@ __device__ __forceinline__ void add_token(Acc& s, float k, float v, float w) {
   const float Md = fmaf(-nf1, w, s.ma);  // max exponent after the decay
   const float D2 = k - Md;
   const float x = ex2(-fabsf(D2) * kLog2e);
-  const bool reset = D2 > 0.f;  // the new key becomes the maximum (and the anchor)
+  const bool reset = k > Md;  // the new key becomes the maximum (and the anchor)
   const float a = reset ? x : 1.f;
   const float b = reset ? 1.f : x;
   s.num = fmaf(a, s.num, b * v);
@@ -391,7 +391,7 @@ __device__ __forceinline__ float step_token(Acc& s, float k, float v, float w, f
   const float Md = fmaf(-nf1, w, s.ma);
   const float D2 = k - Md;
   const float x = ex2(-fabsf(D2) * kLog2e);
-  const bool reset = D2 > 0.f;          // the key is the new maximum (and anchor)
+  const bool reset = k > Md;            // the key is the new maximum (and anchor)
   const float a = reset ? x : 1.f;      // weight of the carried state
   const float b = reset ? 1.f : x;      // weight of the current token (no bonus)
   const float bc = b * c;               // ... and with the bonus
@@ -407,8 +407,8 @@ __device__ __forceinline__ bool fast_uw(float u, float w) { return fabsf(u - w) 
 
 // step_token over N consecutive tokens of VEC channels, reorganised for
 // instruction-level parallelism. Only the anchor and count are carried from
-// token to token through a short chain (fma, subtract, compare, select), and
-// only it runs first, for all N tokens; the exponentials, the num/den updates
+// token to token through a short chain (fma, compare, select), and only it
+// runs first, for all N tokens; the exponentials, the num/den updates
 // and the outputs of the N tokens then have no dependency on each other
 // beyond one fma per token, so their latencies overlap. Every token goes
 // through exactly the operations of step_token, in the same order, so the
@@ -418,18 +418,25 @@ __device__ __forceinline__ void step_tokens(Acc (&s)[VEC], const float (&k)[N][V
                                             const float (&w)[VEC], const float (&c)[VEC], float (&out)[N][VEC]) {
   float d2[N][VEC];
   bool rs[N][VEC];
+  // The chain carries the anchor and cnt = (decays since the anchor) + 1, so
+  // that per token it is one fma, one compare and one select; the count's
+  // increment and the difference k - Md stay off it.
+  float cnt[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) cnt[e] = s[e].nf + 1.f;
 #pragma unroll
   for (int i = 0; i < N; ++i) {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      const float nf1 = s[e].nf + 1.f;
-      const float Md = fmaf(-nf1, w[e], s[e].ma);
+      const float Md = fmaf(-cnt[e], w[e], s[e].ma);
+      rs[i][e] = k[i][e] > Md;
       d2[i][e] = k[i][e] - Md;
-      rs[i][e] = d2[i][e] > 0.f;
       s[e].ma = rs[i][e] ? k[i][e] : s[e].ma;
-      s[e].nf = rs[i][e] ? 0.f : nf1;
+      cnt[e] = rs[i][e] ? 1.f : cnt[e] + 1.f;
     }
   }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) s[e].nf = cnt[e] - 1.f;
 #pragma unroll
   for (int i = 0; i < N; ++i) {
 #pragma unroll

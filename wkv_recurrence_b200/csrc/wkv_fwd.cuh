@@ -446,6 +446,21 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   }
 
   if (scan) {
+    // ---- hand the workspace back for the next launch: the CTA that counts
+    // itself last resets the ticket counter and advances the epoch. Every CTA
+    // counts itself only after reading the epoch and taking its ticket (both
+    // before the __syncthreads above), and neither is read again during the
+    // launch, so this can happen at the start instead of at the end, off the
+    // tile's path. The next launch on the stream starts after this one ends.
+    if (lane == 0) {
+      const uint32_t prev = atomicAdd(&p.hdr->done, 1u);
+      if (prev == (uint32_t)p.n_tiles - 1u) {
+        p.hdr->ticket = 0;
+        p.hdr->done = 0;
+        __threadfence();
+        atomicExch(&p.hdr->epoch, target);
+      }
+    }
     // ---- look-back: incoming state of the tile (overlaps the TMA copy)
     Acc x[VEC];
     const int qb = j / p.G;
@@ -629,18 +644,6 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     if (kTMA && !copy_ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
   }
 
-  // ---- hand the workspace back for the next launch once every tile is done
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const uint32_t prev = atomicAdd(&p.hdr->done, 1u);
-    if (prev == (uint32_t)p.n_tiles - 1u) {
-      p.hdr->ticket = 0;
-      p.hdr->done = 0;
-      __threadfence();
-      atomicExch(&p.hdr->epoch, target);
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
