@@ -139,7 +139,7 @@ def step_bytes(wl) -> int:
     return 36 * wl.B * wl.C + 8 * wl.C
 
 
-KERNEL_NAMES = {1: "wkv_fwd_seq", 2: "wkv_fwd_chunk", 3: "wkv_span_totals+scan+replay", 4: "wkv_fwd_pipe"}
+KERNEL_NAMES = {1: "wkv_fwd_seq", 2: "wkv_fwd_chunk", 3: "wkv_tile_totals+scan+replay", 4: "wkv_fwd_pipe"}
 
 
 def forward_kernel_name(wl, options) -> str:
@@ -152,9 +152,12 @@ def forward_kernel_name(wl, options) -> str:
 
 
 def launches_per_step(wl, options) -> int:
-    """Kernel launches of one step: the forward (1, or 3 for the span scan)
-    and one decode launch."""
-    return (3 if forward_kernel_name(wl, options).startswith("wkv_span") else 1) + 1
+    """Kernel launches of one step: the forward (1; for the three-launch scan
+    3, or 2 when the sequence is a single chunk) and one decode launch."""
+    if not forward_kernel_name(wl, options).startswith("wkv_tile"):
+        return 2
+    chunk = (options or {}).get("chunk_len", 0) or 128
+    return (3 if wl.T > chunk else 2) + 1
 
 
 def measured_peaks():

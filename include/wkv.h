@@ -81,18 +81,17 @@ typedef struct {
  * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
  * zero-filled struct also means "defaults".
  *   kernel          0 = choose by shape (sequential for many channels or short
- *                   sequences; otherwise a chunked scan, pipelined from 4096
- *                   tiles of 64 channels x chunk_len tokens on),
+ *                   sequences; otherwise the chunked scan in three launches),
  *                   1 = sequential-over-T kernel,
  *                   2 = chunked scan in one launch (look-back between CTAs),
- *                   3 = span-streaming scan in three launches (span totals,
- *                   their scan, then the replay; for inputs that stay in L2
- *                   between the launches),
+ *                   3 = chunked scan in three launches (chunk totals, their
+ *                   scan, then the replay; k and v are read twice, from L2
+ *                   the second time for inputs that fit there),
  *                   4 = chunked scan in one launch of persistent CTAs that
  *                   pipeline their tiles (look-back of one tile overlapped
  *                   with the next tile's fold and later tiles' copies)
- *   chunk_len       tokens per chunk for the chunked kernels (0 = choose;
- *                   otherwise 32, 64 or 128)
+ *   chunk_len       tokens per chunk for the chunked kernels (0 = choose: 64
+ *                   for the three-launch scan, 128 otherwise; or 32, 64, 128)
  *   lookback_group  G: the chunked kernel publishes a running prefix every G
  *                   chunks and each chunk combines at most G-1 chunk totals
  *                   after the last one (0 = choose; otherwise 1..1024)
@@ -102,9 +101,8 @@ typedef struct {
  *                   pipelined scan, so chunk_len 128 needs span 16 there)
  *   seq_threads     threads per CTA of the sequential kernel: 32, 64 or 128
  *                   (0 = choose); each thread carries 2 channels
- *   replay          how the span-streaming scan (kernel 3) replays its spans:
- *                   0 = choose, 1 = through per-warp TMA rings in shared
- *                   memory, 2 = with loads straight into registers
+ *   scan_segments   three-launch scan (kernel 3): segments per channel in the
+ *                   scan of the chunk totals: 0 = choose, or 1, 4, 16
  *   seq_vec         channels per thread of the sequential kernel: 1 or 2
  *                   (0 = choose: 1 below 151552 channels B*C, else 2)
  *   reserved        must be 0
@@ -127,7 +125,7 @@ typedef struct {
     int64_t inject_unpublished_tile;
     int32_t span;
     int32_t seq_threads;
-    int32_t replay;
+    int32_t scan_segments;
     int32_t stages;
     int32_t seq_vec;
     int32_t reserved;

@@ -61,8 +61,8 @@ def test_forward_kernel_choice(L):
     # many channels or short sequences: the sequential kernel; otherwise a chunked scan
     assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
-    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) in (2, 4)
-    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 4
+    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 3
+    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 3
     assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 2  # rows TMA cannot address
     # an explicit choice stands, except that the TMA-only scans fall back to the
     # single-launch scan when a row pitch is not a multiple of 16 bytes
@@ -117,8 +117,9 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(kernel=1, seq_threads=48)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
-    for bad in (dict(seq_vec=3), dict(seq_vec=-1), dict(reserved=1)):
-        o = _abi.wkv_options(kernel=1, **bad)
+    for bad in (dict(seq_vec=3), dict(seq_vec=-1), dict(reserved=1), dict(kernel=3, scan_segments=8),
+                dict(kernel=3, scan_segments=-1)):
+        o = _abi.wkv_options(**{"kernel": 1, **bad})
         assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
 
 

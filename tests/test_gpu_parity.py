@@ -66,12 +66,14 @@ def compare(oracle, k, v, w, u, state=None, kv="f32", out_dtype=None, options=No
                                   {"kernel": 2, "chunk_len": 64, "span": 8},
                                   TWO, {"kernel": 3, "chunk_len": 32, "span": 8},
                                   {"kernel": 3, "chunk_len": 64},
+                                  {"kernel": 3, "chunk_len": 32, "scan_segments": 4},
+                                  {"kernel": 3, "chunk_len": 32, "span": 8, "scan_segments": 16},
                                   PIPE, {"kernel": 4, "chunk_len": 32, "lookback_group": 1},
                                   {"kernel": 4, "chunk_len": 64, "span": 8, "stages": 2},
                                   {"kernel": 4, "chunk_len": 64, "span": 8, "lookback_group": 3, "stages": 5},
                                   {"kernel": 4, "chunk_len": 32, "span": 8, "lookback_group": 5, "stages": 8}],
                          ids=["auto", "seq", "chunk128", "chunk32g1", "chunk128g3", "chunk32g5s8", "chunk64s8",
-                              "two128", "two32s8", "two64", "pipe128", "pipe32g1", "pipe64s8st2",
+                              "two128", "two32s8", "two64", "two32seg4", "two32s8seg16", "pipe128", "pipe32g1", "pipe64s8st2",
                               "pipe64s8g3st5", "pipe32s8g5st8"])
 @pytest.mark.parametrize("shape", [(1, 1, 64), (2, 33, 64), (3, 1000, 128), (2, 517, 200), (1, 2048, 64)],
                          ids=lambda s: "x".join(map(str, s)))
@@ -384,6 +386,17 @@ def test_workload_full_size(oracle, name):
     _sampled_direct(oracle, k, v, w, u, out, st, wl.kv_dtype, 40 if wl.T > 10000 else 100, 7, sc, rtol,
                     bf16_out=wl.out_dtype == "bf16")
     print(f"{name}: max normalised out error {eo:.2e}, state errors {es}")
+
+
+@pytest.mark.parametrize("name", ["layer", "long", "mixed"])
+def test_workload_full_size_three_launches(oracle, name):
+    """The three-launch chunked scan on the benchmark shapes."""
+    wl = I.WORKLOADS[name]
+    k, v = I.draw_kv(wl)
+    w, u = I.draw_w(wl), I.draw_u(wl)
+    st = I.draw_state(wl)
+    _, _, eo, es = compare(oracle, k, v, w, u, st, kv=wl.kv_dtype, out_dtype=wl.out_dtype, options=TWO)
+    print(f"{name} (three launches): max normalised out error {eo:.2e}, state errors {es}")
 
 
 @pytest.mark.parametrize("name", ["layer", "long", "mixed"])

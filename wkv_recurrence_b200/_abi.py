@@ -43,7 +43,7 @@ class wkv_options(ctypes.Structure):
                 ("lookback_group", ctypes.c_int32), ("inject_enable", ctypes.c_int32),
                 ("wait_timeout_ns", ctypes.c_int64), ("inject_unpublished_tile", ctypes.c_int64),
                 ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32),
-                ("replay", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("scan_segments", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("seq_vec", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 

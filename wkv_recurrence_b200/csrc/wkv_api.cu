@@ -38,14 +38,12 @@ constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 // the automatic choice gives the sequential kernel one channel per thread below
 // this many channels (148 SMs x 16 warps x 64 channels)
 constexpr long long kSeqVec1MaxLanes = 148ll * 16 * 64;
-// the automatic choice takes the pipelined chunked scan from this many tiles on
-constexpr long long kPipeMinTiles = 4096;
 
 struct Plan {
   int kernel;  // 1 seq, 2 chunked single launch, 3 span streaming (three launches), 4 pipelined chunked
   int seq_threads;  // CTA width of the sequential kernel
   int seq_vec;      // channels per thread of the sequential kernel
-  int replay;       // span-streaming replay: 1 TMA rings, 2 loads into registers
+  int scan_segments;  // three-launch scan: segments per channel in the scan of chunk totals
   int stages;       // pipelined chunked scan: ring stages (0 = choose at launch)
   int L;       // chunk length (chunk kernel)
   int J;       // tokens per warp (chunk kernel)
@@ -92,14 +90,17 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     if (lanes >= 65536 || T <= 64) {
       kernel = 1;
     } else {
-      kernel = 2;
+      // chunked: the three-launch scan (measured: layer 27 vs 29 us single
+      // launch; long 465 vs 603 us pipelined, 636 us single launch)
+      kernel = 3;
     }
   }
   const bool three_requested = (kernel == 3);
   if ((kernel == 3 || kernel == 4) && !tma_ok) kernel = 2;
   pl->kernel = kernel;
   pl->bytes = sizeof(WsHeader);
-  if (o && (o->replay < 0 || o->replay > 2)) return false;
+  if (o && o->scan_segments != 0 && o->scan_segments != 1 && o->scan_segments != 4 && o->scan_segments != 16)
+    return false;
   if (o && (o->stages < 0 || o->stages == 1 || o->stages > 8)) return false;
   if (o && (o->seq_vec < 0 || o->seq_vec > 2 || o->reserved != 0)) return false;
   // one channel per thread doubles the warps of the sequential kernel; worth
@@ -107,7 +108,7 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   // 65536 channels: 377 vs 424 us)
   pl->seq_vec = (o && o->seq_vec) ? o->seq_vec : (lanes < kSeqVec1MaxLanes ? 1 : 2);
   pl->stages = o ? o->stages : 0;
-  pl->replay = (o && o->replay) ? o->replay : 2;
+  pl->scan_segments = o ? o->scan_segments : 0;
   int sth = o ? o->seq_threads : 0;
   if (sth == 0) sth = 32;  // many small CTAs: more resident warps per SM
   if (sth != 32 && sth != 64 && sth != 128) return false;
@@ -115,7 +116,7 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   if (kernel == 1) return true;
 
   int L = o ? o->chunk_len : 0;
-  if (L == 0) L = 128;
+  if (L == 0) L = kernel == 3 ? 64 : 128;
   if (L != 32 && L != 64 && L != 128) return false;
   int J = o ? o->span : 0;
   if (J == 0) J = 16;
@@ -135,21 +136,13 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   pl->n_tiles = (long long)pl->nch * BNG;
   if (pl->n_tiles >= (1ll << 31)) return false;
   pl->nblk = (pl->nch + G - 1) / G;
-  // automatic choice between the chunked scans: the pipelined one pays off
-  // once every SM has many tiles to stream (measured: 16384 tiles 9% faster,
-  // 768 tiles 20% slower)
-  if (want == 0 && tma_ok && pl->n_tiles >= kPipeMinTiles && L / J <= 8) {
-    kernel = 4;
-    pl->kernel = 4;
-  }
-  // span-streaming layout: span aggregates, span incoming states
-  const long long n_spans = (long long)((T + J - 1) / J) * BNG;
-  if (n_spans >= (1ll << 31)) return false;
+  // three-launch layout: totals of all chunks but the last, incoming states
+  // of all chunks
   size_t off3 = sizeof(WsHeader);
-  const size_t t_agg_a = off3;
-  off3 = round_up(off3 + sizeof(float4) * (size_t)n_spans * kChunkCG, 256);
+  const size_t t_tot = off3;
+  off3 = round_up(off3 + sizeof(float4) * (size_t)(std::max(pl->nch - 1, 0) * BNG) * kChunkCG, 256);
   const size_t t_x0 = off3;
-  off3 = round_up(off3 + sizeof(float4) * (size_t)n_spans * kChunkCG, 256);
+  off3 = round_up(off3 + sizeof(float4) * (size_t)pl->n_tiles * kChunkCG, 256);
   // single-launch layout: flags, chunk totals, group prefixes
   size_t off = sizeof(WsHeader);
   pl->off_flags_a = off;
@@ -162,9 +155,8 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   off = round_up(off + sizeof(float4) * (size_t)(pl->nblk * BNG) * kChunkCG, 256);
   if (kernel == 3) {
     pl->off_flags_a = pl->off_flags_p = pl->off_agg_p = 0;
-    pl->off_agg_a = t_agg_a;
+    pl->off_agg_a = t_tot;
     pl->off_x0 = t_x0;
-    pl->n_tiles = n_spans;
     pl->bytes = std::max(off3, off);
   } else {
     pl->bytes = three_requested ? std::max(off3, off) : off;
@@ -374,41 +366,55 @@ struct PdlConfig {
   }
 };
 
-template <typename KV, typename OUT, int J>
-wkv_status launch_spans(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev,
-                        int sms) {
+// The three-launch chunked scan: chunk totals (A), their scan (S), the replay
+// (B, launched with programmatic stream serialization so that its tile copies
+// overlap the scan).
+template <typename KV, typename OUT, int NW, int J>
+wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                        cudaStream_t st, int dev) {
   if (!p.agg_a || !p.x0 || !p.hdr) return WKV_ERR_INVALID_ARG;
-  // per-warp rings of 3 span stages; about 192 KB of shared memory per SM
-  constexpr int STAGES = 3;
-  constexpr int kSpanBytes = 2 * J * 64 * (int)sizeof(KV);
-  constexpr int WARPS = (192 * 1024 / (STAGES * kSpanBytes)) > 16 ? 16 : (192 * 1024 / (STAGES * kSpanBytes));
-  const size_t smem = (size_t)WARPS * STAGES * (kSpanBytes + 8);
-  auto fa = wkv_span_totals<KV, J, STAGES, WARPS>;
-  auto fb = wkv_span_replay<KV, OUT, J, STAGES, WARPS>;
-  auto fs = wkv_span_scan<8>;
-  int occ_a = 0, occ_b = 0;
-  if (!kernel_setup(fa, dev, WARPS * 32, smem, &occ_a) || occ_a < 1) return WKV_ERR_CUDA;
-  if (!kernel_setup(fb, dev, WARPS * 32, smem, &occ_b) || occ_b < 1) return WKV_ERR_CUDA;
-  const long long blocks_needed = (p.n_tiles + WARPS - 1) / WARPS;
-  const unsigned ga = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_a * sms, blocks_needed));
-  const unsigned gb = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_b * sms, blocks_needed));
-  fa<<<ga, WARPS * 32, smem, st>>>(p, tk, tv);
-  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
-  PdlConfig cs(dim3((unsigned)((long long)p.B * p.NG)), dim3(64 * 8), 0, st);
-  if (!cuda_ok(cudaLaunchKernelEx(&cs.cfg, fs, p, (int)J))) return WKV_ERR_CUDA;
-  if (p.replay_mode == 1) {
-    // replay straight from L2 into registers
-    auto fr = wkv_span_replay_ldg<KV, OUT, J>;
-    int occ_r = 0;
-    if (!kernel_setup(fr, dev, 256, 0, &occ_r) || occ_r < 1) return WKV_ERR_CUDA;
-    const unsigned gr = (unsigned)std::max<long long>(1, std::min<long long>((long long)occ_r * sms, (p.n_tiles + 7) / 8));
-    PdlConfig cr(dim3(gr), dim3(256), 0, st);
-    if (!cuda_ok(cudaLaunchKernelEx(&cr.cfg, fr, p))) return WKV_ERR_CUDA;
-    return launch_result();
+  constexpr int L = NW * J;
+  const size_t smem = 2ull * L * kChunkCG * sizeof(KV) + sizeof(float4) * NW * kChunkCG + 64;
+  auto fa = wkv_tile_totals<KV, NW, J>;
+  auto fb = wkv_tile_replay<KV, OUT, NW, J>;
+  int occ = 0;
+  if (!kernel_setup(fa, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  if (!kernel_setup(fb, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  const long long BNG = (long long)p.B * p.NG;
+  if (p.nch > 1) {
+    fa<<<(unsigned)((p.nch - 1) * BNG), NW * 32, smem, st>>>(p, tk, tv);
+    if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   }
-  PdlConfig cb(dim3(gb), dim3(WARPS * 32), smem, st);
+  // segments per channel in the scan: about 16 chunk totals each, at most 16
+  const int ntot = p.nch - 1;
+  int seg = pl.scan_segments;
+  if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 128 ? 4 : 16);
+  switch (seg) {
+    case 1: wkv_tile_scan<1><<<(unsigned)BNG, 64 * 1, 0, st>>>(p, L); break;
+    case 4: wkv_tile_scan<4><<<(unsigned)BNG, 64 * 4, 0, st>>>(p, L); break;
+    default: wkv_tile_scan<16><<<(unsigned)BNG, 64 * 16, 0, st>>>(p, L); break;
+  }
+  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  PdlConfig cb(dim3((unsigned)p.n_tiles), dim3(NW * 32), smem, st);
   if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, tk, tv))) return WKV_ERR_CUDA;
   return launch_result();
+}
+
+template <typename KV, typename OUT>
+wkv_status launch_tile3_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                              cudaStream_t st, int dev) {
+  if (pl.J == 8) {
+    switch (pl.L) {
+      case 32: return launch_tile3<KV, OUT, 4, 8>(pl, p, tk, tv, st, dev);
+      case 64: return launch_tile3<KV, OUT, 8, 8>(pl, p, tk, tv, st, dev);
+      default: return launch_tile3<KV, OUT, 16, 8>(pl, p, tk, tv, st, dev);
+    }
+  }
+  switch (pl.L) {
+    case 32: return launch_tile3<KV, OUT, 2, 16>(pl, p, tk, tv, st, dev);
+    case 64: return launch_tile3<KV, OUT, 4, 16>(pl, p, tk, tv, st, dev);
+    default: return launch_tile3<KV, OUT, 8, 16>(pl, p, tk, tv, st, dev);
+  }
 }
 
 template <typename KV, typename OUT, bool kTMA>
@@ -452,7 +458,6 @@ wkv_status launch_seq_tma(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cu
 template <typename KV, typename OUT>
 wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kvdt, cudaStream_t st, int dev,
                             const DevInfo& di) {
-  const int sms = di.sms;
   CUtensorMap tk, tv;
   std::memset(&tk, 0, sizeof tk);
   std::memset(&tv, 0, sizeof tv);
@@ -463,12 +468,11 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
     }
     return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
   }
-  if (pl.kernel == 3) {  // span streaming (make_plan only chooses it when TMA works)
-    if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.J, kChunkCG) ||
-        !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.J, kChunkCG))
+  if (pl.kernel == 3) {  // three launches (make_plan only chooses it when TMA works)
+    if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
+        !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
       return WKV_ERR_CUDA;
-    if (pl.J == 8) return launch_spans<KV, OUT, 8>(p, tk, tv, st, dev, sms);
-    return launch_spans<KV, OUT, 16>(p, tk, tv, st, dev, sms);
+    return launch_tile3_shape<KV, OUT>(pl, p, tk, tv, st, dev);
   }
   if (pl.kernel == 4) {  // pipelined (make_plan only chooses it when TMA works)
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
@@ -614,7 +618,6 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
     if (pl.kernel == 3) {
       p.flags_a = p.flags_p = nullptr;
       p.x0 = reinterpret_cast<float4*>(ws + pl.off_x0);
-      p.replay_mode = pl.replay == 2 ? 1 : 0;
     }
   }
   const size_t oes = out_dtype == WKV_F32 ? 4 : 2;

@@ -70,8 +70,7 @@ struct FwdParams {
   uint32_t* flags_p;   // [nblk * B * NG]
   float4* agg_a;       // [n_tiles][CG]
   float4* agg_p;       // [nblk * B * NG][CG] (single launch) or [n_tiles][NW][CG] (two launches)
-  float4* x0;          // incoming states of spans (span-streaming scan)
-  int replay_mode;     // span-streaming replay: 0 = TMA rings, 1 = loads into registers
+  float4* x0;          // incoming states of chunks (three-launch scan)
   int stages;          // pipelined chunk scan: shared-memory stages in the ring
 };
 
@@ -647,24 +646,27 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 }
 
 // ---------------------------------------------------------------------------
-// span-streaming scan in three launches, for inputs that fit in L2
+// chunked scan in three launches: chunk totals, their scan, the replay
 // ---------------------------------------------------------------------------
 //
-// A span is 64 channels of one batch row by J consecutive tokens. When k and v
-// together fit comfortably in the 126 MB L2:
-//   A (wkv_span_totals): every warp streams spans from HBM through its own
-//     ring of TMA stages and writes each span's aggregate (from the empty
-//     state) to the workspace;
-//   S (wkv_span_scan): for each (batch row, channel), the incoming state of
-//     every span: the state in combined with the aggregates of all earlier
-//     spans, as a two-level scan (segments of spans, then within segments);
-//   B (wkv_span_replay): every warp streams spans again -- from L2 -- and
-//     replays each from its incoming state, writing the outputs.
-// No warp ever waits for another warp or CTA inside a launch. S and B are
-// launched with programmatic stream serialization: B's warps start copying
-// their first spans (inputs only) while S runs, and wait (griddepcontrol.wait)
-// before reading any incoming state. Only S reads the caller's state in, and
-// it completes before B writes the state out, so the two may alias.
+// The tiles of wkv_fwd_chunk (64 channels x L = NW * J tokens, one CTA each),
+// with the look-back replaced by a launch boundary, so that no CTA ever waits
+// for another:
+//   A (wkv_tile_totals): every tile but those of the last chunk is copied in
+//     (TMA), folded from the empty state into its total, and the total is
+//     written to the workspace;
+//   S (wkv_tile_scan): for each (batch row, channel), the incoming state of
+//     every chunk: the state in combined with the totals of the chunks before
+//     it, as a two-level scan (segments of chunks, then within segments);
+//   B (wkv_tile_replay): every tile is copied in again, its warps fold their
+//     spans for the in-tile prefixes and replay them from (incoming state +
+//     prefix), writing the outputs.
+// k and v are read twice from memory: for inputs that fit in L2 the second
+// read hits L2. B is launched with programmatic stream serialization: its
+// CTAs issue their tile copies (inputs only) while S runs and wait
+// (griddepcontrol.wait) before reading an incoming state. Only S reads the
+// caller's state in, and it completes before B writes the state out, so the
+// two may alias. The order of combines depends on the shape only.
 
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -677,161 +679,90 @@ __device__ __forceinline__ float4 ldg_f4(const float4* q) {
   return r;
 }
 
-// Per-warp ring of STAGES span buffers (k box then v box, [J][64] each).
-template <typename KV, int J>
-struct SpanRing {
-  static constexpr int CG = 64;
-  static constexpr int kBox = J * CG;                                     // elements per tensor
-  static constexpr uint32_t kBytes = 2u * kBox * (uint32_t)sizeof(KV);   // per stage
-};
-
-// Span number sp (0 <= sp < n_spans) in time-major order: sp = q * BNG + bg,
-// so consecutive spans cover neighbouring channel groups of the same rows.
-__device__ __forceinline__ void span_coords(const FwdParams& p, int sp, int& q, int& b, int& g, int& bg) {
-  const int BNG = p.B * p.NG;
-  q = sp / BNG;
-  bg = sp % BNG;
-  b = bg / p.NG;
-  g = bg % p.NG;
-}
-
-// Walks a warp's spans sp, sp + GW, sp + 2 GW, ... keeping (q, b, g) up to
-// date with additions only (the divisions happen once, at the start).
-struct SpanWalk {
-  int sp, q, b, g;
-  int step, dq, db, dg, B, NG;
-  __device__ __forceinline__ SpanWalk(const FwdParams& p, int first, int stride) {
-    int bg;
-    sp = first;
-    step = stride;
-    span_coords(p, first, q, b, g, bg);
-    B = p.B;
-    NG = p.NG;
-    const int BNG = p.B * p.NG;
-    dq = stride / BNG;
-    const int rb = stride % BNG;
-    db = rb / p.NG;
-    dg = rb % p.NG;
-  }
-  __device__ __forceinline__ void next() {
-    sp += step;
-    g += dg;
-    int carry = g >= NG;
-    g -= carry ? NG : 0;
-    b += db + carry;
-    carry = b >= B;
-    b -= carry ? B : 0;
-    q += dq + carry;
-  }
-};
-
-template <typename KV, int J>
-__device__ __forceinline__ void span_issue(const FwdParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv, KV* buf,
-                                           uint64_t* bar, int sp) {
-  using R = SpanRing<KV, J>;
-  int q, b, g, bg;
-  span_coords(p, sp, q, b, g, bg);
-  mbar_arrive_expect_tx(bar, R::kBytes);
-  tma_load_3d(buf, tmk, bar, g * R::CG, q * J, b);
-  tma_load_3d(buf + R::kBox, tmv, bar, g * R::CG, q * J, b);
-}
-
-// After a warp stopped on a timeout at its i-th span: give the copies it had
-// in flight (its next STAGES spans) a bounded chance to land before it exits.
-template <int STAGES>
-__device__ __forceinline__ void span_ring_drain(const FwdParams& p, uint64_t* full, int i, int gw, int GW) {
-  if ((threadIdx.x & 31) != 0) return;
-  for (int k = i; k < i + STAGES; ++k)
-    if (gw + k * GW < p.n_tiles) (void)mbar_wait(&full[k % STAGES], (k / STAGES) & 1, p.timeout_ns);
-}
-
-// Common prologue of the streaming kernels: per-warp barriers and the first
-// STAGES copies of this warp's spans. Spans of warp gw: gw, gw + GW, ...
-template <typename KV, int J, int STAGES>
-__device__ __forceinline__ void span_ring_start(const FwdParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                                                KV* ring, uint64_t* full, int gw, int GW) {
-  using R = SpanRing<KV, J>;
-  const int lane = threadIdx.x & 31;
-  if (lane == 0) {
-    for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
-    fence_mbar_init();
-    for (int s = 0; s < STAGES; ++s) {
-      const int sp = gw + s * GW;
-      if (sp < p.n_tiles) span_issue<KV, J>(p, tmk, tmv, ring + (size_t)s * 2 * R::kBox, &full[s], sp);
-    }
-  }
-  __syncwarp();
-}
-
-template <typename KV, int J, int STAGES, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32)
-    wkv_span_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-  using R = SpanRing<KV, J>;
-  constexpr int VEC = 2, CG = R::CG;
+// Pass A. Grid: (nch - 1) * B * NG CTAs of NW warps; tile = blockIdx.x in
+// chunk-major order. Every tile here is a full chunk (the last chunk, which
+// alone can be partial, has no total to compute).
+template <typename KV, int NW, int J>
+__global__ void __launch_bounds__(NW * 32)
+    wkv_tile_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  constexpr int VEC = 2;
+  constexpr int CG = 32 * VEC;
+  constexpr int L = NW * J;
+  constexpr int kTile = L * CG;
+  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
   extern __shared__ __align__(1024) unsigned char smem[];
-  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-  KV* ring = reinterpret_cast<KV*>(smem) + (size_t)wp * STAGES * 2 * R::kBox;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)WARPS * STAGES * R::kBytes) + wp * STAGES;
-  const int GW = gridDim.x * WARPS;
-  const int gw = blockIdx.x * WARPS + wp;
-  if (lane == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
+  KV* ktile = reinterpret_cast<KV*>(smem);
+  float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_agg + NW * CG);
+
+  const int lane = threadIdx.x & 31;
+  const int wp = threadIdx.x >> 5;
+  const int BNG = p.B * p.NG;
+  const int tile = blockIdx.x;
+  const int j = tile / BNG, bg = tile % BNG;
+  const int cl = lane * VEC;
+  const int c0 = (bg % p.NG) * CG + cl;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, kBytes);
+    tma_load_3d(ktile, &tmk, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
+    tma_load_3d(ktile + kTile, &tmv, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
   }
-  span_ring_start<KV, J, STAGES>(p, &tmk, &tmv, ring, full, gw, GW);
-  const int T = p.T, C = p.C, cl = lane * VEC;
-  int i = 0;
-  SpanWalk it(p, gw, GW);
-  for (; it.sp < p.n_tiles; it.next(), ++i) {
-    const int s = i % STAGES;
-    const int sp = it.sp, q = it.q;
-    const int c0 = it.g * CG + cl;
-    float w[VEC];
+  __syncthreads();
+  float w[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < C) ? __ldg(p.w + c0 + e) : 0.f;
-    const int nv = min(J, T - q * J);
-    if (!mbar_wait(&full[s], (i / STAGES) & 1, p.timeout_ns)) {
-      if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
-      span_ring_drain<STAGES>(p, full, i, gw, GW);
-      break;
-    }
-    KV* buf = ring + (size_t)s * 2 * R::kBox;
-    Acc agg[VEC];
-    aggregate_tile_span<KV, J, VEC, CG>(buf + cl, buf + R::kBox + cl, nv, w, agg);
-    float4* dst = p.agg_a + (size_t)sp * CG + cl;
+  for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < p.C) ? __ldg(p.w + c0 + e) : 0.f;
+  const bool ok = mbar_wait(bar, 0, p.timeout_ns);
+  Acc a[VEC];
+  if (ok) {
+    aggregate_tile_span<KV, J, VEC, CG>(ktile + (wp * J) * CG + cl, ktile + kTile + (wp * J) * CG + cl, J, w, a);
+  } else {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(agg[e]);
-    __syncwarp();  // every lane is done with the stage
-    const int nxt = sp + STAGES * GW;
-    if (lane == 0 && nxt < p.n_tiles) {
-      fence_proxy_async_smem();
-      span_issue<KV, J>(p, &tmk, &tmv, buf, &full[s], nxt);
-    }
+    for (int e = 0; e < VEC; ++e) a[e] = acc_empty();
+    if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
   }
-  grid_launch_dependents();
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(a[e]);
+  __syncthreads();
+  if (wp == 0) {
+    Acc t[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) t[e] = acc_unpack(sh_agg[cl + e]);
+    for (int q = 1; q < NW; ++q) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) t[e] = combine(t[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+    }
+    float4* dst = p.agg_a + (size_t)tile * CG + cl;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(t[e]);
+  }
+  if (!ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
 }
 
-// Two-level scan over the spans of one (batch row, channel): SEG threads per
-// channel each own a contiguous segment of spans. The span aggregates are
-// read-only here (written by the previous launch), so they are loaded through
-// the non-coherent path, eight at a time.
+// Pass S. Grid: B * NG CTAs of 64 * SEG threads; SEG threads per channel
+// each own a contiguous segment of the nch - 1 chunk totals: (1) each
+// segment's total; (2) the segment's incoming state (state in, then the
+// totals of the segments before it); (3) each chunk's incoming state, written
+// to p.x0 [nch][B * NG][64]. The totals were written by the previous launch
+// and are read-only here, so they are loaded through the non-coherent path,
+// eight at a time.
 template <int SEG>
-__global__ void __launch_bounds__(64 * SEG) wkv_span_scan(const FwdParams p, int J) {
+__global__ void __launch_bounds__(64 * SEG) wkv_tile_scan(const FwdParams p, int L) {
   constexpr int CG = 64;
   __shared__ float4 seg_tot[SEG][CG];
-  grid_wait_prerequisites();
-  grid_launch_dependents();
+  grid_launch_dependents();  // the replay's CTAs may start copying their tiles
   const int BNG = p.B * p.NG;
   const int bg = blockIdx.x;
   const int cl = threadIdx.x % CG;
   const int sg = threadIdx.x / CG;
   const int b = bg / p.NG, c = (bg % p.NG) * CG + cl;
   const float w = c < p.C ? __ldg(p.w + c) : 0.f;
-  const int nsp = (p.T + J - 1) / J;
-  const int per = (nsp + SEG - 1) / SEG;
-  const int q0 = min(nsp, sg * per), q1 = min(nsp, q0 + per);
-  const float fJ = (float)J;
-  // 1. this segment's total (the spans before the last one are full J tokens)
+  const int ntot = p.nch - 1;
+  const int per = (ntot + SEG - 1) / SEG;
+  const int q0 = min(ntot, sg * per), q1 = min(ntot, q0 + per);
+  const float fL = (float)L;
+  // 1. this segment's total
   Acc tot = acc_empty();
   for (int qq = q0; qq < q1; qq += 8) {
     float4 a[8];
@@ -840,16 +771,17 @@ __global__ void __launch_bounds__(64 * SEG) wkv_span_scan(const FwdParams p, int
       if (qq + r < q1) a[r] = ldg_f4(p.agg_a + ((size_t)(qq + r) * BNG + bg) * CG + cl);
 #pragma unroll
     for (int r = 0; r < 8; ++r)
-      if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), (float)min(J, p.T - (qq + r) * J), w);
+      if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), fL, w);
   }
   seg_tot[sg][cl] = acc_pack(tot);
   __syncthreads();
-  // 2. incoming state of the segment, then of every span in it
+  // 2. incoming state of the segment
   Acc x = state_in_acc(p, b, c);
   for (int k = 0; k < sg; ++k) {
-    const int kq0 = min(nsp, k * per), kq1 = min(nsp, kq0 + per);
-    x = combine(x, acc_unpack(seg_tot[k][cl]), (float)max(0, min(p.T, kq1 * J) - kq0 * J), w);
+    const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
+    x = combine(x, acc_unpack(seg_tot[k][cl]), (float)(kq1 - kq0) * fL, w);
   }
+  // 3. incoming state of every chunk of the segment (and of the last chunk)
   for (int qq = q0; qq < q1; qq += 8) {
     float4 a[8];
 #pragma unroll
@@ -859,208 +791,104 @@ __global__ void __launch_bounds__(64 * SEG) wkv_span_scan(const FwdParams p, int
     for (int r = 0; r < 8; ++r) {
       if (qq + r < q1) {
         p.x0[((size_t)(qq + r) * BNG + bg) * CG + cl] = acc_pack(x);
-        x = combine(x, acc_unpack(a[r]), fJ, w);
+        x = combine(x, acc_unpack(a[r]), fL, w);
       }
     }
   }
+  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.x0[((size_t)ntot * BNG + bg) * CG + cl] = acc_pack(x);
 }
-
-template <typename KV, typename OUT, int J, int STAGES, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32)
-    wkv_span_replay(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-  using R = SpanRing<KV, J>;
-  constexpr int VEC = 2, CG = R::CG;
+// Pass B. Grid: nch * B * NG CTAs of NW warps (tile = blockIdx.x). The tile
+// copy is issued before waiting for the scan (inputs only).
+template <typename KV, typename OUT, int NW, int J>
+__global__ void __launch_bounds__(NW * 32)
+    wkv_tile_replay(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  constexpr int VEC = 2;
+  constexpr int CG = 32 * VEC;
+  constexpr int L = NW * J;
+  constexpr int kTile = L * CG;
+  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
   extern __shared__ __align__(1024) unsigned char smem[];
-  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-  KV* ring = reinterpret_cast<KV*>(smem) + (size_t)wp * STAGES * 2 * R::kBox;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)WARPS * STAGES * R::kBytes) + wp * STAGES;
-  const int GW = gridDim.x * WARPS;
-  const int gw = blockIdx.x * WARPS + wp;
-  if (lane == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
+  KV* ktile = reinterpret_cast<KV*>(smem);
+  KV* vtile = ktile + kTile;
+  float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_agg + NW * CG);
+
+  const int lane = threadIdx.x & 31;
+  const int wp = threadIdx.x >> 5;
+  const int T = p.T, C = p.C;
+  const int BNG = p.B * p.NG;
+  const int tile = blockIdx.x;
+  const int j = tile / BNG, bg = tile % BNG;
+  const int b = bg / p.NG;
+  const int cl = lane * VEC;
+  const int c0 = (bg % p.NG) * CG + cl;
+  const int ts = j * L + wp * J;
+  const int nv = max(0, min(J, T - ts));
+  const bool last_chunk = (j == p.nch - 1);
+  const int p_last = last_chunk ? (T - 1 - j * L) / J : NW - 1;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, kBytes);
+    tma_load_3d(ktile, &tmk, bar, (bg % p.NG) * CG, j * L, b);
+    tma_load_3d(vtile, &tmv, bar, (bg % p.NG) * CG, j * L, b);
   }
-  // the inputs are not written by the earlier launches: start copying now
-  span_ring_start<KV, J, STAGES>(p, &tmk, &tmv, ring, full, gw, GW);
-  grid_wait_prerequisites();  // incoming states are ready
-  const int T = p.T, C = p.C, cl = lane * VEC;
-  const int nsp = (T + J - 1) / J;
-  int i = 0;
-  SpanWalk it(p, gw, GW);
-  // the incoming state and parameters of a span are loaded one span ahead,
-  // so that their latency hides behind the previous span's replay
-  float4 nx[VEC];
-  float nw[VEC], nu[VEC];
-  auto fetch = [&](const SpanWalk& sw) {
-    if (sw.sp < p.n_tiles) {
-      const int cc = sw.g * CG + cl;
-      const float4* px = p.x0 + (size_t)sw.sp * CG + cl;
+  __syncthreads();
+  float w[VEC], u[VEC], cb[VEC];
+  bool fast = true;
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        const bool ok = cc + e < C;
-        nw[e] = ok ? __ldg(p.w + cc + e) : 0.f;
-        nu[e] = ok ? __ldg(p.u + cc + e) : 0.f;
-        nx[e] = px[e];
-      }
-    }
-  };
-  fetch(it);
-  for (; it.sp < p.n_tiles; ++i) {
-    const int s = i % STAGES;
-    const int sp = it.sp, q = it.q, b = it.b;
-    const int c0 = it.g * CG + cl;
-    const int ts = q * J;
-    const int nv = min(J, T - ts);
-    float w[VEC], u[VEC], cb[VEC];
-    bool fast = true;
-    Acc st[VEC];
+  for (int e = 0; e < VEC; ++e) {
+    const bool okc = c0 + e < C;
+    w[e] = okc ? __ldg(p.w + c0 + e) : 0.f;
+    u[e] = okc ? __ldg(p.u + c0 + e) : 0.f;
+    fast &= fast_uw(u[e], w[e]);
+    cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+  }
+  fast = __all_sync(0xffffffffu, fast);
+  const bool ok = mbar_wait(bar, 0, p.timeout_ns);
+  if (!ok && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+  const KV* ks = ktile + (wp * J) * CG + cl;
+  const KV* vs = vtile + (wp * J) * CG + cl;
+  // in-tile prefix: the spans of the warps before this one
+  {
+    Acc agg[VEC];
+    if (!ok || (last_chunk && wp >= p_last)) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      w[e] = nw[e];
-      u[e] = nu[e];
-      st[e] = acc_unpack(nx[e]);
-      fast &= fast_uw(u[e], w[e]);
-      cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
+      for (int e = 0; e < VEC; ++e) agg[e] = acc_empty();
+    } else {
+      aggregate_tile_span<KV, J, VEC, CG>(ks, vs, nv, w, agg);
     }
-    fast = __all_sync(0xffffffffu, fast);
-    it.next();
-    fetch(it);
-    if (!mbar_wait(&full[s], (i / STAGES) & 1, p.timeout_ns)) {
-      if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
-      span_ring_drain<STAGES>(p, full, i, gw, GW);
-      break;
-    }
-    const KV* ks = ring + (size_t)s * 2 * R::kBox + cl;
-    const KV* vs = ks + R::kBox;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(agg[e]);
+  }
+  __syncthreads();
+  Acc pre[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) pre[e] = acc_empty();
+  for (int q = 0; q < wp; ++q) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) pre[e] = combine(pre[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+  }
+  // the chunk's incoming state, from the scan
+  grid_wait_prerequisites();
+  Acc st[VEC];
+  {
+    const float4* xs = p.x0 + (size_t)tile * CG + cl;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) st[e] = combine(acc_unpack(xs[e]), pre[e], (float)(wp * J), w[e]);
+  }
+  if (nv > 0 && ok) {
     OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
     const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
     if (fast && nv == J) {
-#pragma unroll
-      for (int ii = 0; ii < J; ++ii) {
-        float kx[VEC], vx[VEC], o[VEC];
-        load_vec<KV, VEC>(ks + ii * CG, kx);
-        load_vec<KV, VEC>(vs + ii * CG, vx);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
-        if (lane_vec) {
-          stg_stream<OUT, VEC>(orow + (size_t)ii * C, o);
-        } else {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e)
-            if (c0 + e < C) orow[(size_t)ii * C + e] = Elem<OUT>::from_f32(o[e]);
-        }
-      }
-    } else {
-      for (int ii = 0; ii < nv; ++ii) {
-        float kx[VEC], vx[VEC], o[VEC];
-        load_vec<KV, VEC>(ks + ii * CG, kx);
-        load_vec<KV, VEC>(vs + ii * CG, vx);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          if (fast) {
-            o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
-          } else {
-            o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
-            add_token(st[e], kx[e], vx[e], w[e]);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < VEC; ++e)
-          if (c0 + e < C) orow[(size_t)ii * C + e] = Elem<OUT>::from_f32(o[e]);
-      }
-    }
-    if (q == nsp - 1 && p.o_num) {
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        if (c0 + e < C) {
-          const size_t ii = (size_t)b * C + c0 + e;
-          p.o_num[ii] = st[e].num;
-          p.o_den[ii] = st[e].den;
-          p.o_max[ii] = acc_max_e(st[e], w[e]);
-        }
-      }
-    }
-    __syncwarp();
-    const int nxt = sp + STAGES * GW;
-    if (lane == 0 && nxt < p.n_tiles) {
-      fence_proxy_async_smem();
-      span_issue<KV, J>(p, &tmk, &tmv, ring + (size_t)s * 2 * R::kBox, &full[s], nxt);
-    }
-  }
-}
-
-// Replay of the span-streaming scan that reads k and v straight from global
-// memory (they are L2-resident after the totals launch) into registers: no
-// shared memory, so occupancy is bounded by registers, not by staging
-// buffers, and each warp's 16-token span is one batch of coalesced loads.
-template <typename KV, typename OUT, int J>
-__global__ void __launch_bounds__(256) wkv_span_replay_ldg(const FwdParams p) {
-  constexpr int VEC = 2, CG = 64;
-  const int lane = threadIdx.x & 31;
-  const int GW = gridDim.x * (blockDim.x >> 5);
-  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  grid_wait_prerequisites();  // incoming states are ready
-  const int T = p.T, C = p.C, cl = lane * VEC;
-  const int nsp = (T + J - 1) / J;
-  const bool vec_in = p.vec_store != 0;
-  for (SpanWalk it(p, gw, GW); it.sp < p.n_tiles; it.next()) {
-    const int sp = it.sp, q = it.q, b = it.b;
-    const int c0 = it.g * CG + cl;
-    const int ts = q * J;
-    const int nv = min(J, T - ts);
-    const bool lane_vec = vec_in && c0 + VEC <= C;
-    // this span's tokens, all requested at once
-    float kx[J][VEC], vx[J][VEC];
-    const KV* kp = reinterpret_cast<const KV*>(p.k) + ((size_t)b * T + ts) * C + c0;
-    const KV* vp = reinterpret_cast<const KV*>(p.v) + ((size_t)b * T + ts) * C + c0;
-#pragma unroll
-    for (int ii = 0; ii < J; ++ii) {
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) kx[ii][e] = vx[ii][e] = 0.f;
-      if (ii < nv) {
-        if (lane_vec) {
-          ldg_stream<KV, VEC>(kp + (size_t)ii * C, kx[ii]);
-          ldg_stream<KV, VEC>(vp + (size_t)ii * C, vx[ii]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) {
-            if (c0 + e < C) {
-              kx[ii][e] = Elem<KV>::to_f32(kp[(size_t)ii * C + e]);
-              vx[ii][e] = Elem<KV>::to_f32(vp[(size_t)ii * C + e]);
-            }
-          }
-        }
-      }
-    }
-    float w[VEC], u[VEC], cb[VEC];
-    bool fast = true;
-    Acc st[VEC];
-    {
-      const float4* px = p.x0 + (size_t)sp * CG + cl;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        const bool ok = c0 + e < C;
-        w[e] = ok ? __ldg(p.w + c0 + e) : 0.f;
-        u[e] = ok ? __ldg(p.u + c0 + e) : 0.f;
-        fast &= fast_uw(u[e], w[e]);
-        cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
-        st[e] = acc_unpack(ldg_f4(px + e));
-      }
-    }
-    fast = __all_sync(0xffffffffu, fast);
-    OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
-    if (fast && nv == J) {
-      constexpr int NB = 8;  // tokens per block of step_tokens
+      constexpr int NB = J < 8 ? J : 8;  // tokens per block of step_tokens
 #pragma unroll
       for (int i0 = 0; i0 < J; i0 += NB) {
         float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
 #pragma unroll
         for (int ii = 0; ii < NB; ++ii) {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) {
-            kb[ii][e] = kx[i0 + ii][e];
-            vb[ii][e] = vx[i0 + ii][e];
-          }
+          load_vec<KV, VEC>(ks + (i0 + ii) * CG, kb[ii]);
+          load_vec<KV, VEC>(vs + (i0 + ii) * CG, vb[ii]);
         }
         step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
 #pragma unroll
@@ -1075,37 +903,37 @@ __global__ void __launch_bounds__(256) wkv_span_replay_ldg(const FwdParams p) {
         }
       }
     } else {
+      for (int i = 0; i < nv; ++i) {
+        float kx[VEC], vx[VEC], o[VEC];
+        load_vec<KV, VEC>(ks + i * CG, kx);
+        load_vec<KV, VEC>(vs + i * CG, vx);
 #pragma unroll
-      for (int ii = 0; ii < J; ++ii) {
-        if (ii < nv) {
-          float o[VEC];
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) {
-            if (fast) {
-              o[e] = step_token(st[e], kx[ii][e], vx[ii][e], w[e], cb[e]);
-            } else {
-              o[e] = out_token(st[e], kx[ii][e], vx[ii][e], w[e], u[e]);
-              add_token(st[e], kx[ii][e], vx[ii][e], w[e]);
-            }
+        for (int e = 0; e < VEC; ++e) {
+          if (fast) {
+            o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+          } else {
+            o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
+            add_token(st[e], kx[e], vx[e], w[e]);
           }
-#pragma unroll
-          for (int e = 0; e < VEC; ++e)
-            if (c0 + e < C) orow[(size_t)ii * C + e] = Elem<OUT>::from_f32(o[e]);
         }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e)
+          if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
       }
     }
-    if (q == nsp - 1 && p.o_num) {
+    if (last_chunk && wp == p_last && p.o_num) {
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
         if (c0 + e < C) {
-          const size_t ii = (size_t)b * C + c0 + e;
-          p.o_num[ii] = st[e].num;
-          p.o_den[ii] = st[e].den;
-          p.o_max[ii] = acc_max_e(st[e], w[e]);
+          const size_t i = (size_t)b * C + c0 + e;
+          p.o_num[i] = st[e].num;
+          p.o_den[i] = st[e].den;
+          p.o_max[i] = acc_max_e(st[e], w[e]);
         }
       }
     }
   }
+  if (!ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
 }
 
 // ---------------------------------------------------------------------------
