@@ -40,7 +40,7 @@ constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 constexpr long long kSeqVec1MaxLanes = 148ll * 16 * 64;
 
 struct Plan {
-  int kernel;  // 1 seq, 2 chunked single launch, 3 span streaming (three launches), 4 pipelined chunked
+  int kernel;  // 1 seq, 2 chunked single launch, 3 chunked in three launches, 4 pipelined chunked
   int seq_threads;  // CTA width of the sequential kernel
   int seq_vec;      // channels per thread of the sequential kernel
   int scan_segments;  // three-launch scan: segments per channel in the scan of chunk totals

@@ -1,11 +1,14 @@
 // Forward kernels of the WKV operator over [B, T, C] sequences.
 //
-// Both kernels run the recurrence of "Linear attention without writing a CUDA
+// All kernels run the recurrence of "Linear attention without writing a CUDA
 // kernel", section "The recurrence", in the anchored form of wkv_device.cuh,
-// one channel per register lane, VEC adjacent channels per thread. The
-// sequential kernel streams k and v through shared memory with TMA (3-D tiled
-// bulk copies of a [tokens x channel-group] box, completion on an mbarrier);
-// the chunked kernel loads its short spans straight into registers.
+// one channel per register lane, VEC adjacent channels per thread, and stream
+// k and v through shared memory with TMA (3-D tiled bulk copies of a
+// [tokens x channel-group] box, completion on an mbarrier), or with plain
+// loads where TMA cannot address the rows. The chunked scans come in three
+// forms: in one launch with look-back between CTAs (wkv_fwd_chunk), in three
+// launches with no waiting (wkv_tile_totals, wkv_tile_scan, wkv_tile_replay)
+// and in persistent pipelined CTAs (wkv_fwd_pipe).
 //
 // * wkv_fwd_seq: one CTA per (batch row, channel group), walking all T tokens
 //   through a STAGES-deep ring of [LT x CG] tiles. For many channels (B*C
