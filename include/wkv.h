@@ -102,7 +102,7 @@ typedef struct {
  *   seq_threads     threads per CTA of the sequential kernel: 32, 64 or 128
  *                   (0 = choose); each thread carries 2 channels
  *   scan_segments   three-launch scan (kernel 3): segments per channel in the
- *                   scan of the chunk totals: 0 = choose, or 1, 4, 16
+ *                   scan of the chunk totals: 0 = choose, or 1, 4, 16, 64
  *   seq_vec         channels per thread of the sequential kernel: 1 or 2
  *                   (0 = choose: 1 below 151552 channels B*C, else 2)
  *   reserved        must be 0

@@ -99,7 +99,8 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   if ((kernel == 3 || kernel == 4) && !tma_ok) kernel = 2;
   pl->kernel = kernel;
   pl->bytes = sizeof(WsHeader);
-  if (o && o->scan_segments != 0 && o->scan_segments != 1 && o->scan_segments != 4 && o->scan_segments != 16)
+  if (o && o->scan_segments != 0 && o->scan_segments != 1 && o->scan_segments != 4 && o->scan_segments != 16 &&
+      o->scan_segments != 64)
     return false;
   if (o && (o->stages < 0 || o->stages == 1 || o->stages > 8)) return false;
   if (o && (o->seq_vec < 0 || o->seq_vec > 2 || o->reserved != 0)) return false;
@@ -385,14 +386,16 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
     fa<<<(unsigned)((p.nch - 1) * BNG), NW * 32, smem, st>>>(p, tk, tv);
     if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   }
-  // segments per channel in the scan: about 16 chunk totals each, at most 16
+  // segments per channel in the scan: at most about 16 chunk totals each
   const int ntot = p.nch - 1;
   int seg = pl.scan_segments;
-  if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 128 ? 4 : 16);
+  if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 64 ? 4 : (ntot <= 256 ? 16 : 64));
+  const unsigned gs = (unsigned)(BNG * 4);  // 16 channels per CTA
   switch (seg) {
-    case 1: wkv_tile_scan<1><<<(unsigned)BNG, 64 * 1, 0, st>>>(p, L); break;
-    case 4: wkv_tile_scan<4><<<(unsigned)BNG, 64 * 4, 0, st>>>(p, L); break;
-    default: wkv_tile_scan<16><<<(unsigned)BNG, 64 * 16, 0, st>>>(p, L); break;
+    case 1: wkv_tile_scan<1><<<gs, 16 * 1, 0, st>>>(p, L); break;
+    case 4: wkv_tile_scan<4><<<gs, 16 * 4, 0, st>>>(p, L); break;
+    case 16: wkv_tile_scan<16><<<gs, 16 * 16, 0, st>>>(p, L); break;
+    default: wkv_tile_scan<64><<<gs, 16 * 64, 0, st>>>(p, L); break;
   }
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   PdlConfig cb(dim3((unsigned)p.n_tiles), dim3(NW * 32), smem, st);

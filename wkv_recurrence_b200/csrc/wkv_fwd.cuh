@@ -743,22 +743,25 @@ __global__ void __launch_bounds__(NW * 32)
   if (!ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
 }
 
-// Pass S. Grid: B * NG CTAs of 64 * SEG threads; SEG threads per channel
+// Pass S. Grid: B * NG * 4 CTAs of 16 * SEG threads: a CTA takes 16 of the
+// 64 channels of a (batch row, channel group), and SEG threads per channel
 // each own a contiguous segment of the nch - 1 chunk totals: (1) each
-// segment's total; (2) the segment's incoming state (state in, then the
-// totals of the segments before it); (3) each chunk's incoming state, written
-// to p.x0 [nch][B * NG][64]. The totals were written by the previous launch
-// and are read-only here, so they are loaded through the non-coherent path,
-// eight at a time.
+// segment's total; (2) one thread per channel walks the segment totals once,
+// from the state in, leaving each segment's incoming state in shared memory;
+// (3) each thread walks its segment again, writing each chunk's incoming
+// state to p.x0 [nch][B * NG][64] (and the last chunk's). The totals were
+// written by the previous launch and are read-only here, so they are loaded
+// through the non-coherent path, eight at a time.
 template <int SEG>
-__global__ void __launch_bounds__(64 * SEG) wkv_tile_scan(const FwdParams p, int L) {
-  constexpr int CG = 64;
-  __shared__ float4 seg_tot[SEG][CG];
+__global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int L) {
+  constexpr int CG = 64, CH = 16;
+  __shared__ float4 seg_st[SEG][CH];
   grid_launch_dependents();  // the replay's CTAs may start copying their tiles
   const int BNG = p.B * p.NG;
-  const int bg = blockIdx.x;
-  const int cl = threadIdx.x % CG;
-  const int sg = threadIdx.x / CG;
+  const int bg = blockIdx.x >> 2;
+  const int ch = threadIdx.x % CH;
+  const int cl = (blockIdx.x & 3) * CH + ch;
+  const int sg = threadIdx.x / CH;
   const int b = bg / p.NG, c = (bg % p.NG) * CG + cl;
   const float w = c < p.C ? __ldg(p.w + c) : 0.f;
   const int ntot = p.nch - 1;
@@ -776,15 +779,21 @@ __global__ void __launch_bounds__(64 * SEG) wkv_tile_scan(const FwdParams p, int
     for (int r = 0; r < 8; ++r)
       if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), fL, w);
   }
-  seg_tot[sg][cl] = acc_pack(tot);
+  seg_st[sg][ch] = acc_pack(tot);
   __syncthreads();
-  // 2. incoming state of the segment
-  Acc x = state_in_acc(p, b, c);
-  for (int k = 0; k < sg; ++k) {
-    const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
-    x = combine(x, acc_unpack(seg_tot[k][cl]), (float)(kq1 - kq0) * fL, w);
+  // 2. incoming state of every segment (state in, then the segments before)
+  if (sg == 0) {
+    Acc x = state_in_acc(p, b, c);
+    for (int k = 0; k < SEG; ++k) {
+      const Acc t = acc_unpack(seg_st[k][ch]);
+      const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
+      seg_st[k][ch] = acc_pack(x);
+      x = combine(x, t, (float)(kq1 - kq0) * fL, w);
+    }
   }
+  __syncthreads();
   // 3. incoming state of every chunk of the segment (and of the last chunk)
+  Acc x = acc_unpack(seg_st[sg][ch]);
   for (int qq = q0; qq < q1; qq += 8) {
     float4 a[8];
 #pragma unroll
@@ -800,6 +809,7 @@ __global__ void __launch_bounds__(64 * SEG) wkv_tile_scan(const FwdParams p, int
   }
   if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.x0[((size_t)ntot * BNG + bg) * CG + cl] = acc_pack(x);
 }
+
 // Pass B. Grid: nch * B * NG CTAs of NW warps (tile = blockIdx.x). The tile
 // copy is issued before waiting for the scan (inputs only).
 template <typename KV, typename OUT, int NW, int J>
