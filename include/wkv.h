@@ -90,8 +90,9 @@ typedef struct {
  *                   4 = chunked scan in one launch of persistent CTAs that
  *                   pipeline their tiles (look-back of one tile overlapped
  *                   with the next tile's fold and later tiles' copies)
- *   chunk_len       tokens per chunk for the chunked kernels (0 = choose: 64
- *                   for the three-launch scan, 128 otherwise; or 32, 64, 128)
+ *   chunk_len       tokens per chunk for the chunked kernels (0 = choose: 32
+ *                   or 64 for the three-launch scan, 128 otherwise; or 32, 64,
+ *                   128)
  *   lookback_group  G: the chunked kernel publishes a running prefix every G
  *                   chunks and each chunk combines at most G-1 chunk totals
  *                   after the last one (0 = choose; otherwise 1..1024)

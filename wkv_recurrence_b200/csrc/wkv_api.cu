@@ -117,7 +117,17 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   if (kernel == 1) return true;
 
   int L = o ? o->chunk_len : 0;
-  if (L == 0) L = kernel == 3 ? 64 : 128;
+  if (L == 0) {
+    // the three-launch scan replays every (batch row, chunk, 32 channels) as
+    // one warp: 32-token chunks where 64-token ones would give fewer than 8192
+    // such warps (measured, layer: 25.3 vs 26.5 us), else 64 (long: 424 us at
+    // both 64 and 128, 440 at 32)
+    if (kernel == 3) {
+      L = (B * C * ((T + 63) / 64)) / 32 < 8192 ? 32 : 64;
+    } else {
+      L = 128;
+    }
+  }
   if (L != 32 && L != 64 && L != 128) return false;
   int J = o ? o->span : 0;
   if (J == 0) J = 16;
@@ -287,7 +297,7 @@ template <typename KV, typename OUT, int THREADS, int VEC, int LT, int STAGES, b
 wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
   constexpr int CG = THREADS * VEC;
   const size_t smem = (size_t)STAGES * 2 * LT * CG * sizeof(KV) + 64 * STAGES;
-  auto fn = wkv_fwd_seq<KV, OUT, VEC, THREADS, LT, STAGES, kTMA>;
+  auto fn = wkv_fwd_seq<KV, OUT, VEC, THREADS, LT, STAGES, kTMA, false>;
   int occ = 0;
   if (!kernel_setup(fn, dev, THREADS, smem, &occ)) return WKV_ERR_CUDA;
   FwdParams q = p;
@@ -372,15 +382,13 @@ struct PdlConfig {
 // overlap the scan).
 template <typename KV, typename OUT, int NW, int J>
 wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                        cudaStream_t st, int dev) {
+                        wkv_dtype kvdt, cudaStream_t st, int dev) {
   if (!p.agg_a || !p.x0 || !p.hdr) return WKV_ERR_INVALID_ARG;
   constexpr int L = NW * J;
   const size_t smem = 2ull * L * kChunkCG * sizeof(KV) + sizeof(float4) * NW * kChunkCG + 64;
   auto fa = wkv_tile_totals<KV, NW, J>;
-  auto fb = wkv_tile_replay<KV, OUT, NW, J>;
   int occ = 0;
   if (!kernel_setup(fa, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
-  if (!kernel_setup(fb, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
   const long long BNG = (long long)p.B * p.NG;
   if (p.nch > 1) {
     fa<<<(unsigned)((p.nch - 1) * BNG), NW * 32, smem, st>>>(p, tk, tv);
@@ -398,25 +406,38 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
     default: wkv_tile_scan<64><<<gs, 16 * 64, 0, st>>>(p, L); break;
   }
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
-  PdlConfig cb(dim3((unsigned)p.n_tiles), dim3(NW * 32), smem, st);
-  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, tk, tv))) return WKV_ERR_CUDA;
+  // B: the sequential kernel over every (batch row, chunk, 32-channel group),
+  // from the chunk's incoming state; one channel per thread, 3 stages
+  constexpr bool kF32 = sizeof(KV) == 4;
+  constexpr int LT = kF32 ? 2 * kSeqLtF32 : 2 * kSeqLtBf16;
+  constexpr int CGB = 32;
+  CUtensorMap bk, bv;
+  if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, CGB) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, CGB))
+    return WKV_ERR_CUDA;
+  auto fb = wkv_fwd_seq<KV, OUT, 1, 32, LT, 3, true, true>;
+  const size_t smem_b = 3ull * 2 * LT * CGB * sizeof(KV) + 64 * 3;
+  if (!kernel_setup(fb, dev, 32, smem_b, &occ) || occ < 1) return WKV_ERR_CUDA;
+  const long long grid_b = (long long)p.B * p.nch * ((p.C + CGB - 1) / CGB);
+  if (grid_b >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  PdlConfig cb(dim3((unsigned)grid_b), dim3(32), smem_b, st);
+  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv))) return WKV_ERR_CUDA;
   return launch_result();
 }
 
 template <typename KV, typename OUT>
 wkv_status launch_tile3_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                              cudaStream_t st, int dev) {
+                              wkv_dtype kvdt, cudaStream_t st, int dev) {
   if (pl.J == 8) {
     switch (pl.L) {
-      case 32: return launch_tile3<KV, OUT, 4, 8>(pl, p, tk, tv, st, dev);
-      case 64: return launch_tile3<KV, OUT, 8, 8>(pl, p, tk, tv, st, dev);
-      default: return launch_tile3<KV, OUT, 16, 8>(pl, p, tk, tv, st, dev);
+      case 32: return launch_tile3<KV, OUT, 4, 8>(pl, p, tk, tv, kvdt, st, dev);
+      case 64: return launch_tile3<KV, OUT, 8, 8>(pl, p, tk, tv, kvdt, st, dev);
+      default: return launch_tile3<KV, OUT, 16, 8>(pl, p, tk, tv, kvdt, st, dev);
     }
   }
   switch (pl.L) {
-    case 32: return launch_tile3<KV, OUT, 2, 16>(pl, p, tk, tv, st, dev);
-    case 64: return launch_tile3<KV, OUT, 4, 16>(pl, p, tk, tv, st, dev);
-    default: return launch_tile3<KV, OUT, 8, 16>(pl, p, tk, tv, st, dev);
+    case 32: return launch_tile3<KV, OUT, 2, 16>(pl, p, tk, tv, kvdt, st, dev);
+    case 64: return launch_tile3<KV, OUT, 4, 16>(pl, p, tk, tv, kvdt, st, dev);
+    default: return launch_tile3<KV, OUT, 8, 16>(pl, p, tk, tv, kvdt, st, dev);
   }
 }
 
@@ -475,7 +496,7 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
         !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, pl.L, kChunkCG))
       return WKV_ERR_CUDA;
-    return launch_tile3_shape<KV, OUT>(pl, p, tk, tv, st, dev);
+    return launch_tile3_shape<KV, OUT>(pl, p, tk, tv, kvdt, st, dev);
   }
   if (pl.kernel == 4) {  // pipelined (make_plan only chooses it when TMA works)
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
@@ -613,6 +634,7 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
     p.NG = pl.NG;
     p.nch = pl.nch;
     p.G = pl.G;
+    p.chunk_len = pl.L;
     p.n_tiles = (int)pl.n_tiles;
     p.flags_a = reinterpret_cast<uint32_t*>(ws + pl.off_flags_a);
     p.flags_p = reinterpret_cast<uint32_t*>(ws + pl.off_flags_p);

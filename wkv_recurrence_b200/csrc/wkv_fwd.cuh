@@ -7,7 +7,8 @@
 // [tokens x channel-group] box, completion on an mbarrier), or with plain
 // loads where TMA cannot address the rows. The chunked scans come in three
 // forms: in one launch with look-back between CTAs (wkv_fwd_chunk), in three
-// launches with no waiting (wkv_tile_totals, wkv_tile_scan, wkv_tile_replay)
+// launches with no waiting (wkv_tile_totals, wkv_tile_scan, then wkv_fwd_seq
+// in chunked mode)
 // and in persistent pipelined CTAs (wkv_fwd_pipe).
 //
 // * wkv_fwd_seq: one CTA per (batch row, channel group), walking all T tokens
@@ -74,8 +75,17 @@ struct FwdParams {
   float4* agg_a;       // [n_tiles][CG]
   float4* agg_p;       // [nblk * B * NG][CG] (single launch) or [n_tiles][NW][CG] (two launches)
   float4* x0;          // incoming states of chunks (three-launch scan)
+  int chunk_len;       // chunked scans: tokens per chunk
   int stages;          // pipelined chunk scan: shared-memory stages in the ring
 };
+
+// Programmatic dependent launch: let the next launch on the stream be
+// scheduled, and wait for the launches before this one to finish (and their
+// writes to be visible).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // State in for one channel, anchored; empty when no state is passed.
 __device__ __forceinline__ Acc state_in_acc(const FwdParams& p, int b, int c) {
@@ -111,7 +121,13 @@ __device__ __forceinline__ void coop_load_tile(KV* dst, const KV* src, int b, in
 // ---------------------------------------------------------------------------
 // sequential-over-T kernel
 // ---------------------------------------------------------------------------
-template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA>
+// kChunked: the replay pass of the three-launch scan. A CTA then takes one
+// chunk (p.chunk_len tokens) of one batch row and starts from the chunk's
+// incoming state, which the scan pass wrote to p.x0 ([nch][B * NG][64] with
+// p.NG 64-channel groups); the grid is B * nch * ceil(C / CG). It issues its
+// first copies (inputs only) before waiting (griddepcontrol.wait) for the
+// scan, and only the last chunk writes the state out.
+template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA, bool kChunked>
 __global__ void __launch_bounds__(THREADS)
     wkv_fwd_seq(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
   constexpr int CG = THREADS * VEC;
@@ -122,11 +138,16 @@ __global__ void __launch_bounds__(THREADS)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
 
   const int tid = threadIdx.x;
-  const int b = blockIdx.x / p.NG;
-  const int g = blockIdx.x % p.NG;
   const int T = p.T, C = p.C;
+  const int ngs = kChunked ? (C + CG - 1) / CG : p.NG;  // channel groups of this kernel
+  const int bj = blockIdx.x / ngs;
+  const int g = blockIdx.x % ngs;
+  const int b = kChunked ? bj / p.nch : bj;
+  const int jc = kChunked ? bj % p.nch : 0;  // chunk
+  const int tbeg = kChunked ? jc * p.chunk_len : 0;
+  const int tend = kChunked ? min(T, tbeg + p.chunk_len) : T;
   const int c0 = g * CG + tid * VEC;
-  const int ntile = (T + LT - 1) / LT;
+  const int ntile = (tend - tbeg + LT - 1) / LT;
 
   if (kTMA && tid == 0) {
     prefetch_tmap(&tmk);
@@ -136,8 +157,8 @@ __global__ void __launch_bounds__(THREADS)
     fence_mbar_init();
     for (int s = 0; s < STAGES && s < ntile; ++s) {
       mbar_arrive_expect_tx(&full[s], kStageBytes);
-      tma_load_3d(tiles + (2 * s) * kTile, &tmk, &full[s], g * CG, s * LT, b);
-      tma_load_3d(tiles + (2 * s + 1) * kTile, &tmv, &full[s], g * CG, s * LT, b);
+      tma_load_3d(tiles + (2 * s) * kTile, &tmk, &full[s], g * CG, tbeg + s * LT, b);
+      tma_load_3d(tiles + (2 * s + 1) * kTile, &tmv, &full[s], g * CG, tbeg + s * LT, b);
     }
   }
 
@@ -153,9 +174,17 @@ __global__ void __launch_bounds__(THREADS)
     fast &= fast_uw(u[e], w[e]);
     cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
     st[e] = acc_empty();
-    if (ok && p.s_num) {
+    if (!kChunked && ok && p.s_num) {
       const size_t i = (size_t)b * C + c;
       st[e] = acc_from_state(p.s_num[i], p.s_den[i], p.s_max[i]);
+    }
+  }
+  if (kChunked) {
+    grid_wait_prerequisites();  // the scan pass has written the incoming states
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const int c = c0 + e;
+      if (c < C) st[e] = acc_unpack(p.x0[((size_t)jc * p.B * p.NG + (size_t)b * p.NG + c / 64) * 64 + c % 64]);
     }
   }
   fast = __all_sync(0xffffffffu, fast);  // one path per warp
@@ -167,7 +196,7 @@ __global__ void __launch_bounds__(THREADS)
   int aborted_at = -1;
   for (int i = 0; i < ntile; ++i) {
     const int s = kTMA ? (i % STAGES) : 0;
-    const int t0 = i * LT;
+    const int t0 = tbeg + i * LT;
     if (kTMA) {
       const bool ok = mbar_wait(&full[s], (i / STAGES) & 1, p.timeout_ns);
       if (__syncthreads_or(!ok)) {
@@ -181,7 +210,7 @@ __global__ void __launch_bounds__(THREADS)
     }
     const KV* ks = tiles + (2 * s) * kTile + tid * VEC;
     const KV* vs = ks + kTile;
-    const int nv = min(LT, T - t0);
+    const int nv = min(LT, tend - t0);
     OUT* orow = out + ((size_t)b * T + t0) * C;
     if (c0 < C) {
       if (nv == LT && fast) {
@@ -228,7 +257,7 @@ __global__ void __launch_bounds__(THREADS)
     __syncthreads();  // every thread is done with stage s
     if (kTMA && tid == 0 && i + STAGES < ntile) {
       fence_proxy_async_smem();
-      const int tn = (i + STAGES) * LT;
+      const int tn = tbeg + (i + STAGES) * LT;
       mbar_arrive_expect_tx(&full[s], kStageBytes);
       tma_load_3d(tiles + (2 * s) * kTile, &tmk, &full[s], g * CG, tn, b);
       tma_load_3d(tiles + (2 * s + 1) * kTile, &tmv, &full[s], g * CG, tn, b);
@@ -246,7 +275,7 @@ __global__ void __launch_bounds__(THREADS)
     return;
   }
 
-  if (p.o_num && c0 < C) {
+  if (p.o_num && c0 < C && (!kChunked || jc == p.nch - 1)) {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       const int c = c0 + e;
@@ -661,20 +690,16 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 //   S (wkv_tile_scan): for each (batch row, channel), the incoming state of
 //     every chunk: the state in combined with the totals of the chunks before
 //     it, as a two-level scan (segments of chunks, then within segments);
-//   B (wkv_tile_replay): every tile is copied in again, its warps fold their
-//     spans for the in-tile prefixes and replay them from (incoming state +
-//     prefix), writing the outputs.
+//   B (wkv_fwd_seq in chunked mode): every (batch row, chunk) is replayed as
+//     an independent sequence of chunk_len tokens from its incoming state, one
+//     channel per thread, streaming k and v again (TMA ring, 3 stages).
 // k and v are read twice from memory: for inputs that fit in L2 the second
 // read hits L2. B is launched with programmatic stream serialization: its
-// CTAs issue their tile copies (inputs only) while S runs and wait
+// CTAs issue their first copies (inputs only) while S runs and wait
 // (griddepcontrol.wait) before reading an incoming state. Only S reads the
-// caller's state in, and it completes before B writes the state out, so the
-// two may alias. The order of combines depends on the shape only.
-
-__device__ __forceinline__ void grid_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void grid_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// caller's state in, and it completes before B writes the state out (from
+// the last chunk), so the two may alias. The order of combines depends on
+// the shape only.
 
 __device__ __forceinline__ float4 ldg_f4(const float4* q) {
   float4 r;
@@ -808,145 +833,6 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
     }
   }
   if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.x0[((size_t)ntot * BNG + bg) * CG + cl] = acc_pack(x);
-}
-
-// Pass B. Grid: nch * B * NG CTAs of NW warps (tile = blockIdx.x). The tile
-// copy is issued before waiting for the scan (inputs only).
-template <typename KV, typename OUT, int NW, int J>
-__global__ void __launch_bounds__(NW * 32)
-    wkv_tile_replay(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
-  constexpr int VEC = 2;
-  constexpr int CG = 32 * VEC;
-  constexpr int L = NW * J;
-  constexpr int kTile = L * CG;
-  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
-  extern __shared__ __align__(1024) unsigned char smem[];
-  KV* ktile = reinterpret_cast<KV*>(smem);
-  KV* vtile = ktile + kTile;
-  float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_agg + NW * CG);
-
-  const int lane = threadIdx.x & 31;
-  const int wp = threadIdx.x >> 5;
-  const int T = p.T, C = p.C;
-  const int BNG = p.B * p.NG;
-  const int tile = blockIdx.x;
-  const int j = tile / BNG, bg = tile % BNG;
-  const int b = bg / p.NG;
-  const int cl = lane * VEC;
-  const int c0 = (bg % p.NG) * CG + cl;
-  const int ts = j * L + wp * J;
-  const int nv = max(0, min(J, T - ts));
-  const bool last_chunk = (j == p.nch - 1);
-  const int p_last = last_chunk ? (T - 1 - j * L) / J : NW - 1;
-  if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(bar, kBytes);
-    tma_load_3d(ktile, &tmk, bar, (bg % p.NG) * CG, j * L, b);
-    tma_load_3d(vtile, &tmv, bar, (bg % p.NG) * CG, j * L, b);
-  }
-  __syncthreads();
-  float w[VEC], u[VEC], cb[VEC];
-  bool fast = true;
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    const bool okc = c0 + e < C;
-    w[e] = okc ? __ldg(p.w + c0 + e) : 0.f;
-    u[e] = okc ? __ldg(p.u + c0 + e) : 0.f;
-    fast &= fast_uw(u[e], w[e]);
-    cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
-  }
-  fast = __all_sync(0xffffffffu, fast);
-  const bool ok = mbar_wait(bar, 0, p.timeout_ns);
-  if (!ok && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
-  const KV* ks = ktile + (wp * J) * CG + cl;
-  const KV* vs = vtile + (wp * J) * CG + cl;
-  // in-tile prefix: the spans of the warps before this one
-  {
-    Acc agg[VEC];
-    if (!ok || (last_chunk && wp >= p_last)) {
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) agg[e] = acc_empty();
-    } else {
-      aggregate_tile_span<KV, J, VEC, CG>(ks, vs, nv, w, agg);
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(agg[e]);
-  }
-  __syncthreads();
-  Acc pre[VEC];
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) pre[e] = acc_empty();
-  for (int q = 0; q < wp; ++q) {
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) pre[e] = combine(pre[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
-  }
-  // the chunk's incoming state, from the scan
-  grid_wait_prerequisites();
-  Acc st[VEC];
-  {
-    const float4* xs = p.x0 + (size_t)tile * CG + cl;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) st[e] = combine(acc_unpack(xs[e]), pre[e], (float)(wp * J), w[e]);
-  }
-  if (nv > 0 && ok) {
-    OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c0;
-    const bool lane_vec = p.vec_store != 0 && c0 + VEC <= C;
-    if (fast && nv == J) {
-      constexpr int NB = J < 8 ? J : 8;  // tokens per block of step_tokens
-#pragma unroll
-      for (int i0 = 0; i0 < J; i0 += NB) {
-        float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
-#pragma unroll
-        for (int ii = 0; ii < NB; ++ii) {
-          load_vec<KV, VEC>(ks + (i0 + ii) * CG, kb[ii]);
-          load_vec<KV, VEC>(vs + (i0 + ii) * CG, vb[ii]);
-        }
-        step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
-#pragma unroll
-        for (int ii = 0; ii < NB; ++ii) {
-          if (lane_vec) {
-            stg_stream<OUT, VEC>(orow + (size_t)(i0 + ii) * C, ob[ii]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e)
-              if (c0 + e < C) orow[(size_t)(i0 + ii) * C + e] = Elem<OUT>::from_f32(ob[ii][e]);
-          }
-        }
-      }
-    } else {
-      for (int i = 0; i < nv; ++i) {
-        float kx[VEC], vx[VEC], o[VEC];
-        load_vec<KV, VEC>(ks + i * CG, kx);
-        load_vec<KV, VEC>(vs + i * CG, vx);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          if (fast) {
-            o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
-          } else {
-            o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
-            add_token(st[e], kx[e], vx[e], w[e]);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < VEC; ++e)
-          if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
-      }
-    }
-    if (last_chunk && wp == p_last && p.o_num) {
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        if (c0 + e < C) {
-          const size_t i = (size_t)b * C + c0 + e;
-          p.o_num[i] = st[e].num;
-          p.o_den[i] = st[e].den;
-          p.o_max[i] = acc_max_e(st[e], w[e]);
-        }
-      }
-    }
-  }
-  if (!ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
 }
 
 // ---------------------------------------------------------------------------
