@@ -380,6 +380,23 @@ struct PdlConfig {
 // The three-launch chunked scan: chunk totals (A), their scan (S), the replay
 // (B, launched with programmatic stream serialization so that its tile copies
 // overlap the scan).
+// The replay pass of the three-launch scan: the sequential kernel in chunked
+// mode, one warp per (batch row, chunk, 32 channels), launched with
+// programmatic stream serialization after the scan.
+template <typename KV, typename OUT, int LT, int STAGES>
+wkv_status launch_seq_chunks(const FwdParams& p, const CUtensorMap& bk, const CUtensorMap& bv, cudaStream_t st,
+                             int dev) {
+  auto fb = wkv_fwd_seq<KV, OUT, 1, 32, LT, STAGES, true, true>;
+  const size_t smem = (size_t)STAGES * 2 * LT * 32 * sizeof(KV) + 64 * STAGES;
+  int occ = 0;
+  if (!kernel_setup(fb, dev, 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  const long long grid = (long long)p.B * p.nch * ((p.C + 31) / 32);
+  if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  PdlConfig cb(dim3((unsigned)grid), dim3(32), smem, st);
+  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv))) return WKV_ERR_CUDA;
+  return launch_result();
+}
+
 template <typename KV, typename OUT, int NW, int J>
 wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                         wkv_dtype kvdt, cudaStream_t st, int dev) {
@@ -407,21 +424,16 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   }
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   // B: the sequential kernel over every (batch row, chunk, 32-channel group),
-  // from the chunk's incoming state; one channel per thread, 3 stages
+  // from the chunk's incoming state; one channel per thread
   constexpr bool kF32 = sizeof(KV) == 4;
   constexpr int LT = kF32 ? 2 * kSeqLtF32 : 2 * kSeqLtBf16;
-  constexpr int CGB = 32;
   CUtensorMap bk, bv;
-  if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, CGB) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, CGB))
+  if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, 32) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, 32))
     return WKV_ERR_CUDA;
-  auto fb = wkv_fwd_seq<KV, OUT, 1, 32, LT, 3, true, true>;
-  const size_t smem_b = 3ull * 2 * LT * CGB * sizeof(KV) + 64 * 3;
-  if (!kernel_setup(fb, dev, 32, smem_b, &occ) || occ < 1) return WKV_ERR_CUDA;
-  const long long grid_b = (long long)p.B * p.nch * ((p.C + CGB - 1) / CGB);
-  if (grid_b >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  PdlConfig cb(dim3((unsigned)grid_b), dim3(32), smem_b, st);
-  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv))) return WKV_ERR_CUDA;
-  return launch_result();
+  // a chunk of at most two stages is prefetched whole with 2 (more CTAs fit
+  // per SM); longer chunks stream through 3
+  if (L <= 2 * LT) return launch_seq_chunks<KV, OUT, LT, 2>(p, bk, bv, st, dev);
+  return launch_seq_chunks<KV, OUT, LT, 3>(p, bk, bv, st, dev);
 }
 
 template <typename KV, typename OUT>
