@@ -131,12 +131,6 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -247,46 +241,7 @@ __device__ __forceinline__ void store_vec<__nv_bfloat16, 8>(__nv_bfloat16* p, co
                                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
 }
 
-// Streaming global loads straight into registers (read once: no L1
-// allocation) and streaming stores (evict-first in L2). `p` is aligned to VEC
-// elements.
-template <typename T, int VEC>
-__device__ __forceinline__ void ldg_stream(const T* p, float (&x)[VEC]);
-
-template <>
-__device__ __forceinline__ void ldg_stream<float, 1>(const float* p, float (&x)[1]) {
-  asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(x[0]) : "l"(p));
-}
-template <>
-__device__ __forceinline__ void ldg_stream<float, 2>(const float* p, float (&x)[2]) {
-  asm volatile("ld.global.nc.L1::no_allocate.v2.f32 {%0, %1}, [%2];" : "=f"(x[0]), "=f"(x[1]) : "l"(p));
-}
-template <>
-__device__ __forceinline__ void ldg_stream<float, 4>(const float* p, float (&x)[4]) {
-  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3])
-               : "l"(p));
-}
-template <>
-__device__ __forceinline__ void ldg_stream<__nv_bfloat16, 1>(const __nv_bfloat16* p, float (&x)[1]) {
-  unsigned short h;
-  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(h) : "l"(p));
-  x[0] = __uint_as_float(((uint32_t)h) << 16);
-}
-template <>
-__device__ __forceinline__ void ldg_stream<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&x)[2]) {
-  uint32_t u;
-  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(u) : "l"(p));
-  unpack_bf16x2(u, x[0], x[1]);
-}
-template <>
-__device__ __forceinline__ void ldg_stream<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&x)[4]) {
-  uint32_t a, b;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "l"(p));
-  unpack_bf16x2(a, x[0], x[1]);
-  unpack_bf16x2(b, x[2], x[3]);
-}
-
+// Streaming stores (evict-first in L2). `p` is aligned to VEC elements.
 template <typename T, int VEC>
 __device__ __forceinline__ void stg_stream(T* p, const float (&x)[VEC]);
 
@@ -450,10 +405,6 @@ __device__ __forceinline__ void step_tokens(Acc (&s)[VEC], const float (&k)[N][V
       s[e].den = fmaf(a, s[e].den, b);
     }
   }
-}
-
-__device__ __forceinline__ float bonus_factor(float u, float w) {
-  return ex2((u - w) * kLog2e);
 }
 
 // Associative combine: `a` covers the tokens before `b`, and `b` spans len_b
