@@ -411,12 +411,17 @@ __device__ __forceinline__ void step_tokens(Acc (&s)[VEC], const float (&k)[N][V
 // tokens. The result covers both: `a` is decayed across b's tokens (its count
 // grows by len_b) and the two are added relative to the larger exponent, which
 // becomes the anchor. The empty state is the identity.
+// The exponent difference (a.ma - na w) - (b.ma - b.nf w) is formed as
+// (a.ma - b.ma) - (na - b.nf) w: the counts are integers (exact), the anchors
+// are keys of similar size (their difference is often exact), so it is rounded
+// about once, at its own magnitude, instead of twice at the magnitude of the
+// anchored exponents (long chains of combines, as in a scan of many chunk
+// totals, keep their accuracy).
 __device__ __forceinline__ Acc combine(const Acc& a, const Acc& b, float len_b, float w) {
   const float na = a.nf + len_b;
-  const float Ma = fmaf(-na, w, a.ma);
-  const float Mb = fmaf(-b.nf, w, b.ma);
-  const bool a_wins = Ma >= Mb;
-  const float s = ex2(-fabsf(Ma - Mb) * kLog2e);
+  const float d = fmaf(-(na - b.nf), w, a.ma - b.ma);
+  const bool a_wins = d >= 0.f;
+  const float s = ex2(-fabsf(d) * kLog2e);
   Acc r;
   r.num = a_wins ? fmaf(s, b.num, a.num) : fmaf(s, a.num, b.num);
   r.den = a_wins ? fmaf(s, b.den, a.den) : fmaf(s, a.den, b.den);
