@@ -100,13 +100,16 @@ typedef struct {
  *   span            tokens per warp in a chunk-scan tile, 8 or 16 (0 = choose);
  *                   chunk_len / span warps share a tile (at most 8 for the
  *                   pipelined scan, so chunk_len 128 needs span 16 there)
- *   seq_threads     threads per CTA of the sequential kernel: 32, 64 or 128
- *                   (0 = choose); each thread carries 2 channels
+ *   seq_threads     threads per CTA of the sequential kernel and of the
+ *                   three-launch scan's replay pass: 32, 64 or 128 (0 =
+ *                   choose: 32); each thread carries seq_vec channels in the
+ *                   sequential kernel, one in the replay pass
  *   scan_segments   three-launch scan (kernel 3): segments per channel in the
  *                   scan of the chunk totals: 0 = choose, or 1, 4, 16, 64
  *   seq_vec         channels per thread of the sequential kernel: 1 or 2
  *                   (0 = choose: 1 below 151552 channels B*C, else 2)
- *   reserved        must be 0
+ *   replay_chunks   three-launch scan (kernel 3): consecutive chunks that
+ *                   one replay warp walks (0 = choose; or 1, 2, 4)
  *   stages          shared-memory ring stages of the pipelined scan
  *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
  *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)
@@ -129,7 +132,7 @@ typedef struct {
     int32_t scan_segments;
     int32_t stages;
     int32_t seq_vec;
-    int32_t reserved;
+    int32_t replay_chunks;
 } wkv_options;
 
 /*

@@ -117,7 +117,7 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(kernel=1, seq_threads=48)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
-    for bad in (dict(seq_vec=3), dict(seq_vec=-1), dict(reserved=1), dict(kernel=3, scan_segments=8), dict(kernel=3, scan_segments=32),
+    for bad in (dict(seq_vec=3), dict(seq_vec=-1), dict(kernel=3, replay_chunks=3), dict(kernel=3, replay_chunks=-1), dict(kernel=3, scan_segments=8), dict(kernel=3, scan_segments=32),
                 dict(kernel=3, scan_segments=-1)):
         o = _abi.wkv_options(**{"kernel": 1, **bad})
         assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG

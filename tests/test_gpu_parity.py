@@ -69,12 +69,16 @@ def compare(oracle, k, v, w, u, state=None, kv="f32", out_dtype=None, options=No
                                   {"kernel": 3, "chunk_len": 32, "scan_segments": 4},
                                   {"kernel": 3, "chunk_len": 32, "span": 8, "scan_segments": 16},
                                   {"kernel": 3, "chunk_len": 32, "scan_segments": 64},
+                                  {"kernel": 3, "chunk_len": 32, "replay_chunks": 2},
+                                  {"kernel": 3, "chunk_len": 64, "scan_segments": 4, "replay_chunks": 4},
+                                  {"kernel": 3, "chunk_len": 32, "seq_threads": 64},
+                                  {"kernel": 3, "chunk_len": 64, "seq_threads": 128, "replay_chunks": 2},
                                   PIPE, {"kernel": 4, "chunk_len": 32, "lookback_group": 1},
                                   {"kernel": 4, "chunk_len": 64, "span": 8, "stages": 2},
                                   {"kernel": 4, "chunk_len": 64, "span": 8, "lookback_group": 3, "stages": 5},
                                   {"kernel": 4, "chunk_len": 32, "span": 8, "lookback_group": 5, "stages": 8}],
                          ids=["auto", "seq", "chunk128", "chunk32g1", "chunk128g3", "chunk32g5s8", "chunk64s8",
-                              "two128", "two32s8", "two64", "two32seg4", "two32s8seg16", "two32seg64", "pipe128", "pipe32g1", "pipe64s8st2",
+                              "two128", "two32s8", "two64", "two32seg4", "two32s8seg16", "two32seg64", "two32r2", "two64seg4r4", "two32t64", "two64t128r2", "pipe128", "pipe32g1", "pipe64s8st2",
                               "pipe64s8g3st5", "pipe32s8g5st8"])
 @pytest.mark.parametrize("shape", [(1, 1, 64), (2, 33, 64), (3, 1000, 128), (2, 517, 200), (1, 2048, 64)],
                          ids=lambda s: "x".join(map(str, s)))

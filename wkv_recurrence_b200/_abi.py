@@ -44,7 +44,7 @@ class wkv_options(ctypes.Structure):
                 ("wait_timeout_ns", ctypes.c_int64), ("inject_unpublished_tile", ctypes.c_int64),
                 ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32),
                 ("scan_segments", ctypes.c_int32), ("stages", ctypes.c_int32),
-                ("seq_vec", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("seq_vec", ctypes.c_int32), ("replay_chunks", ctypes.c_int32)]
 
 
 class WkvError(RuntimeError):

@@ -44,6 +44,8 @@ struct Plan {
   int seq_threads;  // CTA width of the sequential kernel
   int seq_vec;      // channels per thread of the sequential kernel
   int scan_segments;  // three-launch scan: segments per channel in the scan of chunk totals
+  int replay_chunks;  // three-launch scan: consecutive chunks per replay CTA
+  int replay_threads;  // three-launch scan: threads (channels) per replay CTA
   int stages;       // pipelined chunked scan: ring stages (0 = choose at launch)
   int L;       // chunk length (chunk kernel)
   int J;       // tokens per warp (chunk kernel)
@@ -103,7 +105,10 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
       o->scan_segments != 64)
     return false;
   if (o && (o->stages < 0 || o->stages == 1 || o->stages > 8)) return false;
-  if (o && (o->seq_vec < 0 || o->seq_vec > 2 || o->reserved != 0)) return false;
+  if (o && (o->seq_vec < 0 || o->seq_vec > 2)) return false;
+  if (o && o->replay_chunks != 0 && o->replay_chunks != 1 && o->replay_chunks != 2 && o->replay_chunks != 4)
+    return false;
+  pl->replay_chunks = (o && o->replay_chunks) ? o->replay_chunks : 1;
   // one channel per thread doubles the warps of the sequential kernel; worth
   // it while two per thread would leave fewer than ~16 warps per SM (measured,
   // 65536 channels: 377 vs 424 us)
@@ -143,6 +148,10 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   pl->G = G;
   pl->NG = (int)((C + kChunkCG - 1) / kChunkCG);
   pl->nch = (int)((T + L - 1) / L);
+  // the replay pass: 32 channels per CTA unless asked otherwise (the most
+  // resident warps; layer: 23.8 us against 24.2 and 24.7 at 64 and 128; long:
+  // within 1.5% at all three)
+  pl->replay_threads = (o && o->seq_threads) ? o->seq_threads : 32;
   const long long BNG = (long long)B * pl->NG;
   pl->n_tiles = (long long)pl->nch * BNG;
   if (pl->n_tiles >= (1ll << 31)) return false;
@@ -383,16 +392,17 @@ struct PdlConfig {
 // The replay pass of the three-launch scan: the sequential kernel in chunked
 // mode, one warp per (batch row, chunk, 32 channels), launched with
 // programmatic stream serialization after the scan.
-template <typename KV, typename OUT, int LT, int STAGES>
+template <typename KV, typename OUT, int TH, int LT, int STAGES>
 wkv_status launch_seq_chunks(const FwdParams& p, const CUtensorMap& bk, const CUtensorMap& bv, cudaStream_t st,
                              int dev) {
-  auto fb = wkv_fwd_seq<KV, OUT, 1, 32, LT, STAGES, true, true>;
-  const size_t smem = (size_t)STAGES * 2 * LT * 32 * sizeof(KV) + 64 * STAGES;
+  auto fb = wkv_fwd_seq<KV, OUT, 1, TH, LT, STAGES, true, true>;
+  const size_t smem = (size_t)STAGES * 2 * LT * TH * sizeof(KV) + 64 * STAGES;
   int occ = 0;
-  if (!kernel_setup(fb, dev, 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
-  const long long grid = (long long)p.B * p.nch * ((p.C + 31) / 32);
+  if (!kernel_setup(fb, dev, TH, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  const long long nseq = (p.nch + p.replay_chunks - 1) / p.replay_chunks;
+  const long long grid = (long long)p.B * nseq * ((p.C + TH - 1) / TH);
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  PdlConfig cb(dim3((unsigned)grid), dim3(32), smem, st);
+  PdlConfig cb(dim3((unsigned)grid), dim3(TH), smem, st);
   if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv))) return WKV_ERR_CUDA;
   return launch_result();
 }
@@ -416,24 +426,40 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   int seg = pl.scan_segments;
   if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 64 ? 4 : (ntot <= 256 ? 16 : 64));
   const unsigned gs = (unsigned)(BNG * 4);  // 16 channels per CTA
+  PdlConfig cs(dim3(gs), dim3(16 * seg), 0, st);
+  cudaError_t e;
   switch (seg) {
-    case 1: wkv_tile_scan<1><<<gs, 16 * 1, 0, st>>>(p, L); break;
-    case 4: wkv_tile_scan<4><<<gs, 16 * 4, 0, st>>>(p, L); break;
-    case 16: wkv_tile_scan<16><<<gs, 16 * 16, 0, st>>>(p, L); break;
-    default: wkv_tile_scan<64><<<gs, 16 * 64, 0, st>>>(p, L); break;
+    case 1: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<1>, p, L); break;
+    case 4: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<4>, p, L); break;
+    case 16: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<16>, p, L); break;
+    default: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<64>, p, L); break;
   }
-  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  if (!cuda_ok(e) || launch_result() != WKV_OK) return WKV_ERR_CUDA;
   // B: the sequential kernel over every (batch row, chunk, 32-channel group),
   // from the chunk's incoming state; one channel per thread
   constexpr bool kF32 = sizeof(KV) == 4;
   constexpr int LT = kF32 ? 2 * kSeqLtF32 : 2 * kSeqLtBf16;
+  // one channel per thread, replay_threads channels per CTA
+  const int th = pl.replay_threads;
   CUtensorMap bk, bv;
-  if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, 32) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, 32))
+  if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, th) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, th))
     return WKV_ERR_CUDA;
-  // a chunk of at most two stages is prefetched whole with 2 (more CTAs fit
-  // per SM); longer chunks stream through 3
-  if (L <= 2 * LT) return launch_seq_chunks<KV, OUT, LT, 2>(p, bk, bv, st, dev);
-  return launch_seq_chunks<KV, OUT, LT, 3>(p, bk, bv, st, dev);
+  // a replay of at most two stages is prefetched whole with 2 (more CTAs fit
+  // per SM); longer ones stream through 3
+  FwdParams q = p;
+  q.replay_chunks = pl.replay_chunks;
+  const bool two = pl.replay_chunks * L <= 2 * LT;
+  switch (th) {
+    case 64:
+      return two ? launch_seq_chunks<KV, OUT, 64, LT, 2>(q, bk, bv, st, dev)
+                 : launch_seq_chunks<KV, OUT, 64, LT, 3>(q, bk, bv, st, dev);
+    case 128:
+      return two ? launch_seq_chunks<KV, OUT, 128, LT, 2>(q, bk, bv, st, dev)
+                 : launch_seq_chunks<KV, OUT, 128, LT, 3>(q, bk, bv, st, dev);
+    default:
+      return two ? launch_seq_chunks<KV, OUT, 32, LT, 2>(q, bk, bv, st, dev)
+                 : launch_seq_chunks<KV, OUT, 32, LT, 3>(q, bk, bv, st, dev);
+  }
 }
 
 template <typename KV, typename OUT>

@@ -77,6 +77,7 @@ struct FwdParams {
   float4* x0;          // incoming states of chunks (three-launch scan)
   int chunk_len;       // chunked scans: tokens per chunk
   int stages;          // pipelined chunk scan: shared-memory stages in the ring
+  int replay_chunks;   // three-launch scan: consecutive chunks per replay CTA
 };
 
 // Programmatic dependent launch: let the next launch on the stream be
@@ -121,12 +122,13 @@ __device__ __forceinline__ void coop_load_tile(KV* dst, const KV* src, int b, in
 // ---------------------------------------------------------------------------
 // sequential-over-T kernel
 // ---------------------------------------------------------------------------
-// kChunked: the replay pass of the three-launch scan. A CTA then takes one
-// chunk (p.chunk_len tokens) of one batch row and starts from the chunk's
-// incoming state, which the scan pass wrote to p.x0 ([nch][B * NG][64] with
-// p.NG 64-channel groups); the grid is B * nch * ceil(C / CG). It issues its
-// first copies (inputs only) before waiting (griddepcontrol.wait) for the
-// scan, and only the last chunk writes the state out.
+// kChunked: the replay pass of the three-launch scan. A CTA then takes
+// R = p.replay_chunks consecutive chunks (R * p.chunk_len tokens) of one batch
+// row and starts from the incoming state of the first, which the scan pass
+// wrote to p.x0 ([nch][B * NG][64] with p.NG 64-channel groups); the grid is
+// B * ceil(nch / R) * ceil(C / CG). It issues its first copies (inputs only)
+// before waiting (griddepcontrol.wait) for the scan, and only the CTA that
+// ends the sequence writes the state out.
 template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA, bool kChunked>
 __global__ void __launch_bounds__(THREADS)
     wkv_fwd_seq(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
@@ -142,10 +144,12 @@ __global__ void __launch_bounds__(THREADS)
   const int ngs = kChunked ? (C + CG - 1) / CG : p.NG;  // channel groups of this kernel
   const int bj = blockIdx.x / ngs;
   const int g = blockIdx.x % ngs;
-  const int b = kChunked ? bj / p.nch : bj;
-  const int jc = kChunked ? bj % p.nch : 0;  // chunk
+  const int nseq = kChunked ? (p.nch + p.replay_chunks - 1) / p.replay_chunks : 1;  // replays per row
+  const int b = kChunked ? bj / nseq : bj;
+  const int js = kChunked ? bj % nseq : 0;  // replay
+  const int jc = js * (kChunked ? p.replay_chunks : 1);  // its first chunk
   const int tbeg = kChunked ? jc * p.chunk_len : 0;
-  const int tend = kChunked ? min(T, tbeg + p.chunk_len) : T;
+  const int tend = kChunked ? min(T, tbeg + p.replay_chunks * p.chunk_len) : T;
   const int c0 = g * CG + tid * VEC;
   const int ntile = (tend - tbeg + LT - 1) / LT;
 
@@ -275,7 +279,7 @@ __global__ void __launch_bounds__(THREADS)
     return;
   }
 
-  if (p.o_num && c0 < C && (!kChunked || jc == p.nch - 1)) {
+  if (p.o_num && c0 < C && (!kChunked || js == nseq - 1)) {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       const int c = c0 + e;
@@ -737,6 +741,7 @@ __global__ void __launch_bounds__(NW * 32)
     tma_load_3d(ktile, &tmk, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
     tma_load_3d(ktile + kTile, &tmv, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
   }
+  grid_launch_dependents();  // the scan may be scheduled (it waits for this grid)
   __syncthreads();
   float w[VEC];
 #pragma unroll
@@ -774,9 +779,11 @@ __global__ void __launch_bounds__(NW * 32)
 // segment's total; (2) one thread per channel walks the segment totals once,
 // from the state in, leaving each segment's incoming state in shared memory;
 // (3) each thread walks its segment again, writing each chunk's incoming
-// state to p.x0 [nch][B * NG][64] (and the last chunk's). The totals were
-// written by the previous launch and are read-only here, so they are loaded
-// through the non-coherent path, eight at a time.
+// state to p.x0 [nch][B * NG][64] (and the last chunk's). Launched with
+// programmatic stream serialization: it waits (griddepcontrol.wait) for the
+// totals pass before its first load. The totals are read-only from then on,
+// so they are loaded through the non-coherent path, eight at a time; a
+// segment of at most eight is loaded once and kept in registers.
 template <int SEG>
 __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int L) {
   constexpr int CG = 64, CH = 16;
@@ -793,16 +800,31 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   const int per = (ntot + SEG - 1) / SEG;
   const int q0 = min(ntot, sg * per), q1 = min(ntot, q0 + per);
   const float fL = (float)L;
-  // 1. this segment's total
+  const float4* tot_of = p.agg_a + (size_t)bg * CG + cl;  // chunk q's total at tot_of[q * BNG * CG]
+  const size_t qs = (size_t)BNG * CG;
+  grid_wait_prerequisites();  // the totals pass has finished
+  // 1. this segment's total; a segment of at most 8 totals stays in registers
+  // for step 3
+  const bool cached = q1 - q0 <= 8;
+  float4 a0[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (cached && q0 + r < q1) a0[r] = ldg_f4(tot_of + (q0 + r) * qs);
   Acc tot = acc_empty();
-  for (int qq = q0; qq < q1; qq += 8) {
-    float4 a[8];
+  if (cached) {
 #pragma unroll
     for (int r = 0; r < 8; ++r)
-      if (qq + r < q1) a[r] = ldg_f4(p.agg_a + ((size_t)(qq + r) * BNG + bg) * CG + cl);
+      if (q0 + r < q1) tot = combine(tot, acc_unpack(a0[r]), fL, w);
+  } else {
+    for (int qq = q0; qq < q1; qq += 8) {
+      float4 a[8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), fL, w);
+      for (int r = 0; r < 8; ++r)
+        if (qq + r < q1) a[r] = ldg_f4(tot_of + (qq + r) * qs);
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), fL, w);
+    }
   }
   seg_st[sg][ch] = acc_pack(tot);
   __syncthreads();
@@ -819,20 +841,31 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   __syncthreads();
   // 3. incoming state of every chunk of the segment (and of the last chunk)
   Acc x = acc_unpack(seg_st[sg][ch]);
-  for (int qq = q0; qq < q1; qq += 8) {
-    float4 a[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (qq + r < q1) a[r] = ldg_f4(p.agg_a + ((size_t)(qq + r) * BNG + bg) * CG + cl);
+  float4* x0_of = p.x0 + (size_t)bg * CG + cl;
+  if (cached) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      if (qq + r < q1) {
-        p.x0[((size_t)(qq + r) * BNG + bg) * CG + cl] = acc_pack(x);
-        x = combine(x, acc_unpack(a[r]), fL, w);
+      if (q0 + r < q1) {
+        x0_of[(q0 + r) * qs] = acc_pack(x);
+        x = combine(x, acc_unpack(a0[r]), fL, w);
+      }
+    }
+  } else {
+    for (int qq = q0; qq < q1; qq += 8) {
+      float4 a[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (qq + r < q1) a[r] = ldg_f4(tot_of + (qq + r) * qs);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (qq + r < q1) {
+          x0_of[(qq + r) * qs] = acc_pack(x);
+          x = combine(x, acc_unpack(a[r]), fL, w);
+        }
       }
     }
   }
-  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.x0[((size_t)ntot * BNG + bg) * CG + cl] = acc_pack(x);
+  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) x0_of[ntot * qs] = acc_pack(x);
 }
 
 // ---------------------------------------------------------------------------
