@@ -171,10 +171,11 @@ def measured_peaks():
 
 
 def source_digest() -> str:
-    """Hash of the device code (the kernels); host-side dispatch is not included,
-    the launch configuration is recorded next to each capture instead."""
+    """Hash of the kernels and of the code that chooses and launches them (tile
+    shapes, stages and grids change the traffic a capture records)."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "wkv_recurrence_b200", "csrc", "*.cuh"))):
+    csrc = os.path.join(ROOT, "wkv_recurrence_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.cu"))):
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
@@ -182,17 +183,19 @@ def source_digest() -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded by an ncu capture under profiles/, if it
-    was taken on the current kernel sources (else None)."""
+    """(DRAM bytes per launch, XU pipe use in % of its peak or None) recorded
+    by an ncu capture under profiles/, if it was taken on the current kernel
+    sources (else (None, None)). The XU pipe (ex2, rcp) is the path's second
+    ceiling after HBM."""
     digest = source_digest()
     for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         with open(p) as f:
             for line in f:
-                m = re.match(r"traffic:\s*kernel=(\S+)\s+workload=(\S+)\s+source=(\S+)\s+bytes_per_launch=(\d+)",
-                             line.strip())
+                m = re.match(r"traffic:\s*kernel=(\S+)\s+workload=(\S+)\s+source=(\S+)\s+bytes_per_launch=(\d+)"
+                             r"(?:\s+xu_pct=([0-9.]+))?", line.strip())
                 if m and m.group(1) == kernel and m.group(2) == workload and m.group(3) == digest:
-                    return int(m.group(4))
-    return None
+                    return int(m.group(4)), (float(m.group(5)) if m.group(5) else None)
+    return None, None
 
 
 class L2Flusher:
@@ -399,7 +402,7 @@ def run_ours(args):
     algo = forward_bytes(wl)
     achieved = algo / (fwd_mean_ms / 1e3) / 1e9
     kernel_name = forward_kernel_name(wl, options)
-    traffic = recorded_traffic(kernel_name, wl.name)
+    traffic, xu_pct = recorded_traffic(kernel_name, wl.name)
 
     # the same forward timed alone after an L2 flush (launch latency included)
     cold = []
@@ -475,7 +478,7 @@ def run_ours(args):
                        "options": options or "auto"},
             "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic, "algorithmic_bytes": algo,
+                         "traffic": traffic, "xu_pipe_pct_of_peak": xu_pct, "algorithmic_bytes": algo,
                          "launch_ms": fwd_mean_ms},
             "decode_step_ms": dec_total_ms / K_steps,
             "forward_ms": {"back_to_back": fwd_total_ms / K_steps, "cold_after_l2_flush": cold_ms},

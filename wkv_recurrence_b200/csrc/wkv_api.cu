@@ -449,6 +449,14 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   FwdParams q = p;
   q.replay_chunks = pl.replay_chunks;
   const bool two = pl.replay_chunks * L <= 2 * LT;
+  if (kF32 && pl.replay_chunks * L == 32 && th == 32) {
+    // a 32-token fp32 replay as one 32-token stage: one copy pair and one
+    // wait instead of two (layer: 23.5 against 23.8 us)
+    CUtensorMap ck, cv;
+    if (!make_tmap(&ck, p.k, kvdt, p.B, p.T, p.C, 32, th) || !make_tmap(&cv, p.v, kvdt, p.B, p.T, p.C, 32, th))
+      return WKV_ERR_CUDA;
+    return launch_seq_chunks<KV, OUT, 32, 32, 1>(q, ck, cv, st, dev);
+  }
   switch (th) {
     case 64:
       return two ? launch_seq_chunks<KV, OUT, 64, LT, 2>(q, bk, bv, st, dev)
