@@ -290,6 +290,33 @@ def test_kernels_agree_and_are_deterministic(oracle):
         assert np.all(np.abs(a1 - r1) <= 2 * RTOL_F32 * sc), opts
 
 
+@pytest.mark.parametrize("T", [1000, 20], ids=["many_chunks", "one_chunk"])
+def test_back_to_back_calls_see_previous_results(T):
+    """Calls queued with no synchronisation, each taking the previous call's
+    output as its k and its state as the state in: the launches that may
+    start before the one ahead of them ends (programmatic serialization) must
+    still see its results. Bitwise equal to the same calls synchronised."""
+    B, C = 2, 128
+    k, v, w, u, st = I.random_case(B, T, C, seed=53, state=True)
+    K, V, Wt, U = dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u)
+    S0 = tuple(dev_f32(s) for s in st)
+    o1, s1 = W.forward(K, V, Wt, U, S0, options=TWO)
+    torch.cuda.synchronize()
+    o2, s2 = W.forward(o1.clone(), V, Wt, U, tuple(x.clone() for x in s1), options=TWO)
+    torch.cuda.synchronize()
+    for _ in range(10):
+        c1, cs1 = W.forward(K, V, Wt, U, S0, options=TWO)
+        c2, cs2 = W.forward(c1, V, Wt, U, cs1, options=TWO)
+        c3, _ = W.forward(c2, V, Wt, U, cs2, options=TWO)
+    torch.cuda.synchronize()
+    assert torch.equal(c2, o2)
+    for a, b in zip(cs2, s2):
+        assert torch.equal(a, b)
+    o3, _ = W.forward(o2, V, Wt, U, s2, options=TWO)
+    torch.cuda.synchronize()
+    assert torch.equal(c3, o3)
+
+
 @pytest.mark.parametrize("opts", [CHUNK, TWO, PIPE], ids=["chunk", "two", "pipe"])
 def test_workspace_reuse_across_shapes(oracle, opts):
     """One workspace serves successive calls of different shapes (the epoch scheme)."""

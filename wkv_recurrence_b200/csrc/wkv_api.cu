@@ -426,7 +426,11 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   int seg = pl.scan_segments;
   if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 64 ? 4 : (ntot <= 256 ? 16 : 64));
   const unsigned gs = (unsigned)(BNG * 4);  // 16 channels per CTA
+  // programmatic serialization only behind A (an ordinary launch, so S is
+  // scheduled only after the launch ahead of the call has ended: S reads w
+  // before its own wait)
   PdlConfig cs(dim3(gs), dim3(16 * seg), 0, st);
+  if (p.nch <= 1) cs.cfg.numAttrs = 0;
   cudaError_t e;
   switch (seg) {
     case 1: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<1>, p, L); break;

@@ -696,14 +696,20 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 //     it, as a two-level scan (segments of chunks, then within segments);
 //   B (wkv_fwd_seq in chunked mode): every (batch row, chunk) is replayed as
 //     an independent sequence of chunk_len tokens from its incoming state, one
-//     channel per thread, streaming k and v again (TMA ring, 3 stages).
+//     channel per thread, streaming k and v again through TMA stages.
 // k and v are read twice from memory: for inputs that fit in L2 the second
-// read hits L2. B is launched with programmatic stream serialization: its
-// CTAs issue their first copies (inputs only) while S runs and wait
-// (griddepcontrol.wait) before reading an incoming state. Only S reads the
+// read hits L2. A is an ordinary launch; S (behind A) and B are launched with
+// programmatic stream serialization, so that each may be resident before the
+// one ahead of it ends:
+//   A lets S be scheduled once its copies are issued;
+//   S reads w, then waits (griddepcontrol.wait) for A before its first total;
+//   B issues its first copies (inputs only) while S runs and waits for S
+//     before reading an incoming state.
+// Both are scheduled only after A has started, so every read of the call's
+// inputs follows the end of the launch ahead of the call. Only S reads the
 // caller's state in, and it completes before B writes the state out (from
-// the last chunk), so the two may alias. The order of combines depends on
-// the shape only.
+// the last chunk), so the two may alias. The order of combines depends on the
+// shape only.
 
 __device__ __forceinline__ float4 ldg_f4(const float4* q) {
   float4 r;
@@ -779,9 +785,9 @@ __global__ void __launch_bounds__(NW * 32)
 // segment's total; (2) one thread per channel walks the segment totals once,
 // from the state in, leaving each segment's incoming state in shared memory;
 // (3) each thread walks its segment again, writing each chunk's incoming
-// state to p.x0 [nch][B * NG][64] (and the last chunk's). Launched with
-// programmatic stream serialization: it waits (griddepcontrol.wait) for the
-// totals pass before its first load. The totals are read-only from then on,
+// state to p.x0 [nch][B * NG][64] (and the last chunk's). Behind the totals
+// pass it is launched with programmatic stream serialization and waits
+// (griddepcontrol.wait) for that pass before its first load of a total. The totals are read-only from then on,
 // so they are loaded through the non-coherent path, eight at a time; a
 // segment of at most eight is loaded once and kept in registers.
 template <int SEG>
