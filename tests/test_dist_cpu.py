@@ -81,3 +81,28 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run_bench(["--impl", "reference", "--workload", "small", "--steps", "3"],
                    {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_recorded_traffic_follows_the_sources(tmp_path, monkeypatch):
+    """A profile's traffic line counts only while the kernels and their launch
+    code hash to the digest it names; the XU figure is optional."""
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "wkv_recurrence_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cuh").write_text("kernel one")
+    (csrc / "api.cu").write_text("launch one")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d = bench.source_digest()
+    (tmp_path / "profiles" / "a.md").write_text(
+        f"traffic: kernel=kx workload=layer source={d} bytes_per_launch=123 xu_pct=21.5\n"
+        f"traffic: kernel=ky workload=layer source={d} bytes_per_launch=456\n"
+        "traffic: kernel=kz workload=layer source=0000000000000000 bytes_per_launch=789\n")
+    assert bench.recorded_traffic("kx", "layer") == (123, 21.5)
+    assert bench.recorded_traffic("ky", "layer") == (456, None)
+    assert bench.recorded_traffic("kz", "layer") == (None, None)  # another build's capture
+    assert bench.recorded_traffic("kx", "long") == (None, None)
+    (csrc / "api.cu").write_text("launch two")  # launch code changed: the capture no longer counts
+    assert bench.source_digest() != d
+    assert bench.recorded_traffic("kx", "layer") == (None, None)
