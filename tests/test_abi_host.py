@@ -33,6 +33,39 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def test_binding_structs_match_the_header(tmp_path):
+    """The ctypes structs of the binding have the header's fields, sizes and
+    offsets (compiled against include/wkv.h with the host C compiler)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    structs = {"wkv_options": _abi.wkv_options, "wkv_cstate": _abi.wkv_cstate, "wkv_state": _abi.wkv_state}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "wkv.h"', "int main(void) {"]
+    for name, ct in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for field, _ in ct._fields_:
+            lines.append(f'  printf("{name} {field} %zu\\n", offsetof({name}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    want = []
+    for name, ct in structs.items():
+        want.append(f"{name} size {ctypes.sizeof(ct)}")
+        for field, _ in ct._fields_:
+            want.append(f"{name} {field} {getattr(ct, field).offset}")
+    assert [g for g in got if g] == want
+    # and the header has no field the binding lacks
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct \{([^}]*)\} wkv_options;", text).group(1)
+    header_fields = re.findall(r"\b(\w+);", body)
+    assert header_fields == [f for f, _ in _abi.wkv_options._fields_]
+
+
 def test_status_strings(L):
     for code in range(7):
         s = _abi.status_string(code)
