@@ -8,7 +8,14 @@ the B streams from the returned state. Metric: WKV channel-steps per second
 (B*T*C + B*C per step), and the forward kernel's achieved HBM bandwidth against
 the measured B200 copy bandwidth.
 
-    python bench.py [--gpus N --steps K --warmup W] [--workload layer]
+The headline workload is `long` (B=1, T=65536, C=2048 fp32, 1.6 GB per
+forward), the largest single-GPU configuration. At N=1 the same JSON line also
+carries one sub-record per other workload ("workloads": layer 8x1024x768 fp32,
+mixed 16x4096x4096 bf16, the 256-step batched decode of 4096 streams x 768,
+small 1x64x768), each with its own throughput, roofline fraction, clocks and
+CPU-oracle baseline.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload long]
     python -m torch.distributed.run --nproc-per-node N bench.py --gpus N ...
     python bench.py --impl reference ...     # the float64 CPU oracle, timed
 
@@ -109,13 +116,18 @@ def workload_desc(wl):
             f"{' (state in)' if wl.state != 'zero' else ''} + 1 wkv_step decode token")
 
 
-def workload(args):
+def decode_desc(wl):
+    return (f"batched decode: wkv_step over {wl.B} streams x C={wl.C} fp32, state from a {wl.T}-token "
+            f"prefix (wkv_forward), {wl.decode_steps} steps with fresh k, v")
+
+
+def workload(args, name=None):
     """The named workload, with B and/or T overridden for profiling runs."""
     import dataclasses
 
     from wkv_recurrence_b200 import inputs as I
-    wl = I.WORKLOADS[args.workload]
-    if args.batch or args.tokens:
+    wl = I.WORKLOADS[name or args.workload]
+    if name is None and (args.batch or args.tokens):
         wl = dataclasses.replace(wl, B=args.batch or wl.B, T=args.tokens or wl.T)
     return wl
 
@@ -152,12 +164,12 @@ def forward_kernel_name(wl, options) -> str:
 
 
 def launches_per_step(wl, options) -> int:
-    """Kernel launches of one step: the forward (1; for the three-launch scan
-    3, or 2 when the sequence is a single chunk) and one decode launch."""
-    if not forward_kernel_name(wl, options).startswith("wkv_tile"):
-        return 2
-    chunk = (options or {}).get("chunk_len", 0) or 128
-    return (3 if wl.T > chunk else 2) + 1
+    """Kernel launches of one step: the forward's (as the library reports them
+    for this shape and options) and one decode launch."""
+    import torch
+    import wkv_recurrence_b200 as W
+    kv = torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32
+    return W.forward_launches(wl.B, wl.T, wl.C, kv, options) + 1
 
 
 def measured_peaks():
@@ -284,118 +296,113 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args):
+def _to_dev(x, device, as_bf16=False):
+    import numpy as np
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x.view(np.int16) if as_bf16 else x)).to(device)
+    return t.view(torch.bfloat16) if as_bf16 else t
+
+
+def _timed_graph(g, n_rep, stream, device):
+    """Milliseconds of n_rep back-to-back replays of graph g, by CUDA events on
+    `stream`, bracketed by a barrier and a synchronize on both sides."""
+    import torch
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_rep):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return e0.elapsed_time(e1)
+
+
+def _capture(items, body, stream, device):
+    """A CUDA graph of body(item, stream handle) for every item, captured on a
+    side stream."""
+    import torch
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        h = ctypes.c_void_p(side.cuda_stream)
+        with torch.cuda.graph(g, stream=side):
+            for it in items:
+                body(it, h)
+    stream.wait_stream(side)
+    torch.cuda.synchronize(device)
+    return g
+
+
+def measure_forward(wl, args, options, device, rank, world, headline):
+    """Throughput of the step (forward + one decode token) on workload wl, the
+    forward's roofline, and (headline only) the end-to-end number through the
+    public API. Returns the record (a dict) on every rank."""
     import numpy as np
     import torch
 
     import wkv_recurrence_b200 as W
     from wkv_recurrence_b200 import inputs as I
 
-    rank, local_rank, world = dist_env()
-    torch.cuda.set_device(local_rank)
-    device = torch.device("cuda", local_rank)
-    if world > 1:
-        dist_init("nccl")
-    wl = workload(args)
-    options = json.loads(args.options) if args.options else None
-
-    # synthetic inputs, one batch per rank
     k, v = I.draw_kv(wl, seed=rank)
     w, u = I.draw_w(wl, seed=0), I.draw_u(wl, seed=0)
     st = I.draw_state(wl, seed=rank)
     k1, v1 = I.draw_decode_token(wl, 0, seed=rank)
     bf16 = wl.kv_dtype == "bf16"
-
-    def to_dev(x, as_bf16=False):
-        t = torch.from_numpy(np.ascontiguousarray(x.view(np.int16) if as_bf16 else x))
-        t = t.to(device)
-        return t.view(torch.bfloat16) if as_bf16 else t
-
     out_dtype = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
-    Wt, U = to_dev(w), to_dev(u)
-    S_in = None if st is None else tuple(to_dev(s) for s in st)
+    Wt, U = _to_dev(w, device), _to_dev(u, device)
+    S_in = None if st is None else tuple(_to_dev(s, device) for s in st)
     # R independent buffer sets (inputs, outputs, states), used in turn, so
     # that a step never finds its inputs in L2: R sets together exceed 2.5x L2
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     set_bytes = forward_bytes(wl) + step_bytes(wl)
     R = int(min(8, max(2, -(-int(2.5 * l2) // set_bytes))))
     sets = []
-    for r in range(R):
-        K, V = to_dev(k, bf16), to_dev(v, bf16)
-        K1, V1 = to_dev(k1), to_dev(v1)
-        out = torch.empty(wl.B, wl.T, wl.C, dtype=out_dtype, device=device)
-        state = tuple(torch.empty(wl.B, wl.C, device=device) for _ in range(3))
-        out1 = torch.empty(wl.B, wl.C, device=device)
-        sets.append(dict(K=K, V=V, K1=K1, V1=V1, out=out, state=state, out1=out1))
+    for _ in range(R):
+        d = dict(K=_to_dev(k, device, bf16), V=_to_dev(v, device, bf16), K1=_to_dev(k1, device),
+                 V1=_to_dev(v1, device), out=torch.empty(wl.B, wl.T, wl.C, dtype=out_dtype, device=device),
+                 state=tuple(torch.empty(wl.B, wl.C, device=device) for _ in range(3)),
+                 out1=torch.empty(wl.B, wl.C, device=device))
+        sets.append(d)
     ws = W.make_workspace(wl.B, wl.T, wl.C, options=options, device=device)
-    flusher = L2Flusher(l2, device)
     stream = torch.cuda.current_stream(device)
     # arguments checked and marshalled once; each call below is one C-ABI call
     for d in sets:
         d["fwd"] = W.PreparedForward(d["K"], d["V"], Wt, U, S_in, out=d["out"], state_out=d["state"],
                                      workspace=ws, options=options)
         d["dec"] = W.PreparedStep(d["state"], d["K1"], d["V1"], Wt, U, out=d["out1"])
-    K, V, K1, V1, out, out1, state = (sets[0][x] for x in ("K", "V", "K1", "V1", "out", "out1", "state"))
 
     def one_step(d=sets[0], strm=None):
         d["fwd"](strm)
         d["dec"](strm)
 
-    for i in range(max(3, args.warmup)):
+    warm = max(3, args.warmup)
+    for i in range(warm):
         one_step(sets[i % R])
     torch.cuda.synchronize(device)
     if W.query_status(ws) != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
-
-    # CUDA graphs of R steps (one per buffer set), of R forwards, of R decodes
-    def capture(body):
-        side = torch.cuda.Stream(device)
-        side.wait_stream(stream)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(side):
-            h = ctypes.c_void_p(side.cuda_stream)
-            with torch.cuda.graph(g, stream=side):
-                for d in sets:
-                    body(d, h)
-        stream.wait_stream(side)
-        torch.cuda.synchronize(device)
-        return g
-
-    g_step = capture(lambda d, h: one_step(d, h))
-    g_fwd = capture(lambda d, h: d["fwd"](h))
-    g_dec = capture(lambda d, h: d["dec"](h))
-    for g in (g_step, g_fwd, g_dec):
+    g_step = _capture(sets, lambda d, h: one_step(d, h), stream, device)
+    g_fwd = _capture(sets, lambda d, h: d["fwd"](h), stream, device)
+    for g in (g_step, g_fwd):
         g.replay()
     torch.cuda.synchronize(device)
-
     n_rep = max(1, -(-args.steps // R))
     K_steps = n_rep * R
 
-    def timed(g):
-        barrier(device)
-        torch.cuda.synchronize(device)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_rep):
-            g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(device)
-        return e0.elapsed_time(e1)
-
-    sampler = ClockSampler(local_rank) if not args.no_clocks else None
+    sampler = ClockSampler(torch.cuda.current_device()) if not args.no_clocks else None
     if sampler:
         sampler.start()
     t_wall0 = time.perf_counter()
-    total_ms = timed(g_step)
+    total_ms = _timed_graph(g_step, n_rep, stream, device)
     t_wall = time.perf_counter() - t_wall0
-    fwd_total_ms = timed(g_fwd)
-    dec_total_ms = timed(g_dec)
+    fwd_total_ms = _timed_graph(g_fwd, n_rep, stream, device)
     clocks = sampler.stop() if sampler else None
     if W.query_status(ws) != 0:
         raise RuntimeError("device-side wait timed out during the timed steps")
-
     value, total_ms_max = throughput(units_per_step(wl), K_steps, total_ms, device)
 
     # roofline of the dominant kernel (the forward launch), back to back
@@ -407,8 +414,9 @@ def run_ours(args):
     traffic, xu_pct = recorded_traffic(kernel_name, wl.name)
 
     # the same forward timed alone after an L2 flush (launch latency included)
+    flusher = L2Flusher(l2, device)
     cold = []
-    for i in range(20):
+    for i in range(10):
         flusher()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -418,10 +426,12 @@ def run_ours(args):
         cold.append((e0, e1))
     torch.cuda.synchronize(device)
     cold_ms = statistics.median(a.elapsed_time(b) for a, b in cold)
+    del flusher
 
     # end to end through the public API: pinned host -> device, compute, device -> host
     e2e = None
-    if not args.no_e2e:
+    if headline and not args.no_e2e:
+        K, V, K1, V1, out, out1, state = (sets[0][x] for x in ("K", "V", "K1", "V1", "out", "out1", "state"))
         pin = lambda x: torch.from_numpy(np.ascontiguousarray(x)).pin_memory()  # noqa: E731
         hk = pin(k.view(np.int16) if bf16 else k)
         hv = pin(v.view(np.int16) if bf16 else v)
@@ -439,8 +449,8 @@ def run_ours(args):
             one_step()
             hout.copy_(out, non_blocking=True)
             hout1.copy_(out1, non_blocking=True)
-            for h, s in zip(hst, state):
-                h.copy_(s, non_blocking=True)
+            for hh, s in zip(hst, state):
+                hh.copy_(s, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -461,31 +471,150 @@ def run_ours(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
                "ms_per_step": e2e_ms / n_e2e}
 
-    cpu = None
+    rec = {
+        "workload": workload_desc(wl), "name": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+        "kv_dtype": wl.kv_dtype, "out_dtype": wl.out_dtype,
+        "value": value, "unit": UNIT, "steps": K_steps, "warmup": warm, "ms_per_step": total_ms_max / K_steps,
+        "forward_value": wl.B * wl.T * wl.C / (fwd_mean_ms / 1e3) * world,
+        "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "xu_pipe_pct_of_peak": xu_pct, "algorithmic_bytes": algo,
+                     "launch_ms": fwd_mean_ms},
+        "forward_ms": {"back_to_back": fwd_total_ms / K_steps, "cold_after_l2_flush": cold_ms},
+        "gpu_launches": launches_per_step(wl, options) * K_steps,
+        "clocks": clocks, "wall_s_timed_region": t_wall, "buffer_sets": R,
+        "l2": (f"inputs larger than L2: steps rotate over {R} separate buffer sets "
+               f"({R * set_bytes / 2**20:.0f} MiB in total, L2 is {l2 / 2**20:.0f} MiB), so every step reads "
+               "inputs that are not in L2; steps run back to back from a CUDA graph"),
+        "e2e": e2e,
+    }
+    del sets, ws, g_step, g_fwd
+    torch.cuda.empty_cache()
+    return rec
+
+
+def measure_decode(wl, args, device):
+    """The batched decode workload: the per-step time of wkv_step over
+    S streams x C channels, with the state of every stream built by a T-token
+    prefix through wkv_forward. Steps rotate over 4 independent sets of stream
+    states, and the k, v of each step are one of the workload's drawn decode
+    steps, so that neither a step's state nor its tokens are still in L2 from
+    an earlier launch. N=1 only."""
+    import torch
+
+    import wkv_recurrence_b200 as W
+    from wkv_recurrence_b200 import inputs as I
+
+    S, C = wl.B, wl.C
+    w, u = I.draw_w(wl), I.draw_u(wl)
+    Wt, U = _to_dev(w, device), _to_dev(u, device)
+    # the prefix, in slices of streams to bound host memory
+    base = tuple(torch.empty(S, C, device=device) for _ in range(3))
+    slab = 512
+    for s0 in range(0, S, slab):
+        kp, vp = I.draw_kv_rows(wl, range(s0, min(S, s0 + slab)))
+        W.forward(_to_dev(kp, device), _to_dev(vp, device), Wt, U,
+                  state_out=tuple(x[s0:s0 + slab] for x in base))
+        torch.cuda.synchronize(device)
+        del kp, vp
+    n_tok = wl.decode_steps
+    toks = []
+    for j in range(n_tok):
+        kd, vd = I.draw_decode_token(wl, j)
+        toks.append((_to_dev(kd, device), _to_dev(vd, device)))
+    R = 4
+    sets = [tuple(x.clone() for x in base) for _ in range(R)]
+    out = [torch.empty(S, C, device=device) for _ in range(R)]
+    stream = torch.cuda.current_stream(device)
+    # launch n = (step j of set r, n = R*j + r) takes token buffer n mod n_tok:
+    # each set takes fresh tokens every step, and a token buffer is read again
+    # only n_tok launches later
+    calls = []
+    for j in range(n_tok):
+        for r in range(R):
+            kd, vd = toks[(R * j + r) % n_tok]
+            calls.append(W.PreparedStep(sets[r], kd, vd, Wt, U, out=out[r]))
+    for c in calls[:max(3, args.warmup)]:
+        c()
+    torch.cuda.synchronize(device)
+    g = _capture(calls, lambda c, h: c(h), stream, device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    n_rep = max(1, -(-args.steps // len(calls)))
+    sampler = ClockSampler(torch.cuda.current_device()) if not args.no_clocks else None
+    if sampler:
+        sampler.start()
+    ms = _timed_graph(g, n_rep, stream, device)
+    clocks = sampler.stop() if sampler else None
+    launches = n_rep * len(calls)
+    step_ms = ms / launches
+    peak, peak_kind = measured_peaks()
+    algo = step_bytes(wl)
+    achieved = algo / (step_ms / 1e3) / 1e9
+    traffic, xu_pct = recorded_traffic("wkv_step_kernel", "decode")
+    rec = {
+        "workload": decode_desc(wl), "name": "decode", "S": S, "C": C, "prefix_T": wl.T, "steps_per_stream": n_tok,
+        "value": S * C / (step_ms / 1e3), "unit": UNIT, "steps": launches, "ms_per_step": step_ms,
+        "roofline": {"bound": "hbm", "kernel": "wkv_step_kernel", "achieved": achieved, "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "xu_pipe_pct_of_peak": xu_pct, "algorithmic_bytes": algo, "launch_ms": step_ms},
+        "gpu_launches": launches, "clocks": clocks,
+        "l2": (f"{R} independent sets of stream states are stepped in turn and the k, v of each launch are one "
+               f"of {n_tok} drawn decode steps ({n_tok * 2 * S * C * 4 / 2**30:.1f} GiB), so a launch reads "
+               "state and tokens last touched at least 3 launches (340 MB of traffic) earlier; launches run "
+               "back to back from a CUDA graph"),
+    }
+    del g, calls, sets, toks, base
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args):
+    import torch
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist_init("nccl")
+    options = json.loads(args.options) if args.options else None
+    wl = workload(args)
+    main = measure_forward(wl, args, options, device, rank, world, headline=True)
+
+    subs = {}
+    if world == 1 and not args.no_sub:
+        for name in ("layer", "mixed", "decode", "small"):
+            if name == wl.name:
+                continue
+            swl = workload(args, name)
+            if name == "decode":
+                subs[name] = measure_decode(swl, args, device)
+            else:
+                subs[name] = measure_forward(swl, args, None, device, rank, world, headline=False)
+
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds)
+        main["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds, one_core_s=args.cpu_seconds / 2)
+        for name, rec in subs.items():
+            rec["cpu_baseline"] = cpu_baseline(workload(args, name), budget_s=args.cpu_seconds / 3,
+                                               one_core_s=args.cpu_seconds / 4, decode=(name == "decode"))
 
     if rank == 0:
+        bf16 = wl.kv_dtype == "bf16"
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
-            "warmup": max(3, args.warmup), "ms_per_step": total_ms_max / K_steps, "higher_is_better": True,
+            "metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": world, "steps": main["steps"],
+            "warmup": main["warmup"], "ms_per_step": main["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32" if not bf16 else "bf16-io/f32",
             "data": "synthetic (seeded numpy draws of the workload's distributions)",
-            "config": {"workload": workload_desc(wl), "name": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
+            "config": {"workload": main["workload"], "name": wl.name, "B": wl.B, "T": wl.T, "C": wl.C,
                        "kv_dtype": wl.kv_dtype, "out_dtype": wl.out_dtype, "global_batch": wl.B * world,
                        "seq_len": wl.T, "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": (f"inputs larger than L2: steps rotate over {R} separate buffer sets "
-                              f"({R * set_bytes / 2**20:.0f} MiB in total, L2 is {l2 / 2**20:.0f} MiB), so every "
-                              "step reads inputs that are not in L2; steps run back to back from a CUDA graph"),
-                       "options": options or "auto"},
-            "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
-                         "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic, "xu_pipe_pct_of_peak": xu_pct, "algorithmic_bytes": algo,
-                         "launch_ms": fwd_mean_ms},
-            "decode_step_ms": dec_total_ms / K_steps,
-            "forward_ms": {"back_to_back": fwd_total_ms / K_steps, "cold_after_l2_flush": cold_ms},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(wl, options) * K_steps,
-            "clocks": clocks, "wall_s_timed_region": t_wall, "buffer_sets": R,
+                       "l2": main["l2"], "options": options or "auto"},
+            "roofline": main["roofline"], "forward_ms": main["forward_ms"],
+            "forward_value": main["forward_value"],
+            "cpu_baseline": main.get("cpu_baseline"), "e2e": main["e2e"], "gpu_launches": main["gpu_launches"],
+            "clocks": main["clocks"], "wall_s_timed_region": main["wall_s_timed_region"],
+            "buffer_sets": main["buffer_sets"],
+            "workloads": subs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -496,6 +625,18 @@ def run_ours(args):
 # ---------------------------------------------------------------------------
 # the CPU oracle, timed (cpu_baseline leg, and the reference arm)
 # ---------------------------------------------------------------------------
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
 
 def _oracle_sample(wl, rows, cols, seed=0):
     from wkv_recurrence_b200 import inputs as I
@@ -509,9 +650,9 @@ def _oracle_sample(wl, rows, cols, seed=0):
     return k, v, w, u, st, k1[:, :cols].copy(), v1[:, :cols].copy()
 
 
-def _oracle_step(O, sample):
+def _oracle_step(O, sample, threads):
     k, v, w, u, st, k1, v1 = sample
-    _, s = O.recurrence_forward(k, v, w, u, st)
+    _, s = O.recurrence_forward(k, v, w, u, st, threads=threads)
     O.recurrence_step(s, k1, v1, w, u)
 
 
@@ -527,30 +668,67 @@ def _pick_sample(wl, max_units):
     return rows, cols
 
 
-def cpu_baseline(wl, budget_s=10.0):
-    from oracle import oracle as O
-    O.build()
-    # calibrate on a small slice, then size the sample to ~budget_s of CPU work
+def _set_oracle_threads(O, n):
+    """The oracle's OpenMP thread count for the calls that follow (a tiny
+    forward with an explicit count sets it for the process)."""
+    import numpy as np
+    z = np.zeros((1, 1, 1), np.float32)
+    O.recurrence_forward(z, z, np.zeros(1, np.float32), np.zeros(1, np.float32), threads=n)
+
+
+def _rate(O, wl, budget_s, threads, decode):
+    """Channel-steps per second of the oracle on a slice of wl sized to about
+    budget_s of CPU work with `threads` threads; and the slice's description."""
+    from wkv_recurrence_b200 import inputs as I
+    _set_oracle_threads(O, threads)
+    if decode:
+        # one decode step of every stream in a slice, from a state drawn by a short prefix
+        rows = min(wl.B, 64)
+        sample = _oracle_sample(wl, rows, wl.C)
+        _, st = O.recurrence_forward(sample[0][:, :16], sample[1][:, :16], sample[2], sample[3])
+        kd, vd = I.draw_decode_token(wl, 0, rows=range(rows))
+        reps = 0
+        t0 = time.perf_counter()
+        while True:
+            _, st = O.recurrence_step(st, kd, vd, sample[2], sample[3])
+            reps += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return rows * wl.C * reps / dt, (f"float64 C recurrence step on streams 0..{rows - 1} (all {wl.C} "
+                                         f"channels), {reps} decode steps, {dt:.1f} s")
     rows, cols = _pick_sample(wl, 2_000_000)
     sample = _oracle_sample(wl, rows, cols)
     t0 = time.perf_counter()
-    _oracle_step(O, sample)
-    dt = time.perf_counter() - t0
-    rate = rows * cols * (wl.T + 1) / max(dt, 1e-6)
-    rows, cols = _pick_sample(wl, int(rate * budget_s / 3))
+    _oracle_step(O, sample, threads)
+    rate = rows * cols * (wl.T + 1) / max(time.perf_counter() - t0, 1e-6)
+    rows, cols = _pick_sample(wl, max(2_000, int(rate * budget_s / 3)))
     sample = _oracle_sample(wl, rows, cols)
     reps = 0
     t0 = time.perf_counter()
     while True:
-        _oracle_step(O, sample)
+        _oracle_step(O, sample, threads)
         reps += 1
         if time.perf_counter() - t0 >= budget_s or reps >= 50:
             break
     dt = time.perf_counter() - t0
-    units = rows * cols * (wl.T + 1) * reps
-    return {"value": units / dt, "unit": UNIT, "cores": O.max_threads(), "kind": "oracle",
-            "sample": f"float64 C recurrence (OpenMP) on rows 0..{rows - 1}, channels 0..{cols - 1} of the "
-                      f"{wl.name} workload (T={wl.T}, plus one decode token), {reps} repetition(s), {dt:.1f} s"}
+    return (rows * cols * (wl.T + 1) * reps / dt,
+            f"float64 C recurrence on rows 0..{rows - 1}, channels 0..{cols - 1} of the {wl.name} workload "
+            f"(T={wl.T}, plus one decode token), {reps} repetition(s), {dt:.1f} s")
+
+
+def cpu_baseline(wl, budget_s=10.0, one_core_s=5.0, decode=False):
+    """The float64 oracle timed on this host's cores (OpenMP over channels),
+    and on one core, on a bounded slice of the workload."""
+    from oracle import oracle as O
+    O.build()
+    _set_oracle_threads(O, 0)
+    cores = os.cpu_count() or 1
+    value, sample = _rate(O, wl, budget_s, cores, decode)
+    one, one_sample = _rate(O, wl, one_core_s, 1, decode)
+    _set_oracle_threads(O, cores)
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+            "value_1core": one, "sample_1core": one_sample, "cpu_model": cpu_model()}
 
 
 def run_reference(args):
@@ -558,25 +736,25 @@ def run_reference(args):
     if rank != 0:
         return
     from oracle import oracle as O
-    from wkv_recurrence_b200 import inputs as I
     O.build()
     wl = workload(args)
     steps, warm = args.steps, max(3, args.warmup)
     budget = float(args.reference_seconds)
+    cores = os.cpu_count() or 1
     # size each step so that warm-up + timed steps take about `budget` seconds
     rows, cols = _pick_sample(wl, 200_000)
     sample = _oracle_sample(wl, rows, cols)
     t0 = time.perf_counter()
-    _oracle_step(O, sample)
+    _oracle_step(O, sample, cores)
     rate = rows * cols * (wl.T + 1) / max(time.perf_counter() - t0, 1e-6)
     per_step = max(2_000, int(rate * budget / (steps + warm)))
     rows, cols = _pick_sample(wl, per_step)
     sample = _oracle_sample(wl, rows, cols)
     for _ in range(warm):
-        _oracle_step(O, sample)
+        _oracle_step(O, sample, cores)
     t0 = time.perf_counter()
     for _ in range(steps):
-        _oracle_step(O, sample)
+        _oracle_step(O, sample, cores)
     dt = time.perf_counter() - t0
     units = rows * cols * (wl.T + 1) * steps
     value = units / dt
@@ -586,8 +764,8 @@ def run_reference(args):
             "steps": steps, "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_desc(wl), "name": wl.name, "B": wl.B, "T": wl.T, "C": wl.C},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.max_threads(), "kind": "oracle",
-                             "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -595,18 +773,19 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="layer", help="tiny|small|layer|decode|long|mixed")
+    ap.add_argument("--workload", default="long", help="tiny|small|layer|decode|long|mixed (the headline)")
     ap.add_argument("--options", default="", help='JSON wkv_options, e.g. {"kernel": 2, "chunk_len": 64}')
     ap.add_argument("--batch", type=int, default=0, help="override B of the workload (profiling)")
     ap.add_argument("--tokens", type=int, default=0, help="override T of the workload (profiling)")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-sub", action="store_true", help="headline workload only (no per-workload sub-records)")
     ap.add_argument("--no-clocks", action="store_true")
     args = ap.parse_args(argv)
     _, _, world = dist_env()

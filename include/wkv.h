@@ -54,7 +54,7 @@ typedef enum {
     WKV_OK = 0,
     WKV_ERR_INVALID_ARG = 1,        /* negative size, NULL pointer, bad option value */
     WKV_ERR_UNSUPPORTED_DTYPE = 2,  /* dtype combination not in the list below */
-    WKV_ERR_MISALIGNED = 3,         /* reserved: misaligned inputs take a slower path instead */
+    WKV_ERR_MISALIGNED = 3,         /* workspace not 256-byte aligned (misaligned k, v, out: slower path, no error) */
     WKV_ERR_WORKSPACE_TOO_SMALL = 4,
     WKV_ERR_CUDA = 5,               /* a CUDA runtime call failed (no device, launch error) */
     WKV_ERR_WAIT_TIMEOUT = 6        /* device side: a bounded wait gave up (see wkv_query_status) */
@@ -149,6 +149,13 @@ WKV_API size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const
  * are 16-byte aligned; 0 for invalid arguments. Host-only; touches no device.
  */
 WKV_API int32_t wkv_forward_kernel(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype, const wkv_options *opts);
+
+/*
+ * How many kernels one wkv_forward call launches for these sizes, input dtype
+ * and options (16-byte aligned k and v, T > 0); 0 for invalid arguments or
+ * when there is nothing to compute. Host-only; touches no device.
+ */
+WKV_API int32_t wkv_forward_launches(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype, const wkv_options *opts);
 
 /*
  * Sequence forward: for every (b, c), run the recurrence over t = 0..T-1,

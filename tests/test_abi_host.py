@@ -181,3 +181,24 @@ def test_binding_fails_loudly_without_cuda_tensors():
     x = torch.zeros(1, 4, 8)
     with pytest.raises(ValueError):
         W.forward(x, x, torch.zeros(8), torch.zeros(8))
+
+
+def test_noalloc_rejects_bad_arguments_before_any_device_work(L):
+    """wkv_forward_noalloc runs every argument check of wkv_forward before it
+    looks up its scratch array or queues anything (no device exists here, so
+    reaching the device would return WKV_ERR_CUDA instead)."""
+    def na(B=1, T=4, C=8, k=FAKE, v=FAKE, kvd=0, w=FAKE, u=FAKE, out=FAKE, od=0, sin=None, sout=None):
+        return L.wkv_forward_noalloc(B, T, C, k, v, kvd, w, u, out, od, sin, sout, None)
+    assert na(kvd=7) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert na(kvd=_abi.WKV_F32, od=_abi.WKV_BF16) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert na(k=None) == _abi.WKV_ERR_INVALID_ARG
+    assert na(out=None) == _abi.WKV_ERR_INVALID_ARG
+    assert na(u=None) == _abi.WKV_ERR_INVALID_ARG
+    assert na(sin=ctypes.byref(_abi.wkv_cstate(0x1000, None, 0x1000))) == _abi.WKV_ERR_INVALID_ARG
+    assert na(sout=ctypes.byref(_abi.wkv_state(0x1000, 0x1000, None))) == _abi.WKV_ERR_INVALID_ARG
+    # sizes out of range are refused before any plan is made from them
+    assert na(B=-1) == _abi.WKV_ERR_INVALID_ARG
+    assert na(T=1 << 24) == _abi.WKV_ERR_INVALID_ARG
+    assert na(B=1 << 40, C=1 << 40) == _abi.WKV_ERR_INVALID_ARG
+    assert L.wkv_forward_workspace_size(1 << 40, 4, 1 << 40, None) == 0
+    assert na(B=0, k=None, v=None, out=None) == _abi.WKV_OK

@@ -4,9 +4,10 @@ Some callers cannot allocate device memory: a host application whose own pool
 owns the whole GPU and hands a plug-in only its inputs and outputs, or code
 with hard latency limits that cannot take the device-wide synchronisation of
 cudaMalloc. For them the library keeps its scratch in a fixed device array.
-This test calls that entry point through the C ABI, twice in a row on
-different inputs, and checks each result against the ordinary wkv_forward
-(which takes a caller-allocated workspace). Collected last on purpose: if it
+These tests call that entry point through the C ABI several times in a row on
+different inputs and check every result against the float64 oracle at the
+same bar as the other parity tests, and against the ordinary wkv_forward
+(which takes a caller-allocated workspace). Collected last on purpose: if one
 fails, every other test has already run.
 """
 import ctypes
@@ -18,7 +19,7 @@ import torch
 import wkv_recurrence_b200 as W
 from wkv_recurrence_b200 import _abi
 from wkv_recurrence_b200 import inputs as I
-from parity_util import RTOL_F32, assert_out, dev_f32, host
+from parity_util import RTOL_F32, assert_out, assert_state, dev_f32, host
 
 pytestmark = pytest.mark.gpu
 
@@ -35,28 +36,55 @@ def _noalloc(L, K, V, Wt, U, out, state_in=None, state_out=None):
                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-def test_noalloc_matches_forward_on_two_calls(oracle):
+def _offset_by_one(x: np.ndarray, shape) -> torch.Tensor:
+    """A device copy of x whose base address is 4 bytes past a 16-byte boundary
+    (so TMA cannot address it and the plain-load kernels run)."""
+    return dev_f32(np.concatenate([[0.0], x.ravel()]).astype(np.float32))[1:].view(*shape)
+
+
+def _check_call(oracle, L, B, T, C, seed, with_state, misaligned, what):
+    k, v, w, u, st = I.random_case(B, T, C, seed=seed, k_spike=30.0, w_range=(1e-4, 8.0), state=with_state)
+    assert W.workspace_size(B, T, C) > 256  # scratch beyond the header is in use
+    if misaligned:
+        K, V = _offset_by_one(k, (B, T, C)), _offset_by_one(v, (B, T, C))
+        out = torch.full((B * T * C + 1,), float("nan"), device="cuda")[1:].view(B, T, C)
+    else:
+        K, V = dev_f32(k), dev_f32(v)
+        out = torch.full((B, T, C), float("nan"), device="cuda")
+    Wt, U = dev_f32(w), dev_f32(u)
+    S = None if st is None else tuple(dev_f32(s) for s in st)
+    so = tuple(torch.full((B, C), float("nan"), device="cuda") for _ in range(3))
+    assert _noalloc(L, K, V, Wt, U, out, S, so) == _abi.WKV_OK
+    torch.cuda.synchronize()
+    # against the float64 oracle, at the same bar as every parity test
+    ref, rst = oracle.recurrence_forward(k, v, w, u, st)
+    sc, sst = oracle.abs_scale_forward(k, v, w, u, st)
+    assert_out(host(out), ref, sc, RTOL_F32, what=what)
+    assert_state(tuple(host(s) for s in so), rst, sst[0], RTOL_F32, what=what + " state")
+    # and against the entry point with a caller-allocated workspace
+    ref_out, ref_state = W.forward(K, V, Wt, U, S)
+    torch.cuda.synchronize()
+    assert_out(host(out), host(ref_out), sc, RTOL_F32, what=what + " vs wkv_forward")
+    for a, b in zip(so, ref_state):
+        assert np.allclose(host(a), host(b), rtol=RTOL_F32, atol=0)
+
+
+def test_noalloc_matches_oracle_on_calls_in_a_row(oracle):
+    """Two aligned calls (the three-launch scan, whose scratch holds chunk totals
+    and incoming states), then two misaligned calls (the single-launch scan,
+    whose flags and epoch must start from zero in the shared array after the
+    other kernel used it), each against the oracle."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from wkv_recurrence_b200 import build
     build.build()
     L = _abi.lib()
-    cases = [(4, 1000, 256, True), (3, 2049, 192, False)]  # both take the chunked-scan kernel
-    for call, (B, T, C, with_state) in enumerate(cases):
-        k, v, w, u, st = I.random_case(B, T, C, seed=500 + call, k_spike=30.0, w_range=(1e-4, 8.0),
-                                       state=with_state)
-        assert W.workspace_size(B, T, C) > 256  # scratch beyond the header is in use
-        K, V, Wt, U = dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u)
-        S = None if st is None else tuple(dev_f32(s) for s in st)
-        out = torch.full((B, T, C), float("nan"), device="cuda")
-        so = tuple(torch.full((B, C), float("nan"), device="cuda") for _ in range(3))
-        assert _noalloc(L, K, V, Wt, U, out, S, so) == _abi.WKV_OK
-        ref_out, ref_state = W.forward(K, V, Wt, U, S)
-        torch.cuda.synchronize()
-        sc, sst = oracle.abs_scale_forward(k, v, w, u, st)
-        assert_out(host(out), host(ref_out), sc, RTOL_F32, what=f"noalloc call {call + 1}")
-        for a, b in zip(so, ref_state):
-            assert np.allclose(host(a), host(b), rtol=RTOL_F32, atol=0)
+    assert W.forward_kernel(4, 1000, 256) == 3 and W.forward_kernel(3, 2049, 192) == 3
+    cases = [(4, 1000, 256, True, False), (3, 2049, 192, False, False),
+             (2, 1500, 128, True, True), (3, 777, 64, False, True)]
+    for call, (B, T, C, with_state, misaligned) in enumerate(cases):
+        _check_call(oracle, L, B, T, C, 500 + call, with_state, misaligned,
+                    f"noalloc call {call + 1} ({'misaligned' if misaligned else 'aligned'})")
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():

@@ -14,7 +14,7 @@ fails loudly if it is missing or no CUDA device is present.
 """
 
 from .api import (PreparedForward, PreparedStep, WkvError, empty_state, forward,  # noqa: F401
-                  forward_kernel, make_workspace, query_status, step, workspace_size)
+                  forward_kernel, forward_launches, make_workspace, query_status, step, workspace_size)
 
-__all__ = ["forward", "step", "workspace_size", "forward_kernel", "make_workspace", "query_status", "empty_state",
+__all__ = ["forward", "step", "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
            "PreparedForward", "PreparedStep", "WkvError"]

@@ -23,7 +23,7 @@ WKV_F32 = 0
 WKV_BF16 = 1
 
 # entry points declared in include/wkv.h
-EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward", "wkv_step", "wkv_query_status",
+EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward_launches", "wkv_forward", "wkv_step", "wkv_query_status",
            "wkv_status_string", "wkv_version", "wkv_forward_noalloc", "wkv_last_cuda_error")
 
 # size of the library's built-in scratch array used by wkv_forward_noalloc
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.wkv_forward_workspace_size.restype = SZ
         L.wkv_forward_kernel.argtypes = [I64, I64, I64, I, ctypes.POINTER(wkv_options)]
         L.wkv_forward_kernel.restype = ctypes.c_int32
+        L.wkv_forward_launches.argtypes = [I64, I64, I64, I, ctypes.POINTER(wkv_options)]
+        L.wkv_forward_launches.restype = ctypes.c_int32
         L.wkv_forward.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
                                   ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state),
                                   P, SZ, P, ctypes.POINTER(wkv_options)]

@@ -80,6 +80,14 @@ def forward_kernel(B: int, T: int, C: int, kv_dtype: torch.dtype = torch.float32
     return int(n)
 
 
+def forward_launches(B: int, T: int, C: int, kv_dtype: torch.dtype = torch.float32,
+                     options: Optional[dict] = None) -> int:
+    """How many kernels one ``forward`` call launches for this shape (host-only)."""
+    if kv_dtype not in _DT:
+        raise TypeError(f"dtype {kv_dtype} is not supported (float32 or bfloat16)")
+    return int(_abi.lib().wkv_forward_launches(int(B), int(T), int(C), _DT[kv_dtype], _options(options)))
+
+
 def make_workspace(B: int, T: int, C: int, options: Optional[dict] = None, device=None) -> torch.Tensor:
     """A zero-filled workspace for ``forward`` (zero once; the library keeps it ready)."""
     return torch.zeros(workspace_size(B, T, C, options), dtype=torch.uint8,

@@ -80,10 +80,8 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // which need TMA, into the single-launch one (the pipelined scan uses the same
 // workspace layout as the single-launch one). A three-launch plan reserves enough workspace
 // for either, so a workspace sized by wkv_forward_workspace_size always fits.
-bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, int kv_bytes = 4,
-               bool tma_ok = true) {
+bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, bool tma_ok = true) {
   std::memset(pl, 0, sizeof *pl);
-  (void)kv_bytes;
   const int want = o ? o->kernel : 0;
   if (want < 0 || want > 4) return false;
   const int64_t lanes = B * C;
@@ -182,6 +180,33 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     pl->bytes = three_requested ? std::max(off3, off) : off;
   }
   return true;
+}
+
+// Sizes wkv_forward accepts: B, T, C >= 0, T < 2^24, B and C < 2^31 and
+// B*T*C < 2^62 (checked without overflow).
+bool sizes_ok(int64_t B, int64_t T, int64_t C) {
+  if (B < 0 || T < 0 || C < 0) return false;
+  if (T >= (1ll << 24) || C >= (1ll << 31) || B >= (1ll << 31)) return false;
+  if (B > 0 && C > 0 && T > (int64_t)((1ull << 62) / (uint64_t)(B * C))) return false;
+  return true;
+}
+
+// Every check of wkv_forward's arguments that needs no plan and no workspace:
+// sizes, dtypes, state structs, options, and the pointers the sizes require.
+wkv_status check_forward_args(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
+                              const float* w, const float* u, const void* out, wkv_dtype out_dtype,
+                              const wkv_cstate* state_in, const wkv_state* state_out, const wkv_options* opts) {
+  if (!sizes_ok(B, T, C)) return WKV_ERR_INVALID_ARG;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (out_dtype != WKV_F32 && out_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (kv_dtype == WKV_F32 && out_dtype != WKV_F32) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (state_in && (!state_in->num || !state_in->den || !state_in->max_e)) return WKV_ERR_INVALID_ARG;
+  if (state_out && (!state_out->num || !state_out->den || !state_out->max_e)) return WKV_ERR_INVALID_ARG;
+  if (opts && opts->wait_timeout_ns < 0) return WKV_ERR_INVALID_ARG;
+  if (opts && (opts->inject_enable != 0 && opts->inject_enable != 1)) return WKV_ERR_INVALID_ARG;
+  if (B * T * C > 0 && (!k || !v || !out)) return WKV_ERR_INVALID_ARG;
+  if (B * C > 0 && T > 0 && (!w || !u)) return WKV_ERR_INVALID_ARG;
+  return WKV_OK;
 }
 
 bool tma_usable(const void* k, const void* v, int64_t C, size_t es) {
@@ -590,18 +615,28 @@ const char* wkv_status_string(wkv_status s) {
 size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, const wkv_options* opts) {
   // the automatic choice of kernel may depend on the input dtype, which is
   // not an argument here: return what either choice needs
-  Plan a, b;
-  if (B < 0 || T < 0 || C < 0 || !make_plan(B, T, C, opts, &a, 4) || !make_plan(B, T, C, opts, &b, 2)) return 0;
-  return std::max(a.bytes, b.bytes);
+  Plan pl;
+  if (!sizes_ok(B, T, C) || !make_plan(B, T, C, opts, &pl)) return 0;
+  return pl.bytes;
 }
 
 int32_t wkv_forward_kernel(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype, const wkv_options* opts) {
-  if (B < 0 || T < 0 || C < 0) return 0;
+  if (!sizes_ok(B, T, C)) return 0;
   if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return 0;
   const size_t es = kv_dtype == WKV_F32 ? 4 : 2;
   Plan pl;
-  if (!make_plan(B, T, C, opts, &pl, (int)es, (C * (int64_t)es) % 16 == 0)) return 0;
+  if (!make_plan(B, T, C, opts, &pl, (C * (int64_t)es) % 16 == 0)) return 0;
   return pl.kernel;
+}
+
+int32_t wkv_forward_launches(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype, const wkv_options* opts) {
+  if (!sizes_ok(B, T, C) || B * C == 0 || T == 0) return 0;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return 0;
+  const size_t es = kv_dtype == WKV_F32 ? 4 : 2;
+  Plan pl;
+  if (!make_plan(B, T, C, opts, &pl, (C * (int64_t)es) % 16 == 0)) return 0;
+  if (pl.kernel == 3) return pl.nch > 1 ? 3 : 2;  // chunk totals (when there is more than one chunk), scan, replay
+  return 1;
 }
 
 wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
@@ -609,28 +644,17 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
                        const wkv_state* state_out, void* workspace, size_t workspace_bytes, void* stream,
                        const wkv_options* opts) {
   // ---- argument checks: nothing is launched before they pass
-  if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
-  if (T >= (1ll << 24) || C >= (1ll << 31) || B >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  if (B > 0 && C > 0 && T > (int64_t)((1ull << 62) / (uint64_t)(B * C))) return WKV_ERR_INVALID_ARG;
-  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
-  if (out_dtype != WKV_F32 && out_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
-  if (kv_dtype == WKV_F32 && out_dtype != WKV_F32) return WKV_ERR_UNSUPPORTED_DTYPE;
-  if (state_in && (!state_in->num || !state_in->den || !state_in->max_e)) return WKV_ERR_INVALID_ARG;
-  if (state_out && (!state_out->num || !state_out->den || !state_out->max_e)) return WKV_ERR_INVALID_ARG;
-  if (opts && opts->wait_timeout_ns < 0) return WKV_ERR_INVALID_ARG;
-  if (opts && (opts->inject_enable != 0 && opts->inject_enable != 1)) return WKV_ERR_INVALID_ARG;
+  const wkv_status chk = check_forward_args(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, opts);
+  if (chk != WKV_OK) return chk;
   const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
   // TMA needs 16-byte aligned bases and row pitches; otherwise the kernels
   // fill their tiles with plain loads
   const bool tma = tma_usable(k, v, C, kes);
   Plan pl;
-  if (!make_plan(B, T, C, opts, &pl, (int)kes, tma)) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, opts, &pl, tma)) return WKV_ERR_INVALID_ARG;
   if (!workspace) return WKV_ERR_INVALID_ARG;
   if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
-  const int64_t n = B * T * C;
-  if (n > 0 && (!k || !v || !out)) return WKV_ERR_INVALID_ARG;
-  if (B * C > 0 && T > 0 && (!w || !u)) return WKV_ERR_INVALID_ARG;
 
   const int64_t BC = B * C;
   if (BC == 0) return WKV_OK;  // nothing to compute or write
@@ -807,10 +831,13 @@ bool noalloc_scratch(int dev, void** ptr) {
 wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
                                const float* w, const float* u, void* out, wkv_dtype out_dtype,
                                const wkv_cstate* state_in, const wkv_state* state_out, void* stream) {
-  if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
+  // every argument check of wkv_forward, before anything is queued on the stream
+  const wkv_status chk =
+      check_forward_args(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, nullptr);
+  if (chk != WKV_OK) return chk;
   Plan pl;
   const size_t kes = kv_dtype == WKV_BF16 ? 2 : 4;
-  if (!make_plan(B, T, C, nullptr, &pl, (int)kes, tma_usable(k, v, C, kes))) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, nullptr, &pl, tma_usable(k, v, C, kes))) return WKV_ERR_INVALID_ARG;
   if (pl.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (B * C == 0) {
     // nothing to compute: wkv_forward checks the other arguments and returns

@@ -197,16 +197,30 @@ def draw_state(wl: Workload, rows=None, seed: int = 0):
     return num, den, mx
 
 
+_DEC_BLOCK = 256         # streams per independently seeded block of a decode token
+
+
 def draw_decode_token(wl: Workload, step: int, rows=None, seed: int = 0):
-    """Fresh k, v ~ N(0, 1) for one decode step: fp32 [len(rows), C]."""
-    rows = range(wl.B) if rows is None else list(rows)
-    k = np.empty((len(rows), wl.C), np.float32)
-    v = np.empty((len(rows), wl.C), np.float32)
-    for i, s in enumerate(rows):
-        g = _rng(seed, wl.code, _DK, step * 1_000_003 + s)
-        k[i] = g.standard_normal(wl.C, dtype=np.float32)
-        g = _rng(seed, wl.code, _DV, step * 1_000_003 + s)
-        v[i] = g.standard_normal(wl.C, dtype=np.float32)
+    """Fresh k, v ~ N(0, 1) for one decode step: fp32 [len(rows), C].
+
+    The streams are drawn in blocks of 256, each block from its own generator
+    seeded by (seed, workload, tensor, step, block), so any subset of streams
+    can be regenerated by drawing only the blocks that hold them.
+    """
+    rows = np.asarray(range(wl.B) if rows is None else list(rows), np.int64)
+    k = np.empty((rows.size, wl.C), np.float32)
+    v = np.empty((rows.size, wl.C), np.float32)
+
+    def one(blk):
+        n = min(_DEC_BLOCK, wl.B - int(blk) * _DEC_BLOCK)
+        sel = np.flatnonzero(rows // _DEC_BLOCK == blk)
+        local = rows[sel] - int(blk) * _DEC_BLOCK
+        kb = _rng5(seed, wl.code, _DK, step, int(blk)).standard_normal((n, wl.C), dtype=np.float32)
+        vb = _rng5(seed, wl.code, _DV, step, int(blk)).standard_normal((n, wl.C), dtype=np.float32)
+        k[sel] = kb[local]
+        v[sel] = vb[local]
+
+    _pool_map(one, np.unique(rows // _DEC_BLOCK).tolist())
     return k, v
 
 
