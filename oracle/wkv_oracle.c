@@ -162,3 +162,85 @@ int wkv_oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * Two extensions of the same recurrence, from "RWKV-v6 Architecture:
+ * Attention-Free Linear Transformers":
+ *
+ *   - section "2. Dynamic Data-Dependent Decay": the decay becomes a per-token
+ *     vector w_t. Here w_t takes the place of w in the step above at token t
+ *     (the state is multiplied by e^{-w_t} when token t is added), so an
+ *     earlier token i reaches the output of token t with the exponent
+ *     k_i - (w_{i+1} + ... + w_{t-1}).
+ *   - section "3. Matrix-Valued Hidden State" (the readout) and the
+ *     Time-Mixing description of "RWKV: Merging Transformer Training with RNN
+ *     Speed": the output is gated by the receptance, y_t = sigmoid(r_t) * wkv_t.
+ *
+ * w_t: NULL (use w for every token) or [B, T, C] fp32. r: NULL (no gate) or
+ * [B, T, C] of element type kv_dtype. Everything else as wkv_oracle_forward.
+ */
+void wkv_oracle_forward_ext(int64_t B, int64_t T, int64_t C,
+                            const void *k, const void *v, int kv_dtype,
+                            const float *w, const float *w_t, const float *u, const void *r,
+                            const double *num_in, const double *den_in, const double *max_in,
+                            double *out,
+                            double *num_out, double *den_out, double *max_out,
+                            int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t s = 0; s < B * C; ++s) {
+        const int64_t b = s / C, c = s % C;
+        double num = 0.0, den = 0.0, m = -INFINITY;
+        if (num_in) {
+            num = num_in[s];
+            den = den_in[s];
+            m = max_in[s];
+        }
+        const double uc = (double)u[c];
+        for (int64_t t = 0; t < T; ++t) {
+            const size_t i = ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;
+            const double kt = widen(k, kv_dtype, i);
+            const double vt = widen(v, kv_dtype, i);
+            const double wt = w_t ? (double)w_t[i] : (double)w[c];
+            double y = wkv_token(kt, vt, wt, uc, &num, &den, &m);
+            if (r) y = y / (1.0 + exp(-widen(r, kv_dtype, i)));
+            out[i] = y;
+        }
+        if (num_out) {
+            num_out[s] = num;
+            den_out[s] = den;
+            max_out[s] = m;
+        }
+    }
+}
+
+/*
+ * One decode token for S streams with the same two extensions: w is [C]
+ * (w_per_stream = 0) or [S, C] (the per-token decay of this step for every
+ * stream); r is NULL or [S, C] fp32. Everything else as wkv_oracle_step.
+ */
+void wkv_oracle_step_ext(int64_t S, int64_t C, const float *k, const float *v,
+                         const float *w, int w_per_stream, const float *u, const float *r,
+                         const double *num_in, const double *den_in, const double *max_in,
+                         double *out, double *num_out, double *den_out, double *max_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < S * C; ++i) {
+        const int64_t c = i % C;
+        double num = num_in[i], den = den_in[i], m = max_in[i];
+        const double wi = (double)(w_per_stream ? w[i] : w[c]);
+        double y = wkv_token((double)k[i], (double)v[i], wi, (double)u[c], &num, &den, &m);
+        if (r) y = y / (1.0 + exp(-(double)r[i]));
+        out[i] = y;
+        num_out[i] = num;
+        den_out[i] = den;
+        max_out[i] = m;
+    }
+}

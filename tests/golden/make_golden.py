@@ -33,6 +33,32 @@ def main():
                             f"{float(w[c])!r} {float(u[c])!r} {res[b][t][c]:.30e}\n")
     print("wrote", path)
 
+    # the same tiny case with per-token decays w_t = exp(N(-1, 1)) and a
+    # receptance gate r ~ N(0, 1) ("RWKV-v6 Architecture: Attention-Free Linear
+    # Transformers", sections "2. Dynamic Data-Dependent Decay" and the gated
+    # readout of "3. Matrix-Valued Hidden State")
+    import numpy as np
+    g = np.random.default_rng(2024)
+    wt = np.exp(g.normal(-1.0, 1.0, k.shape)).astype(np.float32)
+    r = g.normal(0.0, 1.0, k.shape).astype(np.float32)
+    res = O.decimal_forward(k, v, w, u, digits=50, w_t=wt, r=r)
+    path = os.path.join(HERE, "wkv_tiny_wt_gate_decimal.txt")
+    with open(path, "w") as f:
+        f.write("# sigmoid(r_t) * wkv_t by the direct sum of the equation in 'Linear attention without\n")
+        f.write("# writing a CUDA kernel', section 'The recurrence', with the per-token decay w_t of\n")
+        f.write("# 'RWKV-v6 Architecture', section '2. Dynamic Data-Dependent Decay' in place of w\n")
+        f.write("# (token i reaches token t with exponent k_i - (w_{i+1} + ... + w_{t-1})); 50-digit\n")
+        f.write("# decimal arithmetic. Workload tiny (B=1, T=8, C=4, seed 0), zero initial state;\n")
+        f.write("# w_t = exp(N(-1, 1)), r ~ N(0, 1) from numpy seed 2024. Written by make_golden.py.\n")
+        f.write("# columns: b t c k v w_t u r out   (inputs: the fp32 values, printed exactly)\n")
+        for b in range(wl.B):
+            for t in range(wl.T):
+                for c in range(wl.C):
+                    f.write(f"{b} {t} {c} {float(k[b, t, c])!r} {float(v[b, t, c])!r} "
+                            f"{float(wt[b, t, c])!r} {float(u[c])!r} {float(r[b, t, c])!r} "
+                            f"{res[b][t][c]:.30e}\n")
+    print("wrote", path)
+
 
 if __name__ == "__main__":
     main()

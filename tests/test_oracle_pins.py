@@ -381,3 +381,231 @@ def test_pins_catch_planted_mistakes(mistake):
         except AssertionError:
             failed.append(check.__name__)
     assert failed, f"no check caught the planted mistake {mistake!r}"
+
+
+# ---------------------------------------------------------------------------
+# the two extensions of "RWKV-v6 Architecture: Attention-Free Linear
+# Transformers": per-token decay w_t (section "2. Dynamic Data-Dependent
+# Decay") and the receptance gate sigmoid(r) * wkv. Checks take
+# impl(k, v, w, u, state, w_t, r) -> (out, state).
+# ---------------------------------------------------------------------------
+
+GOLDEN_EXT = os.path.join(os.path.dirname(__file__), "golden", "wkv_tiny_wt_gate_decimal.txt")
+
+
+def load_golden_ext():
+    rows = [ln.split() for ln in open(GOLDEN_EXT) if not ln.startswith("#")]
+    B = 1 + max(int(r[0]) for r in rows)
+    T = 1 + max(int(r[1]) for r in rows)
+    C = 1 + max(int(r[2]) for r in rows)
+    k, v, wt, r_ = (np.zeros((B, T, C), np.float32) for _ in range(4))
+    w = np.zeros(C, np.float32)
+    u = np.zeros(C, np.float32)
+    ref = np.zeros((B, T, C))
+    for row in rows:
+        b, t, c = int(row[0]), int(row[1]), int(row[2])
+        k[b, t, c], v[b, t, c], wt[b, t, c], u[c], r_[b, t, c] = (np.float32(float(x)) for x in row[3:8])
+        ref[b, t, c] = float(row[8])
+    return k, v, w, u, wt, r_, ref
+
+
+def check_ext_hand_worked(impl):
+    """Three tokens, one channel, worked by hand, with per-token decays
+    w_t = (ln 2, ln 3, ln 5), k = 0, v = (1, 2, 4), u = 0 and no gate.
+
+    Token 1 sees only itself: 1. Token 2 sees token 1 undecayed and itself:
+    (1 + 2) / 2 = 3/2. Token 2's advance decays the state by e^{-ln 3}: the
+    pair becomes N = 1/3 + 2, D = 1/3 + 1, so token 3 gives (7/3 + 4) / (4/3 + 1)
+    = 19/7. Token 3's advance decays by 1/5: N = 67/15, D = 19/15 over the
+    largest exponent 0 (token 3's key).
+    """
+    k = np.zeros((1, 3, 1), np.float32)
+    v = np.array([1.0, 2.0, 4.0], np.float32).reshape(1, 3, 1)
+    wt = np.log(np.array([2.0, 3.0, 5.0])).astype(np.float32).reshape(1, 3, 1)
+    out, (num, den, mx) = impl(k, v, np.zeros(1, np.float32), np.zeros(1, np.float32), None, wt, None)
+    assert out[0, :, 0] == pytest.approx([1.0, 1.5, 19.0 / 7.0], rel=1e-6)
+    assert num[0, 0] == pytest.approx(67.0 / 15.0, rel=1e-6)
+    assert den[0, 0] == pytest.approx(19.0 / 15.0, rel=1e-6)
+    assert mx[0, 0] == pytest.approx(0.0, abs=1e-7)
+
+
+def check_ext_golden_decimal(impl, tol=1e-12):
+    k, v, w, u, wt, r, ref = load_golden_ext()
+    out, _ = impl(k, v, w, u, None, wt, r)
+    assert np.abs(out - ref).max() <= tol * max(1.0, np.abs(ref).max())
+
+
+def check_ext_constant_decay_reduces(impl):
+    """w_t equal to w at every token is the per-channel equation (whose pins
+    are above): compared with the hand-worked and golden-pinned recurrence."""
+    from oracle import oracle as O
+    k, v, w, u, st = I.random_case(2, 40, 6, 31, k_scale=2.0, k_spike=30.0, state=True)
+    wt = np.broadcast_to(w, k.shape).copy()
+    out, s = impl(k, v, w, u, st, wt, None)
+    ref, rs = O.recurrence_forward(k, v, w, u, st)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-13)
+    assert np.allclose(s[2] + np.log(s[1]), rs[2] + np.log(rs[1]), rtol=0, atol=1e-12)
+
+
+def check_ext_reset(impl):
+    """A decay of 1e4 at token j erases every earlier token from the outputs
+    after j: they equal a run that starts at token j from the empty state."""
+    k, v, w, u, _ = I.random_case(1, 30, 5, 32, k_scale=2.0)
+    g = np.random.default_rng(32)
+    wt = np.exp(g.normal(-1.0, 1.0, k.shape)).astype(np.float32)
+    j = 11
+    wt[:, j] = np.float32(1e4)
+    out, _ = impl(k, v, w, u, None, wt, None)
+    out_j, _ = impl(k[:, j:], v[:, j:], w, u, None, wt[:, j:], None)
+    assert np.allclose(out[:, j + 1:], out_j[:, 1:], rtol=1e-12, atol=1e-14)
+    assert not np.allclose(out[:, j], out_j[:, 0])  # token j itself still sees the past
+
+
+def check_ext_split(impl):
+    """Per-token decays and the gate: T1 tokens then the rest from the state = one pass."""
+    k, v, w, u, st = I.random_case(2, 41, 5, 33, k_scale=2.0, state=True)
+    g = np.random.default_rng(33)
+    wt = np.exp(g.normal(-2.0, 1.5, k.shape)).astype(np.float32)
+    r = g.normal(0.0, 2.0, k.shape).astype(np.float32)
+    out, s = impl(k, v, w, u, st, wt, r)
+    o1, s1 = impl(k[:, :13], v[:, :13], w, u, st, wt[:, :13], r[:, :13])
+    o2, s2 = impl(k[:, 13:], v[:, 13:], w, u, s1, wt[:, 13:], r[:, 13:])
+    assert np.allclose(np.concatenate([o1, o2], 1), out, rtol=1e-12, atol=1e-13)
+    assert np.allclose(s2[2] + np.log(s2[1]), s[2] + np.log(s[1]), rtol=0, atol=1e-12)
+
+
+def check_gate_values(impl):
+    """r = 0 halves every output exactly (sigmoid(0) = 1/2) and leaves the state
+    alone; r = +40 leaves it (to 1e-17); r = -40 sends it to zero (e^-40)."""
+    k, v, w, u, st = I.random_case(2, 25, 4, 34, k_scale=2.0, state=True)
+    plain, s0 = impl(k, v, w, u, st, None, None)
+    half, s1 = impl(k, v, w, u, st, None, np.zeros_like(k))
+    assert np.array_equal(half, plain * 0.5)
+    for a, b in zip(s0, s1):
+        assert np.array_equal(a, b)
+    hi, _ = impl(k, v, w, u, st, None, np.full_like(k, 40.0))
+    assert np.allclose(hi, plain, rtol=1e-16, atol=0)
+    lo, _ = impl(k, v, w, u, st, None, np.full_like(k, -40.0))
+    assert np.all(np.abs(lo) <= 5e-18 * np.abs(plain) + 1e-300)
+
+
+EXT_CHECKS = [check_ext_hand_worked, check_ext_golden_decimal, check_ext_constant_decay_reduces,
+              check_ext_reset, check_ext_split, check_gate_values]
+
+
+def _recurrence_ext(O):
+    return lambda k, v, w, u, st, wt, r: O.recurrence_forward(k, v, w, u, st, w_t=wt, r=r)
+
+
+def _direct_ext(O):
+    return lambda k, v, w, u, st, wt, r: O.direct_forward(k, v, w, u, st, w_t=wt, r=r)
+
+
+@pytest.mark.parametrize("check", EXT_CHECKS, ids=lambda f: f.__name__)
+def test_recurrence_ext_pins(oracle, check):
+    check(_recurrence_ext(oracle))
+
+
+@pytest.mark.parametrize("check", EXT_CHECKS, ids=lambda f: f.__name__)
+def test_direct_sum_ext_pins(oracle, check):
+    check(_direct_ext(oracle))
+
+
+def test_decimal_ext_matches_golden(oracle):
+    k, v, w, u, wt, r, ref = load_golden_ext()
+    res = oracle.decimal_forward(k, v, w, u, digits=50, w_t=wt, r=r)
+    for (b, t, c), x in np.ndenumerate(ref):
+        assert abs(float(res[b][t][c]) - x) <= 1e-15 * max(1.0, abs(x))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_recurrence_ext_equals_direct_sum(oracle, seed):
+    T = [9, 33, 64, 50][seed]
+    k, v, w, u, st = I.random_case(2, T, 7, 200 + seed, k_scale=1.0 + seed, k_spike=[0, 40, 0, 60][seed],
+                                   state=bool(seed % 2))
+    g = np.random.default_rng(200 + seed)
+    wt = np.exp(g.normal(-1.0 - seed, 1.5, k.shape)).astype(np.float32)
+    r = g.normal(0.0, 2.0, k.shape).astype(np.float32) if seed % 2 == 0 else None
+    o1, s1 = oracle.recurrence_forward(k, v, w, u, st, w_t=wt, r=r)
+    o2, s2 = oracle.direct_forward(k, v, w, u, st, w_t=wt, r=r)
+    scale, _ = oracle.abs_scale_forward(k, v, w, u, st, w_t=wt, r=r)
+    assert np.all(np.abs(o1 - o2) <= 1e-12 * scale + 1e-300)
+    assert np.allclose(s1[2] + np.log(s1[1]), s2[2] + np.log(s2[1]), rtol=0, atol=1e-12)
+    assert np.allclose(s1[0] / s1[1], s2[0] / s2[1], rtol=1e-12, atol=1e-13)
+    assert np.all(np.abs(o1) <= scale * (1 + 1e-12))
+
+
+def test_ext_direct_output_and_step(oracle):
+    """direct_output and recurrence_step (per-stream decay, gate) against the forward."""
+    k, v, w, u, st = I.random_case(2, 20, 3, 35, state=True)
+    g = np.random.default_rng(35)
+    wt = np.exp(g.normal(-1.0, 1.0, k.shape)).astype(np.float32)
+    r = g.normal(0.0, 1.0, k.shape).astype(np.float32)
+    out, s = oracle.recurrence_forward(k, v, w, u, st, w_t=wt, r=r)
+    for t in (0, 1, 19):
+        o = oracle.direct_output(k[1, :, 2], v[1, :, 2], w[2], u[2], t, (st[0][1, 2], st[1][1, 2], st[2][1, 2]),
+                                 w_t=wt[1, :, 2], r=r[1, t, 2])
+        assert o == pytest.approx(out[1, t, 2], rel=1e-13, abs=1e-15)
+    state = tuple(x.astype(np.float64) for x in st)
+    for t in range(k.shape[1]):
+        o, state = oracle.recurrence_step(state, k[:, t], v[:, t], wt[:, t], u, r=r[:, t])
+        assert np.array_equal(o, out[:, t])
+    for a, b in zip(state, s):
+        assert np.array_equal(a, b)
+
+
+def _python_recurrence_ext(mistake=None):
+    """A Python copy of the recurrence with w_t and the gate, and one thing broken."""
+    def impl(k, v, w, u, st, wt, r):
+        k = np.asarray(k, np.float64)
+        v = np.asarray(v, np.float64)
+        B, T, C = k.shape
+        wt = np.broadcast_to(np.asarray(w, np.float64), k.shape) if wt is None else np.asarray(wt, np.float64)
+        out = np.empty((B, T, C))
+        if st is None:
+            num, den, m = np.zeros((B, C)), np.zeros((B, C)), np.full((B, C), -np.inf)
+        else:
+            num, den, m = (np.array(x, np.float64) for x in st)
+        ud = np.asarray(u, np.float64)
+        with np.errstate(invalid="ignore"):
+            for t in range(T):
+                kt, vt = k[:, t], v[:, t]
+                kb = kt + ud
+                e = np.maximum(m, kb)
+                a, b = np.exp(m - e), np.exp(kb - e)
+                y = (a * num + b * vt) / (a * den + b)
+                if r is not None:
+                    rr = np.asarray(r, np.float64)[:, t]
+                    y = y / (1 + np.exp(rr if mistake == "gate_sign" else -rr))
+                out[:, t] = y
+                if mistake == "decay_next_token":
+                    wd = wt[:, min(t + 1, T - 1)]
+                elif mistake == "decay_prev_token":
+                    wd = wt[:, max(t - 1, 0)]
+                else:
+                    wd = wt[:, t]
+                md = m - wd
+                e2 = np.maximum(md, kt)
+                a2, b2 = np.exp(md - e2), np.exp(kt - e2)
+                num = a2 * num + b2 * vt
+                den = a2 * den + b2
+                m = e2
+        return out, (num, den, m)
+    return impl
+
+
+def test_python_recurrence_ext_passes():
+    for check in EXT_CHECKS:
+        check(_python_recurrence_ext())
+
+
+@pytest.mark.parametrize("mistake", ["decay_next_token", "decay_prev_token", "gate_sign"])
+def test_ext_pins_catch_planted_mistakes(mistake):
+    impl = _python_recurrence_ext(mistake)
+    failed = []
+    for check in EXT_CHECKS:
+        try:
+            check(impl)
+        except AssertionError:
+            failed.append(check.__name__)
+    assert failed, f"no check caught the planted mistake {mistake!r}"
