@@ -81,7 +81,8 @@ typedef struct {
  * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
  * zero-filled struct also means "defaults".
  *   kernel          0 = choose by shape (sequential for many channels or short
- *                   sequences; otherwise the chunked scan in three launches),
+ *                   sequences; the cluster scan for T up to 2048; otherwise
+ *                   the chunked scan in three launches),
  *                   1 = sequential-over-T kernel,
  *                   2 = chunked scan in one launch (look-back between CTAs),
  *                   3 = chunked scan in three launches (chunk totals, their
@@ -89,7 +90,13 @@ typedef struct {
  *                   the second time for inputs that fit there),
  *                   4 = chunked scan in one launch of persistent CTAs that
  *                   pipeline their tiles (look-back of one tile overlapped
- *                   with the next tile's fold and later tiles' copies)
+ *                   with the next tile's fold and later tiles' copies),
+ *                   5 = chunked scan inside one thread-block cluster per
+ *                   (batch row, 32 channels): the cluster's shared memory
+ *                   holds the whole sequence (T <= 8 x cta_warps x span), the
+ *                   CTAs exchange their totals through distributed shared
+ *                   memory; one launch, k and v read once, no waiting
+ *                   between clusters
  *   chunk_len       tokens per chunk for the chunked kernels (0 = choose: 32
  *                   or 64 for the three-launch scan, 128 otherwise; or 32, 64,
  *                   128)
@@ -99,7 +106,8 @@ typedef struct {
  *   wait_timeout_ns limit of every device-side wait (0 = 1 second)
  *   span            tokens per warp in a chunk-scan tile, 8 or 16 (0 = choose);
  *                   chunk_len / span warps share a tile (at most 8 for the
- *                   pipelined scan, so chunk_len 128 needs span 16 there)
+ *                   pipelined scan, so chunk_len 128 needs span 16 there);
+ *                   the cluster scan (kernel 5) takes 16 or 32 (0 = 32)
  *   seq_threads     threads per CTA of the sequential kernel and of the
  *                   three-launch scan's replay pass: 32, 64 or 128 (0 =
  *                   choose: 32); each thread carries seq_vec channels in the
@@ -110,6 +118,8 @@ typedef struct {
  *                   (0 = choose: 1 below 151552 channels B*C, else 2)
  *   replay_chunks   three-launch scan (kernel 3): consecutive chunks that
  *                   one replay warp walks (0 = choose; or 1, 2, 4)
+ *   cta_warps       cluster scan (kernel 5): warps (spans) per CTA, 4, 8 or
+ *                   16 (0 = 8)
  *   stages          shared-memory ring stages of the pipelined scan
  *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
  *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)
@@ -133,6 +143,7 @@ typedef struct {
     int32_t stages;
     int32_t seq_vec;
     int32_t replay_chunks;
+    int32_t cta_warps;
 } wkv_options;
 
 /*
@@ -188,6 +199,41 @@ WKV_API wkv_status wkv_forward(int64_t B, int64_t T, int64_t C,
                        void *stream, const wkv_options *opts);
 
 /*
+ * Two optional inputs of the RWKV-v6 time-mixing block ("RWKV-v6
+ * Architecture: Attention-Free Linear Transformers"), for wkv_forward_ext and
+ * wkv_step_ext:
+ *   w_t  NULL, or fp32 decays of every token ([B, T, C] for a forward, [S, C]
+ *        for a decode step), in place of w: token t's advance multiplies the
+ *        state by e^{-w_t} (section "2. Dynamic Data-Dependent Decay"; the
+ *        page's multiplicative factor exp(-exp(.)) is e^{-w_t} here). An
+ *        earlier token i then reaches token t with the exponent
+ *        k_i - (w_{i+1} + ... + w_{t-1}).
+ *   r    NULL, or the receptance, same shape and element type as k: every
+ *        output is gated, out = sigmoid(r) * wkv (the readout of section
+ *        "3. Matrix-Valued Hidden State"). The state is not gated.
+ */
+typedef struct {
+    const float *w_t;
+    const void *r;
+} wkv_ext;
+
+/*
+ * wkv_forward with the optional inputs of wkv_ext (ext = NULL, or both of its
+ * pointers NULL, is exactly wkv_forward). With w_t, the w argument is not read
+ * and may be NULL. Kernels: r works with every kernel; w_t with the
+ * sequential kernel (1), the three-launch scan (3) and the cluster scan (5);
+ * an explicit kernel 2 or 4 with w_t is WKV_ERR_INVALID_ARG, and the automatic
+ * choice never takes them with w_t.
+ */
+WKV_API wkv_status wkv_forward_ext(int64_t B, int64_t T, int64_t C,
+                           const void *k, const void *v, wkv_dtype kv_dtype,
+                           const float *w, const float *u,
+                           void *out, wkv_dtype out_dtype,
+                           const wkv_cstate *state_in, const wkv_state *state_out,
+                           void *workspace, size_t workspace_bytes,
+                           void *stream, const wkv_options *opts, const wkv_ext *ext);
+
+/*
  * Batched one-token decode (the constant-cost step of the recurrence): S
  * independent streams of C channels each take one token.
  *
@@ -207,6 +253,18 @@ WKV_API wkv_status wkv_step(int64_t S, int64_t C,
                     void *out, wkv_dtype out_dtype,
                     const wkv_cstate *state_in, const wkv_state *state_out,
                     void *stream);
+
+/*
+ * wkv_step with the optional inputs of wkv_ext: w_t [S, C] (this token's decay
+ * for every stream, in place of w, which may then be NULL) and r [S, C]
+ * (element type kv_dtype). ext = NULL is exactly wkv_step.
+ */
+WKV_API wkv_status wkv_step_ext(int64_t S, int64_t C,
+                        const void *k, const void *v, wkv_dtype kv_dtype,
+                        const float *w, const float *u,
+                        void *out, wkv_dtype out_dtype,
+                        const wkv_cstate *state_in, const wkv_state *state_out,
+                        void *stream, const wkv_ext *ext);
 
 /*
  * wkv_forward without a caller-provided workspace. The pages have no

@@ -41,7 +41,8 @@ def test_binding_structs_match_the_header(tmp_path):
     cc = shutil.which("gcc") or shutil.which("cc")
     if cc is None:
         pytest.skip("no host C compiler")
-    structs = {"wkv_options": _abi.wkv_options, "wkv_cstate": _abi.wkv_cstate, "wkv_state": _abi.wkv_state}
+    structs = {"wkv_options": _abi.wkv_options, "wkv_cstate": _abi.wkv_cstate, "wkv_state": _abi.wkv_state,
+               "wkv_ext": _abi.wkv_ext}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "wkv.h"', "int main(void) {"]
     for name, ct in structs.items():
         lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
@@ -91,18 +92,33 @@ def test_workspace_size(L):
 
 def test_forward_kernel_choice(L):
     F32, BF16 = _abi.WKV_F32, _abi.WKV_BF16
-    # many channels or short sequences: the sequential kernel; otherwise a chunked scan
+    # many channels or short sequences: the sequential kernel; up to 2048 tokens
+    # the cluster scan; otherwise a chunked scan
     assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
-    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 3
+    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 5
+    assert L.wkv_forward_kernel(8, 2048, 768, F32, None) == 5
+    assert L.wkv_forward_kernel(8, 2049, 768, F32, None) == 3
     assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 3
     assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 2  # rows TMA cannot address
+    assert L.wkv_forward_kernel(8, 1024, 769, F32, None) == 2
     # an explicit choice stands, except that the TMA-only scans fall back to the
     # single-launch scan when a row pitch is not a multiple of 16 bytes
-    for kernel in (1, 2, 3, 4):
+    for kernel in (1, 2, 3, 4, 5):
         o = _abi.wkv_options(kernel=kernel)
         assert L.wkv_forward_kernel(2, 500, 64, F32, ctypes.byref(o)) == kernel
-        assert L.wkv_forward_kernel(2, 500, 65, F32, ctypes.byref(o)) == (2 if kernel in (3, 4) else kernel)
+        assert L.wkv_forward_kernel(2, 500, 65, F32, ctypes.byref(o)) == (2 if kernel in (3, 4, 5) else kernel)
+    # the cluster scan holds at most 8 CTAs x cta_warps x span tokens
+    o = _abi.wkv_options(kernel=5, cta_warps=4, span=16)
+    assert L.wkv_forward_kernel(2, 512, 64, F32, ctypes.byref(o)) == 5
+    assert L.wkv_forward_kernel(2, 513, 64, F32, ctypes.byref(o)) == 0
+    for bad in (dict(cta_warps=3), dict(cta_warps=32), dict(span=8)):
+        o = _abi.wkv_options(kernel=5, **bad)
+        assert L.wkv_forward_kernel(2, 100, 64, F32, ctypes.byref(o)) == 0
+    assert L.wkv_forward_launches(8, 1024, 768, F32, None) == 1
+    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 3
+    assert L.wkv_forward_launches(2, 20, 64, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 2
+    assert L.wkv_forward_launches(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(-1, 4, 4, F32, None) == 0
     assert L.wkv_forward_kernel(1, 4, 4, 9, None) == 0
     o = _abi.wkv_options(kernel=4, stages=1)
@@ -133,8 +149,18 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, sin=ctypes.byref(bad_state)) == _abi.WKV_ERR_INVALID_ARG
     bad_out = _abi.wkv_state(0x1000, 0x1000, None)
     assert fwd(L, sout=ctypes.byref(bad_out)) == _abi.WKV_ERR_INVALID_ARG
-    o = _abi.wkv_options(kernel=5)
+    o = _abi.wkv_options(kernel=6)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    o = _abi.wkv_options(kernel=5, cta_warps=5)
+    assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
+    # per-token decays with a look-back kernel, or without w_t and without w
+    ext = _abi.wkv_ext(0x2000, None)
+    for kernel in (2, 4):
+        o = _abi.wkv_options(kernel=kernel)
+        assert L.wkv_forward_ext(1, 4, 8, FAKE, FAKE, 0, FAKE, FAKE, FAKE, 0, None, None, ctypes.c_void_p(0x100000),
+                                 1 << 20, None, ctypes.byref(o), ctypes.byref(ext)) == _abi.WKV_ERR_INVALID_ARG
+    assert L.wkv_forward_ext(1, 4, 8, FAKE, FAKE, 0, None, FAKE, FAKE, 0, None, None, ctypes.c_void_p(0x100000),
+                             1 << 20, None, None, None) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(kernel=4, chunk_len=128, span=8)  # 16 warps per role: too many
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     for bad_stages in (1, 9, -1):

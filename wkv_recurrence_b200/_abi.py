@@ -23,8 +23,9 @@ WKV_F32 = 0
 WKV_BF16 = 1
 
 # entry points declared in include/wkv.h
-EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward_launches", "wkv_forward", "wkv_step", "wkv_query_status",
-           "wkv_status_string", "wkv_version", "wkv_forward_noalloc", "wkv_last_cuda_error")
+EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward_launches", "wkv_forward",
+           "wkv_forward_ext", "wkv_step", "wkv_step_ext", "wkv_query_status", "wkv_status_string", "wkv_version",
+           "wkv_forward_noalloc", "wkv_last_cuda_error")
 
 # size of the library's built-in scratch array used by wkv_forward_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -44,7 +45,12 @@ class wkv_options(ctypes.Structure):
                 ("wait_timeout_ns", ctypes.c_int64), ("inject_unpublished_tile", ctypes.c_int64),
                 ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32),
                 ("scan_segments", ctypes.c_int32), ("stages", ctypes.c_int32),
-                ("seq_vec", ctypes.c_int32), ("replay_chunks", ctypes.c_int32)]
+                ("seq_vec", ctypes.c_int32), ("replay_chunks", ctypes.c_int32),
+                ("cta_warps", ctypes.c_int32)]
+
+
+class wkv_ext(ctypes.Structure):
+    _fields_ = [("w_t", ctypes.c_void_p), ("r", ctypes.c_void_p)]
 
 
 class WkvError(RuntimeError):
@@ -80,6 +86,14 @@ def lib() -> ctypes.CDLL:
         L.wkv_step.argtypes = [I64, I64, P, P, I, P, P, P, I,
                                ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P]
         L.wkv_step.restype = I
+        L.wkv_forward_ext.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
+                                      ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state),
+                                      P, SZ, P, ctypes.POINTER(wkv_options), ctypes.POINTER(wkv_ext)]
+        L.wkv_forward_ext.restype = I
+        L.wkv_step_ext.argtypes = [I64, I64, P, P, I, P, P, P, I,
+                                   ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P,
+                                   ctypes.POINTER(wkv_ext)]
+        L.wkv_step_ext.restype = I
         L.wkv_forward_noalloc.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
                                           ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P]
         L.wkv_forward_noalloc.restype = I

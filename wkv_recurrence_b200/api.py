@@ -103,25 +103,44 @@ def _default_workspace(nbytes: int, device: torch.device) -> torch.Tensor:
     return ws
 
 
-def forward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+def _ext(w_t: Optional[torch.Tensor], r: Optional[torch.Tensor], shape, kv_dtype):
+    """The wkv_ext struct for optional per-token decays and receptance, or None."""
+    if w_t is None and r is None:
+        return None
+    if w_t is not None:
+        _need_cuda(w_t, "w_t", torch.float32)
+        if tuple(w_t.shape) != tuple(shape):
+            raise ValueError(f"w_t must be {tuple(shape)}")
+    if r is not None:
+        _need_cuda(r, "r", kv_dtype)
+        if tuple(r.shape) != tuple(shape):
+            raise ValueError(f"r must be {tuple(shape)}")
+    return _abi.wkv_ext(None if w_t is None else w_t.data_ptr(), None if r is None else r.data_ptr())
+
+
+def forward(k: torch.Tensor, v: torch.Tensor, w: Optional[torch.Tensor], u: torch.Tensor,
             state: Optional[State] = None, *, out_dtype: Optional[torch.dtype] = None,
             out: Optional[torch.Tensor] = None, state_out: Optional[State] = None,
             workspace: Optional[torch.Tensor] = None, options: Optional[dict] = None,
-            return_state: bool = True):
+            return_state: bool = True, w_t: Optional[torch.Tensor] = None, r: Optional[torch.Tensor] = None):
     """WKV over a sequence. k, v: [B, T, C] (float32 or bfloat16); w, u: [C] float32.
 
     state: optional (num, den, max_e), each float32 [B, C]. Returns
     (out [B, T, C], (num, den, max_e)) -- the state after the last token.
+    w_t: optional float32 [B, T, C] per-token decays in place of w (w may then
+    be None). r: optional receptance [B, T, C] (dtype of k): out = sigmoid(r) wkv.
     """
     _need_cuda(k, "k")
     _need_cuda(v, "v", k.dtype)
-    _need_cuda(w, "w", torch.float32)
+    if w_t is None or w is not None:
+        _need_cuda(w, "w", torch.float32)
     _need_cuda(u, "u", torch.float32)
     if k.dim() != 3 or v.shape != k.shape:
         raise ValueError("k and v must both be [B, T, C]")
     B, T, C = k.shape
-    if w.shape != (C,) or u.shape != (C,):
+    if (w is not None and w.shape != (C,)) or u.shape != (C,):
         raise ValueError("w and u must be [C]")
+    ext = _ext(w_t, r, (B, T, C), k.dtype)
     dev = k.device
     out_dtype = out_dtype or k.dtype
     if out is None:
@@ -148,31 +167,36 @@ def forward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
     if workspace is None:
         workspace = _default_workspace(need, dev)
     _need_cuda(workspace, "workspace")
-    code = _abi.lib().wkv_forward(
+    code = _abi.lib().wkv_forward_ext(
         B, T, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u),
         _ptr(out), _dtype_code(out, "out"),
         ctypes.byref(sin) if sin is not None else None,
         ctypes.byref(sout) if sout is not None else None,
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(), opts)
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(), opts,
+        ctypes.byref(ext) if ext is not None else None)
     _abi.check(code, "wkv_forward")
     return out, state_out
 
 
-def step(state: State, k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor, *,
+def step(state: State, k: torch.Tensor, v: torch.Tensor, w: Optional[torch.Tensor], u: torch.Tensor, *,
          out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
-         state_out: Optional[State] = None, inplace: bool = False):
+         state_out: Optional[State] = None, inplace: bool = False,
+         w_t: Optional[torch.Tensor] = None, r: Optional[torch.Tensor] = None):
     """One decode token for S streams. k, v: [S, C]; state: (num, den, max_e) [S, C].
 
     Returns (out [S, C], new state). With ``inplace=True`` the state tensors
-    are updated in place and returned.
+    are updated in place and returned. w_t: optional float32 [S, C] decays of
+    this token in place of w; r: optional receptance [S, C] (out = sigmoid(r) wkv).
     """
     _need_cuda(k, "k")
     _need_cuda(v, "v", k.dtype)
-    _need_cuda(w, "w", torch.float32)
+    if w_t is None or w is not None:
+        _need_cuda(w, "w", torch.float32)
     _need_cuda(u, "u", torch.float32)
     if k.dim() != 2 or v.shape != k.shape:
         raise ValueError("k and v must both be [S, C]")
     S, C = k.shape
+    ext = _ext(w_t, r, (S, C), k.dtype)
     for i, s in enumerate(state):
         _need_cuda(s, f"state[{i}]", torch.float32)
         if s.shape != (S, C):
@@ -187,9 +211,9 @@ def step(state: State, k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: tor
         state_out = tuple(torch.empty_like(s) for s in state)
     sin = _abi.wkv_cstate(*(s.data_ptr() for s in state))
     sout = _abi.wkv_state(*(s.data_ptr() for s in state_out))
-    code = _abi.lib().wkv_step(S, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u),
-                               _ptr(out), _dtype_code(out, "out"), ctypes.byref(sin),
-                               ctypes.byref(sout), _stream())
+    code = _abi.lib().wkv_step_ext(S, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u),
+                                   _ptr(out), _dtype_code(out, "out"), ctypes.byref(sin),
+                                   ctypes.byref(sout), _stream(), ctypes.byref(ext) if ext is not None else None)
     _abi.check(code, "wkv_step")
     return out, state_out
 
@@ -216,16 +240,18 @@ class PreparedForward:
     """
 
     def __init__(self, k, v, w, u, state=None, *, out, state_out=None, workspace=None,
-                 options: Optional[dict] = None):
+                 options: Optional[dict] = None, w_t=None, r=None):
         _need_cuda(k, "k")
         _need_cuda(v, "v", k.dtype)
-        _need_cuda(w, "w", torch.float32)
+        if w_t is None or w is not None:
+            _need_cuda(w, "w", torch.float32)
         _need_cuda(u, "u", torch.float32)
         B, T, C = k.shape
-        if v.shape != k.shape or w.shape != (C,) or u.shape != (C,) or out.shape != k.shape:
+        if v.shape != k.shape or (w is not None and w.shape != (C,)) or u.shape != (C,) or out.shape != k.shape:
             raise ValueError("shapes must be k, v, out [B, T, C] and w, u [C]")
         _need_cuda(out, "out")
-        self._keep = [k, v, w, u, out]
+        self._ext = _ext(w_t, r, (B, T, C), k.dtype)
+        self._keep = [k, v, w, u, out, w_t, r]
         self._sin = self._sout = None
         if state is not None:
             for i, s in enumerate(state):
@@ -251,7 +277,7 @@ class PreparedForward:
         _need_cuda(workspace, "workspace")
         self.workspace = workspace
         self._keep.append(workspace)
-        self._fn = _abi.lib().wkv_forward
+        self._fn = _abi.lib().wkv_forward_ext
         self._args = (B, T, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u), _ptr(out),
                       _dtype_code(out, "out"),
                       ctypes.byref(self._sin) if self._sin is not None else None,
@@ -259,9 +285,10 @@ class PreparedForward:
                       _ptr(workspace), workspace.numel() * workspace.element_size())
         self._stream = _stream()
         self._opts = opts
+        self._ext_ref = ctypes.byref(self._ext) if self._ext is not None else None
 
     def __call__(self, stream=None) -> None:
-        code = self._fn(*self._args, self._stream if stream is None else stream, self._opts)
+        code = self._fn(*self._args, self._stream if stream is None else stream, self._opts, self._ext_ref)
         if code:
             _abi.check(code, "wkv_forward")
 

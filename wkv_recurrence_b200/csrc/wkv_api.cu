@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "../../include/wkv.h"
+#include "wkv_cluster.cuh"
 #include "wkv_device.cuh"
 #include "wkv_fwd.cuh"
 #include "wkv_step.cuh"
@@ -40,7 +41,10 @@ constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 constexpr long long kSeqVec1MaxLanes = 148ll * 16 * 64;
 
 struct Plan {
-  int kernel;  // 1 seq, 2 chunked single launch, 3 chunked in three launches, 4 pipelined chunked
+  int kernel;  // 1 seq, 2 chunked single launch, 3 chunked in three launches, 4 pipelined chunked, 5 cluster
+  int cw;      // cluster scan: warps (spans) per CTA
+  int cj;      // cluster scan: tokens per span
+  int ncl;     // cluster scan: CTAs per cluster
   int seq_threads;  // CTA width of the sequential kernel
   int seq_vec;      // channels per thread of the sequential kernel
   int scan_segments;  // three-launch scan: segments per channel in the scan of chunk totals
@@ -54,7 +58,7 @@ struct Plan {
   int nch;     // chunks per sequence
   long long n_tiles;
   long long nblk;  // look-back groups per sequence
-  size_t off_flags_a, off_flags_p, off_agg_a, off_agg_p, off_x0, bytes;
+  size_t off_flags_a, off_flags_p, off_agg_a, off_agg_p, off_x0, off_wtot, bytes;
 };
 
 
@@ -80,24 +84,41 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // which need TMA, into the single-launch one (the pipelined scan uses the same
 // workspace layout as the single-launch one). A three-launch plan reserves enough workspace
 // for either, so a workspace sized by wkv_forward_workspace_size always fits.
-bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, bool tma_ok = true) {
+bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, bool tma_ok = true,
+               bool wt = false) {
   std::memset(pl, 0, sizeof *pl);
   const int want = o ? o->kernel : 0;
-  if (want < 0 || want > 4) return false;
+  if (want < 0 || want > 5) return false;
   const int64_t lanes = B * C;
+  // the cluster scan's CTA shape: cw spans of cj tokens per CTA, up to 8 CTAs
+  if (o && o->cta_warps != 0 && o->cta_warps != 4 && o->cta_warps != 8 && o->cta_warps != 16) return false;
+  const int cw = (o && o->cta_warps) ? o->cta_warps : 8;
+  const int cj = (want == 5 && o && o->span) ? o->span : 32;
+  if (cj != 16 && cj != 32) return false;
+  const int64_t cluster_tokens = 8ll * cw * cj;
   int kernel = want;
   if (kernel == 0) {
     if (lanes >= 65536 || T <= 64) {
       kernel = 1;
+    } else if (T <= cluster_tokens) {
+      // the whole sequence of a channel group fits in one cluster's shared
+      // memory: one launch, one read of k and v
+      kernel = 5;
     } else {
       // chunked: the three-launch scan (measured: layer 27 vs 29 us single
       // launch; long 465 vs 603 us pipelined, 636 us single launch)
       kernel = 3;
     }
   }
+  // per-token decays: the sequential, three-launch and cluster kernels only
+  if (wt && (kernel == 2 || kernel == 4)) return false;
+  if (kernel == 5 && T > cluster_tokens) return false;
   const bool three_requested = (kernel == 3);
-  if ((kernel == 3 || kernel == 4) && !tma_ok) kernel = 2;
+  if ((kernel == 3 || kernel == 4 || kernel == 5) && !tma_ok) kernel = wt ? 1 : 2;
   pl->kernel = kernel;
+  pl->cw = cw;
+  pl->cj = cj;
+  pl->ncl = (int)std::max<int64_t>(1, (T + (int64_t)cw * cj - 1) / ((int64_t)cw * cj));
   pl->bytes = sizeof(WsHeader);
   if (o && o->scan_segments != 0 && o->scan_segments != 1 && o->scan_segments != 4 && o->scan_segments != 16 &&
       o->scan_segments != 64)
@@ -118,6 +139,24 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   if (sth != 32 && sth != 64 && sth != 128) return false;
   pl->seq_threads = sth;
   if (kernel == 1) return true;
+  if (kernel == 5) {
+    // the header only; but a call whose k or v TMA cannot address falls back
+    // to the single-launch scan (or, with per-token decays, the sequential
+    // kernel), so reserve that kernel's layout too
+    pl->bytes = sizeof(WsHeader);
+    if (!wt) {
+      wkv_options o2;
+      std::memset(&o2, 0, sizeof o2);
+      if (o) o2 = *o;
+      o2.kernel = 2;
+      o2.span = 0;
+      o2.chunk_len = 0;
+      Plan p2;
+      if (!make_plan(B, T, C, &o2, &p2, true, false)) return false;
+      pl->bytes = std::max(pl->bytes, p2.bytes);
+    }
+    return true;
+  }
 
   int L = o ? o->chunk_len : 0;
   if (L == 0) {
@@ -135,6 +174,7 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   int J = o ? o->span : 0;
   if (J == 0) J = 16;
   if (J != 8 && J != 16) return false;
+  if (wt && kernel == 3 && J != 16) return false;  // per-token decays: 16-token spans
   // the pipelined scan runs L/J fold and L/J replay warps plus two: at most 8
   // of each keeps the CTA within 1024 threads
   if (kernel == 4 && L / J > 8) return false;
@@ -161,6 +201,9 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   off3 = round_up(off3 + sizeof(float4) * (size_t)(std::max(pl->nch - 1, 0) * BNG) * kChunkCG, 256);
   const size_t t_x0 = off3;
   off3 = round_up(off3 + sizeof(float4) * (size_t)pl->n_tiles * kChunkCG, 256);
+  // with per-token decays, the decay sum of each chunk total
+  const size_t t_w = off3;
+  off3 = round_up(off3 + sizeof(float) * (size_t)(std::max(pl->nch - 1, 0) * BNG) * kChunkCG, 256);
   // single-launch layout: flags, chunk totals, group prefixes
   size_t off = sizeof(WsHeader);
   pl->off_flags_a = off;
@@ -175,6 +218,7 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     pl->off_flags_a = pl->off_flags_p = pl->off_agg_p = 0;
     pl->off_agg_a = t_tot;
     pl->off_x0 = t_x0;
+    pl->off_wtot = t_w;
     pl->bytes = std::max(off3, off);
   } else {
     pl->bytes = three_requested ? std::max(off3, off) : off;
@@ -327,18 +371,19 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-template <typename KV, typename OUT, int THREADS, int VEC, int LT, int STAGES, bool kTMA>
-wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st, int dev) {
+template <typename KV, typename OUT, int THREADS, int VEC, int LT, int STAGES, bool kTMA, bool kWT = false>
+wkv_status launch_seq(const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tw,
+                      cudaStream_t st, int dev) {
   constexpr int CG = THREADS * VEC;
-  const size_t smem = (size_t)STAGES * 2 * LT * CG * sizeof(KV) + 64 * STAGES;
-  auto fn = wkv_fwd_seq<KV, OUT, VEC, THREADS, LT, STAGES, kTMA, false>;
+  const size_t smem = (size_t)STAGES * seq_stage_bytes<KV, LT, CG, kWT>() + 64 * STAGES;
+  auto fn = wkv_fwd_seq<KV, OUT, VEC, THREADS, LT, STAGES, kTMA, false, kWT>;
   int occ = 0;
   if (!kernel_setup(fn, dev, THREADS, smem, &occ)) return WKV_ERR_CUDA;
   FwdParams q = p;
   q.NG = (p.C + CG - 1) / CG;
   const long long grid = (long long)p.B * q.NG;
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  fn<<<(unsigned)grid, THREADS, smem, st>>>(q, tk, tv);
+  fn<<<(unsigned)grid, THREADS, smem, st>>>(q, tk, tv, tw);
   return launch_result();
 }
 
@@ -417,33 +462,37 @@ struct PdlConfig {
 // The replay pass of the three-launch scan: the sequential kernel in chunked
 // mode, one warp per (batch row, chunk, 32 channels), launched with
 // programmatic stream serialization after the scan.
-template <typename KV, typename OUT, int TH, int LT, int STAGES>
+template <typename KV, typename OUT, int TH, int LT, int STAGES, bool kWT = false>
 wkv_status launch_seq_chunks(const FwdParams& p, const CUtensorMap& bk, const CUtensorMap& bv, cudaStream_t st,
-                             int dev) {
-  auto fb = wkv_fwd_seq<KV, OUT, 1, TH, LT, STAGES, true, true>;
-  const size_t smem = (size_t)STAGES * 2 * LT * TH * sizeof(KV) + 64 * STAGES;
+                             int dev, const CUtensorMap* bw = nullptr) {
+  auto fb = wkv_fwd_seq<KV, OUT, 1, TH, LT, STAGES, true, true, kWT>;
+  const size_t smem = (size_t)STAGES * seq_stage_bytes<KV, LT, TH, kWT>() + 64 * STAGES;
   int occ = 0;
   if (!kernel_setup(fb, dev, TH, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
   const long long nseq = (p.nch + p.replay_chunks - 1) / p.replay_chunks;
   const long long grid = (long long)p.B * nseq * ((p.C + TH - 1) / TH);
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
   PdlConfig cb(dim3((unsigned)grid), dim3(TH), smem, st);
-  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv))) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv, bw ? *bw : bv))) return WKV_ERR_CUDA;
   return launch_result();
 }
 
-template <typename KV, typename OUT, int NW, int J>
+template <typename KV, typename OUT, int NW, int J, bool kWT>
 wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                         wkv_dtype kvdt, cudaStream_t st, int dev) {
-  if (!p.agg_a || !p.x0 || !p.hdr) return WKV_ERR_INVALID_ARG;
+  if (!p.agg_a || !p.x0 || !p.hdr || (kWT && !p.wtot)) return WKV_ERR_INVALID_ARG;
   constexpr int L = NW * J;
-  const size_t smem = 2ull * L * kChunkCG * sizeof(KV) + sizeof(float4) * NW * kChunkCG + 64;
-  auto fa = wkv_tile_totals<KV, NW, J>;
+  CUtensorMap tw;
+  std::memset(&tw, 0, sizeof tw);
+  if (kWT && !make_tmap(&tw, p.w_t, WKV_F32, p.B, p.T, p.C, L, kChunkCG)) return WKV_ERR_CUDA;
+  const size_t smem = 2ull * L * kChunkCG * sizeof(KV) + (kWT ? sizeof(float) * L * kChunkCG : 0) +
+                      sizeof(float4) * NW * kChunkCG + (kWT ? sizeof(float) * NW * kChunkCG : 0) + 64;
+  auto fa = wkv_tile_totals<KV, NW, J, kWT>;
   int occ = 0;
   if (!kernel_setup(fa, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
   const long long BNG = (long long)p.B * p.NG;
   if (p.nch > 1) {
-    fa<<<(unsigned)((p.nch - 1) * BNG), NW * 32, smem, st>>>(p, tk, tv);
+    fa<<<(unsigned)((p.nch - 1) * BNG), NW * 32, smem, st>>>(p, tk, tv, tw);
     if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   }
   // segments per channel in the scan: at most about 16 chunk totals each
@@ -458,19 +507,20 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   if (p.nch <= 1) cs.cfg.numAttrs = 0;
   cudaError_t e;
   switch (seg) {
-    case 1: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<1>, p, L); break;
-    case 4: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<4>, p, L); break;
-    case 16: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<16>, p, L); break;
-    default: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<64>, p, L); break;
+    case 1: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<1, kWT>, p, L); break;
+    case 4: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<4, kWT>, p, L); break;
+    case 16: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<16, kWT>, p, L); break;
+    default: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<64, kWT>, p, L); break;
   }
   if (!cuda_ok(e) || launch_result() != WKV_OK) return WKV_ERR_CUDA;
   // B: the sequential kernel over every (batch row, chunk, 32-channel group),
   // from the chunk's incoming state; one channel per thread
   constexpr bool kF32 = sizeof(KV) == 4;
   constexpr int LT = kF32 ? 2 * kSeqLtF32 : 2 * kSeqLtBf16;
-  // one channel per thread, replay_threads channels per CTA
-  const int th = pl.replay_threads;
-  CUtensorMap bk, bv;
+  // one channel per thread, replay_threads channels per CTA (32 with
+  // per-token decays)
+  const int th = kWT ? 32 : pl.replay_threads;
+  CUtensorMap bk, bv, bw;
   if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, th) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, th))
     return WKV_ERR_CUDA;
   // a replay of at most two stages is prefetched whole with 2 (more CTAs fit
@@ -478,41 +528,54 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   FwdParams q = p;
   q.replay_chunks = pl.replay_chunks;
   const bool two = pl.replay_chunks * L <= 2 * LT;
-  if (kF32 && pl.replay_chunks * L == 32 && th == 32) {
-    // a 32-token fp32 replay as one 32-token stage: one copy pair and one
-    // wait instead of two (layer: 23.5 against 23.8 us)
-    CUtensorMap ck, cv;
-    if (!make_tmap(&ck, p.k, kvdt, p.B, p.T, p.C, 32, th) || !make_tmap(&cv, p.v, kvdt, p.B, p.T, p.C, 32, th))
-      return WKV_ERR_CUDA;
-    return launch_seq_chunks<KV, OUT, 32, 32, 1>(q, ck, cv, st, dev);
-  }
-  switch (th) {
-    case 64:
-      return two ? launch_seq_chunks<KV, OUT, 64, LT, 2>(q, bk, bv, st, dev)
-                 : launch_seq_chunks<KV, OUT, 64, LT, 3>(q, bk, bv, st, dev);
-    case 128:
-      return two ? launch_seq_chunks<KV, OUT, 128, LT, 2>(q, bk, bv, st, dev)
-                 : launch_seq_chunks<KV, OUT, 128, LT, 3>(q, bk, bv, st, dev);
-    default:
-      return two ? launch_seq_chunks<KV, OUT, 32, LT, 2>(q, bk, bv, st, dev)
-                 : launch_seq_chunks<KV, OUT, 32, LT, 3>(q, bk, bv, st, dev);
+  if (kWT) {
+    if (!make_tmap(&bw, p.w_t, WKV_F32, p.B, p.T, p.C, LT, th)) return WKV_ERR_CUDA;
+    return two ? launch_seq_chunks<KV, OUT, 32, LT, 2, true>(q, bk, bv, st, dev, &bw)
+               : launch_seq_chunks<KV, OUT, 32, LT, 3, true>(q, bk, bv, st, dev, &bw);
+  } else {
+    if (kF32 && pl.replay_chunks * L == 32 && th == 32) {
+      // a 32-token fp32 replay as one 32-token stage: one copy pair and one
+      // wait instead of two (layer: 23.5 against 23.8 us)
+      CUtensorMap ck, cv;
+      if (!make_tmap(&ck, p.k, kvdt, p.B, p.T, p.C, 32, th) || !make_tmap(&cv, p.v, kvdt, p.B, p.T, p.C, 32, th))
+        return WKV_ERR_CUDA;
+      return launch_seq_chunks<KV, OUT, 32, 32, 1>(q, ck, cv, st, dev);
+    }
+    switch (th) {
+      case 64:
+        return two ? launch_seq_chunks<KV, OUT, 64, LT, 2>(q, bk, bv, st, dev)
+                   : launch_seq_chunks<KV, OUT, 64, LT, 3>(q, bk, bv, st, dev);
+      case 128:
+        return two ? launch_seq_chunks<KV, OUT, 128, LT, 2>(q, bk, bv, st, dev)
+                   : launch_seq_chunks<KV, OUT, 128, LT, 3>(q, bk, bv, st, dev);
+      default:
+        return two ? launch_seq_chunks<KV, OUT, 32, LT, 2>(q, bk, bv, st, dev)
+                   : launch_seq_chunks<KV, OUT, 32, LT, 3>(q, bk, bv, st, dev);
+    }
   }
 }
 
 template <typename KV, typename OUT>
 wkv_status launch_tile3_shape(const Plan& pl, const FwdParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                               wkv_dtype kvdt, cudaStream_t st, int dev) {
+  if (p.w_t) {  // make_plan takes 16-token spans with per-token decays
+    switch (pl.L) {
+      case 32: return launch_tile3<KV, OUT, 2, 16, true>(pl, p, tk, tv, kvdt, st, dev);
+      case 64: return launch_tile3<KV, OUT, 4, 16, true>(pl, p, tk, tv, kvdt, st, dev);
+      default: return launch_tile3<KV, OUT, 8, 16, true>(pl, p, tk, tv, kvdt, st, dev);
+    }
+  }
   if (pl.J == 8) {
     switch (pl.L) {
-      case 32: return launch_tile3<KV, OUT, 4, 8>(pl, p, tk, tv, kvdt, st, dev);
-      case 64: return launch_tile3<KV, OUT, 8, 8>(pl, p, tk, tv, kvdt, st, dev);
-      default: return launch_tile3<KV, OUT, 16, 8>(pl, p, tk, tv, kvdt, st, dev);
+      case 32: return launch_tile3<KV, OUT, 4, 8, false>(pl, p, tk, tv, kvdt, st, dev);
+      case 64: return launch_tile3<KV, OUT, 8, 8, false>(pl, p, tk, tv, kvdt, st, dev);
+      default: return launch_tile3<KV, OUT, 16, 8, false>(pl, p, tk, tv, kvdt, st, dev);
     }
   }
   switch (pl.L) {
-    case 32: return launch_tile3<KV, OUT, 2, 16>(pl, p, tk, tv, kvdt, st, dev);
-    case 64: return launch_tile3<KV, OUT, 4, 16>(pl, p, tk, tv, kvdt, st, dev);
-    default: return launch_tile3<KV, OUT, 8, 16>(pl, p, tk, tv, kvdt, st, dev);
+    case 32: return launch_tile3<KV, OUT, 2, 16, false>(pl, p, tk, tv, kvdt, st, dev);
+    case 64: return launch_tile3<KV, OUT, 4, 16, false>(pl, p, tk, tv, kvdt, st, dev);
+    default: return launch_tile3<KV, OUT, 8, 16, false>(pl, p, tk, tv, kvdt, st, dev);
   }
 }
 
@@ -548,9 +611,73 @@ wkv_status launch_seq_tma(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cu
   if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, cg) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, cg))
     return WKV_ERR_CUDA;
   switch (pl.seq_threads) {
-    case 32: return launch_seq<KV, OUT, 32, VEC, LT, STG, true>(p, tk, tv, st, dev);
-    case 64: return launch_seq<KV, OUT, 64, VEC, LT, STG, true>(p, tk, tv, st, dev);
-    default: return launch_seq<KV, OUT, 128, VEC, LT, STG, true>(p, tk, tv, st, dev);
+    case 32: return launch_seq<KV, OUT, 32, VEC, LT, STG, true>(p, tk, tv, tv, st, dev);
+    case 64: return launch_seq<KV, OUT, 64, VEC, LT, STG, true>(p, tk, tv, tv, st, dev);
+    default: return launch_seq<KV, OUT, 128, VEC, LT, STG, true>(p, tk, tv, tv, st, dev);
+  }
+}
+
+// The sequential kernel with per-token decays: one channel per thread,
+// 32-thread CTAs, k, v and w_t in TMA-fed stages of 16 (fp32) or 32 (bf16)
+// tokens, 3 stages.
+template <typename KV, typename OUT>
+wkv_status launch_seq_tma_wt(const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
+  constexpr bool kF32 = sizeof(KV) == 4;
+  constexpr int LT = kF32 ? 2 * kSeqLtF32 : 2 * kSeqLtBf16;
+  CUtensorMap tk, tv, tw;
+  if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, LT, 32) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, LT, 32) ||
+      !make_tmap(&tw, p.w_t, WKV_F32, p.B, p.T, p.C, LT, 32))
+    return WKV_ERR_CUDA;
+  return launch_seq<KV, OUT, 32, 1, LT, 3, true, true>(p, tk, tv, tw, st, dev);
+}
+
+// The cluster scan: one cluster of pl.ncl CTAs per (batch row, 32 channels),
+// k, v (and w_t) copied in by TMA in boxes of one span (J tokens x 32 channels).
+template <typename KV, typename OUT, int NW, int J, bool kWT>
+wkv_status launch_cluster(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
+  CUtensorMap tk, tv, tw;
+  std::memset(&tw, 0, sizeof tw);
+  if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, J, 32) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, J, 32))
+    return WKV_ERR_CUDA;
+  if (kWT && !make_tmap(&tw, p.w_t, WKV_F32, p.B, p.T, p.C, J, 32)) return WKV_ERR_CUDA;
+  constexpr size_t smem = cluster_smem_bytes<KV, NW, J, kWT>();
+  auto fn = wkv_fwd_cluster<KV, OUT, NW, J, kWT>;
+  int occ = 0;
+  if (!kernel_setup(fn, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  FwdParams q = p;
+  q.cluster = pl.ncl;
+  const long long items = (long long)p.B * ((p.C + 31) / 32);
+  const long long grid = items * pl.ncl;
+  if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)pl.ncl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!cuda_ok(cudaLaunchKernelEx(&cfg, fn, q, tk, tv, tw))) return WKV_ERR_CUDA;
+  return launch_result();
+}
+
+template <typename KV, typename OUT, bool kWT>
+wkv_status launch_cluster_shape(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
+  if (pl.cj == 16) {
+    switch (pl.cw) {
+      case 4: return launch_cluster<KV, OUT, 4, 16, kWT>(pl, p, kvdt, st, dev);
+      case 16: return launch_cluster<KV, OUT, 16, 16, kWT>(pl, p, kvdt, st, dev);
+      default: return launch_cluster<KV, OUT, 8, 16, kWT>(pl, p, kvdt, st, dev);
+    }
+  }
+  switch (pl.cw) {
+    case 4: return launch_cluster<KV, OUT, 4, 32, kWT>(pl, p, kvdt, st, dev);
+    case 16: return launch_cluster<KV, OUT, 16, 32, kWT>(pl, p, kvdt, st, dev);
+    default: return launch_cluster<KV, OUT, 8, 32, kWT>(pl, p, kvdt, st, dev);
   }
 }
 
@@ -560,12 +687,21 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
   CUtensorMap tk, tv;
   std::memset(&tk, 0, sizeof tk);
   std::memset(&tv, 0, sizeof tv);
+  if (pl.kernel == 5) {
+    return p.w_t ? launch_cluster_shape<KV, OUT, true>(pl, p, kvdt, st, dev)
+                 : launch_cluster_shape<KV, OUT, false>(pl, p, kvdt, st, dev);
+  }
   if (pl.kernel == 1) {
+    if (p.w_t) {
+      // per-token decays: one channel per thread, 32-thread CTAs
+      if (tma) return launch_seq_tma_wt<KV, OUT>(p, kvdt, st, dev);
+      return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false, true>(p, tk, tv, tv, st, dev);
+    }
     if (tma) {
       if (pl.seq_vec == 1) return launch_seq_tma<KV, OUT, 1>(pl, p, kvdt, st, dev);
       return launch_seq_tma<KV, OUT, 2>(pl, p, kvdt, st, dev);
     }
-    return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false>(p, tk, tv, st, dev);
+    return launch_seq<KV, OUT, 128, kSeqFallbackVec, kSeqFallbackLt, 1, false, false>(p, tk, tv, tv, st, dev);
   }
   if (pl.kernel == 3) {  // three launches (make_plan only chooses it when TMA works)
     if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, pl.L, kChunkCG) ||
@@ -639,19 +775,23 @@ int32_t wkv_forward_launches(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype
   return 1;
 }
 
-wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
-                       const float* w, const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
-                       const wkv_state* state_out, void* workspace, size_t workspace_bytes, void* stream,
-                       const wkv_options* opts) {
+wkv_status wkv_forward_ext(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
+                           const float* w, const float* u, void* out, wkv_dtype out_dtype,
+                           const wkv_cstate* state_in, const wkv_state* state_out, void* workspace,
+                           size_t workspace_bytes, void* stream, const wkv_options* opts, const wkv_ext* ext) {
+  const float* w_t = ext ? ext->w_t : nullptr;
+  const void* r = ext ? ext->r : nullptr;
   // ---- argument checks: nothing is launched before they pass
-  const wkv_status chk = check_forward_args(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, opts);
+  const wkv_status chk =
+      check_forward_args(B, T, C, k, v, kv_dtype, w_t ? u : w, u, out, out_dtype, state_in, state_out, opts);
   if (chk != WKV_OK) return chk;
+  if (B * T * C > 0 && (w_t || r) && !aligned(w_t ? (const void*)w_t : r, 4)) return WKV_ERR_INVALID_ARG;
   const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
   // TMA needs 16-byte aligned bases and row pitches; otherwise the kernels
   // fill their tiles with plain loads
-  const bool tma = tma_usable(k, v, C, kes);
+  const bool tma = tma_usable(k, v, C, kes) && (!w_t || tma_usable(w_t, w_t, C, 4));
   Plan pl;
-  if (!make_plan(B, T, C, opts, &pl, tma)) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, opts, &pl, tma, w_t != nullptr)) return WKV_ERR_INVALID_ARG;
   if (!workspace) return WKV_ERR_INVALID_ARG;
   if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
@@ -690,6 +830,8 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   p.w = w;
   p.u = u;
   p.out = out;
+  p.w_t = w_t;
+  p.r = r;
   if (state_in) {
     p.s_num = state_in->num;
     p.s_den = state_in->den;
@@ -717,6 +859,7 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
     if (pl.kernel == 3) {
       p.flags_a = p.flags_p = nullptr;
       p.x0 = reinterpret_cast<float4*>(ws + pl.off_x0);
+      p.wtot = reinterpret_cast<float*>(ws + pl.off_wtot);
     }
   }
   const size_t oes = out_dtype == WKV_F32 ? 4 : 2;
@@ -732,9 +875,19 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const voi
   return dispatch_forward<__nv_bfloat16, float>(pl, p, tma, kv_dtype, st, dev, di);
 }
 
-wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype, const float* w,
-                    const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
-                    const wkv_state* state_out, void* stream) {
+wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
+                       const float* w, const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
+                       const wkv_state* state_out, void* workspace, size_t workspace_bytes, void* stream,
+                       const wkv_options* opts) {
+  return wkv_forward_ext(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, workspace,
+                         workspace_bytes, stream, opts, nullptr);
+}
+
+wkv_status wkv_step_ext(int64_t S, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype, const float* w,
+                        const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
+                        const wkv_state* state_out, void* stream, const wkv_ext* ext) {
+  const float* w_t = ext ? ext->w_t : nullptr;
+  const void* r = ext ? ext->r : nullptr;
   if (S < 0 || C < 0) return WKV_ERR_INVALID_ARG;
   if (S > 0 && C > (int64_t)((1ull << 62) / (uint64_t)S)) return WKV_ERR_INVALID_ARG;
   if (C >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
@@ -746,7 +899,7 @@ wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtyp
   if (!state_out->num || !state_out->den || !state_out->max_e) return WKV_ERR_INVALID_ARG;
   const int64_t n = S * C;
   if (n == 0) return WKV_OK;
-  if (!k || !v || !w || !u || !out) return WKV_ERR_INVALID_ARG;
+  if (!k || !v || (!w && !w_t) || !u || !out) return WKV_ERR_INVALID_ARG;
 
   StepParams p;
   p.n = n;
@@ -762,12 +915,15 @@ wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtyp
   p.o_num = state_out->num;
   p.o_den = state_out->den;
   p.o_max = state_out->max_e;
+  p.w_t = w_t;
+  p.r = r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t kes = kv_dtype == WKV_F32 ? 4 : 2, oes = out_dtype == WKV_F32 ? 4 : 2;
   constexpr int VEC = 4;
   const bool vec = (C % VEC) == 0 && aligned(k, kes * VEC) && aligned(v, kes * VEC) && aligned(out, oes * VEC) &&
-                   aligned(w, 16) && aligned(u, 16) && aligned(p.s_num, 16) && aligned(p.s_den, 16) &&
-                   aligned(p.s_max, 16) && aligned(p.o_num, 16) && aligned(p.o_den, 16) && aligned(p.o_max, 16);
+                   (w_t ? aligned(w_t, 16) : aligned(w, 16)) && (!r || aligned(r, kes * VEC)) && aligned(u, 16) &&
+                   aligned(p.s_num, 16) && aligned(p.s_den, 16) && aligned(p.s_max, 16) && aligned(p.o_num, 16) &&
+                   aligned(p.o_den, 16) && aligned(p.o_max, 16);
   const int per = vec ? VEC : 1;
   const long long threads = (n + per - 1) / per;
   const unsigned blocks = (unsigned)((threads + 255) / 256);
@@ -782,6 +938,12 @@ wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtyp
     else wkv_step_kernel<__nv_bfloat16, float, 1><<<blocks, 256, 0, st>>>(p);
   }
   return launch_result();
+}
+
+wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype, const float* w,
+                    const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
+                    const wkv_state* state_out, void* stream) {
+  return wkv_step_ext(S, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, stream, nullptr);
 }
 
 wkv_status wkv_query_status(void* workspace, void* stream) {

@@ -444,6 +444,107 @@ __device__ __forceinline__ Acc acc_from_state(float num, float den, float max_e)
   return Acc{num, den, max_e, 0.f};
 }
 
+// ---------------------------------------------------------------------------
+// Per-token decay w_t ("RWKV-v6 Architecture", section "2. Dynamic
+// Data-Dependent Decay"): the decay since the anchor is no longer count * w but
+// a running sum of the tokens' decays. Acc.nf then holds that sum, and sums
+// over many tokens are compensated (the rounding error of each addition is
+// carried separately, Knuth's TwoSum), so that a long memory of small decays
+// does not drift the way a plain fp32 running sum would.
+// ---------------------------------------------------------------------------
+
+// hi + lo = a + b exactly, hi = fl(a + b) (Knuth's TwoSum, no precondition on
+// the magnitudes)
+__device__ __forceinline__ void two_sum(float a, float b, float& hi, float& lo) {
+  hi = a + b;
+  const float bp = hi - a;
+  lo = (a - (hi - bp)) + (b - bp);
+}
+
+// Combine with per-token decays: `b` covers tokens whose decays sum to w_b, so
+// `a` is decayed by w_b across them. Same structure as combine().
+__device__ __forceinline__ Acc combine_wt(const Acc& a, const Acc& b, float w_b) {
+  const float na = a.nf + w_b;
+  const float d = (a.ma - b.ma) - (na - b.nf);
+  const bool a_wins = d >= 0.f;
+  const float s = ex2(-fabsf(d) * kLog2e);
+  Acc r;
+  r.num = a_wins ? fmaf(s, b.num, a.num) : fmaf(s, a.num, b.num);
+  r.den = a_wins ? fmaf(s, b.den, a.den) : fmaf(s, a.den, b.den);
+  r.ma = a_wins ? a.ma : b.ma;
+  r.nf = a_wins ? na : b.nf;
+  return r;
+}
+
+// One token with its own decay wt: output from the state before it (with the
+// bonus u), then the advance (decay by e^{-wt}, add the token without bonus).
+// `lo` carries the compensation of the running decay sum s.nf; it is reset
+// with the anchor.
+__device__ __forceinline__ float step_token_wt(Acc& s, float& lo, float k, float v, float wt, float u) {
+  // output: the undecayed state (exponent ma - nf - lo) against k + u
+  const float M = (s.ma - s.nf) - lo;
+  const float D = (k + u) - M;
+  const float beta = ex2(fminf(D, kBonusClamp) * kLog2e);
+  const float out = fmaf(beta, v, s.num) * rcp(s.den + beta);
+  // advance
+  float hi, e;
+  two_sum(s.nf, wt, hi, e);
+  const float lo1 = lo + e;
+  const float Md = (s.ma - hi) - lo1;
+  const float D2 = k - Md;
+  const float x = ex2(-fabsf(D2) * kLog2e);
+  const bool reset = D2 > 0.f;
+  const float a = reset ? x : 1.f;
+  const float b = reset ? 1.f : x;
+  s.num = fmaf(a, s.num, b * v);
+  s.den = fmaf(a, s.den, b);
+  s.ma = reset ? k : s.ma;
+  s.nf = reset ? 0.f : hi;
+  lo = reset ? 0.f : lo1;
+  return out;
+}
+
+// The state's max exponent with per-token decays (ma - nf, and the
+// compensation of nf).
+__device__ __forceinline__ float acc_max_e_wt(const Acc& s, float lo) { return (s.ma - s.nf) - lo; }
+
+// ---------------------------------------------------------------------------
+// The receptance gate of the Time-Mixing block: y = sigmoid(r) * wkv.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float gate(float y, float r) { return y * rcp(1.f + ex2(-r * kLog2e)); }
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, barrier, and loads from another CTA's shared
+// memory (distributed shared memory).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// (the non-.aligned forms: callers need not be converged)
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+// shared-memory address of the same variable in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t map_shared_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float4 acc_pack(const Acc& s) { return make_float4(s.num, s.den, s.ma, s.nf); }
 __device__ __forceinline__ Acc acc_unpack(const float4& f) { return Acc{f.x, f.y, f.z, f.w}; }
 

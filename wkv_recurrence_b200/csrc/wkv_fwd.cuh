@@ -78,6 +78,10 @@ struct FwdParams {
   int chunk_len;       // chunked scans: tokens per chunk
   int stages;          // pipelined chunk scan: shared-memory stages in the ring
   int replay_chunks;   // three-launch scan: consecutive chunks per replay CTA
+  int cluster;         // cluster kernel: CTAs per cluster
+  const float* w_t;    // per-token decay [B, T, C] in place of w, or NULL
+  const void* r;       // receptance [B, T, C] (element type of k, v): out = sigmoid(r) wkv; or NULL
+  float* wtot;         // three-launch scan with w_t: decay sum of each chunk total, [nch-1][B * NG][64]
 };
 
 // Programmatic dependent launch: let the next launch on the stream be
@@ -106,6 +110,25 @@ __device__ __forceinline__ void store_out(OUT* row, int c0, int C, bool vec_ok, 
   }
 }
 
+// The receptance gate on VEC outputs of one token row (out = sigmoid(r) wkv),
+// when the call has one: r is [B, T, C] with the element type of k and v;
+// `row` is the offset of (b, t, 0).
+template <typename KV, int VEC>
+__device__ __forceinline__ void gate_row(const FwdParams& p, size_t row, int c0, float (&o)[VEC]) {
+  if (!p.r) return;
+  const KV* rr = reinterpret_cast<const KV*>(p.r) + row;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e)
+    if (c0 + e < p.C) o[e] = gate(o[e], Elem<KV>::to_f32(rr[c0 + e]));
+}
+
+// Bytes of one shared-memory stage of the sequential kernel: LT tokens x CG
+// channels of k and v, and of w_t with per-token decays.
+template <typename KV, int LT, int CG, bool kWT>
+__host__ __device__ constexpr uint32_t seq_stage_bytes() {
+  return (uint32_t)(LT * CG * (2 * sizeof(KV) + (kWT ? sizeof(float) : 0)));
+}
+
 template <typename KV>
 __device__ __forceinline__ void coop_load_tile(KV* dst, const KV* src, int b, int t0, int rows, int cbase, int CG,
                                                int T, int C) {
@@ -129,15 +152,21 @@ __device__ __forceinline__ void coop_load_tile(KV* dst, const KV* src, int b, in
 // B * ceil(nch / R) * ceil(C / CG). It issues its first copies (inputs only)
 // before waiting (griddepcontrol.wait) for the scan, and only the CTA that
 // ends the sequence writes the state out.
-template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA, bool kChunked>
+template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA, bool kChunked,
+          bool kWT>
 __global__ void __launch_bounds__(THREADS)
-    wkv_fwd_seq(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    wkv_fwd_seq(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                const __grid_constant__ CUtensorMap tmw) {
   constexpr int CG = THREADS * VEC;
   constexpr int kTile = LT * CG;  // elements per tensor per stage
-  constexpr uint32_t kStageBytes = 2u * kTile * sizeof(KV);
+  constexpr uint32_t kStageBytes = seq_stage_bytes<KV, LT, CG, kWT>();
   extern __shared__ __align__(1024) unsigned char smem[];
-  KV* tiles = reinterpret_cast<KV*>(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
+  // stage s: k tile, v tile (KV), then the w_t tile (fp32)
+  auto ktile = [&](int s) { return reinterpret_cast<KV*>(smem + (size_t)s * kStageBytes); };
+  auto wtile = [&](int s) {
+    return reinterpret_cast<float*>(smem + (size_t)s * kStageBytes + 2 * kTile * sizeof(KV));
+  };
 
   const int tid = threadIdx.x;
   const int T = p.T, C = p.C;
@@ -153,28 +182,31 @@ __global__ void __launch_bounds__(THREADS)
   const int c0 = g * CG + tid * VEC;
   const int ntile = (tend - tbeg + LT - 1) / LT;
 
+  auto issue = [&](int s, int t) {
+    mbar_arrive_expect_tx(&full[s], kStageBytes);
+    tma_load_3d(ktile(s), &tmk, &full[s], g * CG, t, b);
+    tma_load_3d(ktile(s) + kTile, &tmv, &full[s], g * CG, t, b);
+    if (kWT) tma_load_3d(wtile(s), &tmw, &full[s], g * CG, t, b);
+  };
   if (kTMA && tid == 0) {
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
-    for (int s = 0; s < STAGES && s < ntile; ++s) {
-      mbar_arrive_expect_tx(&full[s], kStageBytes);
-      tma_load_3d(tiles + (2 * s) * kTile, &tmk, &full[s], g * CG, tbeg + s * LT, b);
-      tma_load_3d(tiles + (2 * s + 1) * kTile, &tmv, &full[s], g * CG, tbeg + s * LT, b);
-    }
+    for (int s = 0; s < STAGES && s < ntile; ++s) issue(s, tbeg + s * LT);
   }
 
-  float w[VEC], u[VEC], cb[VEC];
+  float w[VEC], u[VEC], cb[VEC], lo[VEC];
   Acc st[VEC];
   bool fast = true;
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
     const int c = c0 + e;
     const bool ok = c < C;
-    w[e] = ok ? p.w[c] : 0.f;
+    w[e] = (ok && !kWT) ? p.w[c] : 0.f;
     u[e] = ok ? p.u[c] : 0.f;
+    lo[e] = 0.f;
     fast &= fast_uw(u[e], w[e]);
     cb[e] = ex2(fminf(fmaxf(u[e] - w[e], -kFastUW), kFastUW) * kLog2e);
     st[e] = acc_empty();
@@ -208,16 +240,30 @@ __global__ void __launch_bounds__(THREADS)
         break;
       }
     } else {
-      coop_load_tile<KV>(tiles, reinterpret_cast<const KV*>(p.k), b, t0, LT, g * CG, CG, T, C);
-      coop_load_tile<KV>(tiles + kTile, reinterpret_cast<const KV*>(p.v), b, t0, LT, g * CG, CG, T, C);
+      coop_load_tile<KV>(ktile(0), reinterpret_cast<const KV*>(p.k), b, t0, LT, g * CG, CG, T, C);
+      coop_load_tile<KV>(ktile(0) + kTile, reinterpret_cast<const KV*>(p.v), b, t0, LT, g * CG, CG, T, C);
+      if (kWT) coop_load_tile<float>(wtile(0), p.w_t, b, t0, LT, g * CG, CG, T, C);
       __syncthreads();
     }
-    const KV* ks = tiles + (2 * s) * kTile + tid * VEC;
+    const KV* ks = ktile(s) + tid * VEC;
     const KV* vs = ks + kTile;
+    const float* wsm = wtile(s) + tid * VEC;
     const int nv = min(LT, tend - t0);
     OUT* orow = out + ((size_t)b * T + t0) * C;
+    const size_t rrow = ((size_t)b * T + t0) * C;
     if (c0 < C) {
-      if (nv == LT && fast) {
+      if (kWT) {
+        for (int j = 0; j < nv; ++j) {
+          float kx[VEC], vx[VEC], wx[VEC], o[VEC];
+          load_vec<KV, VEC>(ks + j * CG, kx);
+          load_vec<KV, VEC>(vs + j * CG, vx);
+          load_vec<float, VEC>(wsm + j * CG, wx);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) o[e] = step_token_wt(st[e], lo[e], kx[e], vx[e], wx[e], u[e]);
+          gate_row<KV, VEC>(p, rrow + (size_t)j * C, c0, o);
+          store_out<OUT, VEC>(orow + (size_t)j * C, c0, C, vec_ok, o);
+        }
+      } else if (nv == LT && fast) {
         constexpr int NB = LT < 8 ? LT : 8;  // tokens per block of step_tokens
 #pragma unroll
         for (int j0 = 0; j0 < LT; j0 += NB) {
@@ -229,7 +275,10 @@ __global__ void __launch_bounds__(THREADS)
           }
           step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
 #pragma unroll
-          for (int jj = 0; jj < NB; ++jj) store_out<OUT, VEC>(orow + (size_t)(j0 + jj) * C, c0, C, vec_ok, ob[jj]);
+          for (int jj = 0; jj < NB; ++jj) {
+            gate_row<KV, VEC>(p, rrow + (size_t)(j0 + jj) * C, c0, ob[jj]);
+            store_out<OUT, VEC>(orow + (size_t)(j0 + jj) * C, c0, C, vec_ok, ob[jj]);
+          }
         }
       } else if (nv == LT) {
 #pragma unroll 4
@@ -242,6 +291,7 @@ __global__ void __launch_bounds__(THREADS)
             o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
             add_token(st[e], kx[e], vx[e], w[e]);
           }
+          gate_row<KV, VEC>(p, rrow + (size_t)j * C, c0, o);
           store_out<OUT, VEC>(orow + (size_t)j * C, c0, C, vec_ok, o);
         }
       } else {
@@ -254,6 +304,7 @@ __global__ void __launch_bounds__(THREADS)
             o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
             add_token(st[e], kx[e], vx[e], w[e]);
           }
+          gate_row<KV, VEC>(p, rrow + (size_t)j * C, c0, o);
           store_out<OUT, VEC>(orow + (size_t)j * C, c0, C, vec_ok, o);
         }
       }
@@ -261,10 +312,7 @@ __global__ void __launch_bounds__(THREADS)
     __syncthreads();  // every thread is done with stage s
     if (kTMA && tid == 0 && i + STAGES < ntile) {
       fence_proxy_async_smem();
-      const int tn = tbeg + (i + STAGES) * LT;
-      mbar_arrive_expect_tx(&full[s], kStageBytes);
-      tma_load_3d(tiles + (2 * s) * kTile, &tmk, &full[s], g * CG, tn, b);
-      tma_load_3d(tiles + (2 * s + 1) * kTile, &tmv, &full[s], g * CG, tn, b);
+      issue(s, tbeg + (i + STAGES) * LT);
       ++issued;
     }
   }
@@ -287,7 +335,7 @@ __global__ void __launch_bounds__(THREADS)
         const size_t i = (size_t)b * C + c;
         p.o_num[i] = st[e].num;
         p.o_den[i] = st[e].den;
-        p.o_max[i] = acc_max_e(st[e], w[e]);
+        p.o_max[i] = kWT ? acc_max_e_wt(st[e], lo[e]) : acc_max_e(st[e], w[e]);
       }
     }
   }
@@ -374,6 +422,71 @@ __device__ __forceinline__ void aggregate_tile_span(const KV* ks, const KV* vs, 
       agg[e] = acc_empty();
     } else {
       // all weights share the factor 2^{M log2e - ML} from rounding ML
+      const float corr = fmaf(M[e], kLog2e, -ML[e]);
+      const float fix = fmaf(-corr, 0.6931471805599453f, 1.f);
+      agg[e] = Acc{num[e] * fix, den[e] * fix, M[e], 0.f};
+    }
+  }
+}
+
+// Aggregate of one span of n <= J tokens with per-token decays ("RWKV-v6
+// Architecture", section "2. Dynamic Data-Dependent Decay"), anchored at the
+// span's end: token i has exponent s_i = k_i - (w_{i+1} + ... + w_{n-1})
+// there. The suffix sums are compensated (two_sum). Also returns the span's
+// decay sum (what the span does to everything before it). `ws` points at this
+// lane's channels of the span's w_t rows, CG apart like k and v.
+template <typename KV, int J, int VEC, int CG>
+__device__ __forceinline__ void aggregate_span_wt(const KV* ks, const KV* vs, const float* ws, int n,
+                                                  Acc (&agg)[VEC], float (&wsum)[VEC]) {
+  float sx[J][VEC];
+  float hi[VEC], lo[VEC], M[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    hi[e] = lo[e] = 0.f;
+    M[e] = kNegBig;
+  }
+#pragma unroll
+  for (int i = J - 1; i >= 0; --i) {
+    if (i < n) {
+      float kx[VEC], wx[VEC];
+      load_vec<KV, VEC>(ks + i * CG, kx);
+      load_vec<float, VEC>(ws + i * CG, wx);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        sx[i][e] = (kx[e] - hi[e]) - lo[e];
+        M[e] = fmaxf(M[e], sx[i][e]);
+        float h, er;
+        two_sum(hi[e], wx[e], h, er);
+        hi[e] = h;
+        lo[e] += er;
+      }
+    }
+  }
+  float ML[VEC], num[VEC], den[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    ML[e] = M[e] * kLog2e;
+    num[e] = den[e] = 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < J; ++i) {
+    if (i < n) {
+      float vx[VEC];
+      load_vec<KV, VEC>(vs + i * CG, vx);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float x = ex2(fmaf(sx[i][e], kLog2e, -ML[e]));
+        num[e] = fmaf(x, vx[e], num[e]);
+        den[e] += x;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    wsum[e] = hi[e] + lo[e];
+    if (n <= 0) {
+      agg[e] = acc_empty();
+    } else {
       const float corr = fmaf(M[e], kLog2e, -ML[e]);
       const float fix = fmaf(-corr, 0.6931471805599453f, 1.f);
       agg[e] = Acc{num[e] * fix, den[e] * fix, M[e], 0.f};
@@ -629,6 +742,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
           step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
 #pragma unroll
           for (int ii = 0; ii < NB; ++ii) {
+            gate_row<KV, VEC>(p, ((size_t)b * T + ts + i0 + ii) * C, c0, ob[ii]);
             if (lane_vec) {
               stg_stream<OUT, VEC>(orow + (size_t)(i0 + ii) * C, ob[ii]);
             } else {
@@ -645,6 +759,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
           load_vec<KV, VEC>(vs + i * CG, vx);
 #pragma unroll
           for (int e = 0; e < VEC; ++e) o[e] = step_token(st[e], kx[e], vx[e], w[e], cb[e]);
+          gate_row<KV, VEC>(p, ((size_t)b * T + ts + i) * C, c0, o);
 #pragma unroll
           for (int e = 0; e < VEC; ++e)
             if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
@@ -659,6 +774,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
             o[e] = out_token(st[e], kx[e], vx[e], w[e], u[e]);
             add_token(st[e], kx[e], vx[e], w[e]);
           }
+          gate_row<KV, VEC>(p, ((size_t)b * T + ts + i) * C, c0, o);
 #pragma unroll
           for (int e = 0; e < VEC; ++e)
             if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);
@@ -720,18 +836,21 @@ __device__ __forceinline__ float4 ldg_f4(const float4* q) {
 // Pass A. Grid: (nch - 1) * B * NG CTAs of NW warps; tile = blockIdx.x in
 // chunk-major order. Every tile here is a full chunk (the last chunk, which
 // alone can be partial, has no total to compute).
-template <typename KV, int NW, int J>
+template <typename KV, int NW, int J, bool kWT>
 __global__ void __launch_bounds__(NW * 32)
-    wkv_tile_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    wkv_tile_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                    const __grid_constant__ CUtensorMap tmw) {
   constexpr int VEC = 2;
   constexpr int CG = 32 * VEC;
   constexpr int L = NW * J;
   constexpr int kTile = L * CG;
-  constexpr uint32_t kBytes = 2u * kTile * sizeof(KV);
+  constexpr uint32_t kBytes = (uint32_t)(2u * kTile * sizeof(KV) + (kWT ? kTile * sizeof(float) : 0));
   extern __shared__ __align__(1024) unsigned char smem[];
   KV* ktile = reinterpret_cast<KV*>(smem);
+  float* wtile = reinterpret_cast<float*>(smem + 2u * kTile * sizeof(KV));  // (kWT)
   float4* sh_agg = reinterpret_cast<float4*>(smem + kBytes);  // [NW][CG]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_agg + NW * CG);
+  float* sh_w = reinterpret_cast<float*>(sh_agg + NW * CG);   // [NW][CG] (kWT)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sh_w + (kWT ? NW * CG : 0));
 
   const int lane = threadIdx.x & 31;
   const int wp = threadIdx.x >> 5;
@@ -746,35 +865,62 @@ __global__ void __launch_bounds__(NW * 32)
     mbar_arrive_expect_tx(bar, kBytes);
     tma_load_3d(ktile, &tmk, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
     tma_load_3d(ktile + kTile, &tmv, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
+    if (kWT) tma_load_3d(wtile, &tmw, bar, (bg % p.NG) * CG, j * L, bg / p.NG);
   }
   grid_launch_dependents();  // the scan may be scheduled (it waits for this grid)
   __syncthreads();
   float w[VEC];
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) w[e] = (c0 + e < p.C) ? __ldg(p.w + c0 + e) : 0.f;
+  for (int e = 0; e < VEC; ++e) w[e] = (!kWT && c0 + e < p.C) ? __ldg(p.w + c0 + e) : 0.f;
   const bool ok = mbar_wait(bar, 0, p.timeout_ns);
   Acc a[VEC];
+  float ws[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) ws[e] = 0.f;
   if (ok) {
-    aggregate_tile_span<KV, J, VEC, CG>(ktile + (wp * J) * CG + cl, ktile + kTile + (wp * J) * CG + cl, J, w, a);
+    const int o = (wp * J) * CG + cl;
+    if (kWT) {
+      aggregate_span_wt<KV, J, VEC, CG>(ktile + o, ktile + kTile + o, wtile + o, J, a, ws);
+    } else {
+      aggregate_tile_span<KV, J, VEC, CG>(ktile + o, ktile + kTile + o, J, w, a);
+    }
   } else {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) a[e] = acc_empty();
     if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
   }
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) sh_agg[wp * CG + cl + e] = acc_pack(a[e]);
+  for (int e = 0; e < VEC; ++e) {
+    sh_agg[wp * CG + cl + e] = acc_pack(a[e]);
+    if (kWT) sh_w[wp * CG + cl + e] = ws[e];
+  }
   __syncthreads();
   if (wp == 0) {
     Acc t[VEC];
+    float wt[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) t[e] = acc_unpack(sh_agg[cl + e]);
+    for (int e = 0; e < VEC; ++e) {
+      t[e] = acc_unpack(sh_agg[cl + e]);
+      wt[e] = kWT ? sh_w[cl + e] : 0.f;
+    }
     for (int q = 1; q < NW; ++q) {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) t[e] = combine(t[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+      for (int e = 0; e < VEC; ++e) {
+        if (kWT) {
+          const float wq = sh_w[q * CG + cl + e];
+          t[e] = combine_wt(t[e], acc_unpack(sh_agg[q * CG + cl + e]), wq);
+          wt[e] += wq;
+        } else {
+          t[e] = combine(t[e], acc_unpack(sh_agg[q * CG + cl + e]), (float)J, w[e]);
+        }
+      }
     }
     float4* dst = p.agg_a + (size_t)tile * CG + cl;
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) dst[e] = acc_pack(t[e]);
+    for (int e = 0; e < VEC; ++e) {
+      dst[e] = acc_pack(t[e]);
+      if (kWT) p.wtot[(size_t)tile * CG + cl + e] = wt[e];
+    }
   }
   if (!ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
 }
@@ -790,10 +936,11 @@ __global__ void __launch_bounds__(NW * 32)
 // (griddepcontrol.wait) for that pass before its first load of a total. The totals are read-only from then on,
 // so they are loaded through the non-coherent path, eight at a time; a
 // segment of at most eight is loaded once and kept in registers.
-template <int SEG>
+template <int SEG, bool kWT>
 __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int L) {
   constexpr int CG = 64, CH = 16;
   __shared__ float4 seg_st[SEG][CH];
+  __shared__ float seg_w[SEG][CH];  // decay sum of each segment (kWT)
   grid_launch_dependents();  // the replay's CTAs may start copying their tiles
   const int BNG = p.B * p.NG;
   const int bg = blockIdx.x >> 2;
@@ -801,38 +948,63 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   const int cl = (blockIdx.x & 3) * CH + ch;
   const int sg = threadIdx.x / CH;
   const int b = bg / p.NG, c = (bg % p.NG) * CG + cl;
-  const float w = c < p.C ? __ldg(p.w + c) : 0.f;
+  const float w = (!kWT && c < p.C) ? __ldg(p.w + c) : 0.f;
   const int ntot = p.nch - 1;
   const int per = (ntot + SEG - 1) / SEG;
   const int q0 = min(ntot, sg * per), q1 = min(ntot, q0 + per);
   const float fL = (float)L;
   const float4* tot_of = p.agg_a + (size_t)bg * CG + cl;  // chunk q's total at tot_of[q * BNG * CG]
+  const float* wtot_of = kWT ? p.wtot + (size_t)bg * CG + cl : nullptr;
   const size_t qs = (size_t)BNG * CG;
+  // one combine of a chunk total (its decay sum wq with per-token decays)
+  auto comb = [&](const Acc& x, const float4& t, float wq) {
+    return kWT ? combine_wt(x, acc_unpack(t), wq) : combine(x, acc_unpack(t), fL, w);
+  };
   grid_wait_prerequisites();  // the totals pass has finished
   // 1. this segment's total; a segment of at most 8 totals stays in registers
   // for step 3
   const bool cached = q1 - q0 <= 8;
   float4 a0[8];
+  float w0[8];
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
-    if (cached && q0 + r < q1) a0[r] = ldg_f4(tot_of + (q0 + r) * qs);
+  for (int r = 0; r < 8; ++r) {
+    if (cached && q0 + r < q1) {
+      a0[r] = ldg_f4(tot_of + (q0 + r) * qs);
+      w0[r] = kWT ? __ldg(wtot_of + (q0 + r) * qs) : 0.f;
+    }
+  }
   Acc tot = acc_empty();
+  float wseg = 0.f;
   if (cached) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (q0 + r < q1) tot = combine(tot, acc_unpack(a0[r]), fL, w);
+    for (int r = 0; r < 8; ++r) {
+      if (q0 + r < q1) {
+        tot = comb(tot, a0[r], w0[r]);
+        wseg += w0[r];
+      }
+    }
   } else {
     for (int qq = q0; qq < q1; qq += 8) {
       float4 a[8];
+      float wa[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (qq + r < q1) a[r] = ldg_f4(tot_of + (qq + r) * qs);
+      for (int r = 0; r < 8; ++r) {
+        if (qq + r < q1) {
+          a[r] = ldg_f4(tot_of + (qq + r) * qs);
+          wa[r] = kWT ? __ldg(wtot_of + (qq + r) * qs) : 0.f;
+        }
+      }
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (qq + r < q1) tot = combine(tot, acc_unpack(a[r]), fL, w);
+      for (int r = 0; r < 8; ++r) {
+        if (qq + r < q1) {
+          tot = comb(tot, a[r], wa[r]);
+          wseg += wa[r];
+        }
+      }
     }
   }
   seg_st[sg][ch] = acc_pack(tot);
+  seg_w[sg][ch] = wseg;
   __syncthreads();
   // 2. incoming state of every segment (state in, then the segments before)
   if (sg == 0) {
@@ -841,7 +1013,7 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
       const Acc t = acc_unpack(seg_st[k][ch]);
       const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
       seg_st[k][ch] = acc_pack(x);
-      x = combine(x, t, (float)(kq1 - kq0) * fL, w);
+      x = kWT ? combine_wt(x, t, seg_w[k][ch]) : combine(x, t, (float)(kq1 - kq0) * fL, w);
     }
   }
   __syncthreads();
@@ -853,20 +1025,25 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
     for (int r = 0; r < 8; ++r) {
       if (q0 + r < q1) {
         x0_of[(q0 + r) * qs] = acc_pack(x);
-        x = combine(x, acc_unpack(a0[r]), fL, w);
+        x = comb(x, a0[r], w0[r]);
       }
     }
   } else {
     for (int qq = q0; qq < q1; qq += 8) {
       float4 a[8];
+      float wa[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (qq + r < q1) a[r] = ldg_f4(tot_of + (qq + r) * qs);
+      for (int r = 0; r < 8; ++r) {
+        if (qq + r < q1) {
+          a[r] = ldg_f4(tot_of + (qq + r) * qs);
+          wa[r] = kWT ? __ldg(wtot_of + (qq + r) * qs) : 0.f;
+        }
+      }
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         if (qq + r < q1) {
           x0_of[(qq + r) * qs] = acc_pack(x);
-          x = combine(x, acc_unpack(a[r]), fL, w);
+          x = comb(x, a[r], wa[r]);
         }
       }
     }
@@ -1164,6 +1341,7 @@ __global__ void __launch_bounds__((2 * NC + 2) * 32)
             step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
 #pragma unroll
             for (int ii = 0; ii < NB; ++ii) {
+              gate_row<KV, VEC>(p, ((size_t)b * T + ts + i0 + ii) * C, c0, ob[ii]);
               if (lane_vec) {
                 stg_stream<OUT, VEC>(orow + (size_t)(i0 + ii) * C, ob[ii]);
               } else {
@@ -1187,6 +1365,7 @@ __global__ void __launch_bounds__((2 * NC + 2) * 32)
                 add_token(st[e], kx[e], vx[e], w[e]);
               }
             }
+            gate_row<KV, VEC>(p, ((size_t)b * T + ts + i) * C, c0, o);
 #pragma unroll
             for (int e = 0; e < VEC; ++e)
               if (c0 + e < C) orow[(size_t)i * C + e] = Elem<OUT>::from_f32(o[e]);

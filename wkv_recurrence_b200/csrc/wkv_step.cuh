@@ -33,6 +33,8 @@ struct StepParams {
   float* o_num;
   float* o_den;
   float* o_max;
+  const float* w_t;  // this token's decay of every stream [S, C] in place of w, or NULL
+  const void* r;     // receptance [S, C] (element type of k, v): out = sigmoid(r) wkv; or NULL
 };
 
 __device__ __forceinline__ void decode_token(float k, float v, float w, float u, float& num, float& den, float& m,
@@ -75,10 +77,20 @@ __global__ void __launch_bounds__(256) wkv_step_kernel(const StepParams p) {
     load_vec<float, VEC>(p.s_num + i0, num);
     load_vec<float, VEC>(p.s_den + i0, den);
     load_vec<float, VEC>(p.s_max + i0, mx);
-    load_vec<float, VEC>(p.w + c0, w);
+    if (p.w_t) {
+      load_vec<float, VEC>(p.w_t + i0, w);
+    } else {
+      load_vec<float, VEC>(p.w + c0, w);
+    }
     load_vec<float, VEC>(p.u + c0, u);
 #pragma unroll
     for (int e = 0; e < VEC; ++e) decode_token(kx[e], vx[e], w[e], u[e], num[e], den[e], mx[e], o[e]);
+    if (p.r) {
+      float rx[VEC];
+      load_vec<KV, VEC>(reinterpret_cast<const KV*>(p.r) + i0, rx);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) o[e] = gate(o[e], rx[e]);
+    }
     store_vec<OUT, VEC>(reinterpret_cast<OUT*>(p.out) + i0, o);
     store_vec<float, VEC>(p.o_num + i0, num);
     store_vec<float, VEC>(p.o_den + i0, den);
@@ -90,7 +102,8 @@ __global__ void __launch_bounds__(256) wkv_step_kernel(const StepParams p) {
       float num = p.s_num[i], den = p.s_den[i], mx = p.s_max[i], o;
       const float kk = Elem<KV>::to_f32(reinterpret_cast<const KV*>(p.k)[i]);
       const float vv = Elem<KV>::to_f32(reinterpret_cast<const KV*>(p.v)[i]);
-      decode_token(kk, vv, p.w[c], p.u[c], num, den, mx, o);
+      decode_token(kk, vv, p.w_t ? p.w_t[i] : p.w[c], p.u[c], num, den, mx, o);
+      if (p.r) o = gate(o, Elem<KV>::to_f32(reinterpret_cast<const KV*>(p.r)[i]));
       reinterpret_cast<OUT*>(p.out)[i] = Elem<OUT>::from_f32(o);
       p.o_num[i] = num;
       p.o_den[i] = den;

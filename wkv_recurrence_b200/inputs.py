@@ -34,7 +34,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 # tensor codes for the per-row generators
-_W, _U, _K, _V, _SNUM, _SDEN, _SMAX, _DK, _DV = range(9)
+_W, _U, _K, _V, _SNUM, _SDEN, _SMAX, _DK, _DV, _WT, _R = range(11)
 
 
 @dataclass(frozen=True)
@@ -176,6 +176,49 @@ def draw_kv_rows(wl: Workload, rows, seed: int = 0, T: int | None = None):
 
 def draw_kv(wl: Workload, seed: int = 0):
     return draw_kv_rows(wl, range(wl.B), seed)
+
+
+def draw_wt_rows(wl: Workload, rows, seed: int = 0, T: int | None = None) -> np.ndarray:
+    """Per-token decays w_t for the given rows, fp32 [len(rows), T, C], drawn
+    per token from the workload's w distribution (log-normal exp(N(-1, 1))
+    clipped to [1e-3, 8], or log-uniform in [1e-4, 4]); in 512-token blocks
+    seeded by (seed, workload, tensor, row, block), like k and v."""
+    T = wl.T if T is None else T
+    rows = list(rows)
+    out = np.empty((len(rows), T, wl.C), np.float32)
+    nblk = max(1, -(-T // _BLOCK_T))
+
+    def one(job):
+        i, b, j = job
+        t0, t1 = j * _BLOCK_T, min(T, (j + 1) * _BLOCK_T)
+        g = _rng5(seed, wl.code, _WT, b, j)
+        if wl.w_dist == "loguniform":
+            x = np.exp(g.uniform(np.log(1e-4), np.log(4.0), (t1 - t0, wl.C)))
+        else:
+            x = np.clip(np.exp(g.normal(-1.0, 1.0, (t1 - t0, wl.C))), 1e-3, 8.0)
+        out[i, t0:t1] = x.astype(np.float32)
+
+    _pool_map(one, [(i, b, j) for i, b in enumerate(rows) for j in range(nblk)])
+    return out
+
+
+def draw_r_rows(wl: Workload, rows, seed: int = 0, T: int | None = None) -> np.ndarray:
+    """Receptance r ~ N(0, 1) for the given rows, [len(rows), T, C] in the
+    element type of k and v (uint16 bf16 codes for bf16 workloads)."""
+    T = wl.T if T is None else T
+    rows = list(rows)
+    bf16 = wl.kv_dtype == "bf16"
+    out = np.empty((len(rows), T, wl.C), np.uint16 if bf16 else np.float32)
+    nblk = max(1, -(-T // _BLOCK_T))
+
+    def one(job):
+        i, b, j = job
+        t0, t1 = j * _BLOCK_T, min(T, (j + 1) * _BLOCK_T)
+        x = _rng5(seed, wl.code, _R, b, j).standard_normal((t1 - t0, wl.C), dtype=np.float32)
+        out[i, t0:t1] = f32_to_bf16_bits(x) if bf16 else x
+
+    _pool_map(one, [(i, b, j) for i, b in enumerate(rows) for j in range(nblk)])
+    return out
 
 
 def draw_state(wl: Workload, rows=None, seed: int = 0):
