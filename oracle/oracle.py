@@ -26,6 +26,10 @@ Functions
                         channels): the O(T) oracle used at full size. Pinned to
                         the sum by the tests.
 ``recurrence_step``     one decode token for S streams, same recurrence.
+``recurrence_backward`` the gradients of sum(g * wkv) with respect to k, v,
+                        w, u and the state passed in, by the chain rule run
+                        backwards through the same recurrence (float64 C), with
+                        the magnitude scale of each gradient.
 ``abs_scale_*``         the same oracles run with |v| (and |num_in|): the
                         per-output scale sum_i p_i |v_i| used by the parity
                         metric.
@@ -105,6 +109,8 @@ def _load():
         lib.wkv_oracle_forward_ext.restype = None
         lib.wkv_oracle_step_ext.argtypes = [I64, I64, P, P, P, I, P, P, P, P, P, P, P, P, P]
         lib.wkv_oracle_step_ext.restype = None
+        lib.wkv_oracle_backward.argtypes = [I64, I64, I64, P, P, I] + [P] * 20 + [I]
+        lib.wkv_oracle_backward.restype = None
         _lib = lib
     return _lib
 
@@ -191,6 +197,36 @@ def recurrence_step(state, k, v, w, u, r=None):
     lib.wkv_oracle_step_ext(S, C, _p(k), _p(v), _p(w), per_stream, _p(u), _p(rr),
                             _p(si[0]), _p(si[1]), _p(si[2]), _p(out), _p(so[0]), _p(so[1]), _p(so[2]))
     return out, tuple(so)
+
+
+def recurrence_backward(k, v, w, u, gout, state=None, kv_dtype: str = "f32", threads: int = 0):
+    """Gradients of sum(gout * wkv) by the float64 backward recurrence.
+
+    gout: [B, T, C] (float64 or float32), dL/d wkv. No loss term on the final
+    state. Returns two dicts, the gradients and their scales (the same
+    formulas on magnitudes: the sum of |terms| of each gradient):
+      dk, dv [B, T, C]; dw, du [C] (summed over the batch rows);
+      dnum, dden, dmax [B, C] (the state passed in; zeros without one).
+    """
+    lib = _load()
+    k, v, code = _kv_arrays(k, v, kv_dtype)
+    B, T, C = k.shape
+    w = np.ascontiguousarray(w, np.float32)
+    u = np.ascontiguousarray(u, np.float32)
+    g = np.ascontiguousarray(gout, np.float64)
+    assert g.shape == (B, T, C)
+    si = [None, None, None]
+    if state is not None:
+        si = [np.ascontiguousarray(np.broadcast_to(s, (B, C)), np.float64) for s in state]
+    d = {n: np.zeros(sh) for n, sh in (("dk", (B, T, C)), ("dv", (B, T, C)), ("dw", (C,)), ("du", (C,)),
+                                        ("dnum", (B, C)), ("dden", (B, C)), ("dmax", (B, C)))}
+    sc = {n: np.zeros_like(a) for n, a in d.items()}
+    lib.wkv_oracle_backward(B, T, C, _p(k), _p(v), code, _p(w), _p(u), _p(si[0]), _p(si[1]), _p(si[2]), _p(g),
+                            _p(d["dk"]), _p(d["dv"]), _p(d["dw"]), _p(d["du"]),
+                            _p(d["dnum"]), _p(d["dden"]), _p(d["dmax"]),
+                            _p(sc["dk"]), _p(sc["dv"]), _p(sc["dw"]), _p(sc["du"]),
+                            _p(sc["dnum"]), _p(sc["dden"]), _p(sc["dmax"]), int(threads))
+    return d, sc
 
 
 # ---------------------------------------------------------------------------

@@ -28,6 +28,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #ifdef _OPENMP
@@ -243,4 +244,149 @@ void wkv_oracle_step_ext(int64_t S, int64_t C, const float *k, const float *v,
         den_out[i] = den;
         max_out[i] = m;
     }
+}
+
+/*
+ * Gradients of the forward for a loss whose gradient with respect to every
+ * output is given (gout = dL/d wkv, [B, T, C]); no loss term on the final
+ * state. This is the chain rule applied to the step function of "The
+ * recurrence", backwards in time:
+ *
+ *   Write the state before token t as the pair (N_t, D_t) = (num, den) e^{m}
+ *   and the output as wkv_t = A_t / Z_t with A_t = N_t + e^{u+k_t} v_t,
+ *   Z_t = D_t + e^{u+k_t}. The state advances as N_{t+1} = e^{-w} N_t +
+ *   e^{k_t} v_t (D likewise with v = 1). With dN_t = dL/dN_t (the total effect
+ *   through every later output) and dD_t likewise:
+ *     dN_t = g_t / Z_t + e^{-w} dN_{t+1},  dD_t = -g_t wkv_t / Z_t + e^{-w} dD_{t+1},
+ *     dN_T = dD_T = 0,
+ *     dv_t = g_t e^{u+k_t} / Z_t + e^{k_t} dN_{t+1},
+ *     dk_t = g_t e^{u+k_t} (v_t - wkv_t) / Z_t + e^{k_t} (v_t dN_{t+1} + dD_{t+1}),
+ *     du  += g_t e^{u+k_t} (v_t - wkv_t) / Z_t,
+ *     dw  -= e^{-w} (N_t dN_{t+1} + D_t dD_{t+1}),
+ *   and for the state passed in, (N_0, D_0) = (num0, den0) e^{m0}:
+ *     dnum0 = e^{m0} dN_0, dden0 = e^{m0} dD_0, dm0 = num0 dnum0 + den0 dden0.
+ *
+ * Every exponential is taken relative to a running maximum, as in the forward:
+ * Z_t relative to e_t = max(m_t, u + k_t), and (dN_t, dD_t) = (rn, rd) e^{Q_t}
+ * with Q_t the largest exponent contributing to them.
+ *
+ * The s* outputs (optional, NULL to skip) are the same formulas with every
+ * signed quantity replaced by its magnitude (g, v, wkv, num0, and the
+ * accumulators run on |g|): the sum of the magnitudes of the terms that make
+ * up each gradient, the scale against which its rounding error is measured.
+ *
+ * dw and du are [C], summed over the batch rows; the state gradients are
+ * [B, C] (NULL to skip).
+ */
+void wkv_oracle_backward(int64_t B, int64_t T, int64_t C,
+                         const void *k, const void *v, int kv_dtype,
+                         const float *w, const float *u,
+                         const double *num_in, const double *den_in, const double *max_in,
+                         const double *gout,
+                         double *dk, double *dv, double *dw, double *du,
+                         double *dnum, double *dden, double *dmax,
+                         double *sk, double *sv, double *sw, double *su,
+                         double *snum, double *sden, double *smax,
+                         int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    /* per (b, c) partial sums of dw, du (and their scales), summed over b below */
+    double *pw = (double *)calloc((size_t)(B * C) * 4, sizeof(double));
+
+#pragma omp parallel
+    {
+        double *st = (double *)malloc(sizeof(double) * 3 * (size_t)(T > 0 ? T : 1));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t s = 0; s < B * C; ++s) {
+            const int64_t b = s / C, c = s % C;
+            const double wc = (double)w[c], uc = (double)u[c];
+            double num = 0.0, den = 0.0, m = -INFINITY;
+            if (num_in) {
+                num = num_in[s];
+                den = den_in[s];
+                m = max_in[s];
+            }
+            const double num0 = num, den0 = den, m0 = m;
+            /* forward: the state before every token */
+            for (int64_t t = 0; t < T; ++t) {
+                const size_t i = ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;
+                st[3 * t] = num;
+                st[3 * t + 1] = den;
+                st[3 * t + 2] = m;
+                (void)wkv_token(widen(k, kv_dtype, i), widen(v, kv_dtype, i), wc, uc, &num, &den, &m);
+            }
+            /* backward */
+            double rn = 0.0, rd = 0.0, an = 0.0, ad = 0.0, Q = -INFINITY;
+            double gu = 0.0, gw = 0.0, au = 0.0, aw = 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {
+                const size_t i = ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;
+                const double kt = widen(k, kv_dtype, i), vt = widen(v, kv_dtype, i), g = gout[i];
+                const double nt = st[3 * t], dt = st[3 * t + 1], mt = st[3 * t + 2];
+                const double e = fmax(mt, kt + uc);
+                const double a = exp(mt - e), bb = exp(kt + uc - e);
+                const double z = a * dt + bb;
+                const double out = (a * nt + bb * vt) / z;
+                const double p = g / z, q = -g * out / z;
+                const double pa = fabs(g) / z, qa = fabs(g) * fabs(out) / z;
+                const double E1 = exp(kt + Q);          /* e^{k_t} relative to dN_{t+1}'s exponent */
+                const double E2 = exp(mt + Q - wc);     /* e^{m_t - w}, likewise */
+                dv[i] = p * bb + rn * E1;
+                dk[i] = p * bb * (vt - out) + E1 * (vt * rn + rd);
+                gu += p * bb * (vt - out);
+                gw -= E2 * (nt * rn + dt * rd);
+                if (sv) {
+                    sv[i] = pa * bb + an * E1;
+                    sk[i] = pa * bb * (fabs(vt) + fabs(out)) + E1 * (fabs(vt) * an + ad);
+                }
+                au += pa * bb * (fabs(vt) + fabs(out));
+                aw += E2 * (fabs(nt) * an + dt * ad);
+                /* move the accumulators to position t: decay by w, add token t */
+                const double Qn = fmax(Q - wc, -e);
+                const double x1 = exp(Q - wc - Qn), x2 = exp(-e - Qn);
+                rn = rn * x1 + p * x2;
+                rd = rd * x1 + q * x2;
+                an = an * x1 + pa * x2;
+                ad = ad * x1 + qa * x2;
+                Q = Qn;
+            }
+            pw[4 * s] = gw;
+            pw[4 * s + 1] = gu;
+            pw[4 * s + 2] = aw;
+            pw[4 * s + 3] = au;
+            if (dnum) {
+                const double f = (m0 == -INFINITY || !(den0 > 0.0)) ? 0.0 : exp(m0 + Q);
+                dnum[s] = rn * f;
+                dden[s] = rd * f;
+                dmax[s] = num0 * dnum[s] + den0 * dden[s];
+                if (snum) {
+                    snum[s] = an * f;
+                    sden[s] = ad * f;
+                    smax[s] = fabs(num0) * snum[s] + den0 * sden[s];
+                }
+            }
+        }
+        free(st);
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        double gw = 0.0, gu = 0.0, aw = 0.0, au = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            const int64_t s = b * C + c;
+            gw += pw[4 * s];
+            gu += pw[4 * s + 1];
+            aw += pw[4 * s + 2];
+            au += pw[4 * s + 3];
+        }
+        dw[c] = gw;
+        du[c] = gu;
+        if (sw) {
+            sw[c] = aw;
+            su[c] = au;
+        }
+    }
+    free(pw);
 }
