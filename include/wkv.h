@@ -267,6 +267,43 @@ WKV_API wkv_status wkv_step_ext(int64_t S, int64_t C,
                         void *stream, const wkv_ext *ext);
 
 /*
+ * Backward of wkv_forward (per-channel w, no w_t or r): the gradients of a
+ * loss L given gout = dL/d wkv for every output, with no loss term on the
+ * final state. The chain rule through the step function of "The recurrence"
+ * run backwards in time; the pages' claim that the recurrence trains like a
+ * transformer ("What held up": it trains; "RWKV-v6 Architecture", "Key
+ * Mechanics: Architectural Duality", time-parallel mode) is what makes it
+ * part of the operator:
+ *     dv_t = g_t e^{u+k_t}/Z_t + e^{k_t} dN_{t+1}
+ *     dk_t = g_t e^{u+k_t}(v_t - wkv_t)/Z_t + e^{k_t}(v_t dN_{t+1} + dD_{t+1})
+ *     du   = sum_{b,t} g_t e^{u+k_t}(v_t - wkv_t)/Z_t
+ *     dw   = -sum_{b,t} e^{-w}(N_t dN_{t+1} + D_t dD_{t+1})
+ * with (N_t, D_t) the state pair before token t, Z_t = D_t + e^{u+k_t}, and
+ * dN_t = g_t/Z_t + e^{-w} dN_{t+1}, dD_t = -g_t wkv_t/Z_t + e^{-w} dD_{t+1}.
+ *
+ *   k, v       [B, T, C], element type kv_dtype, base addresses 16-byte
+ *              aligned and C * element size a multiple of 16 bytes (else
+ *              WKV_ERR_MISALIGNED)
+ *   w, u       [C] fp32;  state_in  NULL or three fp32 [B, C] (as wkv_forward)
+ *   gout       [B, T, C] fp32
+ *   dk, dv     [B, T, C] fp32 (written)
+ *   dw, du     [C] fp32 (written; summed over the batch rows)
+ *   dstate_in  NULL, or three fp32 [B, C] arrays receiving dL/dnum, dL/dden,
+ *              dL/dmax_e of state_in (zeros where it was empty or absent)
+ *   workspace  at least wkv_backward_workspace_size(B, T, C) bytes, 256-byte
+ *              aligned; no zero-fill needed (every byte read is written first)
+ * Results are bitwise reproducible. Launches six kernels (four when T <= 32).
+ */
+WKV_API size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C);
+WKV_API wkv_status wkv_backward(int64_t B, int64_t T, int64_t C,
+                        const void *k, const void *v, wkv_dtype kv_dtype,
+                        const float *w, const float *u,
+                        const wkv_cstate *state_in, const float *gout,
+                        float *dk, float *dv, float *dw, float *du,
+                        const wkv_state *dstate_in,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * wkv_forward without a caller-provided workspace. The pages have no
  * counterpart to this entry point; it exists for callers that cannot allocate
  * device memory themselves: hosts that hand a plug-in only its input and

@@ -13,8 +13,8 @@ Importing the package does not load the library; the first call does, and
 fails loudly if it is missing or no CUDA device is present.
 """
 
-from .api import (PreparedForward, PreparedStep, WkvError, empty_state, forward,  # noqa: F401
+from .api import (WKV, PreparedForward, PreparedStep, WkvError, backward, empty_state, forward,  # noqa: F401
                   forward_kernel, forward_launches, make_workspace, query_status, step, workspace_size)
 
-__all__ = ["forward", "step", "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
+__all__ = ["forward", "step", "backward", "WKV", "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
            "PreparedForward", "PreparedStep", "WkvError"]

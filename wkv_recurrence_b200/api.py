@@ -218,6 +218,71 @@ def step(state: State, k: torch.Tensor, v: torch.Tensor, w: Optional[torch.Tenso
     return out, state_out
 
 
+def backward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor, gout: torch.Tensor,
+             state: Optional[State] = None, *, need_state_grad: bool = True,
+             workspace: Optional[torch.Tensor] = None):
+    """Gradients of a loss with dL/d wkv = gout [B, T, C] (float32).
+
+    Returns (dk, dv, dw, du, dstate): dk, dv float32 [B, T, C]; dw, du float32
+    [C] summed over the batch; dstate the gradients of (num, den, max_e) of
+    ``state`` (zeros without one), or None if not needed.
+    """
+    _need_cuda(k, "k")
+    _need_cuda(v, "v", k.dtype)
+    _need_cuda(w, "w", torch.float32)
+    _need_cuda(u, "u", torch.float32)
+    _need_cuda(gout, "gout", torch.float32)
+    if k.dim() != 3 or v.shape != k.shape or gout.shape != k.shape:
+        raise ValueError("k, v and gout must be [B, T, C]")
+    B, T, C = k.shape
+    dev = k.device
+    dk = torch.empty((B, T, C), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    dw = torch.empty(C, dtype=torch.float32, device=dev)
+    du = torch.empty_like(dw)
+    sin = None
+    if state is not None:
+        for i, s in enumerate(state):
+            _need_cuda(s, f"state[{i}]", torch.float32)
+        sin = _abi.wkv_cstate(*(s.data_ptr() for s in state))
+    dstate = None
+    dsout = None
+    if need_state_grad:
+        dstate = tuple(torch.empty((B, C), dtype=torch.float32, device=dev) for _ in range(3))
+        dsout = _abi.wkv_state(*(s.data_ptr() for s in dstate))
+    need = _abi.lib().wkv_backward_workspace_size(B, T, C)
+    if need == 0:
+        raise ValueError("invalid sizes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _need_cuda(workspace, "workspace")
+    code = _abi.lib().wkv_backward(
+        B, T, C, _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(w), _ptr(u),
+        ctypes.byref(sin) if sin is not None else None, _ptr(gout), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
+        ctypes.byref(dsout) if dsout is not None else None, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream())
+    _abi.check(code, "wkv_backward")
+    return dk, dv, dw, du, dstate
+
+
+class WKV(torch.autograd.Function):
+    """The operator as a torch autograd function: forward through wkv_forward,
+    backward through wkv_backward (per-channel w, float32 or bfloat16 k and v,
+    gradients in float32). ``WKV.apply(k, v, w, u)`` returns wkv [B, T, C]."""
+
+    @staticmethod
+    def forward(ctx, k, v, w, u):
+        out, _ = forward(k, v, w, u, return_state=False)
+        ctx.save_for_backward(k, v, w, u)
+        return out
+
+    @staticmethod
+    def backward(ctx, gout):
+        k, v, w, u = ctx.saved_tensors
+        dk, dv, dw, du, _ = backward(k, v, w, u, gout.float().contiguous(), need_state_grad=False)
+        return dk.to(k.dtype), dv.to(v.dtype), dw, du
+
+
 def query_status(workspace: torch.Tensor) -> int:
     """Synchronise the current stream; return and clear the device-side status of a workspace."""
     return int(_abi.lib().wkv_query_status(_ptr(workspace), _stream()))

@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "../../include/wkv.h"
+#include "wkv_bwd.cuh"
 #include "wkv_cluster.cuh"
 #include "wkv_device.cuh"
 #include "wkv_fwd.cuh"
@@ -724,6 +725,97 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
   return launch_chunk_shape<KV, OUT, false>(pl, p, tk, tv, st, dev);
 }
 
+// ---------------------------------------------------------------------------
+// backward
+// ---------------------------------------------------------------------------
+constexpr int kBwdL = 32;  // tokens per chunk of the backward
+
+struct BwdPlan {
+  int NG, nch;
+  size_t off_agg, off_x0, off_rtot, off_rin, off_pdu, off_pdw, bytes;
+};
+
+bool make_bwd_plan(int64_t B, int64_t T, int64_t C, BwdPlan* pl) {
+  std::memset(pl, 0, sizeof *pl);
+  if (!sizes_ok(B, T, C)) return false;
+  pl->NG = (int)((C + kChunkCG - 1) / kChunkCG);
+  pl->nch = (int)std::max<int64_t>(1, (T + kBwdL - 1) / kBwdL);
+  const size_t slots = (size_t)B * pl->NG * kChunkCG;  // float4 slots per chunk
+  size_t off = sizeof(WsHeader);
+  pl->off_agg = off;
+  off = round_up(off + sizeof(float4) * slots * (size_t)std::max(pl->nch - 1, 1), 256);
+  pl->off_x0 = off;
+  off = round_up(off + sizeof(float4) * slots * pl->nch, 256);
+  pl->off_rtot = off;
+  off = round_up(off + sizeof(float4) * slots * pl->nch, 256);
+  pl->off_rin = off;
+  off = round_up(off + sizeof(float4) * slots * pl->nch, 256);
+  pl->off_pdu = off;
+  off = round_up(off + sizeof(float) * (size_t)pl->nch * B * C, 256);
+  pl->off_pdw = off;
+  off = round_up(off + sizeof(float) * (size_t)pl->nch * B * C, 256);
+  pl->bytes = off;
+  return true;
+}
+
+template <int SEG_MAX>
+int scan_segments_for(int ntot) {
+  const int seg = ntot <= 16 ? 1 : (ntot <= 64 ? 4 : (ntot <= 256 ? 16 : 64));
+  return std::min(seg, SEG_MAX);
+}
+
+template <typename KV>
+wkv_status launch_backward(const BwdPlan& pl, const FwdParams& fp, const BwdParams& bp, wkv_dtype kvdt,
+                           cudaStream_t st, int dev) {
+  // A, S: the forward state entering every chunk (the forward's passes)
+  constexpr int NW = kBwdL / 16, J = 16;
+  const long long BNG = (long long)fp.B * fp.NG;
+  if (pl.nch > 1) {
+    CUtensorMap tk, tv;
+    if (!make_tmap(&tk, fp.k, kvdt, fp.B, fp.T, fp.C, kBwdL, kChunkCG) ||
+        !make_tmap(&tv, fp.v, kvdt, fp.B, fp.T, fp.C, kBwdL, kChunkCG))
+      return WKV_ERR_CUDA;
+    const size_t smem = 2ull * kBwdL * kChunkCG * sizeof(KV) + sizeof(float4) * NW * kChunkCG + 64;
+    auto fa = wkv_tile_totals<KV, NW, J, false>;
+    int occ = 0;
+    if (!kernel_setup(fa, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+    fa<<<(unsigned)((pl.nch - 1) * BNG), NW * 32, smem, st>>>(fp, tk, tv, tv);
+    if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  }
+  const int seg = scan_segments_for<64>(pl.nch - 1);
+  const unsigned gs = (unsigned)(BNG * 4);
+  switch (seg) {
+    case 1: wkv_tile_scan<1, false><<<gs, 16, 0, st>>>(fp, kBwdL); break;
+    case 4: wkv_tile_scan<4, false><<<gs, 64, 0, st>>>(fp, kBwdL); break;
+    case 16: wkv_tile_scan<16, false><<<gs, 256, 0, st>>>(fp, kBwdL); break;
+    default: wkv_tile_scan<64, false><<<gs, 1024, 0, st>>>(fp, kBwdL); break;
+  }
+  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  // R1: reverse aggregates of chunks 1 .. nch-1
+  const long long ngw = (fp.C + 31) / 32;
+  if (pl.nch > 1) {
+    const long long items = (long long)fp.B * (pl.nch - 1) * ngw;
+    wkv_bwd_rev_totals<KV><<<(unsigned)((items + 3) / 4), 128, 0, st>>>(bp);
+    if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  }
+  // RS: the reverse state entering every chunk from its end
+  switch (seg) {
+    case 1: wkv_bwd_rev_scan<1><<<gs, 16, 0, st>>>(bp); break;
+    case 4: wkv_bwd_rev_scan<4><<<gs, 64, 0, st>>>(bp); break;
+    case 16: wkv_bwd_rev_scan<16><<<gs, 256, 0, st>>>(bp); break;
+    default: wkv_bwd_rev_scan<64><<<gs, 1024, 0, st>>>(bp); break;
+  }
+  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  // R2: the gradients
+  const long long items = (long long)fp.B * pl.nch * ngw;
+  if ((items + 3) / 4 >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  wkv_bwd_chunk<KV, kBwdL><<<(unsigned)((items + 3) / 4), 128, 0, st>>>(bp);
+  if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  // RED: du, dw
+  wkv_bwd_reduce<<<(unsigned)((fp.C + 255) / 256), 256, 0, st>>>(bp);
+  return launch_result();
+}
+
 }  // namespace
 }  // namespace wkv
 
@@ -944,6 +1036,106 @@ wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtyp
                     const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
                     const wkv_state* state_out, void* stream) {
   return wkv_step_ext(S, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, stream, nullptr);
+}
+
+size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C) {
+  BwdPlan pl;
+  if (!make_bwd_plan(B, T, C, &pl)) return 0;
+  return pl.bytes;
+}
+
+wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const void* k, const void* v, wkv_dtype kv_dtype,
+                        const float* w, const float* u, const wkv_cstate* state_in, const float* gout, float* dk,
+                        float* dv, float* dw, float* du, const wkv_state* dstate_in, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  // ---- argument checks: nothing is launched before they pass
+  if (!sizes_ok(B, T, C)) return WKV_ERR_INVALID_ARG;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (state_in && (!state_in->num || !state_in->den || !state_in->max_e)) return WKV_ERR_INVALID_ARG;
+  if (dstate_in && (!dstate_in->num || !dstate_in->den || !dstate_in->max_e)) return WKV_ERR_INVALID_ARG;
+  if (B * T * C > 0 && (!k || !v || !gout || !dk || !dv)) return WKV_ERR_INVALID_ARG;
+  if (C > 0 && (!w || !u || !dw || !du)) return WKV_ERR_INVALID_ARG;
+  const size_t kes = kv_dtype == WKV_F32 ? 4 : 2;
+  BwdPlan pl;
+  if (!make_bwd_plan(B, T, C, &pl)) return WKV_ERR_INVALID_ARG;
+  if (!workspace) return WKV_ERR_INVALID_ARG;
+  if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
+  // the forward pass inside uses TMA on k and v
+  if (B * T * C > 0 && !tma_usable(k, v, C, kes)) return WKV_ERR_MISALIGNED;
+  if (C == 0) return WKV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || T == 0) {
+    // no tokens: every gradient is zero
+    if (!cuda_ok(cudaMemsetAsync(dw, 0, sizeof(float) * C, st)) ||
+        !cuda_ok(cudaMemsetAsync(du, 0, sizeof(float) * C, st)))
+      return WKV_ERR_CUDA;
+    if (dstate_in && B > 0) {
+      float* d[3] = {dstate_in->num, dstate_in->den, dstate_in->max_e};
+      for (float* x : d)
+        if (!cuda_ok(cudaMemsetAsync(x, 0, sizeof(float) * B * C, st))) return WKV_ERR_CUDA;
+    }
+    return WKV_OK;
+  }
+  int dev = 0;
+  if (!cuda_ok(cudaGetDevice(&dev))) return WKV_ERR_CUDA;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  FwdParams fp;
+  std::memset(&fp, 0, sizeof fp);
+  fp.B = (int)B;
+  fp.T = (int)T;
+  fp.C = (int)C;
+  fp.NG = pl.NG;
+  fp.nch = pl.nch;
+  fp.chunk_len = kBwdL;
+  fp.k = k;
+  fp.v = v;
+  fp.w = w;
+  fp.u = u;
+  if (state_in) {
+    fp.s_num = state_in->num;
+    fp.s_den = state_in->den;
+    fp.s_max = state_in->max_e;
+  }
+  fp.hdr = reinterpret_cast<WsHeader*>(ws);
+  fp.timeout_ns = kDefaultTimeoutNs;
+  fp.inject_tile = -1;
+  fp.agg_a = reinterpret_cast<float4*>(ws + pl.off_agg);
+  fp.x0 = reinterpret_cast<float4*>(ws + pl.off_x0);
+
+  BwdParams bp;
+  std::memset(&bp, 0, sizeof bp);
+  bp.B = (int)B;
+  bp.T = (int)T;
+  bp.C = (int)C;
+  bp.NG = pl.NG;
+  bp.nch = pl.nch;
+  bp.chunk_len = kBwdL;
+  bp.k = k;
+  bp.v = v;
+  bp.w = w;
+  bp.u = u;
+  bp.g = gout;
+  bp.s_num = fp.s_num;
+  bp.s_den = fp.s_den;
+  bp.s_max = fp.s_max;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.dw = dw;
+  bp.du = du;
+  if (dstate_in) {
+    bp.d_num = dstate_in->num;
+    bp.d_den = dstate_in->den;
+    bp.d_max = dstate_in->max_e;
+  }
+  bp.x0 = fp.x0;
+  bp.rtot = reinterpret_cast<float4*>(ws + pl.off_rtot);
+  bp.rin = reinterpret_cast<float4*>(ws + pl.off_rin);
+  bp.pdu = reinterpret_cast<float*>(ws + pl.off_pdu);
+  bp.pdw = reinterpret_cast<float*>(ws + pl.off_pdw);
+  if (kv_dtype == WKV_F32) return launch_backward<float>(pl, fp, bp, kv_dtype, st, dev);
+  return launch_backward<__nv_bfloat16>(pl, fp, bp, kv_dtype, st, dev);
 }
 
 wkv_status wkv_query_status(void* workspace, void* stream) {

@@ -1,0 +1,346 @@
+// Backward of the WKV forward: the gradients of a loss L with respect to k, v,
+// w, u and the state passed in, given g = dL/d wkv for every output (no loss
+// term on the final state).
+//
+// The chain rule through the step function of "Linear attention without
+// writing a CUDA kernel", section "The recurrence", run backwards in time.
+// With the state before token t as the pair (N_t, D_t) and the output
+// wkv_t = A_t / Z_t, A_t = N_t + e^{u+k_t} v_t, Z_t = D_t + e^{u+k_t}, the
+// reverse accumulators dN_t = dL/dN_t and dD_t = dL/dD_t obey
+//     dN_t = g_t / Z_t + e^{-w} dN_{t+1},   dD_t = -g_t wkv_t / Z_t + e^{-w} dD_{t+1},
+// a linear recurrence of exactly the forward's shape running the other way:
+// its "keys" are -M_t (M_t the largest exponent in Z_t) and its two value
+// streams are p_t = g_t / z_t and q_t = -g_t wkv_t / z_t (z_t = Z_t e^{-M_t}).
+// So the reverse accumulators use the same anchored arithmetic (Acc: num and
+// den hold the two value streams, the anchor and count give their exponent)
+// and the same associative combine. Then, with R = (dN_{t+1}, dD_{t+1}):
+//     dv_t = g_t e^{u+k_t} / Z_t + e^{k_t} dN_{t+1}
+//     dk_t = g_t e^{u+k_t} (v_t - wkv_t) / Z_t + e^{k_t} (v_t dN_{t+1} + dD_{t+1})
+//     du  += g_t e^{u+k_t} (v_t - wkv_t) / Z_t
+//     dw  -= e^{-w} (N_t dN_{t+1} + D_t dD_{t+1})
+// and dnum0 = e^{m0} dN_0, dden0 = e^{m0} dD_0, dm0 = num0 dnum0 + den0 dden0.
+//
+// The work is cut into chunks of L tokens like the forward's three-launch
+// scan, so that every pass is parallel over (batch row, chunk, channel):
+//   A, S  the forward's chunk totals and their scan: the forward state
+//         entering every chunk (x0);
+//   R1    wkv_bwd_rev_totals: per chunk, the forward replayed from x0 and the
+//         chunk's reverse aggregate (its tokens' contributions to dN, dD at
+//         the chunk's start);
+//   RS    the scan of R1's aggregates from the last chunk backwards: the
+//         reverse state entering every chunk from its end (rin);
+//   R2    wkv_bwd_chunk: per chunk, the forward replayed from x0 (states kept
+//         at every 4th token in registers, the others recomputed), then the
+//         tokens in reverse from rin, writing dk, dv and per-chunk partial sums
+//         of du, dw; chunk 0 also yields the state gradients;
+//   RED   wkv_bwd_reduce: du, dw as compensated sums of the partials over the
+//         chunks and batch rows, in a fixed order.
+// One warp per (batch row, chunk, 32 channels) in R1 and R2; k, v and g are
+// read with coalesced 128-byte loads straight into registers (the second
+// read of a chunk hits L1/L2). All orders of accumulation depend on the shape
+// only, so results are bitwise reproducible.
+#pragma once
+
+#include "wkv_device.cuh"
+#include "wkv_fwd.cuh"
+
+namespace wkv {
+
+struct BwdParams {
+  int B, T, C;
+  int NG;            // 64-channel groups per batch row (layout of x0, rtot, rin)
+  int nch;           // chunks per sequence
+  int chunk_len;
+  const void* k;
+  const void* v;
+  const float* w;
+  const float* u;
+  const float* g;    // dL/d wkv [B, T, C] fp32
+  const float* s_num;  // state in (NULL = empty)
+  const float* s_den;
+  const float* s_max;
+  float* dk;         // [B, T, C] fp32
+  float* dv;
+  float* dw;         // [C] fp32
+  float* du;
+  float* d_num;      // [B, C] state gradients (NULL = not written)
+  float* d_den;
+  float* d_max;
+  const float4* x0;  // forward state entering every chunk [nch][B*NG][64]
+  float4* rtot;      // reverse aggregate of every chunk [nch][B*NG][64] (chunk 0 unused)
+  float4* rin;       // reverse state entering every chunk from its end [nch][B*NG][64]
+  float* pdw;        // per-chunk partial sums [nch][B][C]
+  float* pdu;
+};
+
+__device__ __forceinline__ size_t bwd_slot(const BwdParams& p, int j, int b, int c) {
+  return ((size_t)j * p.B * p.NG + (size_t)b * p.NG + c / 64) * 64 + c % 64;
+}
+
+// The forward state before token t in plain form: num, den and the max
+// exponent m (m = ma - nf w of the anchored state).
+struct Fwd3 {
+  float num, den, m;
+};
+
+// Output statistics of token t from the state before it: the exponent M_t of
+// Z_t, z_t = Z_t e^{-M_t} (>= 1), the current token's weight b_t = e^{u+k_t-M_t}
+// and wkv_t.
+struct OutStat {
+  float M, z, b, out;
+};
+
+__device__ __forceinline__ OutStat out_stat(const Fwd3& s, float k, float v, float u) {
+  const float ku = k + u;
+  const float D = ku - s.m;
+  const float x = ex2(-fabsf(D) * kLog2e);
+  const bool tok = D > 0.f;  // the current token carries the largest exponent
+  const float a = tok ? x : 1.f;
+  const float b = tok ? 1.f : x;
+  OutStat o;
+  o.M = tok ? ku : s.m;
+  o.z = fmaf(a, s.den, b);
+  o.out = fmaf(a, s.num, b * v) * rcp(o.z);
+  o.b = b;
+  return o;
+}
+
+// Adds token t to a reverse accumulator that stands at position t+1: decay by
+// one token, then the token's contribution (p, q) with exponent -M. The
+// accumulator is an Acc: num, den hold the two streams; max exponent
+// ma - nf w relative to its position.
+__device__ __forceinline__ void rev_add(Acc& r, float M, float p, float q, float w) {
+  const float nf1 = r.nf + 1.f;
+  const float Qd = fmaf(-nf1, w, r.ma);
+  const float y = -M;
+  const float d = y - Qd;
+  const float x = ex2(-fabsf(d) * kLog2e);
+  const bool reset = d > 0.f;
+  const float a = reset ? x : 1.f;
+  const float bb = reset ? 1.f : x;
+  r.num = fmaf(a, r.num, bb * p);
+  r.den = fmaf(a, r.den, bb * q);
+  r.ma = reset ? y : r.ma;
+  r.nf = reset ? 0.f : nf1;
+}
+
+template <typename KV>
+__device__ __forceinline__ float ldk(const void* base, size_t i) {
+  return Elem<KV>::to_f32(reinterpret_cast<const KV*>(base)[i]);
+}
+
+// R1. One warp per (batch row, chunk j >= 1, 32 channels); grid
+// B * (nch - 1) * ceil(C / 32) warps, 4 per CTA. The forward is replayed from
+// x0[j] to get M_t, z_t, wkv_t of every token; the chunk's reverse aggregate
+// (relative to its first token: token t enters with exponent
+// -M_t - (t - t0) w) is folded in token order.
+template <typename KV>
+__global__ void __launch_bounds__(128) wkv_bwd_rev_totals(const BwdParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int ngw = (p.C + 31) / 32;
+  const long long n_items = (long long)p.B * (p.nch - 1) * ngw;
+  if (item >= n_items) return;
+  const int gw = (int)(item % ngw);
+  const int j = 1 + (int)((item / ngw) % (p.nch - 1));
+  const int b = (int)(item / ((long long)ngw * (p.nch - 1)));
+  const int c = gw * 32 + lane;
+  if (c >= p.C) return;
+  const float w = __ldg(p.w + c), u = __ldg(p.u + c);
+  Acc s = acc_unpack(p.x0[bwd_slot(p, j, b, c)]);
+  const int t0 = j * p.chunk_len;
+  const int t1 = min(p.T, t0 + p.chunk_len);
+  Acc r = acc_empty();
+  for (int t = t0; t < t1; ++t) {
+    const size_t i = ((size_t)b * p.T + t) * p.C + c;
+    const float k = ldk<KV>(p.k, i), v = ldk<KV>(p.v, i), g = __ldg(p.g + i);
+    const OutStat o = out_stat(Fwd3{s.num, s.den, acc_max_e(s, w)}, k, v, u);
+    const float rz = rcp(o.z);
+    const float pp = g * rz, qq = -g * o.out * rz;
+    // token t's exponent at the chunk's start: -M_t - (t - t0) w, anchored at
+    // -M_t with count t - t0
+    const float cnt = (float)(t - t0);
+    const float Qd = fmaf(-r.nf, w, r.ma);      // the aggregate's exponent
+    const float y = fmaf(-cnt, w, -o.M);         // this token's
+    const float d = y - Qd;
+    const float x = ex2(-fabsf(d) * kLog2e);
+    const bool reset = d > 0.f;
+    const float a = reset ? x : 1.f;
+    const float bb = reset ? 1.f : x;
+    r.num = fmaf(a, r.num, bb * pp);
+    r.den = fmaf(a, r.den, bb * qq);
+    r.ma = reset ? -o.M : r.ma;
+    r.nf = reset ? cnt : r.nf;
+    add_token(s, k, v, w);
+  }
+  p.rtot[bwd_slot(p, j, b, c)] = acc_pack(r);
+}
+
+// RS. The reverse scan of the chunks' reverse aggregates: rin[j] = the reverse
+// state at the end of chunk j from every later chunk (rin[nch-1] empty),
+// rin[j] = combine(rin[j+1], rtot[j+1]) with rin[j+1] decayed across chunk
+// j+1. Same two-level structure as the forward's wkv_tile_scan (16 channels x
+// SEG segments per CTA, segments of about 16 chunks), walking the chunks from
+// the last: index q stands for chunk nch-1-q.
+template <int SEG>
+__global__ void __launch_bounds__(16 * SEG) wkv_bwd_rev_scan(const BwdParams p) {
+  constexpr int CH = 16;
+  __shared__ float4 seg_st[SEG][CH];
+  const int bg = blockIdx.x >> 2;
+  const int ch = threadIdx.x % CH;
+  const int cl = (blockIdx.x & 3) * CH + ch;
+  const int sg = threadIdx.x / CH;
+  const int b = bg / p.NG, c = (bg % p.NG) * 64 + cl;
+  const float w = c < p.C ? __ldg(p.w + c) : 0.f;
+  const int ntot = p.nch - 1;  // aggregates of chunks nch-1 .. 1
+  const int per = (ntot + SEG - 1) / SEG;
+  const int q0 = min(ntot, sg * per), q1 = min(ntot, q0 + per);
+  const float fL = (float)p.chunk_len;
+  auto tot = [&](int q) { return acc_unpack(p.rtot[bwd_slot(p, p.nch - 1 - q, b, c)]); };
+  // 1. this segment's aggregate
+  Acc t = acc_empty();
+  if (c < p.C)
+    for (int q = q0; q < q1; ++q) t = combine(t, tot(q), fL, w);
+  seg_st[sg][ch] = acc_pack(t);
+  __syncthreads();
+  // 2. the state entering every segment
+  if (sg == 0) {
+    Acc x = acc_empty();
+    for (int k = 0; k < SEG; ++k) {
+      const Acc st = acc_unpack(seg_st[k][ch]);
+      const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
+      seg_st[k][ch] = acc_pack(x);
+      x = combine(x, st, (float)(kq1 - kq0) * fL, w);
+    }
+  }
+  __syncthreads();
+  // 3. the state entering every chunk of the segment
+  if (c >= p.C) return;
+  Acc x = acc_unpack(seg_st[sg][ch]);
+  for (int q = q0; q < q1; ++q) {
+    p.rin[bwd_slot(p, p.nch - 1 - q, b, c)] = acc_pack(x);
+    x = combine(x, tot(q), fL, w);
+  }
+  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.rin[bwd_slot(p, 0, b, c)] = acc_pack(x);
+}
+
+// R2. One warp per (batch row, chunk, 32 channels), 4 warps per CTA. Forward
+// replay of the chunk from x0[j] keeping the state at every 4th token (a
+// checkpoint), then the tokens in reverse in groups of 4: the group's four
+// states are recomputed from its checkpoint, and each token, from the last,
+// gives dk, dv and its du, dw terms, then joins the reverse accumulator.
+template <typename KV, int L>
+__global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
+  constexpr int NGRP = L / 4;
+  const int lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int ngw = (p.C + 31) / 32;
+  const long long n_items = (long long)p.B * p.nch * ngw;
+  if (item >= n_items) return;
+  const int gw = (int)(item % ngw);
+  const int j = (int)((item / ngw) % p.nch);
+  const int b = (int)(item / ((long long)ngw * p.nch));
+  const int c = gw * 32 + lane;
+  if (c >= p.C) return;
+  const float w = __ldg(p.w + c), u = __ldg(p.u + c);
+  const int t0 = j * L;
+  const int n = min(L, p.T - t0);
+  const size_t row0 = ((size_t)b * p.T + t0) * p.C + c;
+  const size_t C = (size_t)p.C;
+
+  // ---- forward replay with a checkpoint every 4 tokens
+  Acc ck[NGRP];
+  Acc s = acc_unpack(p.x0[bwd_slot(p, j, b, c)]);
+#pragma unroll
+  for (int gi = 0; gi < NGRP; ++gi) {
+    ck[gi] = s;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int t = gi * 4 + q;
+      if (t < n) add_token(s, ldk<KV>(p.k, row0 + t * C), ldk<KV>(p.v, row0 + t * C), w);
+    }
+  }
+
+  // ---- reverse
+  Acc r = acc_unpack(p.rin[bwd_slot(p, j, b, c)]);
+  float du = 0.f, dw = 0.f;
+  const float ew = ex2(-w * kLog2e);  // e^{-w}
+#pragma unroll
+  for (int gi = NGRP - 1; gi >= 0; --gi) {
+    if (gi * 4 >= n) continue;
+    Fwd3 st[4];
+    float kk[4], vv[4], gg[4];
+    Acc x = ck[gi];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int t = gi * 4 + q;
+      st[q] = Fwd3{x.num, x.den, acc_max_e(x, w)};
+      if (t < n) {
+        kk[q] = ldk<KV>(p.k, row0 + t * C);
+        vv[q] = ldk<KV>(p.v, row0 + t * C);
+        gg[q] = __ldg(p.g + row0 + t * C);
+        add_token(x, kk[q], vv[q], w);
+      }
+    }
+#pragma unroll
+    for (int q = 3; q >= 0; --q) {
+      const int t = gi * 4 + q;
+      if (t >= n) continue;
+      const OutStat o = out_stat(st[q], kk[q], vv[q], u);
+      const float rz = rcp(o.z);
+      const float pp = gg[q] * rz, qq = -gg[q] * o.out * rz;
+      // the reverse accumulator stands at t+1: exponent Q = ma - nf w
+      const float E1 = ex2(fmaf(-r.nf, w, kk[q] + r.ma) * kLog2e);            // e^{k_t + Q}
+      const float E2 = ex2(fmaf(-r.nf, w, st[q].m + r.ma) * kLog2e) * ew;    // e^{m_t + Q - w}
+      const float pb = pp * o.b;
+      p.dv[row0 + t * C] = fmaf(r.num, E1, pb);
+      p.dk[row0 + t * C] = fmaf(E1, fmaf(vv[q], r.num, r.den), pb * (vv[q] - o.out));
+      du = fmaf(pb, vv[q] - o.out, du);
+      dw = fmaf(-E2, fmaf(st[q].num, r.num, st[q].den * r.den), dw);
+      rev_add(r, o.M, pp, qq, w);
+    }
+  }
+  const size_t pi = ((size_t)j * p.B + b) * p.C + c;
+  p.pdu[pi] = du;
+  p.pdw[pi] = dw;
+  if (j == 0 && p.d_num) {
+    // the state passed in: dN_0 = r.num e^{Q}, dD_0 = r.den e^{Q}
+    const size_t si = (size_t)b * p.C + c;
+    float gn = 0.f, gd = 0.f, gm = 0.f;
+    if (p.s_num) {
+      const float num0 = p.s_num[si], den0 = p.s_den[si], m0 = p.s_max[si];
+      if (den0 > 0.f && m0 > kNegBig) {
+        const float f = ex2(fmaf(-r.nf, w, m0 + r.ma) * kLog2e);
+        gn = r.num * f;
+        gd = r.den * f;
+        gm = fmaf(num0, gn, den0 * gd);
+      }
+    }
+    p.d_num[si] = gn;
+    p.d_den[si] = gd;
+    p.d_max[si] = gm;
+  }
+}
+
+// RED. du[c], dw[c]: compensated sums of the partials over (chunk, batch row)
+// in a fixed order (Kahan-Babuska), one thread per channel.
+__global__ void __launch_bounds__(256) wkv_bwd_reduce(const BwdParams p) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= p.C) return;
+  float su = 0.f, cu = 0.f, sw = 0.f, cw = 0.f;
+  const long long n = (long long)p.nch * p.B;
+  for (long long i = 0; i < n; ++i) {
+    const float xu = p.pdu[i * p.C + c], xw = p.pdw[i * p.C + c];
+    float h, e;
+    two_sum(su, xu, h, e);
+    su = h;
+    cu += e;
+    two_sum(sw, xw, h, e);
+    sw = h;
+    cw += e;
+  }
+  p.du[c] = su + cu;
+  p.dw[c] = sw + cw;
+}
+
+}  // namespace wkv
