@@ -151,7 +151,8 @@ def step_bytes(wl) -> int:
     return 36 * wl.B * wl.C + 8 * wl.C
 
 
-KERNEL_NAMES = {1: "wkv_fwd_seq", 2: "wkv_fwd_chunk", 3: "wkv_tile_totals+scan+replay", 4: "wkv_fwd_pipe"}
+KERNEL_NAMES = {1: "wkv_fwd_seq", 2: "wkv_fwd_chunk", 3: "wkv_tile_totals+scan+replay", 4: "wkv_fwd_pipe",
+                5: "wkv_fwd_cluster"}
 
 
 def forward_kernel_name(wl, options) -> str:
@@ -569,6 +570,158 @@ def measure_decode(wl, args, device):
     return rec
 
 
+def measure_backward(wl, args, device):
+    """wkv_backward over workload wl with g ~ N(0, 1): per-call time in a CUDA
+    graph, buffer sets rotated so that no call finds its inputs in L2.
+    Algorithmic bytes: k, v, g read and dk, dv written once (20 B per
+    channel-step in fp32), w, u read and dw, du written, the state in read and
+    its gradient written."""
+    import torch
+
+    import wkv_recurrence_b200 as W
+    from wkv_recurrence_b200 import _abi
+    from wkv_recurrence_b200 import inputs as I
+
+    k, v = I.draw_kv(wl)
+    w, u = I.draw_w(wl), I.draw_u(wl)
+    st = I.draw_state(wl)
+    g = I.draw_r_rows(wl, range(wl.B))
+    bf16 = wl.kv_dtype == "bf16"
+    n = wl.B * wl.T * wl.C
+    kv_es = 2 if bf16 else 4
+    algo = n * (2 * kv_es + 4 + 8) + 16 * wl.C + (24 * wl.B * wl.C if st is not None else 0)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    R = int(min(6, max(2, -(-int(2.5 * l2) // algo))))
+    Wt, U = _to_dev(w, device), _to_dev(u, device)
+    S_in = None if st is None else tuple(_to_dev(x, device) for x in st)
+    ws_bytes = _abi.lib().wkv_backward_workspace_size(wl.B, wl.T, wl.C)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    L = _abi.lib()
+    P = ctypes.c_void_p
+    sets = []
+    for _ in range(R):
+        d = dict(K=_to_dev(k, device, bf16), V=_to_dev(v, device, bf16), G=_to_dev(g, device),
+                 dk=torch.empty(wl.B, wl.T, wl.C, device=device), dv=torch.empty(wl.B, wl.T, wl.C, device=device),
+                 dw=torch.empty(wl.C, device=device), du=torch.empty(wl.C, device=device),
+                 ds=tuple(torch.empty(wl.B, wl.C, device=device) for _ in range(3)))
+        d["sin"] = None if S_in is None else _abi.wkv_cstate(*(x.data_ptr() for x in S_in))
+        d["sout"] = _abi.wkv_state(*(x.data_ptr() for x in d["ds"]))
+        sets.append(d)
+
+    def call(d, h=None):
+        code = L.wkv_backward(wl.B, wl.T, wl.C, P(d["K"].data_ptr()), P(d["V"].data_ptr()),
+                              _abi.WKV_BF16 if bf16 else _abi.WKV_F32, P(Wt.data_ptr()), P(U.data_ptr()),
+                              ctypes.byref(d["sin"]) if d["sin"] is not None else None, P(d["G"].data_ptr()),
+                              P(d["dk"].data_ptr()), P(d["dv"].data_ptr()), P(d["dw"].data_ptr()),
+                              P(d["du"].data_ptr()), ctypes.byref(d["sout"]), P(ws.data_ptr()), ws_bytes,
+                              h if h is not None else P(torch.cuda.current_stream(device).cuda_stream))
+        if code:
+            _abi.check(code, "wkv_backward")
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(3, args.warmup)):
+        call(sets[i % R])
+    torch.cuda.synchronize(device)
+    g_bwd = _capture(sets, call, stream, device)
+    g_bwd.replay()
+    torch.cuda.synchronize(device)
+    n_rep = max(1, -(-max(1, args.steps // 20) // R))
+    sampler = ClockSampler(torch.cuda.current_device()) if not args.no_clocks else None
+    if sampler:
+        sampler.start()
+    ms = _timed_graph(g_bwd, n_rep, stream, device)
+    clocks = sampler.stop() if sampler else None
+    call_ms = ms / (n_rep * R)
+    peak, peak_kind = measured_peaks()
+    achieved = algo / (call_ms / 1e3) / 1e9
+    traffic, xu_pct = recorded_traffic("wkv_backward", wl.name)
+    launches = 6 if wl.T > 32 else 4
+    rec = {
+        "workload": f"wkv_backward {wl.kv_dtype} B={wl.B} T={wl.T} C={wl.C} (gradients of sum(g * wkv), "
+                    f"g ~ N(0, 1){', state in' if st is not None else ''})",
+        "name": f"backward_{wl.name}", "value": n / (call_ms / 1e3), "unit": UNIT, "steps": n_rep * R,
+        "ms_per_step": call_ms,
+        "roofline": {"bound": "hbm", "kernel": "wkv_backward (6 launches)", "achieved": achieved, "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "xu_pipe_pct_of_peak": xu_pct, "algorithmic_bytes": algo, "launch_ms": call_ms},
+        "gpu_launches": launches * n_rep * R, "clocks": clocks, "buffer_sets": R,
+        "l2": f"calls rotate over {R} separate buffer sets ({R * algo / 2**20:.0f} MiB of algorithmic traffic)",
+    }
+    del g_bwd, sets, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
+# fp32 SIMT peak of a B200 for the matrix-state kernel's roofline: 148 SMs x
+# 128 fp32 lanes x 2 flops per fused multiply-add x the 1965 MHz maximum clock
+V6_FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measure_v6(wl, args, device):
+    """wkv_v6_forward over the v6 workload: per-call time in a CUDA graph over
+    rotating buffer sets. Roofline: fp32 instruction issue, 5 D^2 flops per
+    (token, head) (update: a product and a fused multiply-add per state entry;
+    readout: a fused multiply-add per entry) against the fp32 SIMT peak; HBM
+    bytes (r, w, k, v read, y written) reported beside it."""
+    import torch
+
+    import wkv_recurrence_b200 as W
+    from wkv_recurrence_b200 import inputs as I
+
+    r, w, k, v = I.draw_v6(wl)
+    bf16 = wl.kv_dtype == "bf16"
+    n = wl.B * wl.T * wl.H * wl.D
+    es = 2 if bf16 else 4
+    hbm = n * (3 * es + 4 + (2 if wl.out_dtype == "bf16" else 4))
+    flops = 5 * wl.B * wl.T * wl.H * wl.D * wl.D
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    R = int(min(6, max(2, -(-int(2.5 * l2) // hbm))))
+    out_dtype = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
+    sets = []
+    for _ in range(R):
+        sets.append(dict(r=_to_dev(r, device, bf16), w=_to_dev(w, device), k=_to_dev(k, device, bf16),
+                         v=_to_dev(v, device, bf16),
+                         y=torch.empty(wl.B, wl.T, wl.H, wl.D, dtype=out_dtype, device=device),
+                         s=torch.empty(wl.B, wl.H, wl.D, wl.D, device=device)))
+    stream = torch.cuda.current_stream(device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+
+    def call(d, h=None):
+        # on the current stream: the capture's side stream while capturing
+        W.v6_forward(d["r"], d["w"], d["k"], d["v"], None, out=d["y"], state_out=d["s"], workspace=ws)
+
+    for i in range(max(3, args.warmup)):
+        call(sets[i % R])
+    torch.cuda.synchronize(device)
+    g6 = _capture(sets, call, stream, device)
+    g6.replay()
+    torch.cuda.synchronize(device)
+    n_rep = max(1, -(-max(1, args.steps // 20) // R))
+    sampler = ClockSampler(torch.cuda.current_device()) if not args.no_clocks else None
+    if sampler:
+        sampler.start()
+    ms = _timed_graph(g6, n_rep, stream, device)
+    clocks = sampler.stop() if sampler else None
+    call_ms = ms / (n_rep * R)
+    tflops = flops / (call_ms / 1e3) / 1e12
+    peak, peak_kind = measured_peaks()
+    rec = {
+        "workload": f"wkv_v6_forward {wl.kv_dtype} B={wl.B} T={wl.T} H={wl.H} D={wl.D} (matrix-valued state, "
+                    "zero state in, state out)",
+        "name": wl.name, "value": n / (call_ms / 1e3), "unit": "channel-steps/s (B*T*H*D per s)",
+        "steps": n_rep * R, "ms_per_step": call_ms,
+        "roofline": {"bound": "alu", "kernel": "wkv6_fwd", "achieved": tflops, "peak": V6_FP32_PEAK_TFLOPS,
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz", "unit": "TFLOP/s",
+                     "frac": tflops / V6_FP32_PEAK_TFLOPS, "traffic": None, "algorithmic_flops": flops,
+                     "hbm_achieved_gbs": hbm / (call_ms / 1e3) / 1e9, "hbm_frac_of_measured": hbm / (call_ms / 1e3) / 1e9 / peak,
+                     "launch_ms": call_ms},
+        "gpu_launches": n_rep * R, "clocks": clocks, "buffer_sets": R,
+    }
+    del g6, sets
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args):
     import torch
 
@@ -591,12 +744,23 @@ def run_ours(args):
                 subs[name] = measure_decode(swl, args, device)
             else:
                 subs[name] = measure_forward(swl, args, None, device, rank, world, headline=False)
+        from wkv_recurrence_b200 import inputs as I
+        for name in ("layer", "long"):
+            subs[f"backward_{name}"] = measure_backward(workload(args, name), args, device)
+        subs["v6"] = measure_v6(I.V6_WORKLOADS["v6"], args, device)
 
     if rank == 0 and world == 1 and not args.no_cpu:
         main["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds, one_core_s=args.cpu_seconds / 2)
         for name, rec in subs.items():
+            if name.startswith("backward_") or name == "v6":
+                continue
             rec["cpu_baseline"] = cpu_baseline(workload(args, name), budget_s=args.cpu_seconds / 3,
                                                one_core_s=args.cpu_seconds / 4, decode=(name == "decode"))
+        for name in ("layer", "long"):
+            subs[f"backward_{name}"]["cpu_baseline"] = cpu_baseline_backward(workload(args, name),
+                                                                             budget_s=args.cpu_seconds / 3)
+        from wkv_recurrence_b200 import inputs as I
+        subs["v6"]["cpu_baseline"] = cpu_baseline_v6(I.V6_WORKLOADS["v6"], budget_s=args.cpu_seconds / 3)
 
     if rank == 0:
         bf16 = wl.kv_dtype == "bf16"
@@ -729,6 +893,55 @@ def cpu_baseline(wl, budget_s=10.0, one_core_s=5.0, decode=False):
     _set_oracle_threads(O, cores)
     return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
             "value_1core": one, "sample_1core": one_sample, "cpu_model": cpu_model()}
+
+
+def cpu_baseline_backward(wl, budget_s=3.0):
+    """The float64 oracle backward on a slice of the workload, all host cores."""
+    import numpy as np
+
+    from oracle import oracle as O
+    from wkv_recurrence_b200 import inputs as I
+    O.build()
+    cores = os.cpu_count() or 1
+    _set_oracle_threads(O, cores)
+    rows = 1
+    cols = min(wl.C, 256)
+    T = min(wl.T, 4096)
+    k, v = I.draw_kv_rows(wl, range(rows), T=T)
+    k, v = k[:, :, :cols].copy(), v[:, :, :cols].copy()
+    w, u = I.draw_w(wl)[:cols].copy(), I.draw_u(wl)[:cols].copy()
+    g = np.random.default_rng(0).normal(size=k.shape)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        O.recurrence_backward(k, v, w, u, g, threads=cores)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": rows * T * cols * reps / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"float64 C backward recurrence on row 0, channels 0..{cols - 1}, tokens 0..{T - 1} of the "
+                      f"{wl.name} workload, {reps} repetition(s), {dt:.1f} s", "cpu_model": cpu_model()}
+
+
+def cpu_baseline_v6(wl, budget_s=3.0):
+    """The float64 numpy oracle of the matrix-valued state on a slice of the workload."""
+    from oracle import v6_oracle as V
+    from wkv_recurrence_b200 import inputs as I
+    T = 64
+    r, w, k, v = I.draw_v6(wl, T=T)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        V.recurrence(r, w, k, v)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": wl.B * T * wl.H * wl.D * reps / dt, "unit": "channel-steps/s (B*T*H*D per s)",
+            "cores": 1, "kind": "oracle",
+            "sample": f"float64 numpy recurrence on tokens 0..{T - 1} of every head of the {wl.name} workload, "
+                      f"{reps} repetition(s), {dt:.1f} s", "cpu_model": cpu_model()}
 
 
 def run_reference(args):

@@ -304,6 +304,37 @@ WKV_API wkv_status wkv_backward(int64_t B, int64_t T, int64_t C,
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The RWKV-v6 matrix-valued state ("RWKV-v6 Architecture: Attention-Free
+ * Linear Transformers", section "3. Matrix-Valued Hidden State"): per head a
+ * D x D state S, and for every token
+ *     S_t = diag(w_t) S_{t-1} + k_t v_t^T,     y_t = sigmoid(r_t) * (S_t k_t)
+ * (row i of S decays by w_t[i]; the readout multiplies the updated state by
+ * k_t, as the page writes it). A different operator from wkv_forward: no
+ * denominator and no max exponent.
+ *
+ *   r, k, v    [B, T, H, D], element type kv_dtype
+ *   w          [B, T, H, D] fp32: the decay factor itself, in [0, 1] (the
+ *              page's exp(-exp(.)) of a projection)
+ *   y          [B, T, H, D], element type y_dtype ((F32, F32), (BF16, BF16)
+ *              or (BF16, F32))
+ *   state_in   NULL (zero state) or [B, H, D, D] fp32, S[b][h][i][j] with i
+ *              the row (key) index; state_out NULL or the same shape, may
+ *              alias state_in
+ *   D          32, 64 or 128
+ *   workspace  at least 256 bytes, 256-byte aligned, zero-filled before its
+ *              first use: its status word reports device-side wait timeouts
+ *              (wkv_query_status)
+ * r, w, k, v must be 16-byte aligned (WKV_ERR_MISALIGNED otherwise). The
+ * arithmetic and the state are fp32; results are bitwise reproducible. A
+ * decode step is a call with T = 1.
+ */
+WKV_API wkv_status wkv_v6_forward(int64_t B, int64_t T, int64_t H, int64_t D,
+                        const void *r, const float *w, const void *k, const void *v, wkv_dtype kv_dtype,
+                        void *y, wkv_dtype y_dtype,
+                        const float *state_in, float *state_out,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * wkv_forward without a caller-provided workspace. The pages have no
  * counterpart to this entry point; it exists for callers that cannot allocate
  * device memory themselves: hosts that hand a plug-in only its input and

@@ -70,17 +70,18 @@ def _check_call(oracle, L, B, T, C, seed, with_state, misaligned, what):
 
 
 def test_noalloc_matches_oracle_on_calls_in_a_row(oracle):
-    """Two aligned calls (the three-launch scan, whose scratch holds chunk totals
-    and incoming states), then two misaligned calls (the single-launch scan,
-    whose flags and epoch must start from zero in the shared array after the
-    other kernel used it), each against the oracle."""
+    """Aligned calls (the cluster scan, which uses only the status word, and
+    the three-launch scan, whose scratch holds chunk totals and incoming
+    states), then two misaligned calls (the single-launch scan, whose flags and
+    epoch must start from zero in the shared array after the other kernels
+    used it), each against the oracle."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from wkv_recurrence_b200 import build
     build.build()
     L = _abi.lib()
-    assert W.forward_kernel(4, 1000, 256) == 3 and W.forward_kernel(3, 2049, 192) == 3
-    cases = [(4, 1000, 256, True, False), (3, 2049, 192, False, False),
+    assert W.forward_kernel(4, 1000, 256) == 5 and W.forward_kernel(3, 3000, 192) == 3
+    cases = [(4, 1000, 256, True, False), (3, 3000, 192, False, False), (2, 2049, 128, True, False),
              (2, 1500, 128, True, True), (3, 777, 64, False, True)]
     for call, (B, T, C, with_state, misaligned) in enumerate(cases):
         _check_call(oracle, L, B, T, C, 500 + call, with_state, misaligned,

@@ -14,7 +14,8 @@ fails loudly if it is missing or no CUDA device is present.
 """
 
 from .api import (WKV, PreparedForward, PreparedStep, WkvError, backward, empty_state, forward,  # noqa: F401
-                  forward_kernel, forward_launches, make_workspace, query_status, step, workspace_size)
+                  forward_kernel, forward_launches, make_workspace, query_status, step, v6_forward,
+                  workspace_size)
 
-__all__ = ["forward", "step", "backward", "WKV", "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
+__all__ = ["forward", "step", "backward", "WKV", "v6_forward", "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
            "PreparedForward", "PreparedStep", "WkvError"]

@@ -25,7 +25,8 @@ WKV_BF16 = 1
 # entry points declared in include/wkv.h
 EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward_launches", "wkv_forward",
            "wkv_forward_ext", "wkv_step", "wkv_step_ext", "wkv_query_status", "wkv_status_string", "wkv_version",
-           "wkv_forward_noalloc", "wkv_last_cuda_error", "wkv_backward_workspace_size", "wkv_backward")
+           "wkv_forward_noalloc", "wkv_last_cuda_error", "wkv_backward_workspace_size", "wkv_backward",
+           "wkv_v6_forward")
 
 # size of the library's built-in scratch array used by wkv_forward_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -102,6 +103,8 @@ def lib() -> ctypes.CDLL:
         L.wkv_backward.argtypes = [I64, I64, I64, P, P, I, P, P, ctypes.POINTER(wkv_cstate), P,
                                    P, P, P, P, ctypes.POINTER(wkv_state), P, SZ, P]
         L.wkv_backward.restype = I
+        L.wkv_v6_forward.argtypes = [I64, I64, I64, I64, P, P, P, P, I, P, I, P, P, P, SZ, P]
+        L.wkv_v6_forward.restype = I
         L.wkv_query_status.argtypes = [P, P]
         L.wkv_query_status.restype = I
         L.wkv_status_string.argtypes = [I]

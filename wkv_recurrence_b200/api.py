@@ -265,6 +265,42 @@ def backward(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
     return dk, dv, dw, du, dstate
 
 
+def v6_forward(r: torch.Tensor, w: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+               state: Optional[torch.Tensor] = None, *, out_dtype: Optional[torch.dtype] = None,
+               out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+               return_state: bool = True, workspace: Optional[torch.Tensor] = None):
+    """The RWKV-v6 matrix-valued state over a sequence: r, k, v [B, T, H, D]
+    (float32 or bfloat16), w [B, T, H, D] float32 decay factors; state
+    [B, H, D, D] float32 or None. Returns (y [B, T, H, D], state after the
+    last token or None)."""
+    _need_cuda(k, "k")
+    _need_cuda(v, "v", k.dtype)
+    _need_cuda(r, "r", k.dtype)
+    _need_cuda(w, "w", torch.float32)
+    if k.dim() != 4 or v.shape != k.shape or r.shape != k.shape or w.shape != k.shape:
+        raise ValueError("r, w, k, v must all be [B, T, H, D]")
+    B, T, H, D = k.shape
+    out_dtype = out_dtype or k.dtype
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=out_dtype, device=k.device)
+    _need_cuda(out, "out", out_dtype)
+    if state is not None:
+        _need_cuda(state, "state", torch.float32)
+        if state.shape != (B, H, D, D):
+            raise ValueError("state must be [B, H, D, D]")
+    if return_state and state_out is None:
+        state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=k.device)
+    if state_out is not None:
+        _need_cuda(state_out, "state_out", torch.float32)
+    if workspace is None:
+        workspace = _default_workspace(256, k.device)
+    code = _abi.lib().wkv_v6_forward(B, T, H, D, _ptr(r), _ptr(w), _ptr(k), _ptr(v), _dtype_code(k, "k"), _ptr(out),
+                                   _dtype_code(out, "out"), _ptr(state), _ptr(state_out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream())
+    _abi.check(code, "wkv_v6_forward")
+    return out, state_out
+
+
 class WKV(torch.autograd.Function):
     """The operator as a torch autograd function: forward through wkv_forward,
     backward through wkv_backward (per-channel w, float32 or bfloat16 k and v,

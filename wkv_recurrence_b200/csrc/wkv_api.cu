@@ -19,6 +19,7 @@
 #include "wkv_device.cuh"
 #include "wkv_fwd.cuh"
 #include "wkv_step.cuh"
+#include "wkv_v6.cuh"
 
 namespace wkv {
 namespace {
@@ -726,6 +727,57 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
 }
 
 // ---------------------------------------------------------------------------
+// RWKV-v6 matrix-valued state
+// ---------------------------------------------------------------------------
+// [rows, cols] row-major tensor, box [box_rows, box_cols]
+bool make_tmap_2d(CUtensorMap* m, const void* base, wkv_dtype dt, int64_t rows, int64_t cols, int box_rows,
+                  int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const size_t es = dt == WKV_F32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * es)};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt == WKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr int kV6Rows = 16;  // state rows per CTA
+constexpr int kV6Tokens = 32;  // tokens per staged block
+
+template <typename KV, typename OUT, int D>
+wkv_status launch_v6(const V6Params& p, const void* r, const float* w, const void* k, const void* v, wkv_dtype kvdt,
+                     cudaStream_t st, int dev) {
+  const int64_t rows = (int64_t)p.B * p.T, cols = (int64_t)p.H * D;
+  CUtensorMap tk, tv, tr, tw;
+  if (!make_tmap_2d(&tk, k, kvdt, rows, cols, kV6Tokens, D) || !make_tmap_2d(&tv, v, kvdt, rows, cols, kV6Tokens, D) ||
+      !make_tmap_2d(&tr, r, kvdt, rows, cols, kV6Tokens, kV6Rows) ||
+      !make_tmap_2d(&tw, w, WKV_F32, rows, cols, kV6Tokens, kV6Rows))
+    return WKV_ERR_CUDA;
+  const size_t smem = 2 * v6_stage_bytes<KV, D, kV6Rows, kV6Tokens>() + 16;
+  auto fn = wkv6_fwd<KV, OUT, D, kV6Rows>;
+  int occ = 0;
+  if (!kernel_setup(fn, dev, kV6Rows * 4, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  const long long grid = (long long)p.B * p.H * (D / kV6Rows);
+  if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  fn<<<(unsigned)grid, kV6Rows * 4, smem, st>>>(p, tk, tv, tr, tw);
+  return launch_result();
+}
+
+template <typename KV, typename OUT>
+wkv_status launch_v6_d(int64_t D, const V6Params& p, const void* r, const float* w, const void* k, const void* v,
+                       wkv_dtype kvdt, cudaStream_t st, int dev) {
+  switch (D) {
+    case 32: return launch_v6<KV, OUT, 32>(p, r, w, k, v, kvdt, st, dev);
+    case 64: return launch_v6<KV, OUT, 64>(p, r, w, k, v, kvdt, st, dev);
+    default: return launch_v6<KV, OUT, 128>(p, r, w, k, v, kvdt, st, dev);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // backward
 // ---------------------------------------------------------------------------
 constexpr int kBwdL = 32;  // tokens per chunk of the backward
@@ -1036,6 +1088,53 @@ wkv_status wkv_step(int64_t S, int64_t C, const void* k, const void* v, wkv_dtyp
                     const float* u, void* out, wkv_dtype out_dtype, const wkv_cstate* state_in,
                     const wkv_state* state_out, void* stream) {
   return wkv_step_ext(S, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, stream, nullptr);
+}
+
+wkv_status wkv_v6_forward(int64_t B, int64_t T, int64_t H, int64_t D, const void* r, const float* w, const void* k,
+                        const void* v, wkv_dtype kv_dtype, void* y, wkv_dtype y_dtype, const float* state_in,
+                        float* state_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || T < 0 || H < 0) return WKV_ERR_INVALID_ARG;
+  if (D != 32 && D != 64 && D != 128) return WKV_ERR_INVALID_ARG;
+  if (T >= (1ll << 24) || H >= (1ll << 20) || B >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  if (B > 0 && H > 0 && T > (int64_t)((1ull << 40) / (uint64_t)(B * H))) return WKV_ERR_INVALID_ARG;
+  if (kv_dtype != WKV_F32 && kv_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (y_dtype != WKV_F32 && y_dtype != WKV_BF16) return WKV_ERR_UNSUPPORTED_DTYPE;
+  if (kv_dtype == WKV_F32 && y_dtype != WKV_F32) return WKV_ERR_UNSUPPORTED_DTYPE;
+  const int64_t n = B * T * H * D;
+  if (n > 0 && (!r || !w || !k || !v || !y)) return WKV_ERR_INVALID_ARG;
+  if (!workspace) return WKV_ERR_INVALID_ARG;
+  if (workspace_bytes < sizeof(WsHeader)) return WKV_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
+  // TMA: 16-byte aligned bases (the row pitch H*D*size is a multiple of 16 for D >= 32)
+  if (n > 0 && (!aligned(r, 16) || !aligned(w, 16) || !aligned(k, 16) || !aligned(v, 16))) return WKV_ERR_MISALIGNED;
+  if (B * H == 0) return WKV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // the state passes through
+    if (state_out && state_out != state_in) {
+      const size_t bytes = sizeof(float) * (size_t)(B * H * D * D);
+      if (state_in) {
+        if (!cuda_ok(cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, st))) return WKV_ERR_CUDA;
+      } else if (!cuda_ok(cudaMemsetAsync(state_out, 0, bytes, st))) {
+        return WKV_ERR_CUDA;
+      }
+    }
+    return WKV_OK;
+  }
+  int dev = 0;
+  if (!cuda_ok(cudaGetDevice(&dev))) return WKV_ERR_CUDA;
+  V6Params p;
+  std::memset(&p, 0, sizeof p);
+  p.B = (int)B;
+  p.T = (int)T;
+  p.H = (int)H;
+  p.y = y;
+  p.s_in = state_in;
+  p.s_out = state_out;
+  p.hdr = static_cast<WsHeader*>(workspace);
+  p.timeout_ns = kDefaultTimeoutNs;
+  if (kv_dtype == WKV_F32) return launch_v6_d<float, float>(D, p, r, w, k, v, kv_dtype, st, dev);
+  if (y_dtype == WKV_BF16) return launch_v6_d<__nv_bfloat16, __nv_bfloat16>(D, p, r, w, k, v, kv_dtype, st, dev);
+  return launch_v6_d<__nv_bfloat16, float>(D, p, r, w, k, v, kv_dtype, st, dev);
 }
 
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C) {

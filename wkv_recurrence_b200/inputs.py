@@ -290,3 +290,50 @@ def random_case(B: int, T: int, C: int, seed: int, *, k_scale: float = 1.0,
         mx = g.normal(1.0, 2.0, (B, C)).astype(np.float32)
         st = (num, den, mx)
     return k, v, w, u, st
+
+
+# ---------------------------------------------------------------------------
+# the RWKV-v6 matrix-valued state ("RWKV-v6 Architecture", section
+# "3. Matrix-Valued Hidden State")
+# ---------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class V6Workload:
+    name: str
+    code: int
+    B: int
+    T: int
+    H: int
+    D: int
+    kv_dtype: str = "f32"
+    out_dtype: str = "f32"
+
+
+V6_WORKLOADS = {
+    # the MicroRWKV layer width (768 = 12 heads x 64) at its block length
+    "v6": V6Workload("v6", 20, B=8, T=1024, H=12, D=64),
+    "v6_bf16": V6Workload("v6_bf16", 21, B=8, T=1024, H=12, D=64, kv_dtype="bf16", out_dtype="bf16"),
+}
+
+
+def draw_v6(wl: V6Workload, seed: int = 0, T: int | None = None):
+    """r, w, k, v [B, T, H, D]: r, k, v ~ N(0, 1) (bf16 codes for bf16
+    workloads), w = exp(-exp(N(-1, 1))) fp32 (the page's decay form applied to
+    a standard-normal projection shifted by -1). Each (tensor, batch row) from
+    its own generator."""
+    T = wl.T if T is None else T
+    shape = (T, wl.H, wl.D)
+    bf16 = wl.kv_dtype == "bf16"
+    out = {}
+    for name, code in (("r", 0), ("w", 1), ("k", 2), ("v", 3)):
+        dt = np.float32 if (name == "w" or not bf16) else np.uint16
+        arr = np.empty((wl.B,) + shape, dt)
+        for b in range(wl.B):
+            g = _rng(seed, wl.code, 100 + code, b)
+            if name == "w":
+                arr[b] = np.exp(-np.exp(g.normal(-1.0, 1.0, shape))).astype(np.float32)
+            else:
+                x = g.standard_normal(shape, dtype=np.float32)
+                arr[b] = f32_to_bf16_bits(x) if bf16 else x
+        out[name] = arr
+    return out["r"], out["w"], out["k"], out["v"]
