@@ -57,7 +57,10 @@ typedef enum {
     WKV_ERR_MISALIGNED = 3,         /* workspace not 256-byte aligned (misaligned k, v, out: slower path, no error) */
     WKV_ERR_WORKSPACE_TOO_SMALL = 4,
     WKV_ERR_CUDA = 5,               /* a CUDA runtime call failed (no device, launch error) */
-    WKV_ERR_WAIT_TIMEOUT = 6        /* device side: a bounded wait gave up (see wkv_query_status) */
+    WKV_ERR_WAIT_TIMEOUT = 6,       /* device side: a bounded wait gave up (see wkv_query_status) */
+    WKV_ERR_BOUNDS = 7              /* device side, the bounds-checked build (libwkv_debug.so, compiled
+                                       with -DWKV_DEBUG) only: an index outside its array was caught and
+                                       the access skipped (see wkv_query_status) */
 } wkv_status;
 
 typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
@@ -368,7 +371,8 @@ WKV_API wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C,
 
 /*
  * Synchronises `stream`, then reads and clears the device-side status word in
- * `workspace` (a wkv_forward workspace). Returns WKV_OK, WKV_ERR_WAIT_TIMEOUT
+ * `workspace` (a wkv_forward, wkv_backward or wkv_v6_forward workspace).
+ * Returns WKV_OK, WKV_ERR_BOUNDS (bounds-checked build only), WKV_ERR_WAIT_TIMEOUT
  * if a device-side wait of an earlier call gave up (its outputs are then not
  * valid), or WKV_ERR_CUDA if the synchronisation itself failed.
  */

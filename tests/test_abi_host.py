@@ -68,7 +68,7 @@ def test_binding_structs_match_the_header(tmp_path):
 
 
 def test_status_strings(L):
-    for code in range(7):
+    for code in range(8):
         s = _abi.status_string(code)
         assert s and s != "unknown status"
     assert _abi.status_string(99) == "unknown status"

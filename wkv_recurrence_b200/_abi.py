@@ -9,7 +9,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "_build", "libwkv.so")
+# WKV_LIBRARY=debug selects the bounds-checked build (libwkv_debug.so)
+LIB_PATH = os.path.join(HERE, "_build", "libwkv_debug.so" if os.environ.get("WKV_LIBRARY") == "debug"
+                        else "libwkv.so")
 
 WKV_OK = 0
 WKV_ERR_INVALID_ARG = 1
@@ -18,6 +20,7 @@ WKV_ERR_MISALIGNED = 3
 WKV_ERR_WORKSPACE_TOO_SMALL = 4
 WKV_ERR_CUDA = 5
 WKV_ERR_WAIT_TIMEOUT = 6
+WKV_ERR_BOUNDS = 7
 
 WKV_F32 = 0
 WKV_BF16 = 1

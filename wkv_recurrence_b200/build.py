@@ -2,8 +2,13 @@
 
     python -m wkv_recurrence_b200.build            # build if sources changed
     python -m wkv_recurrence_b200.build --force    # always rebuild
+    python -m wkv_recurrence_b200.build --debug    # also the bounds-checked libwkv_debug.so
 
-nvcc cross-compiles, so this runs on a machine without a GPU.
+nvcc cross-compiles, so this runs on a machine without a GPU. The
+bounds-checked variant (-DWKV_DEBUG) checks the indices of the kernels'
+stores and workspace accesses and reports a violation through the status
+word (WKV_ERR_BOUNDS from wkv_query_status) instead of touching memory; the
+binding loads it instead of libwkv.so when WKV_LIBRARY=debug is set.
 """
 from __future__ import annotations
 
@@ -17,6 +22,7 @@ ROOT = os.path.dirname(HERE)
 SRC_DIR = os.path.join(HERE, "csrc")
 MAIN = os.path.join(SRC_DIR, "wkv_api.cu")
 LIB = os.path.join(HERE, "_build", "libwkv.so")
+LIB_DEBUG = os.path.join(HERE, "_build", "libwkv_debug.so")
 HEADER = os.path.join(ROOT, "include", "wkv.h")
 
 NVCC_FLAGS = [
@@ -39,19 +45,31 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
+    out = LIB_DEBUG if debug else LIB
     newest = max(os.path.getmtime(p) for p in _sources())
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
-        return LIB
-    os.makedirs(os.path.dirname(LIB), exist_ok=True)
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-o", tmp, MAIN]
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest:
+        return out
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DWKV_DEBUG"] if debug else []), *extra_flags, "-o", tmp, MAIN]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
+
+
+def build_all(force: bool = False, verbose: bool = False):
+    """Both variants, compiled concurrently."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(2) as ex:
+        futs = [ex.submit(build, force, verbose, (), d) for d in (False, True)]
+        return [f.result() for f in futs]
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    if "--debug" in sys.argv:
+        print(build_all(force="--force" in sys.argv, verbose=True))
+    else:
+        print(build(force="--force" in sys.argv, verbose=True))

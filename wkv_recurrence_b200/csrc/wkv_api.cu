@@ -888,6 +888,7 @@ const char* wkv_status_string(wkv_status s) {
     case WKV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case WKV_ERR_CUDA: return "CUDA runtime error";
     case WKV_ERR_WAIT_TIMEOUT: return "device-side wait timed out";
+    case WKV_ERR_BOUNDS: return "device-side index out of bounds (bounds-checked build)";
   }
   return "unknown status";
 }
@@ -1233,6 +1234,7 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const void* k, const vo
   bp.rin = reinterpret_cast<float4*>(ws + pl.off_rin);
   bp.pdu = reinterpret_cast<float*>(ws + pl.off_pdu);
   bp.pdw = reinterpret_cast<float*>(ws + pl.off_pdw);
+  bp.hdr = fp.hdr;
   if (kv_dtype == WKV_F32) return launch_backward<float>(pl, fp, bp, kv_dtype, st, dev);
   return launch_backward<__nv_bfloat16>(pl, fp, bp, kv_dtype, st, dev);
 }
@@ -1248,6 +1250,7 @@ wkv_status wkv_query_status(void* workspace, void* stream) {
     const uint32_t zero = 0;
     if (!cuda_ok(cudaMemcpy(&h->status, &zero, sizeof zero, cudaMemcpyHostToDevice))) return WKV_ERR_CUDA;
   }
+  if (bits & kStatusBoundsError) return WKV_ERR_BOUNDS;
   return (bits & kStatusWaitTimeout) ? WKV_ERR_WAIT_TIMEOUT : WKV_OK;
 }
 

@@ -71,6 +71,7 @@ struct BwdParams {
   float4* rin;       // reverse state entering every chunk from its end [nch][B*NG][64]
   float* pdw;        // per-chunk partial sums [nch][B][C]
   float* pdu;
+  WsHeader* hdr;     // status word (bounds-checked build)
 };
 
 __device__ __forceinline__ size_t bwd_slot(const BwdParams& p, int j, int b, int c) {
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(128) wkv_bwd_rev_totals(const BwdParams p) {
     r.nf = reset ? cnt : r.nf;
     add_token(s, k, v, w);
   }
-  p.rtot[bwd_slot(p, j, b, c)] = acc_pack(r);
+  if (WKV_IN(p.hdr, bwd_slot(p, j, b, c), (size_t)p.nch * p.B * p.NG * 64)) p.rtot[bwd_slot(p, j, b, c)] = acc_pack(r);
 }
 
 // RS. The reverse scan of the chunks' reverse aggregates: rin[j] = the reverse
@@ -217,8 +218,10 @@ __global__ void __launch_bounds__(16 * SEG) wkv_bwd_rev_scan(const BwdParams p) 
   // 3. the state entering every chunk of the segment
   if (c >= p.C) return;
   Acc x = acc_unpack(seg_st[sg][ch]);
+  const size_t n_slots = (size_t)p.nch * p.B * p.NG * 64;  // (bounds-checked build)
+  (void)n_slots;
   for (int q = q0; q < q1; ++q) {
-    p.rin[bwd_slot(p, p.nch - 1 - q, b, c)] = acc_pack(x);
+    if (WKV_IN(p.hdr, bwd_slot(p, p.nch - 1 - q, b, c), n_slots)) p.rin[bwd_slot(p, p.nch - 1 - q, b, c)] = acc_pack(x);
     x = combine(x, tot(q), fL, w);
   }
   if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.rin[bwd_slot(p, 0, b, c)] = acc_pack(x);
@@ -247,6 +250,9 @@ __global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
   const int n = min(L, p.T - t0);
   const size_t row0 = ((size_t)b * p.T + t0) * p.C + c;
   const size_t C = (size_t)p.C;
+  if (!WKV_IN(p.hdr, (size_t)b * p.T + t0 + n - 1, (size_t)p.B * p.T) ||
+      !WKV_IN(p.hdr, ((size_t)j * p.B + b) * p.C + c, (size_t)p.nch * p.B * p.C))
+    return;
 
   // ---- forward replay with a checkpoint every 4 tokens
   Acc ck[NGRP];

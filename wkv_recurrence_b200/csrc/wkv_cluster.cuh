@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(NW * 32)
   cluster_arrive();  // done with the other CTAs' shared memory
 
   // ---- 4. replay the span
-  if (nv > 0 && copy_ok) {
+  if (nv > 0 && copy_ok && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
     Acc st = kWT ? combine_wt(x, pre, wpre) : combine(x, pre, (float)(wp * J), w);
     OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c;
     const KV* rrow = p.r ? reinterpret_cast<const KV*>(p.r) + ((size_t)b * T + ts) * C + c : nullptr;
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(NW * 32)
       st = s1[0];
     }
     // the warp that holds the last token writes the state out
-    if (p.o_num && cok && ts + nv == T) {
+    if (p.o_num && cok && ts + nv == T && WKV_IN(p.hdr, (size_t)b * C + c, (size_t)p.B * C)) {
       const size_t i = (size_t)b * C + c;
       p.o_num[i] = st.num;
       p.o_den[i] = st.den;

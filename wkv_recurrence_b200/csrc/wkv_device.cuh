@@ -23,6 +23,7 @@ constexpr float kBonusClamp = 44.0f;
 
 // device-side status bits, kept in the workspace header
 constexpr uint32_t kStatusWaitTimeout = 1u;
+constexpr uint32_t kStatusBoundsError = 2u;  // bounds-checked build only
 
 struct WsHeader {
   uint32_t ticket;   // next tile to hand out (chunked kernel)
@@ -32,6 +33,23 @@ struct WsHeader {
   uint32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+// ---------------------------------------------------------------------------
+// Index checks of the bounds-checked build (compiled with -DWKV_DEBUG): an
+// index outside its array sets kStatusBoundsError in the status word of the
+// call's workspace header and the access is skipped; nothing traps, so the
+// context stays usable and wkv_query_status reports it. In the ordinary build
+// every check is the constant true and compiles away.
+// ---------------------------------------------------------------------------
+#ifdef WKV_DEBUG
+__device__ __forceinline__ bool dbg_ok(WsHeader* h, bool in_bounds) {
+  if (!in_bounds && h) atomicOr(&h->status, kStatusBoundsError);
+  return in_bounds;
+}
+#define WKV_IN(h, i, n) ::wkv::dbg_ok((h), (unsigned long long)(i) < (unsigned long long)(n))
+#else
+#define WKV_IN(h, i, n) true
+#endif
 
 // ---------------------------------------------------------------------------
 // PTX wrappers

@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       const int c = c0 + e;
-      if (c < C) st[e] = acc_unpack(p.x0[((size_t)jc * p.B * p.NG + (size_t)b * p.NG + c / 64) * 64 + c % 64]);
+      const size_t xi = ((size_t)jc * p.B * p.NG + (size_t)b * p.NG + c / 64) * 64 + c % 64;
+      if (c < C && WKV_IN(p.hdr, xi, (size_t)p.nch * p.B * p.NG * 64)) st[e] = acc_unpack(p.x0[xi]);
     }
   }
   fast = __all_sync(0xffffffffu, fast);  // one path per warp
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(THREADS)
     const int nv = min(LT, tend - t0);
     OUT* orow = out + ((size_t)b * T + t0) * C;
     const size_t rrow = ((size_t)b * T + t0) * C;
-    if (c0 < C) {
+    if (c0 < C && WKV_IN(p.hdr, (size_t)b * T + t0 + nv - 1, (size_t)p.B * T)) {
       if (kWT) {
         for (int j = 0; j < nv; ++j) {
           float kx[VEC], vx[VEC], wx[VEC], o[VEC];
@@ -331,8 +332,8 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       const int c = c0 + e;
-      if (c < C) {
-        const size_t i = (size_t)b * C + c;
+      const size_t i = (size_t)b * C + c;
+      if (c < C && WKV_IN(p.hdr, i, (size_t)p.B * C)) {
         p.o_num[i] = st[e].num;
         p.o_den[i] = st[e].den;
         p.o_max[i] = kWT ? acc_max_e_wt(st[e], lo[e]) : acc_max_e(st[e], w[e]);
@@ -693,7 +694,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     if (wp == NW - 1) {
 #pragma unroll
       for (int e = 0; e < VEC; ++e) tot[e] = combine(pre[e], acc_unpack(sh_agg[wp * CG + cl + e]), (float)nv, w[e]);
-      if (!last_chunk) {
+      if (!last_chunk && WKV_IN(p.hdr, (size_t)tile * CG + cl + VEC - 1, (size_t)p.n_tiles * CG)) {
         float4* dst = p.agg_a + (size_t)tile * CG + cl;
 #pragma unroll
         for (int e = 0; e < VEC; ++e)
@@ -715,7 +716,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       if (lane == 0 && !inject) st_release_u32(p.flags_p + (size_t)qb * BNG + bg, target);
     }
     // 3. replay this warp's tokens from shared memory
-    if (nv > 0 && copy_ok) {
+    if (nv > 0 && copy_ok && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
       float cb[VEC];
       bool fast = true;
 #pragma unroll
@@ -918,6 +919,7 @@ __global__ void __launch_bounds__(NW * 32)
     float4* dst = p.agg_a + (size_t)tile * CG + cl;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
+      if (!WKV_IN(p.hdr, (size_t)tile * CG + cl + e, (size_t)(p.nch - 1) * BNG * CG)) continue;
       dst[e] = acc_pack(t[e]);
       if (kWT) p.wtot[(size_t)tile * CG + cl + e] = wt[e];
     }
@@ -956,6 +958,8 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   const float4* tot_of = p.agg_a + (size_t)bg * CG + cl;  // chunk q's total at tot_of[q * BNG * CG]
   const float* wtot_of = kWT ? p.wtot + (size_t)bg * CG + cl : nullptr;
   const size_t qs = (size_t)BNG * CG;
+  const size_t n_x0 = (size_t)p.nch * qs;  // x0 entries (bounds-checked build)
+  (void)n_x0;
   // one combine of a chunk total (its decay sum wq with per-token decays)
   auto comb = [&](const Acc& x, const float4& t, float wq) {
     return kWT ? combine_wt(x, acc_unpack(t), wq) : combine(x, acc_unpack(t), fL, w);
@@ -1024,7 +1028,7 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       if (q0 + r < q1) {
-        x0_of[(q0 + r) * qs] = acc_pack(x);
+        if (WKV_IN(p.hdr, (size_t)bg * CG + cl + (q0 + r) * qs, n_x0)) x0_of[(q0 + r) * qs] = acc_pack(x);
         x = comb(x, a0[r], w0[r]);
       }
     }
@@ -1042,13 +1046,15 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         if (qq + r < q1) {
-          x0_of[(qq + r) * qs] = acc_pack(x);
+          if (WKV_IN(p.hdr, (size_t)bg * CG + cl + (qq + r) * qs, n_x0)) x0_of[(qq + r) * qs] = acc_pack(x);
           x = comb(x, a[r], wa[r]);
         }
       }
     }
   }
-  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) x0_of[ntot * qs] = acc_pack(x);
+  if (((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) &&
+      WKV_IN(p.hdr, (size_t)bg * CG + cl + (size_t)ntot * qs, n_x0))
+    x0_of[ntot * qs] = acc_pack(x);
 }
 
 // ---------------------------------------------------------------------------
@@ -1269,7 +1275,7 @@ __global__ void __launch_bounds__((2 * NC + 2) * 32)
           tt[e] = combine(tt[e], a[e], (float)nv, w[e]);
           tot[(size_t)s * CG + cl + e] = acc_pack(tt[e]);
         }
-        if (j != p.nch - 1) {
+        if (j != p.nch - 1 && WKV_IN(p.hdr, (size_t)tile * CG + cl + VEC - 1, (size_t)p.n_tiles * CG)) {
           const int b = bg / p.NG;
           float4* dst = p.agg_a + (size_t)tile * CG + cl;
 #pragma unroll
@@ -1300,7 +1306,7 @@ __global__ void __launch_bounds__((2 * NC + 2) * 32)
       const int nv = max(0, min(J, T - ts));
       const bool last_chunk = (j == p.nch - 1);
       const int p_last = last_chunk ? (T - 1 - j * L) / J : NC - 1;
-      if (nv > 0) {
+      if (nv > 0 && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
         float w[VEC], u[VEC], cb[VEC];
         bool fast = true;
 #pragma unroll

@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(RB * 4)
       float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
       a += __shfl_xor_sync(0xffffffffu, a, 1);
       a += __shfl_xor_sync(0xffffffffu, a, 2);
-      if (q == 0) y[(((size_t)row0 + blk * TB + tt) * p.H + h) * D + i] = Elem<OUT>::from_f32(gate(a, rr));
+      const size_t yi = (((size_t)row0 + blk * TB + tt) * p.H + h) * D + i;
+      if (q == 0 && WKV_IN(p.hdr, yi, (size_t)p.B * T * p.H * D)) y[yi] = Elem<OUT>::from_f32(gate(a, rr));
     }
     __syncthreads();  // every thread is done with stage s
     if (tid == 0 && blk + 2 < nblk) {
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(RB * 4)
     }
     return;
   }
-  if (p.s_out) {
+  if (p.s_out && WKV_IN(p.hdr, srow + D - 1, (size_t)p.B * p.H * D * D)) {
 #pragma unroll
     for (int m = 0; m < CPT; ++m)
 #pragma unroll
