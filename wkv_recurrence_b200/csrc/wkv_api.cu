@@ -745,25 +745,25 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, wkv_dtype dt, int64_t rows, 
   return r == CUDA_SUCCESS;
 }
 
-constexpr int kV6Rows = 16;  // state rows per CTA
 constexpr int kV6Tokens = 32;  // tokens per staged block
 
 template <typename KV, typename OUT, int D>
 wkv_status launch_v6(const V6Params& p, const void* r, const float* w, const void* k, const void* v, wkv_dtype kvdt,
                      cudaStream_t st, int dev) {
+  constexpr int RB = V6Shape<KV, D>::kRows;  // state rows per CTA
   const int64_t rows = (int64_t)p.B * p.T, cols = (int64_t)p.H * D;
   CUtensorMap tk, tv, tr, tw;
   if (!make_tmap_2d(&tk, k, kvdt, rows, cols, kV6Tokens, D) || !make_tmap_2d(&tv, v, kvdt, rows, cols, kV6Tokens, D) ||
-      !make_tmap_2d(&tr, r, kvdt, rows, cols, kV6Tokens, kV6Rows) ||
-      !make_tmap_2d(&tw, w, WKV_F32, rows, cols, kV6Tokens, kV6Rows))
+      !make_tmap_2d(&tr, r, kvdt, rows, cols, kV6Tokens, RB) ||
+      !make_tmap_2d(&tw, w, WKV_F32, rows, cols, kV6Tokens, RB))
     return WKV_ERR_CUDA;
-  const size_t smem = 2 * v6_stage_bytes<KV, D, kV6Rows, kV6Tokens>() + 16;
-  auto fn = wkv6_fwd<KV, OUT, D, kV6Rows>;
+  const size_t smem = 2 * v6_stage_bytes<KV, D, RB, kV6Tokens>() + 16;
+  auto fn = wkv6_fwd<KV, OUT, D, RB>;
   int occ = 0;
-  if (!kernel_setup(fn, dev, kV6Rows * 4, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
-  const long long grid = (long long)p.B * p.H * (D / kV6Rows);
+  if (!kernel_setup(fn, dev, 128, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  const long long grid = (long long)p.B * p.H * (D / RB);
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  fn<<<(unsigned)grid, kV6Rows * 4, smem, st>>>(p, tk, tv, tr, tw);
+  fn<<<(unsigned)grid, 128, smem, st>>>(p, tk, tv, tr, tw);
   return launch_result();
 }
 

@@ -78,51 +78,91 @@ __device__ __forceinline__ size_t bwd_slot(const BwdParams& p, int j, int b, int
   return ((size_t)j * p.B * p.NG + (size_t)b * p.NG + c / 64) * 64 + c % 64;
 }
 
-// The forward state before token t in plain form: num, den and the max
-// exponent m (m = ma - nf w of the anchored state).
-struct Fwd3 {
-  float num, den, m;
-};
-
-// Output statistics of token t from the state before it: the exponent M_t of
-// Z_t, z_t = Z_t e^{-M_t} (>= 1), the current token's weight b_t = e^{u+k_t-M_t}
-// and wkv_t.
+// Exponents are kept ANCHORED, as in the forward: never as one rounded fp32
+// number of large magnitude, but as an exact key plus integer multiples of w
+// (and, for the output's largest exponent, possibly u), so that the difference
+// of two exponents -- the only thing an exponential here ever needs -- is
+// formed at its own magnitude. (With keys of +-60 and the reverse exponents
+// near -60, rounding the exponents themselves would cost ~1e-5 of relative
+// accuracy per gradient.)
+//
+// The output's largest exponent of token t is M_t = max(m_t, k_t + u) with
+// m_t = ma - nf w the state's: anchored as (key, uf, cnt) with
+// M_t = key - cnt w + uf u, either (ma, 0, nf) or (k_t, 1, 0).
 struct OutStat {
-  float M, z, b, out;
+  float key, uf, cnt;  // M_t = key - cnt w + uf u
+  float z;             // Z_t e^{-M_t} (>= 1)
+  float b;             // e^{u + k_t - M_t}, the current token's weight
+  float out;           // wkv_t
 };
 
-__device__ __forceinline__ OutStat out_stat(const Fwd3& s, float k, float v, float u) {
-  const float ku = k + u;
-  const float D = ku - s.m;
+__device__ __forceinline__ OutStat out_stat(const Acc& s, float k, float v, float u, float w) {
+  // D = (k + u) - m, formed as (k - ma) + u + nf w
+  const float D = fmaf(s.nf, w, (k - s.ma) + u);
   const float x = ex2(-fabsf(D) * kLog2e);
   const bool tok = D > 0.f;  // the current token carries the largest exponent
   const float a = tok ? x : 1.f;
   const float b = tok ? 1.f : x;
   OutStat o;
-  o.M = tok ? ku : s.m;
+  o.key = tok ? k : s.ma;
+  o.uf = tok ? 1.f : 0.f;
+  o.cnt = tok ? 0.f : s.nf;
   o.z = fmaf(a, s.den, b);
   o.out = fmaf(a, s.num, b * v) * rcp(o.z);
   o.b = b;
   return o;
 }
 
-// Adds token t to a reverse accumulator that stands at position t+1: decay by
-// one token, then the token's contribution (p, q) with exponent -M. The
-// accumulator is an Acc: num, den hold the two streams; max exponent
-// ma - nf w relative to its position.
-__device__ __forceinline__ void rev_add(Acc& r, float M, float p, float q, float w) {
-  const float nf1 = r.nf + 1.f;
-  const float Qd = fmaf(-nf1, w, r.ma);
-  const float y = -M;
-  const float d = y - Qd;
+// A reverse accumulator (dN, dD) = (rn, rd) e^{Q} at some position, with
+// Q = -qk - qu u + qc w: the anchor token's -M (qk its key, qu its u flag) and
+// qc = its count minus its distance from the position (an integer).
+struct RAcc {
+  float rn, rd, qk, qc, qu;
+};
+
+constexpr float kPosBig = 1.0e30f;  // qk of the empty accumulator (Q = -1e30)
+
+__device__ __forceinline__ RAcc racc_empty() { return RAcc{0.f, 0.f, kPosBig, 0.f, 0.f}; }
+
+// Packed as a float4: qc + qu / 2 in the last slot (qc is an integer below
+// 2^22 in magnitude, so the half is exact).
+__device__ __forceinline__ float4 racc_pack(const RAcc& r) { return make_float4(r.rn, r.rd, r.qk, r.qc + 0.5f * r.qu); }
+__device__ __forceinline__ RAcc racc_unpack(const float4& f) {
+  const float qc = floorf(f.w);
+  return RAcc{f.x, f.y, f.z, qc, 2.f * (f.w - qc)};
+}
+
+// Adds a token whose exponent at the accumulator's position is
+// -key - uf u + cnt w, with value streams (p, q).
+__device__ __forceinline__ void racc_add(RAcc& r, float key, float uf, float cnt, float p, float q, float w,
+                                         float u) {
+  const float d = fmaf(cnt - r.qc, w, (r.qk - key) + (r.qu - uf) * u);  // token's exponent - Q
   const float x = ex2(-fabsf(d) * kLog2e);
-  const bool reset = d > 0.f;
-  const float a = reset ? x : 1.f;
-  const float bb = reset ? 1.f : x;
-  r.num = fmaf(a, r.num, bb * p);
-  r.den = fmaf(a, r.den, bb * q);
-  r.ma = reset ? y : r.ma;
-  r.nf = reset ? 0.f : nf1;
+  const bool tok = d > 0.f;
+  const float a = tok ? x : 1.f;
+  const float bb = tok ? 1.f : x;
+  r.rn = fmaf(a, r.rn, bb * p);
+  r.rd = fmaf(a, r.rd, bb * q);
+  r.qk = tok ? key : r.qk;
+  r.qu = tok ? uf : r.qu;
+  r.qc = tok ? cnt : r.qc;
+}
+
+// `a` stands `len` tokens after `b`'s position (it covers the tokens after
+// b's): moved to b's position and merged. Associative, the empty accumulator
+// is the identity.
+__device__ __forceinline__ RAcc racc_combine(const RAcc& a, const RAcc& b, float len, float w, float u) {
+  const float ac = a.qc - len;
+  const float d = fmaf(ac - b.qc, w, (b.qk - a.qk) + (b.qu - a.qu) * u);  // a's exponent - b's
+  const bool a_wins = d >= 0.f;
+  const float s = ex2(-fabsf(d) * kLog2e);
+  RAcc r;
+  r.rn = a_wins ? fmaf(s, b.rn, a.rn) : fmaf(s, a.rn, b.rn);
+  r.rd = a_wins ? fmaf(s, b.rd, a.rd) : fmaf(s, a.rd, b.rd);
+  r.qk = a_wins ? a.qk : b.qk;
+  r.qu = a_wins ? a.qu : b.qu;
+  r.qc = a_wins ? ac : b.qc;
+  return r;
 }
 
 template <typename KV>
@@ -151,30 +191,17 @@ __global__ void __launch_bounds__(128) wkv_bwd_rev_totals(const BwdParams p) {
   Acc s = acc_unpack(p.x0[bwd_slot(p, j, b, c)]);
   const int t0 = j * p.chunk_len;
   const int t1 = min(p.T, t0 + p.chunk_len);
-  Acc r = acc_empty();
+  RAcc r = racc_empty();  // at the chunk's first token
   for (int t = t0; t < t1; ++t) {
     const size_t i = ((size_t)b * p.T + t) * p.C + c;
     const float k = ldk<KV>(p.k, i), v = ldk<KV>(p.v, i), g = __ldg(p.g + i);
-    const OutStat o = out_stat(Fwd3{s.num, s.den, acc_max_e(s, w)}, k, v, u);
+    const OutStat o = out_stat(s, k, v, u, w);
     const float rz = rcp(o.z);
-    const float pp = g * rz, qq = -g * o.out * rz;
-    // token t's exponent at the chunk's start: -M_t - (t - t0) w, anchored at
-    // -M_t with count t - t0
-    const float cnt = (float)(t - t0);
-    const float Qd = fmaf(-r.nf, w, r.ma);      // the aggregate's exponent
-    const float y = fmaf(-cnt, w, -o.M);         // this token's
-    const float d = y - Qd;
-    const float x = ex2(-fabsf(d) * kLog2e);
-    const bool reset = d > 0.f;
-    const float a = reset ? x : 1.f;
-    const float bb = reset ? 1.f : x;
-    r.num = fmaf(a, r.num, bb * pp);
-    r.den = fmaf(a, r.den, bb * qq);
-    r.ma = reset ? -o.M : r.ma;
-    r.nf = reset ? cnt : r.nf;
+    // token t's exponent at the chunk's start: -M_t - (t - t0) w
+    racc_add(r, o.key, o.uf, o.cnt - (float)(t - t0), g * rz, -g * o.out * rz, w, u);
     add_token(s, k, v, w);
   }
-  if (WKV_IN(p.hdr, bwd_slot(p, j, b, c), (size_t)p.nch * p.B * p.NG * 64)) p.rtot[bwd_slot(p, j, b, c)] = acc_pack(r);
+  if (WKV_IN(p.hdr, bwd_slot(p, j, b, c), (size_t)p.nch * p.B * p.NG * 64)) p.rtot[bwd_slot(p, j, b, c)] = racc_pack(r);
 }
 
 // RS. The reverse scan of the chunks' reverse aggregates: rin[j] = the reverse
@@ -193,38 +220,39 @@ __global__ void __launch_bounds__(16 * SEG) wkv_bwd_rev_scan(const BwdParams p) 
   const int sg = threadIdx.x / CH;
   const int b = bg / p.NG, c = (bg % p.NG) * 64 + cl;
   const float w = c < p.C ? __ldg(p.w + c) : 0.f;
+  const float u = c < p.C ? __ldg(p.u + c) : 0.f;
   const int ntot = p.nch - 1;  // aggregates of chunks nch-1 .. 1
   const int per = (ntot + SEG - 1) / SEG;
   const int q0 = min(ntot, sg * per), q1 = min(ntot, q0 + per);
   const float fL = (float)p.chunk_len;
-  auto tot = [&](int q) { return acc_unpack(p.rtot[bwd_slot(p, p.nch - 1 - q, b, c)]); };
+  auto tot = [&](int q) { return racc_unpack(p.rtot[bwd_slot(p, p.nch - 1 - q, b, c)]); };
   // 1. this segment's aggregate
-  Acc t = acc_empty();
+  RAcc t = racc_empty();
   if (c < p.C)
-    for (int q = q0; q < q1; ++q) t = combine(t, tot(q), fL, w);
-  seg_st[sg][ch] = acc_pack(t);
+    for (int q = q0; q < q1; ++q) t = racc_combine(t, tot(q), fL, w, u);
+  seg_st[sg][ch] = racc_pack(t);
   __syncthreads();
   // 2. the state entering every segment
   if (sg == 0) {
-    Acc x = acc_empty();
+    RAcc x = racc_empty();
     for (int k = 0; k < SEG; ++k) {
-      const Acc st = acc_unpack(seg_st[k][ch]);
+      const RAcc st = racc_unpack(seg_st[k][ch]);
       const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
-      seg_st[k][ch] = acc_pack(x);
-      x = combine(x, st, (float)(kq1 - kq0) * fL, w);
+      seg_st[k][ch] = racc_pack(x);
+      x = racc_combine(x, st, (float)(kq1 - kq0) * fL, w, u);
     }
   }
   __syncthreads();
   // 3. the state entering every chunk of the segment
   if (c >= p.C) return;
-  Acc x = acc_unpack(seg_st[sg][ch]);
+  RAcc x = racc_unpack(seg_st[sg][ch]);
   const size_t n_slots = (size_t)p.nch * p.B * p.NG * 64;  // (bounds-checked build)
   (void)n_slots;
   for (int q = q0; q < q1; ++q) {
-    if (WKV_IN(p.hdr, bwd_slot(p, p.nch - 1 - q, b, c), n_slots)) p.rin[bwd_slot(p, p.nch - 1 - q, b, c)] = acc_pack(x);
-    x = combine(x, tot(q), fL, w);
+    if (WKV_IN(p.hdr, bwd_slot(p, p.nch - 1 - q, b, c), n_slots)) p.rin[bwd_slot(p, p.nch - 1 - q, b, c)] = racc_pack(x);
+    x = racc_combine(x, tot(q), fL, w, u);
   }
-  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.rin[bwd_slot(p, 0, b, c)] = acc_pack(x);
+  if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.rin[bwd_slot(p, 0, b, c)] = racc_pack(x);
 }
 
 // R2. One warp per (batch row, chunk, 32 channels), 4 warps per CTA. Forward
@@ -268,19 +296,18 @@ __global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
   }
 
   // ---- reverse
-  Acc r = acc_unpack(p.rin[bwd_slot(p, j, b, c)]);
+  RAcc r = racc_unpack(p.rin[bwd_slot(p, j, b, c)]);  // at the chunk's end
   float du = 0.f, dw = 0.f;
-  const float ew = ex2(-w * kLog2e);  // e^{-w}
 #pragma unroll
   for (int gi = NGRP - 1; gi >= 0; --gi) {
     if (gi * 4 >= n) continue;
-    Fwd3 st[4];
+    Acc st[4];
     float kk[4], vv[4], gg[4];
     Acc x = ck[gi];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int t = gi * 4 + q;
-      st[q] = Fwd3{x.num, x.den, acc_max_e(x, w)};
+      st[q] = x;
       if (t < n) {
         kk[q] = ldk<KV>(p.k, row0 + t * C);
         vv[q] = ldk<KV>(p.v, row0 + t * C);
@@ -292,33 +319,35 @@ __global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
     for (int q = 3; q >= 0; --q) {
       const int t = gi * 4 + q;
       if (t >= n) continue;
-      const OutStat o = out_stat(st[q], kk[q], vv[q], u);
+      const OutStat o = out_stat(st[q], kk[q], vv[q], u, w);
       const float rz = rcp(o.z);
       const float pp = gg[q] * rz, qq = -gg[q] * o.out * rz;
-      // the reverse accumulator stands at t+1: exponent Q = ma - nf w
-      const float E1 = ex2(fmaf(-r.nf, w, kk[q] + r.ma) * kLog2e);            // e^{k_t + Q}
-      const float E2 = ex2(fmaf(-r.nf, w, st[q].m + r.ma) * kLog2e) * ew;    // e^{m_t + Q - w}
+      // the reverse accumulator stands at t+1: Q = -qk - qu u + qc w
+      const float E1 = ex2(fmaf(r.qc, w, (kk[q] - r.qk) - r.qu * u) * kLog2e);                     // e^{k_t + Q}
+      const float E2 = ex2(fmaf(r.qc - st[q].nf - 1.f, w, (st[q].ma - r.qk) - r.qu * u) * kLog2e);  // e^{m_t + Q - w}
       const float pb = pp * o.b;
-      p.dv[row0 + t * C] = fmaf(r.num, E1, pb);
-      p.dk[row0 + t * C] = fmaf(E1, fmaf(vv[q], r.num, r.den), pb * (vv[q] - o.out));
+      p.dv[row0 + t * C] = fmaf(r.rn, E1, pb);
+      p.dk[row0 + t * C] = fmaf(E1, fmaf(vv[q], r.rn, r.rd), pb * (vv[q] - o.out));
       du = fmaf(pb, vv[q] - o.out, du);
-      dw = fmaf(-E2, fmaf(st[q].num, r.num, st[q].den * r.den), dw);
-      rev_add(r, o.M, pp, qq, w);
+      dw = fmaf(-E2, fmaf(st[q].num, r.rn, st[q].den * r.rd), dw);
+      // move the accumulator to position t and add token t
+      r.qc -= 1.f;
+      racc_add(r, o.key, o.uf, o.cnt, pp, qq, w, u);
     }
   }
   const size_t pi = ((size_t)j * p.B + b) * p.C + c;
   p.pdu[pi] = du;
   p.pdw[pi] = dw;
   if (j == 0 && p.d_num) {
-    // the state passed in: dN_0 = r.num e^{Q}, dD_0 = r.den e^{Q}
+    // the state passed in: dN_0 = rn e^{Q}, dD_0 = rd e^{Q}
     const size_t si = (size_t)b * p.C + c;
     float gn = 0.f, gd = 0.f, gm = 0.f;
     if (p.s_num) {
       const float num0 = p.s_num[si], den0 = p.s_den[si], m0 = p.s_max[si];
       if (den0 > 0.f && m0 > kNegBig) {
-        const float f = ex2(fmaf(-r.nf, w, m0 + r.ma) * kLog2e);
-        gn = r.num * f;
-        gd = r.den * f;
+        const float f = ex2(fmaf(r.qc, w, (m0 - r.qk) - r.qu * u) * kLog2e);  // e^{m0 + Q}
+        gn = r.rn * f;
+        gd = r.rd * f;
         gm = fmaf(num0, gn, den0 * gd);
       }
     }

@@ -186,22 +186,31 @@ __global__ void __launch_bounds__(NW * 32)
       const float w1[1] = {w};
       Acc s1[1] = {st};
       if (fast && nv == J) {
-        constexpr int NB = J < 8 ? J : 8;
+        // the span's hot loop, compiled once with and once without the gate
+        auto span = [&](auto gated) {
+          constexpr bool kGate = decltype(gated)::value;
+          constexpr int NB = J < 8 ? J : 8;
 #pragma unroll
-        for (int j0 = 0; j0 < J; j0 += NB) {
-          float kb[NB][1], vb[NB][1], ob[NB][1], rb[NB];
+          for (int j0 = 0; j0 < J; j0 += NB) {
+            float kb[NB][1], vb[NB][1], ob[NB][1], rb[NB];
 #pragma unroll
-          for (int jj = 0; jj < NB; ++jj) {
-            load_vec<KV, 1>(ks + (j0 + jj) * CG, kb[jj]);
-            load_vec<KV, 1>(vs + (j0 + jj) * CG, vb[jj]);
-            rb[jj] = rrow ? Elem<KV>::to_f32(rrow[(size_t)(j0 + jj) * C]) : 0.f;
+            for (int jj = 0; jj < NB; ++jj) {
+              load_vec<KV, 1>(ks + (j0 + jj) * CG, kb[jj]);
+              load_vec<KV, 1>(vs + (j0 + jj) * CG, vb[jj]);
+              if (kGate) rb[jj] = Elem<KV>::to_f32(rrow[(size_t)(j0 + jj) * C]);
+            }
+            step_tokens<NB, 1>(s1, kb, vb, w1, cb, ob);
+#pragma unroll
+            for (int jj = 0; jj < NB; ++jj) {
+              const float o = kGate ? gate(ob[jj][0], rb[jj]) : ob[jj][0];
+              if (cok) orow[(size_t)(j0 + jj) * C] = Elem<OUT>::from_f32(o);
+            }
           }
-          step_tokens<NB, 1>(s1, kb, vb, w1, cb, ob);
-#pragma unroll
-          for (int jj = 0; jj < NB; ++jj) {
-            const float o = rrow ? gate(ob[jj][0], rb[jj]) : ob[jj][0];
-            if (cok) orow[(size_t)(j0 + jj) * C] = Elem<OUT>::from_f32(o);
-          }
+        };
+        if (rrow) {
+          span(Flag<true>{});
+        } else {
+          span(Flag<false>{});
         }
       } else {
         for (int i = 0; i < nv; ++i) {

@@ -110,6 +110,13 @@ __device__ __forceinline__ void store_out(OUT* row, int c0, int C, bool vec_ok, 
   }
 }
 
+// A compile-time flag passed to generic lambdas (so that one body is compiled
+// once per value).
+template <bool V>
+struct Flag {
+  static constexpr bool value = V;
+};
+
 // The receptance gate on VEC outputs of one token row (out = sigmoid(r) wkv),
 // when the call has one: r is [B, T, C] with the element type of k and v;
 // `row` is the offset of (b, t, 0).
@@ -265,21 +272,31 @@ __global__ void __launch_bounds__(THREADS)
           store_out<OUT, VEC>(orow + (size_t)j * C, c0, C, vec_ok, o);
         }
       } else if (nv == LT && fast) {
-        constexpr int NB = LT < 8 ? LT : 8;  // tokens per block of step_tokens
+        // the tile's hot loop, compiled once with and once without the gate
+        // (no per-token test of p.r)
+        auto tile = [&](auto gated) {
+          constexpr bool kGate = decltype(gated)::value;
+          constexpr int NB = LT < 8 ? LT : 8;  // tokens per block of step_tokens
 #pragma unroll
-        for (int j0 = 0; j0 < LT; j0 += NB) {
-          float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
+          for (int j0 = 0; j0 < LT; j0 += NB) {
+            float kb[NB][VEC], vb[NB][VEC], ob[NB][VEC];
 #pragma unroll
-          for (int jj = 0; jj < NB; ++jj) {
-            load_vec<KV, VEC>(ks + (j0 + jj) * CG, kb[jj]);
-            load_vec<KV, VEC>(vs + (j0 + jj) * CG, vb[jj]);
+            for (int jj = 0; jj < NB; ++jj) {
+              load_vec<KV, VEC>(ks + (j0 + jj) * CG, kb[jj]);
+              load_vec<KV, VEC>(vs + (j0 + jj) * CG, vb[jj]);
+            }
+            step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
+#pragma unroll
+            for (int jj = 0; jj < NB; ++jj) {
+              if (kGate) gate_row<KV, VEC>(p, rrow + (size_t)(j0 + jj) * C, c0, ob[jj]);
+              store_out<OUT, VEC>(orow + (size_t)(j0 + jj) * C, c0, C, vec_ok, ob[jj]);
+            }
           }
-          step_tokens<NB, VEC>(st, kb, vb, w, cb, ob);
-#pragma unroll
-          for (int jj = 0; jj < NB; ++jj) {
-            gate_row<KV, VEC>(p, rrow + (size_t)(j0 + jj) * C, c0, ob[jj]);
-            store_out<OUT, VEC>(orow + (size_t)(j0 + jj) * C, c0, C, vec_ok, ob[jj]);
-          }
+        };
+        if (p.r) {
+          tile(Flag<true>{});
+        } else {
+          tile(Flag<false>{});
         }
       } else if (nv == LT) {
 #pragma unroll 4

@@ -5,8 +5,8 @@
 // Row i of the state evolves on its own (it decays by w_t[i] and gains
 // k_t[i] v_t^T) and y_t[i] reads only row i, so the rows are independent
 // recurrences: this kernel gives each CTA a block of RB rows of one head and
-// walks the sequence, each row's state in registers of 4 threads (16
-// columns each for D = 64).
+// walks the sequence, each row's state in registers of NQ threads (8 for
+// D >= 64: 8 columns each in fp32 at D = 64), 128 threads per CTA.
 //
 // Why no tensor cores here: the readout and the update are per-row dot
 // products and rank-1 updates with a decay that differs per row, so the only
@@ -20,9 +20,9 @@
 // Inputs stream through shared memory in blocks of TB tokens (TMA, two stages
 // on mbarriers): the block's k and v rows of the head (every row block needs
 // all D columns) and the block's r and w for this CTA's rows. Thread q of a
-// row owns the 16-byte column chunks q, q+4, q+8, ... so that the four
-// threads of a row read four different bank groups, and the rows of a warp
-// read the same addresses (broadcast).
+// row owns the 16-byte column chunks q, q+NQ, q+2NQ, ... so that the threads
+// of a row read different bank groups, and the rows of a warp read the same
+// addresses (broadcast).
 #pragma once
 
 #include "wkv_device.cuh"
@@ -52,11 +52,20 @@ __host__ __device__ constexpr size_t v6_stage_bytes() {
   return (size_t)TB * (2 * D * sizeof(KV) + RB * sizeof(KV) + RB * sizeof(float));
 }
 
+// Threads per state row and rows per CTA (128 threads) for head size D.
+template <typename KV, int D>
+struct V6Shape {
+  static constexpr int kChunks = D * (int)sizeof(KV) / 16;           // 16-byte chunks per row
+  static constexpr int kThreadsPerRow = kChunks < 8 ? kChunks : 8;
+  static constexpr int kRows = 128 / kThreadsPerRow;
+};
+
 template <typename KV, typename OUT, int D, int RB>
-__global__ void __launch_bounds__(RB * 4)
+__global__ void __launch_bounds__(128)
     wkv6_fwd(const V6Params p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
              const __grid_constant__ CUtensorMap tmr, const __grid_constant__ CUtensorMap tmw) {
-  constexpr int NQ = 4;                        // threads per row
+  constexpr int NQ = V6Shape<KV, D>::kThreadsPerRow;  // threads per row
+  static_assert(RB * NQ == 128, "128 threads per CTA");
   constexpr int TB = 32;                       // tokens per staged block
   constexpr int EPC = 16 / sizeof(KV);         // elements per 16-byte chunk
   constexpr int NCH = D / EPC;                 // chunks per row
@@ -142,8 +151,8 @@ __global__ void __launch_bounds__(RB * 4)
         }
       }
       float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
+#pragma unroll
+      for (int o = 1; o < NQ; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
       const size_t yi = (((size_t)row0 + blk * TB + tt) * p.H + h) * D + i;
       if (q == 0 && WKV_IN(p.hdr, yi, (size_t)p.B * T * p.H * D)) y[yi] = Elem<OUT>::from_f32(gate(a, rr));
     }
