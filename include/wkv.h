@@ -288,7 +288,7 @@ WKV_API wkv_status wkv_step_ext(int64_t S, int64_t C,
  *              aligned and C * element size a multiple of 16 bytes (else
  *              WKV_ERR_MISALIGNED)
  *   w, u       [C] fp32;  state_in  NULL or three fp32 [B, C] (as wkv_forward)
- *   gout       [B, T, C] fp32
+ *   gout       [B, T, C] fp32, base address 16-byte aligned
  *   dk, dv     [B, T, C] fp32 (written)
  *   dw, du     [C] fp32 (written; summed over the batch rows)
  *   dstate_in  NULL, or three fp32 [B, C] arrays receiving dL/dnum, dL/dden,

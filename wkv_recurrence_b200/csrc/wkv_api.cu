@@ -843,11 +843,19 @@ wkv_status launch_backward(const BwdPlan& pl, const FwdParams& fp, const BwdPara
     default: wkv_tile_scan<64, false><<<gs, 1024, 0, st>>>(fp, kBwdL); break;
   }
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  // the chunks' k, v, g tiles (32 channels x kBwdL tokens) for R1 and R2
+  CUtensorMap rk, rv, rg;
+  if (!make_tmap(&rk, fp.k, kvdt, fp.B, fp.T, fp.C, kBwdL, 32) ||
+      !make_tmap(&rv, fp.v, kvdt, fp.B, fp.T, fp.C, kBwdL, 32) ||
+      !make_tmap(&rg, bp.g, WKV_F32, fp.B, fp.T, fp.C, kBwdL, 32))
+    return WKV_ERR_CUDA;
+  const size_t tsmem = bwd_tile_bytes<KV, kBwdL>() + 16;
   // R1: reverse aggregates of chunks 1 .. nch-1
   const long long ngw = (fp.C + 31) / 32;
   if (pl.nch > 1) {
     const long long items = (long long)fp.B * (pl.nch - 1) * ngw;
-    wkv_bwd_rev_totals<KV><<<(unsigned)((items + 3) / 4), 128, 0, st>>>(bp);
+    if (items >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+    wkv_bwd_rev_totals<KV, kBwdL><<<(unsigned)items, 32, tsmem, st>>>(bp, rk, rv, rg);
     if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   }
   // RS: the reverse state entering every chunk from its end
@@ -860,11 +868,11 @@ wkv_status launch_backward(const BwdPlan& pl, const FwdParams& fp, const BwdPara
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
   // R2: the gradients
   const long long items = (long long)fp.B * pl.nch * ngw;
-  if ((items + 3) / 4 >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
-  wkv_bwd_chunk<KV, kBwdL><<<(unsigned)((items + 3) / 4), 128, 0, st>>>(bp);
+  if (items >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
+  wkv_bwd_chunk<KV, kBwdL><<<(unsigned)items, 32, tsmem, st>>>(bp, rk, rv, rg);
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
-  // RED: du, dw
-  wkv_bwd_reduce<<<(unsigned)((fp.C + 255) / 256), 256, 0, st>>>(bp);
+  // RED: du, dw (one warp per channel)
+  wkv_bwd_reduce<<<(unsigned)((fp.C + 7) / 8), 256, 0, st>>>(bp);
   return launch_result();
 }
 
@@ -1161,8 +1169,8 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const void* k, const vo
   if (!workspace) return WKV_ERR_INVALID_ARG;
   if (workspace_bytes < pl.bytes) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(workspace, 256)) return WKV_ERR_MISALIGNED;
-  // the forward pass inside uses TMA on k and v
-  if (B * T * C > 0 && !tma_usable(k, v, C, kes)) return WKV_ERR_MISALIGNED;
+  // the kernels copy k, v and gout with TMA
+  if (B * T * C > 0 && (!tma_usable(k, v, C, kes) || !tma_usable(gout, gout, C, 4))) return WKV_ERR_MISALIGNED;
   if (C == 0) return WKV_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (B == 0 || T == 0) {
@@ -1235,6 +1243,7 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const void* k, const vo
   bp.pdu = reinterpret_cast<float*>(ws + pl.off_pdu);
   bp.pdw = reinterpret_cast<float*>(ws + pl.off_pdw);
   bp.hdr = fp.hdr;
+  bp.timeout_ns = kDefaultTimeoutNs;
   if (kv_dtype == WKV_F32) return launch_backward<float>(pl, fp, bp, kv_dtype, st, dev);
   return launch_backward<__nv_bfloat16>(pl, fp, bp, kv_dtype, st, dev);
 }

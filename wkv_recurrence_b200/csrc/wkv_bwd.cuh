@@ -34,11 +34,10 @@
 //         tokens in reverse from rin, writing dk, dv and per-chunk partial sums
 //         of du, dw; chunk 0 also yields the state gradients;
 //   RED   wkv_bwd_reduce: du, dw as compensated sums of the partials over the
-//         chunks and batch rows, in a fixed order.
-// One warp per (batch row, chunk, 32 channels) in R1 and R2; k, v and g are
-// read with coalesced 128-byte loads straight into registers (the second
-// read of a chunk hits L1/L2). All orders of accumulation depend on the shape
-// only, so results are bitwise reproducible.
+//         chunks and batch rows (a warp per channel), in a fixed order.
+// One 32-thread CTA per (batch row, chunk, 32 channels) in R1 and R2, the
+// chunk's k, v and g copied into shared memory by TMA. All orders of
+// accumulation depend on the shape only, so results are bitwise reproducible.
 #pragma once
 
 #include "wkv_device.cuh"
@@ -71,7 +70,8 @@ struct BwdParams {
   float4* rin;       // reverse state entering every chunk from its end [nch][B*NG][64]
   float* pdw;        // per-chunk partial sums [nch][B][C]
   float* pdu;
-  WsHeader* hdr;     // status word (bounds-checked build)
+  WsHeader* hdr;     // status word: wait timeouts (and index errors in the bounds-checked build)
+  uint64_t timeout_ns;
 };
 
 __device__ __forceinline__ size_t bwd_slot(const BwdParams& p, int j, int b, int c) {
@@ -165,40 +165,72 @@ __device__ __forceinline__ RAcc racc_combine(const RAcc& a, const RAcc& b, float
   return r;
 }
 
-template <typename KV>
-__device__ __forceinline__ float ldk(const void* base, size_t i) {
-  return Elem<KV>::to_f32(reinterpret_cast<const KV*>(base)[i]);
+
+// The chunk's tiles in shared memory: k, v (element type KV) and g (fp32), L
+// tokens x 32 channels each, copied by TMA on one mbarrier. Returns false if
+// the copy did not land within the wait limit (the status word is set).
+template <typename KV, int L>
+__host__ __device__ constexpr uint32_t bwd_tile_bytes() {
+  return (uint32_t)(L * 32 * (2 * sizeof(KV) + sizeof(float)));
 }
 
-// R1. One warp per (batch row, chunk j >= 1, 32 channels); grid
-// B * (nch - 1) * ceil(C / 32) warps, 4 per CTA. The forward is replayed from
-// x0[j] to get M_t, z_t, wkv_t of every token; the chunk's reverse aggregate
-// (relative to its first token: token t enters with exponent
-// -M_t - (t - t0) w) is folded in token order.
-template <typename KV>
-__global__ void __launch_bounds__(128) wkv_bwd_rev_totals(const BwdParams p) {
-  const int lane = threadIdx.x & 31;
-  const long long item = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+template <typename KV, int L>
+__device__ __forceinline__ bool bwd_load_tile(const BwdParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
+                                              const CUtensorMap* tg, unsigned char* smem, uint64_t* bar, int gw,
+                                              int t0, int b) {
+  KV* ks = reinterpret_cast<KV*>(smem);
+  if ((threadIdx.x & 31) == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, bwd_tile_bytes<KV, L>());
+    tma_load_3d(ks, tk, bar, gw * 32, t0, b);
+    tma_load_3d(ks + L * 32, tv, bar, gw * 32, t0, b);
+    tma_load_3d(reinterpret_cast<float*>(ks + 2 * L * 32), tg, bar, gw * 32, t0, b);
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(bar, 0, p.timeout_ns);
+  if (!ok && (threadIdx.x & 31) == 0) {
+    atomicOr(&p.hdr->status, kStatusWaitTimeout);
+    (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// R1. One 32-thread CTA per (batch row, chunk j >= 1, 32 channels). The
+// forward is replayed from x0[j] out of the chunk's tiles to get M_t, z_t,
+// wkv_t of every token; the chunk's reverse aggregate (relative to its first
+// token: token t enters with exponent -M_t - (t - t0) w) is folded in token
+// order.
+template <typename KV, int L>
+__global__ void __launch_bounds__(32)
+    wkv_bwd_rev_totals(const BwdParams p, const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmg) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const KV* ks = reinterpret_cast<const KV*>(smem);
+  const KV* vs = ks + L * 32;
+  const float* gs = reinterpret_cast<const float*>(vs + L * 32);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + bwd_tile_bytes<KV, L>());
+  const int lane = threadIdx.x;
   const int ngw = (p.C + 31) / 32;
-  const long long n_items = (long long)p.B * (p.nch - 1) * ngw;
-  if (item >= n_items) return;
+  const long long item = blockIdx.x;
   const int gw = (int)(item % ngw);
   const int j = 1 + (int)((item / ngw) % (p.nch - 1));
   const int b = (int)(item / ((long long)ngw * (p.nch - 1)));
+  const int t0 = j * L;
+  if (!bwd_load_tile<KV, L>(p, &tmk, &tmv, &tmg, smem, bar, gw, t0, b)) return;
   const int c = gw * 32 + lane;
   if (c >= p.C) return;
   const float w = __ldg(p.w + c), u = __ldg(p.u + c);
   Acc s = acc_unpack(p.x0[bwd_slot(p, j, b, c)]);
-  const int t0 = j * p.chunk_len;
-  const int t1 = min(p.T, t0 + p.chunk_len);
+  const int n = min(L, p.T - t0);
   RAcc r = racc_empty();  // at the chunk's first token
-  for (int t = t0; t < t1; ++t) {
-    const size_t i = ((size_t)b * p.T + t) * p.C + c;
-    const float k = ldk<KV>(p.k, i), v = ldk<KV>(p.v, i), g = __ldg(p.g + i);
+  for (int t = 0; t < n; ++t) {
+    const float k = Elem<KV>::to_f32(ks[t * 32 + lane]), v = Elem<KV>::to_f32(vs[t * 32 + lane]);
+    const float g = gs[t * 32 + lane];
     const OutStat o = out_stat(s, k, v, u, w);
     const float rz = rcp(o.z);
-    // token t's exponent at the chunk's start: -M_t - (t - t0) w
-    racc_add(r, o.key, o.uf, o.cnt - (float)(t - t0), g * rz, -g * o.out * rz, w, u);
+    // token t's exponent at the chunk's start: -M_t - t w
+    racc_add(r, o.key, o.uf, o.cnt - (float)t, g * rz, -g * o.out * rz, w, u);
     add_token(s, k, v, w);
   }
   if (WKV_IN(p.hdr, bwd_slot(p, j, b, c), (size_t)p.nch * p.B * p.NG * 64)) p.rtot[bwd_slot(p, j, b, c)] = racc_pack(r);
@@ -255,32 +287,41 @@ __global__ void __launch_bounds__(16 * SEG) wkv_bwd_rev_scan(const BwdParams p) 
   if ((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) p.rin[bwd_slot(p, 0, b, c)] = racc_pack(x);
 }
 
-// R2. One warp per (batch row, chunk, 32 channels), 4 warps per CTA. Forward
-// replay of the chunk from x0[j] keeping the state at every 4th token (a
-// checkpoint), then the tokens in reverse in groups of 4: the group's four
-// states are recomputed from its checkpoint, and each token, from the last,
-// gives dk, dv and its du, dw terms, then joins the reverse accumulator.
+// R2. One 32-thread CTA per (batch row, chunk, 32 channels), the chunk's k, v
+// and g in shared memory (TMA). Forward replay of the chunk from x0[j]
+// keeping the state at every 4th token (a checkpoint, in registers), then the
+// tokens in reverse in groups of 4: the group's four states are recomputed
+// from its checkpoint, and each token, from the last, gives dk, dv and its
+// du, dw terms, then joins the reverse accumulator.
 template <typename KV, int L>
-__global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
+__global__ void __launch_bounds__(32)
+    wkv_bwd_chunk(const BwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                  const __grid_constant__ CUtensorMap tmg) {
   constexpr int NGRP = L / 4;
-  const int lane = threadIdx.x & 31;
-  const long long item = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const KV* ks = reinterpret_cast<const KV*>(smem);
+  const KV* vs = ks + L * 32;
+  const float* gs = reinterpret_cast<const float*>(vs + L * 32);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + bwd_tile_bytes<KV, L>());
+  const int lane = threadIdx.x;
   const int ngw = (p.C + 31) / 32;
-  const long long n_items = (long long)p.B * p.nch * ngw;
-  if (item >= n_items) return;
+  const long long item = blockIdx.x;
   const int gw = (int)(item % ngw);
   const int j = (int)((item / ngw) % p.nch);
   const int b = (int)(item / ((long long)ngw * p.nch));
+  const int t0 = j * L;
+  if (!bwd_load_tile<KV, L>(p, &tmk, &tmv, &tmg, smem, bar, gw, t0, b)) return;
   const int c = gw * 32 + lane;
   if (c >= p.C) return;
   const float w = __ldg(p.w + c), u = __ldg(p.u + c);
-  const int t0 = j * L;
   const int n = min(L, p.T - t0);
   const size_t row0 = ((size_t)b * p.T + t0) * p.C + c;
   const size_t C = (size_t)p.C;
   if (!WKV_IN(p.hdr, (size_t)b * p.T + t0 + n - 1, (size_t)p.B * p.T) ||
       !WKV_IN(p.hdr, ((size_t)j * p.B + b) * p.C + c, (size_t)p.nch * p.B * p.C))
     return;
+  auto kat = [&](int t) { return Elem<KV>::to_f32(ks[t * 32 + lane]); };
+  auto vat = [&](int t) { return Elem<KV>::to_f32(vs[t * 32 + lane]); };
 
   // ---- forward replay with a checkpoint every 4 tokens
   Acc ck[NGRP];
@@ -291,7 +332,7 @@ __global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int t = gi * 4 + q;
-      if (t < n) add_token(s, ldk<KV>(p.k, row0 + t * C), ldk<KV>(p.v, row0 + t * C), w);
+      if (t < n) add_token(s, kat(t), vat(t), w);
     }
   }
 
@@ -309,9 +350,9 @@ __global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
       const int t = gi * 4 + q;
       st[q] = x;
       if (t < n) {
-        kk[q] = ldk<KV>(p.k, row0 + t * C);
-        vv[q] = ldk<KV>(p.v, row0 + t * C);
-        gg[q] = __ldg(p.g + row0 + t * C);
+        kk[q] = kat(t);
+        vv[q] = vat(t);
+        gg[q] = gs[t * 32 + lane];
         add_token(x, kk[q], vv[q], w);
       }
     }
@@ -357,14 +398,17 @@ __global__ void __launch_bounds__(128) wkv_bwd_chunk(const BwdParams p) {
   }
 }
 
-// RED. du[c], dw[c]: compensated sums of the partials over (chunk, batch row)
-// in a fixed order (Kahan-Babuska), one thread per channel.
+// RED. du[c], dw[c] from the partials over (chunk, batch row): one warp per
+// channel, lane l summing partials l, l+32, ... with compensation
+// (Kahan-Babuska), then a fixed shuffle tree: the order depends on the shape
+// only.
 __global__ void __launch_bounds__(256) wkv_bwd_reduce(const BwdParams p) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const long long c = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (c >= p.C) return;
   float su = 0.f, cu = 0.f, sw = 0.f, cw = 0.f;
   const long long n = (long long)p.nch * p.B;
-  for (long long i = 0; i < n; ++i) {
+  for (long long i = lane; i < n; i += 32) {
     const float xu = p.pdu[i * p.C + c], xw = p.pdw[i * p.C + c];
     float h, e;
     two_sum(su, xu, h, e);
@@ -374,8 +418,17 @@ __global__ void __launch_bounds__(256) wkv_bwd_reduce(const BwdParams p) {
     sw = h;
     cw += e;
   }
-  p.du[c] = su + cu;
-  p.dw[c] = sw + cw;
+  su += cu;
+  sw += cw;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    su += __shfl_xor_sync(0xffffffffu, su, o);
+    sw += __shfl_xor_sync(0xffffffffu, sw, o);
+  }
+  if (lane == 0) {
+    p.du[c] = su;
+    p.dw[c] = sw;
+  }
 }
 
 }  // namespace wkv
