@@ -271,9 +271,12 @@ void wkv_oracle_step_ext(int64_t S, int64_t C, const float *k, const float *v,
  * with Q_t the largest exponent contributing to them.
  *
  * The s* outputs (optional, NULL to skip) are the same formulas with every
- * signed quantity replaced by its magnitude (g, v, wkv, num0, and the
- * accumulators run on |g|): the sum of the magnitudes of the terms that make
- * up each gradient, the scale against which its rounding error is measured.
+ * signed quantity replaced by the sum of the magnitudes of its own terms: g by
+ * |g|, v by |v|, the state's numerator and wkv_t by the same sums taken over
+ * |v| (for wkv_t that is sum_i p_i |v_i|, the scale the forward is measured
+ * against), and the accumulators run on those. The result bounds the sum of
+ * the magnitudes of every term that makes up each gradient: the scale against
+ * which its rounding error is measured.
  *
  * dw and du are [C], summed over the batch rows; the state gradients are
  * [B, C] (NULL to skip).
@@ -300,7 +303,7 @@ void wkv_oracle_backward(int64_t B, int64_t T, int64_t C,
 
 #pragma omp parallel
     {
-        double *st = (double *)malloc(sizeof(double) * 3 * (size_t)(T > 0 ? T : 1));
+        double *st = (double *)malloc(sizeof(double) * 4 * (size_t)(T > 0 ? T : 1));
 #pragma omp for schedule(dynamic, 16)
         for (int64_t s = 0; s < B * C; ++s) {
             const int64_t b = s / C, c = s % C;
@@ -312,13 +315,18 @@ void wkv_oracle_backward(int64_t B, int64_t T, int64_t C,
                 m = max_in[s];
             }
             const double num0 = num, den0 = den, m0 = m;
+            /* the numerator over |v| (same exponents and denominator) */
+            double numa = fabs(num), dena = den, ma = m;
             /* forward: the state before every token */
             for (int64_t t = 0; t < T; ++t) {
                 const size_t i = ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;
-                st[3 * t] = num;
-                st[3 * t + 1] = den;
-                st[3 * t + 2] = m;
-                (void)wkv_token(widen(k, kv_dtype, i), widen(v, kv_dtype, i), wc, uc, &num, &den, &m);
+                st[4 * t] = num;
+                st[4 * t + 1] = den;
+                st[4 * t + 2] = m;
+                st[4 * t + 3] = numa;
+                const double kt = widen(k, kv_dtype, i), vt = widen(v, kv_dtype, i);
+                (void)wkv_token(kt, vt, wc, uc, &num, &den, &m);
+                (void)wkv_token(kt, fabs(vt), wc, uc, &numa, &dena, &ma);
             }
             /* backward */
             double rn = 0.0, rd = 0.0, an = 0.0, ad = 0.0, Q = -INFINITY;
@@ -326,13 +334,14 @@ void wkv_oracle_backward(int64_t B, int64_t T, int64_t C,
             for (int64_t t = T - 1; t >= 0; --t) {
                 const size_t i = ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;
                 const double kt = widen(k, kv_dtype, i), vt = widen(v, kv_dtype, i), g = gout[i];
-                const double nt = st[3 * t], dt = st[3 * t + 1], mt = st[3 * t + 2];
+                const double nt = st[4 * t], dt = st[4 * t + 1], mt = st[4 * t + 2], nta = st[4 * t + 3];
                 const double e = fmax(mt, kt + uc);
                 const double a = exp(mt - e), bb = exp(kt + uc - e);
                 const double z = a * dt + bb;
                 const double out = (a * nt + bb * vt) / z;
+                const double outa = (a * nta + bb * fabs(vt)) / z;  /* sum_i p_i |v_i| */
                 const double p = g / z, q = -g * out / z;
-                const double pa = fabs(g) / z, qa = fabs(g) * fabs(out) / z;
+                const double pa = fabs(g) / z, qa = fabs(g) * outa / z;
                 const double E1 = exp(kt + Q);          /* e^{k_t} relative to dN_{t+1}'s exponent */
                 const double E2 = exp(mt + Q - wc);     /* e^{m_t - w}, likewise */
                 dv[i] = p * bb + rn * E1;
@@ -341,10 +350,10 @@ void wkv_oracle_backward(int64_t B, int64_t T, int64_t C,
                 gw -= E2 * (nt * rn + dt * rd);
                 if (sv) {
                     sv[i] = pa * bb + an * E1;
-                    sk[i] = pa * bb * (fabs(vt) + fabs(out)) + E1 * (fabs(vt) * an + ad);
+                    sk[i] = pa * bb * (fabs(vt) + outa) + E1 * (fabs(vt) * an + ad);
                 }
-                au += pa * bb * (fabs(vt) + fabs(out));
-                aw += E2 * (fabs(nt) * an + dt * ad);
+                au += pa * bb * (fabs(vt) + outa);
+                aw += E2 * (nta * an + dt * ad);
                 /* move the accumulators to position t: decay by w, add token t */
                 const double Qn = fmax(Q - wc, -e);
                 const double x1 = exp(Q - wc - Qn), x2 = exp(-e - Qn);
