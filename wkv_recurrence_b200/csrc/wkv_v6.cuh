@@ -133,7 +133,48 @@ __global__ void __launch_bounds__(128)
     const int nt = min(TB, T - blk * TB);
     const KV* K = sk(s);
     const KV* V = sv(s);
-    for (int tt = 0; tt < nt; ++tt) {
+    int tt = 0;
+    // full groups of G tokens: the state updates run token after token, but
+    // the four-level reductions and gates of the group's outputs overlap
+    constexpr int G = 4;
+    for (; tt + G <= nt; tt += G) {
+      float ki[G], wi[G], rr[G], a[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        ki[j] = Elem<KV>::to_f32(K[(tt + j) * D + i]);
+        wi[j] = sw(s)[(tt + j) * RB + ri];
+        rr[j] = Elem<KV>::to_f32(sr(s)[(tt + j) * RB + ri]);
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < CPT; ++m) {
+          float kv[EPC], vv[EPC];
+          load_vec<KV, EPC>(K + (tt + j) * D + (m * NQ + q) * EPC, kv);
+          load_vec<KV, EPC>(V + (tt + j) * D + (m * NQ + q) * EPC, vv);
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) {
+            float& x = S[m * EPC + e];
+            x = fmaf(wi[j], x, ki[j] * vv[e]);
+            acc[e & 3] = fmaf(x, kv[e], acc[e & 3]);
+          }
+        }
+        a[j] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      }
+#pragma unroll
+      for (int o = 1; o < NQ; o <<= 1)
+#pragma unroll
+        for (int j = 0; j < G; ++j) a[j] += __shfl_xor_sync(0xffffffffu, a[j], o);
+      if (q == 0) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const size_t yi = (((size_t)row0 + blk * TB + tt + j) * p.H + h) * D + i;
+          if (WKV_IN(p.hdr, yi, (size_t)p.B * T * p.H * D)) y[yi] = Elem<OUT>::from_f32(gate(a[j], rr[j]));
+        }
+      }
+    }
+    for (; tt < nt; ++tt) {
       const float ki = Elem<KV>::to_f32(K[tt * D + i]);
       const float wi = sw(s)[tt * RB + ri];
       const float rr = Elem<KV>::to_f32(sr(s)[tt * RB + ri]);
