@@ -84,8 +84,7 @@ typedef struct {
  * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
  * zero-filled struct also means "defaults".
  *   kernel          0 = choose by shape (sequential for many channels or short
- *                   sequences; the cluster scan for T up to 2048; otherwise
- *                   the chunked scan in three launches),
+ *                   sequences, otherwise the cluster scan),
  *                   1 = sequential-over-T kernel,
  *                   2 = chunked scan in one launch (look-back between CTAs),
  *                   3 = chunked scan in three launches (chunk totals, their
@@ -94,12 +93,14 @@ typedef struct {
  *                   4 = chunked scan in one launch of persistent CTAs that
  *                   pipeline their tiles (look-back of one tile overlapped
  *                   with the next tile's fold and later tiles' copies),
- *                   5 = chunked scan inside one thread-block cluster per
- *                   (batch row, 32 channels): the cluster's shared memory
- *                   holds the whole sequence (T <= 8 x cta_warps x span), the
- *                   CTAs exchange their totals through distributed shared
- *                   memory; one launch, k and v read once, no waiting
- *                   between clusters
+ *                   5 = chunked scan in thread-block clusters: a cluster of
+ *                   up to 8 CTAs takes a segment of 8 x cta_warps x span
+ *                   tokens of one (batch row, 32 channels), its CTAs exchange
+ *                   their totals through distributed shared memory, and the
+ *                   segments of a channel group chain through the inclusive
+ *                   prefix each publishes for the next; one launch, k and v
+ *                   read once from memory (the replay re-reads them from L2),
+ *                   any alignment (no TMA)
  *   chunk_len       tokens per chunk for the chunked kernels (0 = choose: 32
  *                   or 64 for the three-launch scan, 128 otherwise; or 32, 64,
  *                   128)
@@ -110,7 +111,7 @@ typedef struct {
  *   span            tokens per warp in a chunk-scan tile, 8 or 16 (0 = choose);
  *                   chunk_len / span warps share a tile (at most 8 for the
  *                   pipelined scan, so chunk_len 128 needs span 16 there);
- *                   the cluster scan (kernel 5) takes 16 or 32 (0 = 32)
+ *                   the cluster scan (kernel 5) takes 16 or 32 (0 = 16)
  *   seq_threads     threads per CTA of the sequential kernel and of the
  *                   three-launch scan's replay pass: 32, 64 or 128 (0 =
  *                   choose: 32); each thread carries seq_vec channels in the
@@ -121,14 +122,15 @@ typedef struct {
  *                   (0 = choose: 1 below 151552 channels B*C, else 2)
  *   replay_chunks   three-launch scan (kernel 3): consecutive chunks that
  *                   one replay warp walks (0 = choose; or 1, 2, 4)
- *   cta_warps       cluster scan (kernel 5): warps (spans) per CTA, 4, 8 or
- *                   16 (0 = 8)
+ *   cta_warps       cluster scan (kernel 5): warps (spans) per CTA, 8 or 16
+ *                   (0 = 16)
  *   stages          shared-memory ring stages of the pipelined scan
  *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
  *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)
  *   inject_enable, inject_unpublished_tile
  *                   tests of the bounded waits only: with inject_enable = 1,
- *                   chunk-scan tile number inject_unpublished_tile computes
+ *                   chunk-scan tile number inject_unpublished_tile (in the
+ *                   cluster scan: the cluster with that ticket) computes
  *                   but never publishes its result, so the tiles that wait for
  *                   it reach their wait limit, carry on, and the call reports
  *                   WKV_ERR_WAIT_TIMEOUT through wkv_query_status. 0 = off.

@@ -68,32 +68,36 @@ def compare_ext(oracle, k, v, w, u, state=None, kv="f32", out_dtype=None, option
 # the cluster scan
 # ---------------------------------------------------------------------------
 
-CLUSTER_OPTS = [CLUSTER, {"kernel": 5, "cta_warps": 4}, {"kernel": 5, "cta_warps": 16},
-                {"kernel": 5, "span": 16}, {"kernel": 5, "span": 16, "cta_warps": 4},
-                {"kernel": 5, "span": 16, "cta_warps": 16}]
-CLUSTER_IDS = ["w8j32", "w4j32", "w16j32", "w8j16", "w4j16", "w16j16"]
+CLUSTER_OPTS = [CLUSTER, {"kernel": 5, "cta_warps": 8}, {"kernel": 5, "span": 32},
+                {"kernel": 5, "span": 32, "cta_warps": 8}]
+CLUSTER_IDS = ["w16j16", "w8j16", "w16j32", "w8j32"]
 
 
 @pytest.mark.parametrize("opts", CLUSTER_OPTS, ids=CLUSTER_IDS)
-@pytest.mark.parametrize("shape", [(1, 1, 64), (2, 65, 64), (3, 1000, 96), (2, 517, 200), (1, 1024, 36)],
+@pytest.mark.parametrize("shape", [(1, 1, 64), (2, 65, 64), (3, 1000, 96), (2, 517, 200), (1, 1024, 36),
+                                   (2, 2100, 64), (1, 5000, 40), (3, 3001, 33)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_cluster_random_f32(oracle, opts, shape):
+    """One segment (T up to 8 CTAs' worth) and several (the look-back between
+    segments), ragged channel groups, odd C (no 16-byte rows)."""
     B, T, C = shape
     k, v, w, u, st = I.random_case(B, T, C, seed=B * 7 + T + C, k_scale=2.0, k_spike=30.0,
                                    w_range=(1e-4, 8.0), state=(T % 2 == 1))
-    if T > 8 * (opts.get("cta_warps") or 8) * (opts.get("span") or 32):
-        pytest.skip("sequence longer than the cluster holds")
     compare_ext(oracle, k, v, w, u, st, options=opts)
 
 
-def test_cluster_longest_sequences(oracle):
-    """The largest T each CTA shape holds (8 CTAs), and one token less."""
-    for cw, cj in ((8, 32), (16, 32), (4, 16)):
-        for T in (8 * cw * cj, 8 * cw * cj - 1):
-            k, v, w, u, st = I.random_case(2, T, 64, seed=T + cw, k_spike=40.0, w_range=(1e-4, 4.0), state=True)
-            compare_ext(oracle, k, v, w, u, st, options={"kernel": 5, "cta_warps": cw, "span": cj})
-    with pytest.raises((W.WkvError, ValueError)):  # one token more than 8 CTAs hold: refused
-        run_ext(*I.random_case(1, 2049, 32, seed=3)[:4], options={"kernel": 5})
+def test_cluster_segment_boundaries(oracle):
+    """T at, just below and just above multiples of a segment (8 CTAs x 16
+    spans x 16 tokens = 2048 tokens for the default shape)."""
+    for T in (2047, 2048, 2049, 4096, 4097, 6143):
+        k, v, w, u, st = I.random_case(2, T, 64, seed=T, k_spike=40.0, w_range=(1e-4, 4.0), state=True)
+        compare_ext(oracle, k, v, w, u, st, options=CLUSTER)
+
+
+def test_cluster_misaligned_inputs(oracle):
+    """The cluster scan loads k and v with plain loads: any alignment."""
+    k, v, w, u, st = I.random_case(2, 2500, 64, seed=91, k_spike=30.0, state=True)
+    compare_ext(oracle, k, v, w, u, st, options=CLUSTER, aligned=False)
 
 
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
@@ -118,10 +122,10 @@ def test_cluster_in_place_state_and_determinism(oracle):
     assert torch.equal(a, b) and all(torch.equal(x, y) for x, y in zip(sa, sb))
 
 
-def test_cluster_is_the_automatic_choice_up_to_2048_tokens():
+def test_cluster_is_the_automatic_choice_for_few_channels():
     assert W.forward_kernel(8, 1024, 768) == 5
-    assert W.forward_kernel(8, 2048, 768) == 5
-    assert W.forward_kernel(8, 2049, 768) == 3
+    assert W.forward_kernel(1, 65536, 2048) == 5
+    assert W.forward_kernel(16, 4096, 4096, torch.bfloat16) == 1
     assert W.forward_launches(8, 1024, 768) == 1
 
 
@@ -129,20 +133,18 @@ def test_cluster_is_the_automatic_choice_up_to_2048_tokens():
 # per-token decay w_t
 # ---------------------------------------------------------------------------
 
-WT_KERNELS = [SEQ, CLUSTER, TWO, None, {"kernel": 5, "cta_warps": 4, "span": 16},
+WT_KERNELS = [SEQ, CLUSTER, TWO, None, {"kernel": 5, "cta_warps": 8, "span": 32},
               {"kernel": 3, "chunk_len": 64, "scan_segments": 4}, {"kernel": 3, "chunk_len": 128, "replay_chunks": 2},
               {"kernel": 3, "chunk_len": 32, "scan_segments": 16}]
-WT_IDS = ["seq", "cluster", "two", "auto", "cluster_w4j16", "two64seg4", "two128r2", "two32seg16"]
+WT_IDS = ["seq", "cluster", "two", "auto", "cluster_w8j32", "two64seg4", "two128r2", "two32seg16"]
 
 
 @pytest.mark.parametrize("opts", WT_KERNELS, ids=WT_IDS)
-@pytest.mark.parametrize("shape", [(2, 33, 64), (3, 1000, 96), (2, 517, 200), (1, 2048, 64)],
+@pytest.mark.parametrize("shape", [(2, 33, 64), (3, 1000, 96), (2, 517, 200), (1, 2048, 64), (1, 4500, 64)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_per_token_decay(oracle, opts, shape):
     B, T, C = shape
     k, v, w, u, st = I.random_case(B, T, C, seed=T + C, k_scale=2.0, k_spike=30.0, state=(T % 2 == 1))
-    if opts and opts.get("kernel") == 5 and T > 8 * (opts.get("cta_warps") or 8) * (opts.get("span") or 32):
-        pytest.skip("sequence longer than the cluster holds")
     compare_ext(oracle, k, v, w, u, st, options=opts, w_t=_wt(k.shape, T + C))
 
 

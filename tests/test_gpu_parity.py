@@ -330,15 +330,17 @@ def test_workspace_reuse_across_shapes(oracle, opts):
         assert_out(host(out), ref, sc, RTOL_F32)
 
 
-@pytest.mark.parametrize("kernel", [2, 4], ids=["chunk", "pipe"])
+@pytest.mark.parametrize("kernel", [2, 4, 5], ids=["chunk", "pipe", "cluster"])
 def test_bounded_wait_reports_timeout_and_recovers(oracle, kernel):
-    """A chunk tile that never publishes: waiters give up after the limit,
-    report WKV_ERR_WAIT_TIMEOUT, and the next call on the same workspace is
-    correct again."""
+    """A chunk tile (or, in the cluster scan, a segment) that never publishes:
+    waiters give up after the limit, report WKV_ERR_WAIT_TIMEOUT, and the next
+    call on the same workspace is correct again."""
     B, T, C = 2, 4096, 128
     k, v, w, u, _ = I.random_case(B, T, C, seed=41)
     opts = {"kernel": kernel, "chunk_len": 64, "lookback_group": 4, "wait_timeout_ns": 20_000_000,
             "inject_enable": 1, "inject_unpublished_tile": 9}
+    if kernel == 5:  # two segments of 2048 tokens, 8 channel groups: tickets 0-7 publish
+        opts = {"kernel": 5, "wait_timeout_ns": 20_000_000, "inject_enable": 1, "inject_unpublished_tile": 3}
     ws = W.make_workspace(B, T, C, options=opts)
     K, V, Wt, U = dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u)
     t0 = time.time()

@@ -47,6 +47,7 @@ struct Plan {
   int cw;      // cluster scan: warps (spans) per CTA
   int cj;      // cluster scan: tokens per span
   int ncl;     // cluster scan: CTAs per cluster
+  int nseg;    // cluster scan: segments (clusters) per (batch row, 32-channel group)
   int seq_threads;  // CTA width of the sequential kernel
   int seq_vec;      // channels per thread of the sequential kernel
   int scan_segments;  // three-launch scan: segments per channel in the scan of chunk totals
@@ -93,34 +94,33 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   if (want < 0 || want > 5) return false;
   const int64_t lanes = B * C;
   // the cluster scan's CTA shape: cw spans of cj tokens per CTA, up to 8 CTAs
-  if (o && o->cta_warps != 0 && o->cta_warps != 4 && o->cta_warps != 8 && o->cta_warps != 16) return false;
-  const int cw = (o && o->cta_warps) ? o->cta_warps : 8;
-  const int cj = (want == 5 && o && o->span) ? o->span : 32;
+  // per cluster and segment
+  if (o && o->cta_warps != 0 && o->cta_warps != 8 && o->cta_warps != 16) return false;
+  const int cw = (o && o->cta_warps) ? o->cta_warps : 16;
+  const int cj = (want == 5 && o && o->span) ? o->span : 16;
   if (cj != 16 && cj != 32) return false;
-  const int64_t cluster_tokens = 8ll * cw * cj;
   int kernel = want;
   if (kernel == 0) {
     if (lanes >= 65536 || T <= 64) {
       kernel = 1;
-    } else if (T <= cluster_tokens) {
-      // the whole sequence of a channel group fits in one cluster's shared
-      // memory: one launch, one read of k and v
-      kernel = 5;
     } else {
-      // chunked: the three-launch scan (measured: layer 27 vs 29 us single
-      // launch; long 465 vs 603 us pipelined, 636 us single launch)
-      kernel = 3;
+      // the cluster scan: one launch, k and v read once from HBM
+      kernel = 5;
     }
   }
   // per-token decays: the sequential, three-launch and cluster kernels only
   if (wt && (kernel == 2 || kernel == 4)) return false;
-  if (kernel == 5 && T > cluster_tokens) return false;
   const bool three_requested = (kernel == 3);
-  if ((kernel == 3 || kernel == 4 || kernel == 5) && !tma_ok) kernel = wt ? 1 : 2;
+  if ((kernel == 3 || kernel == 4) && !tma_ok) kernel = wt ? 1 : 2;  // the cluster scan needs no TMA
   pl->kernel = kernel;
   pl->cw = cw;
   pl->cj = cj;
-  pl->ncl = (int)std::max<int64_t>(1, (T + (int64_t)cw * cj - 1) / ((int64_t)cw * cj));
+  {
+    const int64_t tpc = (int64_t)cw * cj;
+    pl->ncl = (int)std::min<int64_t>(8, std::max<int64_t>(1, (T + tpc - 1) / tpc));
+    const int64_t seg_tokens = pl->ncl * tpc;
+    pl->nseg = (int)std::max<int64_t>(1, (T + seg_tokens - 1) / seg_tokens);
+  }
   pl->bytes = sizeof(WsHeader);
   if (o && o->scan_segments != 0 && o->scan_segments != 1 && o->scan_segments != 4 && o->scan_segments != 16 &&
       o->scan_segments != 64)
@@ -142,21 +142,16 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   pl->seq_threads = sth;
   if (kernel == 1) return true;
   if (kernel == 5) {
-    // the header only; but a call whose k or v TMA cannot address falls back
-    // to the single-launch scan (or, with per-token decays, the sequential
-    // kernel), so reserve that kernel's layout too
-    pl->bytes = sizeof(WsHeader);
-    if (!wt) {
-      wkv_options o2;
-      std::memset(&o2, 0, sizeof o2);
-      if (o) o2 = *o;
-      o2.kernel = 2;
-      o2.span = 0;
-      o2.chunk_len = 0;
-      Plan p2;
-      if (!make_plan(B, T, C, &o2, &p2, true, false)) return false;
-      pl->bytes = std::max(pl->bytes, p2.bytes);
-    }
+    // one segment: the header only; more: a flag and an inclusive prefix
+    // (32 float4) per (segment but the last, batch row, 32-channel group)
+    const int64_t items = B * ((C + 31) / 32);
+    if ((int64_t)pl->nseg * items * pl->ncl >= (1ll << 31)) return false;
+    size_t off = sizeof(WsHeader);
+    pl->off_flags_a = off;
+    off = round_up(off + sizeof(uint32_t) * (size_t)(pl->nseg - 1) * items, 256);
+    pl->off_agg_a = off;
+    off = round_up(off + sizeof(float4) * (size_t)(pl->nseg - 1) * items * 32, 256);
+    pl->bytes = pl->nseg > 1 ? off : sizeof(WsHeader);
     return true;
   }
 
@@ -633,23 +628,19 @@ wkv_status launch_seq_tma_wt(const FwdParams& p, wkv_dtype kvdt, cudaStream_t st
   return launch_seq<KV, OUT, 32, 1, LT, 3, true, true>(p, tk, tv, tw, st, dev);
 }
 
-// The cluster scan: one cluster of pl.ncl CTAs per (batch row, 32 channels),
-// k, v (and w_t) copied in by TMA in boxes of one span (J tokens x 32 channels).
+// The cluster scan: clusters of pl.ncl CTAs, one per (segment, batch row,
+// 32-channel group); k and v read with plain coalesced loads (no TMA).
 template <typename KV, typename OUT, int NW, int J, bool kWT>
-wkv_status launch_cluster(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
-  CUtensorMap tk, tv, tw;
-  std::memset(&tw, 0, sizeof tw);
-  if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, J, 32) || !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, J, 32))
-    return WKV_ERR_CUDA;
-  if (kWT && !make_tmap(&tw, p.w_t, WKV_F32, p.B, p.T, p.C, J, 32)) return WKV_ERR_CUDA;
-  constexpr size_t smem = cluster_smem_bytes<KV, NW, J, kWT>();
+wkv_status launch_cluster(const Plan& pl, const FwdParams& p, cudaStream_t st, int dev) {
+  constexpr size_t smem = cluster_smem_bytes<NW, kWT>();
   auto fn = wkv_fwd_cluster<KV, OUT, NW, J, kWT>;
   int occ = 0;
   if (!kernel_setup(fn, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
   FwdParams q = p;
   q.cluster = pl.ncl;
+  q.nseg = pl.nseg;
   const long long items = (long long)p.B * ((p.C + 31) / 32);
-  const long long grid = items * pl.ncl;
+  const long long grid = items * pl.nseg * pl.ncl;
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -663,24 +654,18 @@ wkv_status launch_cluster(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cu
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (!cuda_ok(cudaLaunchKernelEx(&cfg, fn, q, tk, tv, tw))) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaLaunchKernelEx(&cfg, fn, q))) return WKV_ERR_CUDA;
   return launch_result();
 }
 
 template <typename KV, typename OUT, bool kWT>
-wkv_status launch_cluster_shape(const Plan& pl, const FwdParams& p, wkv_dtype kvdt, cudaStream_t st, int dev) {
-  if (pl.cj == 16) {
-    switch (pl.cw) {
-      case 4: return launch_cluster<KV, OUT, 4, 16, kWT>(pl, p, kvdt, st, dev);
-      case 16: return launch_cluster<KV, OUT, 16, 16, kWT>(pl, p, kvdt, st, dev);
-      default: return launch_cluster<KV, OUT, 8, 16, kWT>(pl, p, kvdt, st, dev);
-    }
+wkv_status launch_cluster_shape(const Plan& pl, const FwdParams& p, cudaStream_t st, int dev) {
+  if (pl.cj == 32) {
+    return pl.cw == 8 ? launch_cluster<KV, OUT, 8, 32, kWT>(pl, p, st, dev)
+                      : launch_cluster<KV, OUT, 16, 32, kWT>(pl, p, st, dev);
   }
-  switch (pl.cw) {
-    case 4: return launch_cluster<KV, OUT, 4, 32, kWT>(pl, p, kvdt, st, dev);
-    case 16: return launch_cluster<KV, OUT, 16, 32, kWT>(pl, p, kvdt, st, dev);
-    default: return launch_cluster<KV, OUT, 8, 32, kWT>(pl, p, kvdt, st, dev);
-  }
+  return pl.cw == 8 ? launch_cluster<KV, OUT, 8, 16, kWT>(pl, p, st, dev)
+                    : launch_cluster<KV, OUT, 16, 16, kWT>(pl, p, st, dev);
 }
 
 template <typename KV, typename OUT>
@@ -690,8 +675,8 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
   std::memset(&tk, 0, sizeof tk);
   std::memset(&tv, 0, sizeof tv);
   if (pl.kernel == 5) {
-    return p.w_t ? launch_cluster_shape<KV, OUT, true>(pl, p, kvdt, st, dev)
-                 : launch_cluster_shape<KV, OUT, false>(pl, p, kvdt, st, dev);
+    return p.w_t ? launch_cluster_shape<KV, OUT, true>(pl, p, st, dev)
+                 : launch_cluster_shape<KV, OUT, false>(pl, p, st, dev);
   }
   if (pl.kernel == 1) {
     if (p.w_t) {
@@ -999,7 +984,10 @@ wkv_status wkv_forward_ext(int64_t B, int64_t T, int64_t C, const void* k, const
   p.hdr = reinterpret_cast<WsHeader*>(ws);
   p.timeout_ns = (opts && opts->wait_timeout_ns > 0) ? (uint64_t)opts->wait_timeout_ns : kDefaultTimeoutNs;
   p.inject_tile = (opts && opts->inject_enable) ? (int)std::min<int64_t>(opts->inject_unpublished_tile, INT32_MAX) : -1;
-  if (pl.kernel >= 2) {
+  if (pl.kernel == 5) {
+    p.flags_a = reinterpret_cast<uint32_t*>(ws + pl.off_flags_a);
+    p.agg_a = reinterpret_cast<float4*>(ws + pl.off_agg_a);
+  } else if (pl.kernel >= 2) {
     p.NG = pl.NG;
     p.nch = pl.nch;
     p.G = pl.G;
@@ -1316,7 +1304,8 @@ wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, c
   void* scratch = nullptr;
   if (!noalloc_scratch(dev, &scratch)) return WKV_ERR_CUDA;
   // counters, epoch, status and flags start at zero for this call
-  const size_t clear = (pl.kernel == 2 || pl.kernel == 4) ? pl.off_agg_a : sizeof(WsHeader);
+  const size_t clear =
+      (pl.kernel == 2 || pl.kernel == 4 || (pl.kernel == 5 && pl.nseg > 1)) ? pl.off_agg_a : sizeof(WsHeader);
   if (!cuda_ok(cudaMemsetAsync(scratch, 0, clear, reinterpret_cast<cudaStream_t>(stream))))
     return WKV_ERR_CUDA;
   return wkv_forward(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, scratch,

@@ -96,10 +96,53 @@ struct OutStat {
   float out;           // wkv_t
 };
 
+// e^{x} for an exponent given as the unevaluated sum x = hi + lo: 2^{hi log2 e}
+// with the product's rounding error recovered by an fma and the low parts
+// applied as the first-order factor 1 + (...) ln 2 (|lo| is below 2^-20 of
+// |hi|, so the second-order term is far below fp32 resolution).
+constexpr float kLog2eLo = 1.925963e-8f;  // log2(e) minus its nearest fp32 value
+constexpr float kLn2 = 0.69314718f;
+__device__ __forceinline__ float exp_hl(float hi, float lo) {
+  const float y = hi * kLog2e;
+  const float yl = fmaf(hi, kLog2e, -y) + fmaf(hi, kLog2eLo, lo * kLog2e);
+  const float r = ex2(y);
+  return fmaf(r, yl * kLn2, r);
+}
+
+// The exponent n w + (a - b) + c as hi + lo with no rounding lost: TwoSum
+// (Knuth) for the additions and the fma-based TwoProduct (Ogita, Rump and
+// Oishi, "Accurate sum and dot product", 2005) for n w. Gradients that are a
+// single exponential of an exponent near +-60 need this: rounding the
+// exponent to fp32 would cost |x| 2^-24 ~ 4e-6 of relative accuracy per
+// operation, several of which would exceed the 1e-5 bar.
+__device__ __forceinline__ void exponent_hl(float n, float w, float a, float b, float c, float& hi, float& lo) {
+  float s1, e1, s2, e2, e3;
+  two_sum(a, -b, s1, e1);
+  two_sum(s1, c, s2, e2);
+  const float pr = n * w;
+  const float ep = fmaf(n, w, -pr);
+  two_sum(s2, pr, hi, e3);
+  lo = (e1 + e2) + (ep + e3);
+}
+__device__ __forceinline__ float exp_exact(float n, float w, float a, float b, float c) {
+  float hi, lo;
+  exponent_hl(n, w, a, b, c, hi, lo);
+  return exp_hl(hi, lo);
+}
+
+// kExact: the current token's weight b = e^{D} (D < 0) evaluated from the
+// exact exponent (the gradient pass, where b multiplies dk and dv directly);
+// otherwise rounded like everywhere else.
+template <bool kExact = false>
 __device__ __forceinline__ OutStat out_stat(const Acc& s, float k, float v, float u, float w) {
   // D = (k + u) - m, formed as (k - ma) + u + nf w
-  const float D = fmaf(s.nf, w, (k - s.ma) + u);
-  const float x = ex2(-fabsf(D) * kLog2e);
+  float D, Dlo = 0.f;
+  if constexpr (kExact) {
+    exponent_hl(s.nf, w, k, s.ma, u, D, Dlo);
+  } else {
+    D = fmaf(s.nf, w, (k - s.ma) + u);
+  }
+  const float x = kExact ? exp_hl(-fabsf(D), D > 0.f ? -Dlo : Dlo) : ex2(-fabsf(D) * kLog2e);
   const bool tok = D > 0.f;  // the current token carries the largest exponent
   const float a = tok ? x : 1.f;
   const float b = tok ? 1.f : x;
@@ -360,12 +403,12 @@ __global__ void __launch_bounds__(32)
     for (int q = 3; q >= 0; --q) {
       const int t = gi * 4 + q;
       if (t >= n) continue;
-      const OutStat o = out_stat(st[q], kk[q], vv[q], u, w);
+      const OutStat o = out_stat<true>(st[q], kk[q], vv[q], u, w);
       const float rz = rcp(o.z);
       const float pp = gg[q] * rz, qq = -gg[q] * o.out * rz;
       // the reverse accumulator stands at t+1: Q = -qk - qu u + qc w
-      const float E1 = ex2(fmaf(r.qc, w, (kk[q] - r.qk) - r.qu * u) * kLog2e);                     // e^{k_t + Q}
-      const float E2 = ex2(fmaf(r.qc - st[q].nf - 1.f, w, (st[q].ma - r.qk) - r.qu * u) * kLog2e);  // e^{m_t + Q - w}
+      const float E1 = exp_exact(r.qc, w, kk[q], r.qk, -r.qu * u);                     // e^{k_t + Q}
+      const float E2 = exp_exact(r.qc - st[q].nf - 1.f, w, st[q].ma, r.qk, -r.qu * u);  // e^{m_t + Q - w}
       const float pb = pp * o.b;
       p.dv[row0 + t * C] = fmaf(r.rn, E1, pb);
       p.dk[row0 + t * C] = fmaf(E1, fmaf(vv[q], r.rn, r.rd), pb * (vv[q] - o.out));
@@ -386,7 +429,7 @@ __global__ void __launch_bounds__(32)
     if (p.s_num) {
       const float num0 = p.s_num[si], den0 = p.s_den[si], m0 = p.s_max[si];
       if (den0 > 0.f && m0 > kNegBig) {
-        const float f = ex2(fmaf(r.qc, w, (m0 - r.qk) - r.qu * u) * kLog2e);  // e^{m0 + Q}
+        const float f = exp_exact(r.qc, w, m0, r.qk, -r.qu * u);  // e^{m0 + Q}
         gn = r.rn * f;
         gd = r.rd * f;
         gm = fmaf(num0, gn, den0 * gd);

@@ -1,33 +1,44 @@
-// The chunked scan over T in one thread-block cluster: for sequences short
-// enough that one cluster's shared memory holds all of a channel group's k and
-// v (T <= 8 CTAs x NW*J tokens), there is no chunk total in global memory, no
-// look-back between CTAs and no second read of the inputs.
+// The chunked scan over T in thread-block clusters, reading k and v from HBM
+// once.
 //
-// One cluster of ncl CTAs takes one (batch row, 32-channel group) and the
-// whole sequence; CTA `rank` of the cluster holds tokens
-// [rank*TPC, (rank+1)*TPC) (TPC = NW*J) in shared memory, one span of J tokens
+// A cluster of ncl CTAs (at most 8) takes one SEGMENT of ncl * NW * J tokens
+// of one (batch row, 32-channel group); CTA `rank` holds tokens
+// [rank*TPC, (rank+1)*TPC) of the segment (TPC = NW*J), one span of J tokens
 // per warp, one channel per lane:
-//   1. each warp copies its span of k and v in (TMA, one mbarrier per span) and
-//      folds it from the empty state into an aggregate (largest end-of-span
-//      exponent first, then the weighted sums);
+//   1. each warp loads its span of k and v (and w_t) straight from global
+//      memory into registers (coalesced 128-byte rows, the whole span in
+//      flight at once) and folds it from the empty state into an aggregate
+//      (largest end-of-span exponent first, then the weighted sums);
 //   2. each warp combines the aggregates of the warps before it (its prefix
-//      inside the CTA); the last warp also forms the CTA's total;
-//   3. after a cluster barrier, every CTA reads the totals of the CTAs before
-//      it from their shared memory (distributed shared memory) and combines
-//      them in order, starting from the state in: its incoming state;
-//   4. each warp replays its span from (incoming state + prefix) out of shared
-//      memory and writes the outputs (gated by sigmoid(r) when r is given);
-//      the warp that holds token T-1 writes the state out.
-// The order of every combine depends on the shape only (results are bitwise
+//      inside the CTA); the last warp forms the CTA's total;
+//   3. after a cluster barrier, each CTA combines the totals of the CTAs
+//      before it, read from their shared memory (distributed shared memory);
+//   4. the segment's incoming state: the state in for the first segment,
+//      else the inclusive prefix the previous segment of the same channel
+//      group published in global memory (flag + payload, a bounded wait);
+//      the last CTA publishes this segment's inclusive prefix at once;
+//   5. each warp replays its span from (incoming state + prefixes), reading k
+//      and v again -- from L2, where the fold put them moments before (only
+//      the data of resident CTAs, a few tens of MB, is between the two reads)
+//      -- gated by sigmoid(r) when r is given; the warp holding token T-1
+//      writes the state out.
+// Segments take their work item from a ticket counter in segment-major order,
+// so a segment's predecessor (same channel group, previous segment) always
+// took its ticket earlier: every wait is for a cluster that is running or
+// done. With a single segment there is no ticket and no wait.
+//
+// The order of every combine depends on the shape only (bitwise
 // reproducible). With kWT the decay is per token ("RWKV-v6 Architecture",
-// section "2. Dynamic Data-Dependent Decay"): w_t comes in as a third tile and
+// section "2. Dynamic Data-Dependent Decay"): w_t is loaded with k and v and
 // the combines carry each span's decay sum.
 //
-// Every CTA reads the state in before the first cluster barrier and the state
-// out is written after it, so state_out may alias state_in. A second cluster
-// barrier (arrive after the last remote read, wait before exit) keeps every
-// CTA's shared memory alive while others may read it. All threads of every CTA
-// take both barriers; no thread returns early.
+// The state in is read by the first segment's CTAs, and the state out is
+// written by the last segment, which (through the published prefixes, or the
+// cluster barrier when there is one segment) runs after those reads, so the
+// two may alias. A second cluster barrier (arrive after the last remote read,
+// wait before exit) keeps every CTA's shared memory alive while others may
+// read it. All threads of every CTA take every barrier; no thread returns
+// early.
 #pragma once
 
 #include "wkv_device.cuh"
@@ -36,89 +47,171 @@
 namespace wkv {
 
 // Shared-memory bytes of wkv_fwd_cluster.
-template <typename KV, int NW, int J, bool kWT>
+template <int NW, bool kWT>
 __host__ __device__ constexpr size_t cluster_smem_bytes() {
-  return (size_t)NW * J * 32 * (2 * sizeof(KV) + (kWT ? 4 : 0))  // k, v (and w_t) tiles
-         + (size_t)NW * 32 * (16 + (kWT ? 4 : 0))                 // span aggregates (and decay sums)
-         + 32 * (16 + 4)                                          // the CTA's total and decay sum
-         + (size_t)NW * 8;                                        // one mbarrier per span
+  return (size_t)NW * 32 * (16 + (kWT ? 4 : 0))  // span aggregates (and decay sums)
+         + 32 * (16 + 4)                         // the CTA's total and decay sum
+         + 32 * (16 + 4)                         // the segment's incoming state and decay sum
+         + 16;                                   // the cluster's ticket
+}
+
+// Aggregate of n <= J tokens held in registers, anchored at the span's end
+// (the register twin of aggregate_tile_span): s_i = k_i - (n-1-i) w.
+template <int J>
+__device__ __forceinline__ Acc fold_regs(const float (&kx)[J], const float (&vx)[J], int n, float w) {
+  float M = kNegBig;
+  const float last = (float)(n - 1);
+#pragma unroll
+  for (int i = 0; i < J; ++i)
+    if (i < n) M = fmaxf(M, fmaf((float)i - last, w, kx[i]));
+  const float ML = M * kLog2e;
+  float num = 0.f, den = 0.f;
+#pragma unroll
+  for (int i = 0; i < J; ++i) {
+    if (i < n) {
+      const float x = ex2(fmaf(fmaf((float)i - last, w, kx[i]), kLog2e, -ML));
+      num = fmaf(x, vx[i], num);
+      den += x;
+    }
+  }
+  if (n <= 0) return acc_empty();
+  const float corr = fmaf(M, kLog2e, -ML);
+  const float fix = fmaf(-corr, 0.6931471805599453f, 1.f);
+  return Acc{num * fix, den * fix, M, 0.f};
+}
+
+// The same with per-token decays (the register twin of aggregate_span_wt):
+// s_i = k_i - (w_{i+1} + ... + w_{n-1}), compensated suffix sums; also the
+// span's decay sum.
+template <int J>
+__device__ __forceinline__ Acc fold_regs_wt(const float (&kx)[J], const float (&vx)[J], const float (&wx)[J], int n,
+                                            float& wsum) {
+  float sx[J];
+  float hi = 0.f, lo = 0.f, M = kNegBig;
+#pragma unroll
+  for (int i = J - 1; i >= 0; --i) {
+    if (i < n) {
+      sx[i] = (kx[i] - hi) - lo;
+      M = fmaxf(M, sx[i]);
+      float h, e;
+      two_sum(hi, wx[i], h, e);
+      hi = h;
+      lo += e;
+    }
+  }
+  wsum = hi + lo;
+  const float ML = M * kLog2e;
+  float num = 0.f, den = 0.f;
+#pragma unroll
+  for (int i = 0; i < J; ++i) {
+    if (i < n) {
+      const float x = ex2(fmaf(sx[i], kLog2e, -ML));
+      num = fmaf(x, vx[i], num);
+      den += x;
+    }
+  }
+  if (n <= 0) return acc_empty();
+  const float corr = fmaf(M, kLog2e, -ML);
+  const float fix = fmaf(-corr, 0.6931471805599453f, 1.f);
+  return Acc{num * fix, den * fix, M, 0.f};
+}
+
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* q) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(q) : "memory");
+  return v;
 }
 
 template <typename KV, typename OUT, int NW, int J, bool kWT>
-__global__ void __launch_bounds__(NW * 32)
-    wkv_fwd_cluster(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                    const __grid_constant__ CUtensorMap tmw) {
+__global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
   constexpr int CG = 32;
   constexpr int TPC = NW * J;
-  constexpr int kSpan = J * CG;  // elements of one tensor in one span
-  constexpr uint32_t kSpanBytes = (uint32_t)(2 * kSpan * sizeof(KV) + (kWT ? kSpan * 4 : 0));
   extern __shared__ __align__(1024) unsigned char smem[];
-  KV* ktile = reinterpret_cast<KV*>(smem);  // [TPC][CG]
-  KV* vtile = ktile + TPC * CG;             // [TPC][CG]
-  float* wtile = reinterpret_cast<float*>(vtile + TPC * CG);                                   // [TPC][CG] (kWT)
-  float4* sagg = reinterpret_cast<float4*>(wtile + (kWT ? TPC * CG : 0));                      // [NW][CG]
-  float* swsum = reinterpret_cast<float*>(sagg + NW * CG);                                     // [NW][CG] (kWT)
-  float4* stot = reinterpret_cast<float4*>(swsum + (kWT ? NW * CG : 0));                       // [CG]
-  float* stotw = reinterpret_cast<float*>(stot + CG);                                          // [CG]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(stotw + CG);                                     // [NW]
+  float4* sagg = reinterpret_cast<float4*>(smem);                           // [NW][CG]
+  float* swsum = reinterpret_cast<float*>(sagg + NW * CG);                  // [NW][CG] (kWT)
+  float4* stot = reinterpret_cast<float4*>(swsum + (kWT ? NW * CG : 0));    // [CG]
+  float* stotw = reinterpret_cast<float*>(stot + CG);                       // [CG]
+  float4* sx = reinterpret_cast<float4*>(stotw + CG);                       // [CG] the segment's incoming state
+  float* sxw = reinterpret_cast<float*>(sx + CG);                           // [CG] (unused slot, kept aligned)
+  uint32_t* sticket = reinterpret_cast<uint32_t*>(sxw + CG);
 
   const int lane = threadIdx.x & 31;
   const int wp = threadIdx.x >> 5;
   const int T = p.T, C = p.C;
   const int ncl = p.cluster;
+  const int nseg = p.nseg;
   const int rank = (int)(blockIdx.x % (unsigned)ncl);
-  const int item = (int)(blockIdx.x / (unsigned)ncl);
   const int ngc = (C + CG - 1) / CG;
-  const int b = item / ngc, g = item % ngc;
+  const int items = p.B * ngc;
+  const uint32_t target = nseg > 1 ? *reinterpret_cast<volatile uint32_t*>(&p.hdr->epoch) + 1u : 0u;
+
+  // ---- the cluster's work item (segment-major ticket order with segments)
+  int cl_id;
+  if (nseg > 1) {
+    if (rank == 0 && threadIdx.x == 0) *sticket = atomicAdd(&p.hdr->ticket, 1u);
+    cluster_arrive();
+    cluster_wait();
+    cl_id = (int)ld_dsmem_u32(map_shared_rank(sticket, 0));
+    if (rank == 0 && threadIdx.x == 0) {
+      // every cluster has read the epoch and taken its ticket before it counts
+      // itself; the last one hands the header back for the next launch
+      const uint32_t prev = atomicAdd(&p.hdr->done, 1u);
+      if (prev == (uint32_t)(nseg * items) - 1u) {
+        p.hdr->ticket = 0;
+        p.hdr->done = 0;
+        __threadfence();
+        atomicExch(&p.hdr->epoch, target);
+      }
+    }
+  } else {
+    cl_id = (int)(blockIdx.x / (unsigned)ncl);
+  }
+  const int seg = cl_id / items, it = cl_id % items;
+  const int b = it / ngc, g = it % ngc;
   const int c = g * CG + lane;
   const bool cok = c < C;
-  const int t_cta = rank * TPC;
+  const int seg_tokens = ncl * TPC;
+  const int t_seg = seg * seg_tokens;
+  const int t_cta = t_seg + rank * TPC;
   const int ts = t_cta + wp * J;
   const int nv = max(0, min(J, T - ts));
+  const size_t row0 = ((size_t)b * T + ts) * C + c;  // (b, ts, c)
+  const KV* kg = reinterpret_cast<const KV*>(p.k) + row0;
+  const KV* vg = reinterpret_cast<const KV*>(p.v) + row0;
 
-  // ---- copy this warp's span in
-  KV* ks = ktile + wp * kSpan + lane;
-  KV* vs = vtile + wp * kSpan + lane;
-  float* wsp = wtile + wp * kSpan + lane;
-  if (lane == 0 && nv > 0) {
-    mbar_init(&bar[wp], 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(&bar[wp], kSpanBytes);
-    tma_load_3d(ktile + wp * kSpan, &tmk, &bar[wp], g * CG, ts, b);
-    tma_load_3d(vtile + wp * kSpan, &tmv, &bar[wp], g * CG, ts, b);
-    if (kWT) tma_load_3d(wtile + wp * kSpan, &tmw, &bar[wp], g * CG, ts, b);
-  }
-  __syncwarp();
-
-  // ---- per-channel constants and the state in (read before the first
-  // cluster barrier: state_out may alias it)
+  // ---- per-channel constants and the state in
   const float w = (!kWT && cok) ? __ldg(p.w + c) : 0.f;
   const float u = cok ? __ldg(p.u + c) : 0.f;
   Acc xin = acc_empty();
-  if (cok && p.s_num) {
+  if (seg == 0 && cok && p.s_num) {
     const size_t i = (size_t)b * C + c;
     xin = acc_from_state(p.s_num[i], p.s_den[i], p.s_max[i]);
   }
 
-  // ---- 1. fold the span
-  bool copy_ok = true;
+  // ---- 1. fold the span from registers
   Acc agg = acc_empty();
   float wsum = 0.f;
-  if (nv > 0) {
-    copy_ok = mbar_wait(&bar[wp], 0, p.timeout_ns);
-    if (!copy_ok) {
-      if (lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
-    } else if (kWT) {
-      Acc a1[1];
-      float s1[1];
-      aggregate_span_wt<KV, J, 1, CG>(ks, vs, wsp, nv, a1, s1);
-      agg = a1[0];
-      wsum = s1[0];
+  {
+    float kx[J], vx[J];
+#pragma unroll
+    for (int i = 0; i < J; ++i) {
+      const bool ok = cok && i < nv;
+      kx[i] = ok ? Elem<KV>::to_f32(kg[(size_t)i * C]) : 0.f;
+      vx[i] = ok ? Elem<KV>::to_f32(vg[(size_t)i * C]) : 0.f;
+    }
+    if constexpr (kWT) {
+      float wx[J];
+#pragma unroll
+      for (int i = 0; i < J; ++i) wx[i] = (cok && i < nv) ? p.w_t[row0 + (size_t)i * C] : 0.f;
+      agg = fold_regs_wt<J>(kx, vx, wx, nv, wsum);
     } else {
-      Acc a1[1];
-      const float w1[1] = {w};
-      aggregate_tile_span<KV, J, 1, CG>(ks, vs, nv, w1, a1);
-      agg = a1[0];
+      agg = fold_regs<J>(kx, vx, nv, w);
     }
   }
   sagg[wp * CG + lane] = acc_pack(agg);
@@ -151,33 +244,82 @@ __global__ void __launch_bounds__(NW * 32)
     stotw[lane] = wtot;
   }
 
-  // ---- 3. incoming state of this CTA from the totals of the CTAs before it
+  // ---- 3. the totals of the CTAs before this one in the segment
   cluster_arrive();
   cluster_wait();
-  Acc x = xin;
+  Acc xl = acc_empty();
+  float xlw = 0.f;
   for (int r = 0; r < rank; ++r) {
     const Acc t = acc_unpack(ld_dsmem_f4(map_shared_rank(&stot[lane], (uint32_t)r)));
     if (kWT) {
-      x = combine_wt(x, t, ld_dsmem_f32(map_shared_rank(&stotw[lane], (uint32_t)r)));
+      const float wr = ld_dsmem_f32(map_shared_rank(&stotw[lane], (uint32_t)r));
+      xl = combine_wt(xl, t, wr);
+      xlw += wr;
     } else {
-      x = combine(x, t, (float)TPC, w);
+      xl = combine(xl, t, (float)TPC, w);
     }
   }
   cluster_arrive();  // done with the other CTAs' shared memory
 
-  // ---- 4. replay the span
-  if (nv > 0 && copy_ok && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
-    Acc st = kWT ? combine_wt(x, pre, wpre) : combine(x, pre, (float)(wp * J), w);
-    OUT* orow = reinterpret_cast<OUT*>(p.out) + ((size_t)b * T + ts) * C + c;
-    const KV* rrow = p.r ? reinterpret_cast<const KV*>(p.r) + ((size_t)b * T + ts) * C + c : nullptr;
+  // ---- 4. the segment's incoming state; the last CTA publishes the
+  // segment's inclusive prefix for the next segment
+  if (wp == 0) {
+    if (seg > 0) {
+      const uint32_t* flag = p.flags_a + (size_t)(seg - 1) * items + it;
+      bool got = ld_acquire_u32(flag) == target;
+      if (!got) {
+        const uint64_t t0 = global_ns();
+        while (!(got = ld_acquire_u32(flag) == target)) {
+          if (global_ns() - t0 > p.timeout_ns) break;
+          __nanosleep(64);
+        }
+      }
+      got = __all_sync(0xffffffffu, got);
+      if (!got && lane == 0) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+      const size_t islot = ((size_t)(seg - 1) * items + it) * CG + lane;
+      sx[lane] = got ? ld_relaxed_f4(p.agg_a + islot) : acc_pack(acc_empty());
+    } else {
+      sx[lane] = acc_pack(xin);
+    }
+  }
+  __syncthreads();
+  const Acc X = acc_unpack(sx[lane]);
+  if (rank == ncl - 1 && seg < nseg - 1 && wp == 0) {
+    // the inclusive prefix of this (full) segment: X, then the CTAs before
+    // this one, then this CTA's total
+    const Acc own = acc_unpack(stot[lane]);
+    Acc incl;
+    if (kWT) {
+      incl = combine_wt(combine_wt(X, xl, xlw), own, stotw[lane]);
+    } else {
+      incl = combine(combine(X, xl, (float)(rank * TPC), w), own, (float)TPC, w);
+    }
+    const size_t oslot = ((size_t)seg * items + it) * CG + lane;
+    if (WKV_IN(p.hdr, oslot, (size_t)(nseg - 1) * items * CG)) p.agg_a[oslot] = acc_pack(incl);
+    __threadfence();
+    __syncwarp();
+    // (inject_tile: the test hook that leaves one segment unpublished)
+    if (lane == 0 && cl_id != p.inject_tile) st_release_u32(p.flags_a + (size_t)seg * items + it, target);
+  }
+
+  // ---- 5. replay the span (k and v again, from L2)
+  if (nv > 0 && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
+    Acc st;
+    if (kWT) {
+      st = combine_wt(combine_wt(X, xl, xlw), pre, wpre);
+    } else {
+      st = combine(combine(X, xl, (float)(rank * TPC), w), pre, (float)(wp * J), w);
+    }
+    OUT* orow = reinterpret_cast<OUT*>(p.out) + row0;
+    const KV* rrow = p.r ? reinterpret_cast<const KV*>(p.r) + row0 : nullptr;
     float lo = 0.f;
     if (kWT) {
       for (int i = 0; i < nv; ++i) {
-        float kx[1], vx[1];
-        load_vec<KV, 1>(ks + i * CG, kx);
-        load_vec<KV, 1>(vs + i * CG, vx);
-        float o = step_token_wt(st, lo, kx[0], vx[0], wsp[i * CG], u);
-        if (rrow) o = gate(o, Elem<KV>::to_f32(rrow[(size_t)i * C]));
+        const float kk = cok ? Elem<KV>::to_f32(kg[(size_t)i * C]) : 0.f;
+        const float vv = cok ? Elem<KV>::to_f32(vg[(size_t)i * C]) : 0.f;
+        const float ww = cok ? p.w_t[row0 + (size_t)i * C] : 0.f;
+        float o = step_token_wt(st, lo, kk, vv, ww, u);
+        if (rrow && cok) o = gate(o, Elem<KV>::to_f32(rrow[(size_t)i * C]));
         if (cok) orow[(size_t)i * C] = Elem<OUT>::from_f32(o);
       }
     } else {
@@ -195,15 +337,15 @@ __global__ void __launch_bounds__(NW * 32)
             float kb[NB][1], vb[NB][1], ob[NB][1], rb[NB];
 #pragma unroll
             for (int jj = 0; jj < NB; ++jj) {
-              load_vec<KV, 1>(ks + (j0 + jj) * CG, kb[jj]);
-              load_vec<KV, 1>(vs + (j0 + jj) * CG, vb[jj]);
-              if (kGate) rb[jj] = Elem<KV>::to_f32(rrow[(size_t)(j0 + jj) * C]);
+              kb[jj][0] = cok ? Elem<KV>::to_f32(kg[(size_t)(j0 + jj) * C]) : 0.f;
+              vb[jj][0] = cok ? Elem<KV>::to_f32(vg[(size_t)(j0 + jj) * C]) : 0.f;
+              if (kGate) rb[jj] = cok ? Elem<KV>::to_f32(rrow[(size_t)(j0 + jj) * C]) : 0.f;
             }
             step_tokens<NB, 1>(s1, kb, vb, w1, cb, ob);
 #pragma unroll
             for (int jj = 0; jj < NB; ++jj) {
-              const float o = kGate ? gate(ob[jj][0], rb[jj]) : ob[jj][0];
-              if (cok) orow[(size_t)(j0 + jj) * C] = Elem<OUT>::from_f32(o);
+              const float o[1] = {kGate ? gate(ob[jj][0], rb[jj]) : ob[jj][0]};
+              if (cok) stg_stream<OUT, 1>(orow + (size_t)(j0 + jj) * C, o);
             }
           }
         };
@@ -214,12 +356,11 @@ __global__ void __launch_bounds__(NW * 32)
         }
       } else {
         for (int i = 0; i < nv; ++i) {
-          float kx[1], vx[1];
-          load_vec<KV, 1>(ks + i * CG, kx);
-          load_vec<KV, 1>(vs + i * CG, vx);
-          float o = out_token(s1[0], kx[0], vx[0], w, u);
-          add_token(s1[0], kx[0], vx[0], w);
-          if (rrow) o = gate(o, Elem<KV>::to_f32(rrow[(size_t)i * C]));
+          const float kk = cok ? Elem<KV>::to_f32(kg[(size_t)i * C]) : 0.f;
+          const float vv = cok ? Elem<KV>::to_f32(vg[(size_t)i * C]) : 0.f;
+          float o = out_token(s1[0], kk, vv, w, u);
+          add_token(s1[0], kk, vv, w);
+          if (rrow && cok) o = gate(o, Elem<KV>::to_f32(rrow[(size_t)i * C]));
           if (cok) orow[(size_t)i * C] = Elem<OUT>::from_f32(o);
         }
       }
@@ -233,7 +374,6 @@ __global__ void __launch_bounds__(NW * 32)
       p.o_max[i] = kWT ? acc_max_e_wt(st, lo) : acc_max_e(st, w);
     }
   }
-  if (nv > 0 && !copy_ok && lane == 0) (void)mbar_wait(&bar[wp], 0, p.timeout_ns);  // bounded drain
   cluster_wait();
 }
 

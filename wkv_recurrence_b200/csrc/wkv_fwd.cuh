@@ -79,6 +79,7 @@ struct FwdParams {
   int stages;          // pipelined chunk scan: shared-memory stages in the ring
   int replay_chunks;   // three-launch scan: consecutive chunks per replay CTA
   int cluster;         // cluster kernel: CTAs per cluster
+  int nseg;            // cluster kernel: segments per (batch row, 32-channel group)
   const float* w_t;    // per-token decay [B, T, C] in place of w, or NULL
   const void* r;       // receptance [B, T, C] (element type of k, v): out = sigmoid(r) wkv; or NULL
   float* wtot;         // three-launch scan with w_t: decay sum of each chunk total, [nch-1][B * NG][64]
