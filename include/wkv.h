@@ -95,12 +95,13 @@ typedef struct {
  *                   with the next tile's fold and later tiles' copies),
  *                   5 = chunked scan in thread-block clusters: a cluster of
  *                   up to 8 CTAs takes a segment of 8 x cta_warps x span
- *                   tokens of one (batch row, 32 channels), its CTAs exchange
- *                   their totals through distributed shared memory, and the
- *                   segments of a channel group chain through the inclusive
- *                   prefix each publishes for the next; one launch, k and v
- *                   read once from memory (the replay re-reads them from L2),
- *                   any alignment (no TMA)
+ *                   tokens of one (batch row, 32 channels); each warp streams
+ *                   its span through its own TMA ring twice (fold, then
+ *                   replay), the CTAs exchange their totals through
+ *                   distributed shared memory, and the segments of a channel
+ *                   group chain through the inclusive prefix each publishes
+ *                   for the next; one launch, k and v read once from memory
+ *                   (the replay re-reads them from L2)
  *   chunk_len       tokens per chunk for the chunked kernels (0 = choose: 32
  *                   or 64 for the three-launch scan, 128 otherwise; or 32, 64,
  *                   128)
@@ -111,7 +112,7 @@ typedef struct {
  *   span            tokens per warp in a chunk-scan tile, 8 or 16 (0 = choose);
  *                   chunk_len / span warps share a tile (at most 8 for the
  *                   pipelined scan, so chunk_len 128 needs span 16 there);
- *                   the cluster scan (kernel 5) takes 16 or 32 (0 = 16)
+ *                   the cluster scan (kernel 5) takes 32 or 64 (0 = 64)
  *   seq_threads     threads per CTA of the sequential kernel and of the
  *                   three-launch scan's replay pass: 32, 64 or 128 (0 =
  *                   choose: 32); each thread carries seq_vec channels in the
@@ -122,8 +123,8 @@ typedef struct {
  *                   (0 = choose: 1 below 151552 channels B*C, else 2)
  *   replay_chunks   three-launch scan (kernel 3): consecutive chunks that
  *                   one replay warp walks (0 = choose; or 1, 2, 4)
- *   cta_warps       cluster scan (kernel 5): warps (spans) per CTA, 8 or 16
- *                   (0 = 16)
+ *   cta_warps       cluster scan (kernel 5): warps (spans) per CTA, 4 or 8
+ *                   (0 = 8)
  *   stages          shared-memory ring stages of the pipelined scan
  *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
  *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)

@@ -84,12 +84,13 @@ def test_workspace_size(L):
     a = L.wkv_forward_workspace_size(8, 1024, 768, ctypes.byref(o3))
     b = L.wkv_forward_workspace_size(8, 2048, 768, ctypes.byref(o3))
     assert 256 < a < b
-    # cluster scan: the header alone for one segment; a flag and a prefix per
-    # later segment and channel group beyond it
-    assert L.wkv_forward_workspace_size(8, 2048, 768, None) == 256
-    a = L.wkv_forward_workspace_size(8, 2049, 768, None)
-    b = L.wkv_forward_workspace_size(8, 8192, 768, None)
-    assert 256 < a < b
+    # cluster scan: a flag and a prefix per segment after the first and channel
+    # group, and room for the single-launch scan that misaligned inputs take
+    o5, o2 = _abi.wkv_options(kernel=5), _abi.wkv_options(kernel=2)
+    for T in (2048, 4096, 4097, 16384):
+        assert L.wkv_forward_workspace_size(8, T, 768, None) == L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o5))
+        assert L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o5)) >= \
+            L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o2))
     assert L.wkv_forward_workspace_size(-1, 4, 4, None) == 0
     o = _abi.wkv_options(kernel=2, chunk_len=48)
     assert L.wkv_forward_workspace_size(1, 64, 64, ctypes.byref(o)) == 0
@@ -100,20 +101,20 @@ def test_workspace_size(L):
 def test_forward_kernel_choice(L):
     F32, BF16 = _abi.WKV_F32, _abi.WKV_BF16
     # many channels or short sequences: the sequential kernel; otherwise the
-    # cluster scan (any T, any alignment)
+    # cluster scan (any T)
     assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
     assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 5
     assert L.wkv_forward_kernel(8, 2049, 768, F32, None) == 5
     assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 5
-    assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 5  # rows TMA cannot address: no TMA needed
-    # an explicit choice stands, except that the TMA-only scans fall back to the
+    assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 2  # rows TMA cannot address
+    # an explicit choice stands, except that the TMA scans fall back to the
     # single-launch scan when a row pitch is not a multiple of 16 bytes
     for kernel in (1, 2, 3, 4, 5):
         o = _abi.wkv_options(kernel=kernel)
         assert L.wkv_forward_kernel(2, 500, 64, F32, ctypes.byref(o)) == kernel
-        assert L.wkv_forward_kernel(2, 500, 65, F32, ctypes.byref(o)) == (2 if kernel in (3, 4) else kernel)
-    for bad in (dict(cta_warps=3), dict(cta_warps=4), dict(cta_warps=32), dict(span=8)):
+        assert L.wkv_forward_kernel(2, 500, 65, F32, ctypes.byref(o)) == (2 if kernel in (3, 4, 5) else kernel)
+    for bad in (dict(cta_warps=3), dict(cta_warps=16), dict(cta_warps=32), dict(span=8), dict(span=16)):
         o = _abi.wkv_options(kernel=5, **bad)
         assert L.wkv_forward_kernel(2, 100, 64, F32, ctypes.byref(o)) == 0
     assert L.wkv_forward_launches(8, 1024, 768, F32, None) == 1
@@ -121,10 +122,6 @@ def test_forward_kernel_choice(L):
     assert L.wkv_forward_launches(1, 65536, 2048, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 3
     assert L.wkv_forward_launches(2, 20, 64, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 2
     assert L.wkv_forward_launches(16, 4096, 4096, BF16, None) == 1
-    # the cluster scan's workspace: the header for one segment, flags and
-    # prefixes for more
-    assert L.wkv_forward_workspace_size(8, 2048, 768, None) == 256
-    assert L.wkv_forward_workspace_size(1, 65536, 2048, None) > 256
     assert L.wkv_forward_kernel(-1, 4, 4, F32, None) == 0
     assert L.wkv_forward_kernel(1, 4, 4, 9, None) == 0
     o = _abi.wkv_options(kernel=4, stages=1)
@@ -157,7 +154,7 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, sout=ctypes.byref(bad_out)) == _abi.WKV_ERR_INVALID_ARG
     o = _abi.wkv_options(kernel=6)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
-    o = _abi.wkv_options(kernel=5, cta_warps=4)
+    o = _abi.wkv_options(kernel=5, cta_warps=16)
     assert fwd(L, opts=ctypes.byref(o)) == _abi.WKV_ERR_INVALID_ARG
     # per-token decays with a look-back kernel, or without w_t and without w
     ext = _abi.wkv_ext(0x2000, None)

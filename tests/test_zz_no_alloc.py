@@ -69,18 +69,19 @@ def _check_call(oracle, L, B, T, C, seed, with_state, misaligned, what):
 
 
 def test_noalloc_matches_oracle_on_calls_in_a_row(oracle):
-    """Calls of the cluster scan in a row: one segment (only the status word in
-    the scratch array), several segments (the scratch holds each segment's
-    flag and prefix, which must start from a clean epoch on every call), and
-    misaligned inputs; each against the oracle."""
+    """Calls in a row: the cluster scan with one segment (only the status word
+    in the scratch array) and several (the scratch holds each segment's flag
+    and prefix, which must start from a clean epoch on every call), and
+    misaligned inputs (the single-launch scan, whose flags share the array);
+    each against the oracle."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from wkv_recurrence_b200 import build
     build.build()
     L = _abi.lib()
     assert W.forward_kernel(4, 1000, 256) == 5 and W.forward_kernel(3, 3000, 192) == 5
-    cases = [(4, 1000, 256, True, False), (3, 3000, 192, False, False), (2, 2049, 128, True, False),
-             (2, 5000, 128, True, True), (3, 777, 64, False, True), (2, 4100, 96, False, False)]
+    cases = [(4, 1000, 256, True, False), (3, 9000, 192, False, False), (2, 4097, 128, True, False),
+             (2, 5000, 128, True, True), (3, 777, 64, False, True), (2, 8200, 96, False, False)]
     for call, (B, T, C, with_state, misaligned) in enumerate(cases):
         _check_call(oracle, L, B, T, C, 500 + call, with_state, misaligned,
                     f"noalloc call {call + 1} ({'misaligned' if misaligned else 'aligned'})")

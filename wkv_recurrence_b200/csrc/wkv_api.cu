@@ -95,10 +95,10 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   const int64_t lanes = B * C;
   // the cluster scan's CTA shape: cw spans of cj tokens per CTA, up to 8 CTAs
   // per cluster and segment
-  if (o && o->cta_warps != 0 && o->cta_warps != 8 && o->cta_warps != 16) return false;
-  const int cw = (o && o->cta_warps) ? o->cta_warps : 16;
-  const int cj = (want == 5 && o && o->span) ? o->span : 16;
-  if (cj != 16 && cj != 32) return false;
+  if (o && o->cta_warps != 0 && o->cta_warps != 4 && o->cta_warps != 8) return false;
+  const int cw = (o && o->cta_warps) ? o->cta_warps : 8;
+  const int cj = (want == 5 && o && o->span) ? o->span : 64;
+  if (cj != 32 && cj != 64) return false;
   int kernel = want;
   if (kernel == 0) {
     if (lanes >= 65536 || T <= 64) {
@@ -111,7 +111,7 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   // per-token decays: the sequential, three-launch and cluster kernels only
   if (wt && (kernel == 2 || kernel == 4)) return false;
   const bool three_requested = (kernel == 3);
-  if ((kernel == 3 || kernel == 4) && !tma_ok) kernel = wt ? 1 : 2;  // the cluster scan needs no TMA
+  if ((kernel == 3 || kernel == 4 || kernel == 5) && !tma_ok) kernel = wt ? 1 : 2;
   pl->kernel = kernel;
   pl->cw = cw;
   pl->cj = cj;
@@ -152,6 +152,20 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     pl->off_agg_a = off;
     off = round_up(off + sizeof(float4) * (size_t)(pl->nseg - 1) * items * 32, 256);
     pl->bytes = pl->nseg > 1 ? off : sizeof(WsHeader);
+    // a call whose inputs TMA cannot address runs the single-launch scan (or,
+    // with per-token decays, the sequential kernel) instead: reserve for it too
+    wkv_options o2;
+    if (o) {
+      o2 = *o;
+    } else {
+      std::memset(&o2, 0, sizeof o2);
+    }
+    o2.kernel = wt ? 1 : 2;
+    o2.cta_warps = 0;
+    o2.span = 0;
+    Plan p2;
+    if (!make_plan(B, T, C, &o2, &p2, false, wt)) return false;
+    pl->bytes = std::max(pl->bytes, p2.bytes);
     return true;
   }
 
@@ -631,11 +645,20 @@ wkv_status launch_seq_tma_wt(const FwdParams& p, wkv_dtype kvdt, cudaStream_t st
 // The cluster scan: clusters of pl.ncl CTAs, one per (segment, batch row,
 // 32-channel group); k and v read with plain coalesced loads (no TMA).
 template <typename KV, typename OUT, int NW, int J, bool kWT>
-wkv_status launch_cluster(const Plan& pl, const FwdParams& p, cudaStream_t st, int dev) {
-  constexpr size_t smem = cluster_smem_bytes<NW, kWT>();
+wkv_status launch_cluster(const Plan& pl, const FwdParams& p, cudaStream_t st, int dev, wkv_dtype kvdt) {
+  constexpr size_t smem = cluster_smem_bytes<KV, NW, kWT>();
   auto fn = wkv_fwd_cluster<KV, OUT, NW, J, kWT>;
   int occ = 0;
   if (!kernel_setup(fn, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
+  CUtensorMap tk, tv, tw;
+  if (!make_tmap(&tk, p.k, kvdt, p.B, p.T, p.C, kClusterLB, 32) ||
+      !make_tmap(&tv, p.v, kvdt, p.B, p.T, p.C, kClusterLB, 32))
+    return WKV_ERR_CUDA;
+  if (kWT) {
+    if (!make_tmap(&tw, p.w_t, WKV_F32, p.B, p.T, p.C, kClusterLB, 32)) return WKV_ERR_CUDA;
+  } else {
+    tw = tk;  // unused
+  }
   FwdParams q = p;
   q.cluster = pl.ncl;
   q.nseg = pl.nseg;
@@ -654,18 +677,18 @@ wkv_status launch_cluster(const Plan& pl, const FwdParams& p, cudaStream_t st, i
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (!cuda_ok(cudaLaunchKernelEx(&cfg, fn, q))) return WKV_ERR_CUDA;
+  if (!cuda_ok(cudaLaunchKernelEx(&cfg, fn, q, tk, tv, tw))) return WKV_ERR_CUDA;
   return launch_result();
 }
 
 template <typename KV, typename OUT, bool kWT>
-wkv_status launch_cluster_shape(const Plan& pl, const FwdParams& p, cudaStream_t st, int dev) {
+wkv_status launch_cluster_shape(const Plan& pl, const FwdParams& p, cudaStream_t st, int dev, wkv_dtype kvdt) {
   if (pl.cj == 32) {
-    return pl.cw == 8 ? launch_cluster<KV, OUT, 8, 32, kWT>(pl, p, st, dev)
-                      : launch_cluster<KV, OUT, 16, 32, kWT>(pl, p, st, dev);
+    return pl.cw == 4 ? launch_cluster<KV, OUT, 4, 32, kWT>(pl, p, st, dev, kvdt)
+                      : launch_cluster<KV, OUT, 8, 32, kWT>(pl, p, st, dev, kvdt);
   }
-  return pl.cw == 8 ? launch_cluster<KV, OUT, 8, 16, kWT>(pl, p, st, dev)
-                    : launch_cluster<KV, OUT, 16, 16, kWT>(pl, p, st, dev);
+  return pl.cw == 4 ? launch_cluster<KV, OUT, 4, 64, kWT>(pl, p, st, dev, kvdt)
+                    : launch_cluster<KV, OUT, 8, 64, kWT>(pl, p, st, dev, kvdt);
 }
 
 template <typename KV, typename OUT>
@@ -675,8 +698,8 @@ wkv_status dispatch_forward(const Plan& pl, FwdParams& p, bool tma, wkv_dtype kv
   std::memset(&tk, 0, sizeof tk);
   std::memset(&tv, 0, sizeof tv);
   if (pl.kernel == 5) {
-    return p.w_t ? launch_cluster_shape<KV, OUT, true>(pl, p, st, dev)
-                 : launch_cluster_shape<KV, OUT, false>(pl, p, st, dev);
+    return p.w_t ? launch_cluster_shape<KV, OUT, true>(pl, p, st, dev, kvdt)
+                 : launch_cluster_shape<KV, OUT, false>(pl, p, st, dev, kvdt);
   }
   if (pl.kernel == 1) {
     if (p.w_t) {

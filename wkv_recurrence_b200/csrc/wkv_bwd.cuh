@@ -408,7 +408,9 @@ __global__ void __launch_bounds__(32)
       const float pp = gg[q] * rz, qq = -gg[q] * o.out * rz;
       // the reverse accumulator stands at t+1: Q = -qk - qu u + qc w
       const float E1 = exp_exact(r.qc, w, kk[q], r.qk, -r.qu * u);                     // e^{k_t + Q}
-      const float E2 = exp_exact(r.qc - st[q].nf - 1.f, w, st[q].ma, r.qk, -r.qu * u);  // e^{m_t + Q - w}
+      // (dw sums these over all tokens; its largest terms have exponents near
+      // zero, so the rounded exponent suffices)
+      const float E2 = ex2(fmaf(r.qc - st[q].nf - 1.f, w, (st[q].ma - r.qk) - r.qu * u) * kLog2e);  // e^{m_t + Q - w}
       const float pb = pp * o.b;
       p.dv[row0 + t * C] = fmaf(r.rn, E1, pb);
       p.dk[row0 + t * C] = fmaf(E1, fmaf(vv[q], r.rn, r.rd), pb * (vv[q] - o.out));

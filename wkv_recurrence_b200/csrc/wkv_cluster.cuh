@@ -4,24 +4,25 @@
 // A cluster of ncl CTAs (at most 8) takes one SEGMENT of ncl * NW * J tokens
 // of one (batch row, 32-channel group); CTA `rank` holds tokens
 // [rank*TPC, (rank+1)*TPC) of the segment (TPC = NW*J), one span of J tokens
-// per warp, one channel per lane:
-//   1. each warp loads its span of k and v (and w_t) straight from global
-//      memory into registers (coalesced 128-byte rows, the whole span in
-//      flight at once) and folds it from the empty state into an aggregate
-//      (largest end-of-span exponent first, then the weighted sums);
-//   2. each warp combines the aggregates of the warps before it (its prefix
-//      inside the CTA); the last warp forms the CTA's total;
-//   3. after a cluster barrier, each CTA combines the totals of the CTAs
-//      before it, read from their shared memory (distributed shared memory);
-//   4. the segment's incoming state: the state in for the first segment,
-//      else the inclusive prefix the previous segment of the same channel
-//      group published in global memory (flag + payload, a bounded wait);
-//      the last CTA publishes this segment's inclusive prefix at once;
-//   5. each warp replays its span from (incoming state + prefixes), reading k
-//      and v again -- from L2, where the fold put them moments before (only
-//      the data of resident CTAs, a few tens of MB, is between the two reads)
-//      -- gated by sigmoid(r) when r is given; the warp holding token T-1
-//      writes the state out.
+// per warp, one channel per lane. Each warp streams its span through a ring of
+// its own: NS shared-memory stages of LB tokens x 32 channels of k and v (and
+// w_t), copied by TMA and completing on one mbarrier per stage. The span goes
+// through the ring twice:
+//   1. fold: block by block from HBM, each block folded in registers (largest
+//      end-of-block exponent first, then the weighted sums) and combined into
+//      the span's aggregate;
+//   2. prefixes: each warp combines the aggregates of the warps before it
+//      (shared memory), the last warp forms the CTA's total, and after a
+//      cluster barrier each CTA combines the totals of the CTAs before it
+//      (distributed shared memory); the segment's incoming state is the state
+//      in for the first segment, else the inclusive prefix that the previous
+//      segment of the same channel group published in global memory (flag +
+//      payload, a bounded wait); the last CTA publishes this segment's
+//      inclusive prefix at once;
+//   3. replay: the same blocks again, from L2, where the fold left them
+//      moments before (the ring's first replay copies are in flight during
+//      step 2), gated by sigmoid(r) when r is given; the warp holding token
+//      T-1 writes the state out.
 // Segments take their work item from a ticket counter in segment-major order,
 // so a segment's predecessor (same channel group, previous segment) always
 // took its ticket earlier: every wait is for a cluster that is running or
@@ -29,8 +30,8 @@
 //
 // The order of every combine depends on the shape only (bitwise
 // reproducible). With kWT the decay is per token ("RWKV-v6 Architecture",
-// section "2. Dynamic Data-Dependent Decay"): w_t is loaded with k and v and
-// the combines carry each span's decay sum.
+// section "2. Dynamic Data-Dependent Decay"): w_t comes through the ring with
+// k and v and the combines carry each block's and span's decay sum.
 //
 // The state in is read by the first segment's CTAs, and the state out is
 // written by the last segment, which (through the published prefixes, or the
@@ -38,7 +39,9 @@
 // two may alias. A second cluster barrier (arrive after the last remote read,
 // wait before exit) keeps every CTA's shared memory alive while others may
 // read it. All threads of every CTA take every barrier; no thread returns
-// early.
+// early, and a warp whose copy wait runs out stops consuming, reports
+// kStatusWaitTimeout, and before the end waits (bounded) for the copies it
+// still has in flight.
 #pragma once
 
 #include "wkv_device.cuh"
@@ -46,16 +49,26 @@
 
 namespace wkv {
 
-// Shared-memory bytes of wkv_fwd_cluster.
-template <int NW, bool kWT>
-__host__ __device__ constexpr size_t cluster_smem_bytes() {
-  return (size_t)NW * 32 * (16 + (kWT ? 4 : 0))  // span aggregates (and decay sums)
-         + 32 * (16 + 4)                         // the CTA's total and decay sum
-         + 32 * (16 + 4)                         // the segment's incoming state and decay sum
-         + 16;                                   // the cluster's ticket
+constexpr int kClusterLB = 8;  // tokens per ring stage
+constexpr int kClusterNS = 4;  // ring stages per warp
+
+template <typename KV, bool kWT>
+__host__ __device__ constexpr uint32_t cluster_stage_bytes() {
+  return (uint32_t)(kClusterLB * 32 * (2 * sizeof(KV) + (kWT ? sizeof(float) : 0)));
 }
 
-// Aggregate of n <= J tokens held in registers, anchored at the span's end
+// Shared-memory bytes of wkv_fwd_cluster.
+template <typename KV, int NW, bool kWT>
+__host__ __device__ constexpr size_t cluster_smem_bytes() {
+  return (size_t)NW * kClusterNS * cluster_stage_bytes<KV, kWT>()  // the warps' rings
+         + (size_t)NW * kClusterNS * 8                             // their mbarriers
+         + (size_t)NW * 32 * (16 + (kWT ? 4 : 0))                  // span aggregates (and decay sums)
+         + 32 * (16 + 4)                                           // the CTA's total and decay sum
+         + 32 * (16 + 4)                                           // the segment's incoming state
+         + 16;                                                     // the cluster's ticket
+}
+
+// Aggregate of n <= J tokens held in registers, anchored at the last one
 // (the register twin of aggregate_tile_span): s_i = k_i - (n-1-i) w.
 template <int J>
 __device__ __forceinline__ Acc fold_regs(const float (&kx)[J], const float (&vx)[J], int n, float w) {
@@ -129,20 +142,29 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* q) {
 }
 
 template <typename KV, typename OUT, int NW, int J, bool kWT>
-__global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
+__global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
+    wkv_fwd_cluster(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                    const __grid_constant__ CUtensorMap tmw) {
   constexpr int CG = 32;
+  constexpr int LB = kClusterLB;
+  constexpr int NS = kClusterNS;
   constexpr int TPC = NW * J;
+  static_assert(J % LB == 0, "a span is whole ring blocks");
+  constexpr uint32_t kStage = cluster_stage_bytes<KV, kWT>();
+  constexpr int kTile = LB * CG;  // elements per tensor per stage
   extern __shared__ __align__(1024) unsigned char smem[];
-  float4* sagg = reinterpret_cast<float4*>(smem);                           // [NW][CG]
-  float* swsum = reinterpret_cast<float*>(sagg + NW * CG);                  // [NW][CG] (kWT)
-  float4* stot = reinterpret_cast<float4*>(swsum + (kWT ? NW * CG : 0));    // [CG]
-  float* stotw = reinterpret_cast<float*>(stot + CG);                       // [CG]
-  float4* sx = reinterpret_cast<float4*>(stotw + CG);                       // [CG] the segment's incoming state
-  float* sxw = reinterpret_cast<float*>(sx + CG);                           // [CG] (unused slot, kept aligned)
-  uint32_t* sticket = reinterpret_cast<uint32_t*>(sxw + CG);
-
   const int lane = threadIdx.x & 31;
   const int wp = threadIdx.x >> 5;
+  unsigned char* ring = smem + (size_t)wp * NS * kStage;                              // this warp's stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * NS * kStage) + wp * NS;
+  float4* sagg = reinterpret_cast<float4*>(smem + (size_t)NW * NS * (kStage + 8));   // [NW][CG]
+  float* swsum = reinterpret_cast<float*>(sagg + NW * CG);                            // [NW][CG] (kWT)
+  float4* stot = reinterpret_cast<float4*>(swsum + (kWT ? NW * CG : 0));              // [CG]
+  float* stotw = reinterpret_cast<float*>(stot + CG);                                 // [CG]
+  float4* sx = reinterpret_cast<float4*>(stotw + CG);                                 // [CG] incoming state
+  float* sxw = reinterpret_cast<float*>(sx + CG);                                     // [CG] (spare, keeps alignment)
+  uint32_t* sticket = reinterpret_cast<uint32_t*>(sxw + CG);
+
   const int T = p.T, C = p.C;
   const int ncl = p.cluster;
   const int nseg = p.nseg;
@@ -176,14 +198,51 @@ __global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
   const int b = it / ngc, g = it % ngc;
   const int c = g * CG + lane;
   const bool cok = c < C;
-  const int seg_tokens = ncl * TPC;
-  const int t_seg = seg * seg_tokens;
+  const int t_seg = seg * ncl * TPC;
   const int t_cta = t_seg + rank * TPC;
-  const int ts = t_cta + wp * J;
-  const int nv = max(0, min(J, T - ts));
+  const int ts = t_cta + wp * J;                // this warp's span
+  const int nv = max(0, min(J, T - ts));        // its tokens
+  const int nb = (nv + LB - 1) / LB;            // its ring blocks
+  const int nl = 2 * nb;                        // copies: the fold's, then the replay's
   const size_t row0 = ((size_t)b * T + ts) * C + c;  // (b, ts, c)
-  const KV* kg = reinterpret_cast<const KV*>(p.k) + row0;
-  const KV* vg = reinterpret_cast<const KV*>(p.v) + row0;
+
+  // ---- this warp's ring: the first NS copies go out at once
+  auto issue = [&](int n) {
+    const int blk = n < nb ? n : n - nb;
+    const int s = n % NS;
+    unsigned char* st = ring + (size_t)s * kStage;
+    mbar_arrive_expect_tx(&bars[s], kStage);
+    tma_load_3d(st, &tmk, &bars[s], g * CG, ts + blk * LB, b);
+    tma_load_3d(st + kTile * sizeof(KV), &tmv, &bars[s], g * CG, ts + blk * LB, b);
+    if (kWT) tma_load_3d(st + 2 * kTile * sizeof(KV), &tmw, &bars[s], g * CG, ts + blk * LB, b);
+  };
+  int issued = 0;  // lane 0's count of copies issued
+  if (lane == 0) {
+    if (wp == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+    }
+#pragma unroll
+    for (int s = 0; s < NS; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+    for (; issued < NS && issued < nl; ++issued) issue(issued);
+  }
+  __syncwarp();
+  bool ok = true;   // every copy this warp waited for arrived in time
+  int n = 0;        // copies consumed
+  auto wait_copy = [&](int x) {
+    const bool got = mbar_wait(&bars[x % NS], (uint32_t)((x / NS) & 1), p.timeout_ns);
+    ok = __all_sync(0xffffffffu, got);
+    return ok;
+  };
+  auto release = [&]() {  // stage n-1 consumed: its slot takes copy n-1+NS
+    __syncwarp();
+    if (lane == 0 && issued < nl) {
+      fence_proxy_async_smem();
+      issue(issued);
+      ++issued;
+    }
+  };
 
   // ---- per-channel constants and the state in
   const float w = (!kWT && cok) ? __ldg(p.w + c) : 0.f;
@@ -194,25 +253,35 @@ __global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
     xin = acc_from_state(p.s_num[i], p.s_den[i], p.s_max[i]);
   }
 
-  // ---- 1. fold the span from registers
+  // ---- 1. fold the span, block by block
   Acc agg = acc_empty();
   float wsum = 0.f;
-  {
-    float kx[J], vx[J];
+#pragma unroll 1
+  for (int blk = 0; blk < nb; ++blk, ++n) {
+    if (!wait_copy(n)) break;
+    const unsigned char* st = ring + (size_t)(n % NS) * kStage;
+    const KV* ks = reinterpret_cast<const KV*>(st) + lane;
+    const KV* vs = ks + kTile;
+    const int nt = min(LB, nv - blk * LB);
+    float kx[LB], vx[LB];
 #pragma unroll
-    for (int i = 0; i < J; ++i) {
-      const bool ok = cok && i < nv;
-      kx[i] = ok ? Elem<KV>::to_f32(kg[(size_t)i * C]) : 0.f;
-      vx[i] = ok ? Elem<KV>::to_f32(vg[(size_t)i * C]) : 0.f;
+    for (int i = 0; i < LB; ++i) {
+      kx[i] = Elem<KV>::to_f32(ks[i * CG]);
+      vx[i] = Elem<KV>::to_f32(vs[i * CG]);
     }
     if constexpr (kWT) {
-      float wx[J];
+      const float* ws = reinterpret_cast<const float*>(st + 2 * kTile * sizeof(KV)) + lane;
+      float wx[LB];
 #pragma unroll
-      for (int i = 0; i < J; ++i) wx[i] = (cok && i < nv) ? p.w_t[row0 + (size_t)i * C] : 0.f;
-      agg = fold_regs_wt<J>(kx, vx, wx, nv, wsum);
+      for (int i = 0; i < LB; ++i) wx[i] = ws[i * CG];
+      float wb;
+      const Acc a = fold_regs_wt<LB>(kx, vx, wx, nt, wb);
+      agg = combine_wt(agg, a, wb);
+      wsum += wb;
     } else {
-      agg = fold_regs<J>(kx, vx, nv, w);
+      agg = combine(agg, fold_regs<LB>(kx, vx, nt, w), (float)nt, w);
     }
+    release();
   }
   sagg[wp * CG + lane] = acc_pack(agg);
   if (kWT) swsum[wp * CG + lane] = wsum;
@@ -244,7 +313,7 @@ __global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
     stotw[lane] = wtot;
   }
 
-  // ---- 3. the totals of the CTAs before this one in the segment
+  // the totals of the CTAs before this one in the segment
   cluster_arrive();
   cluster_wait();
   Acc xl = acc_empty();
@@ -261,8 +330,8 @@ __global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
   }
   cluster_arrive();  // done with the other CTAs' shared memory
 
-  // ---- 4. the segment's incoming state; the last CTA publishes the
-  // segment's inclusive prefix for the next segment
+  // the segment's incoming state; the last CTA publishes the segment's
+  // inclusive prefix for the next segment
   if (wp == 0) {
     if (seg > 0) {
       const uint32_t* flag = p.flags_a + (size_t)(seg - 1) * items + it;
@@ -302,9 +371,10 @@ __global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
     if (lane == 0 && cl_id != p.inject_tile) st_release_u32(p.flags_a + (size_t)seg * items + it, target);
   }
 
-  // ---- 5. replay the span (k and v again, from L2)
-  if (nv > 0 && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
+  // ---- 3. replay the span through the ring (from L2)
+  if (ok && nv > 0 && WKV_IN(p.hdr, (size_t)b * T + ts + nv - 1, (size_t)p.B * T)) {
     Acc st;
+    float lo = 0.f;
     if (kWT) {
       st = combine_wt(combine_wt(X, xl, xlw), pre, wpre);
     } else {
@@ -312,67 +382,75 @@ __global__ void __launch_bounds__(NW * 32) wkv_fwd_cluster(const FwdParams p) {
     }
     OUT* orow = reinterpret_cast<OUT*>(p.out) + row0;
     const KV* rrow = p.r ? reinterpret_cast<const KV*>(p.r) + row0 : nullptr;
-    float lo = 0.f;
-    if (kWT) {
-      for (int i = 0; i < nv; ++i) {
-        const float kk = cok ? Elem<KV>::to_f32(kg[(size_t)i * C]) : 0.f;
-        const float vv = cok ? Elem<KV>::to_f32(vg[(size_t)i * C]) : 0.f;
-        const float ww = cok ? p.w_t[row0 + (size_t)i * C] : 0.f;
-        float o = step_token_wt(st, lo, kk, vv, ww, u);
-        if (rrow && cok) o = gate(o, Elem<KV>::to_f32(rrow[(size_t)i * C]));
-        if (cok) orow[(size_t)i * C] = Elem<OUT>::from_f32(o);
-      }
-    } else {
-      const bool fast = __all_sync(0xffffffffu, fast_uw(u, w));
-      const float cb[1] = {ex2(fminf(fmaxf(u - w, -kFastUW), kFastUW) * kLog2e)};
-      const float w1[1] = {w};
-      Acc s1[1] = {st};
-      if (fast && nv == J) {
-        // the span's hot loop, compiled once with and once without the gate
-        auto span = [&](auto gated) {
+    const bool fast = !kWT && __all_sync(0xffffffffu, fast_uw(u, w));
+    const float cb[1] = {ex2(fminf(fmaxf(u - w, -kFastUW), kFastUW) * kLog2e)};
+    const float w1[1] = {w};
+#pragma unroll 1
+    for (int blk = 0; blk < nb; ++blk, ++n) {
+      if (!wait_copy(n)) break;
+      const unsigned char* sb = ring + (size_t)(n % NS) * kStage;
+      const KV* ks = reinterpret_cast<const KV*>(sb) + lane;
+      const KV* vs = ks + kTile;
+      const int nt = min(LB, nv - blk * LB);
+      OUT* ob = orow + (size_t)blk * LB * C;
+      const KV* rb = rrow ? rrow + (size_t)blk * LB * C : nullptr;
+      if (kWT) {
+        const float* ws = reinterpret_cast<const float*>(sb + 2 * kTile * sizeof(KV)) + lane;
+        for (int i = 0; i < nt; ++i) {
+          float o = step_token_wt(st, lo, Elem<KV>::to_f32(ks[i * CG]), Elem<KV>::to_f32(vs[i * CG]), ws[i * CG], u);
+          if (rb && cok) o = gate(o, Elem<KV>::to_f32(rb[(size_t)i * C]));
+          if (cok) ob[(size_t)i * C] = Elem<OUT>::from_f32(o);
+        }
+      } else if (fast && nt == LB) {
+        // the block's hot loop, compiled once with and once without the gate
+        auto run = [&](auto gated) {
           constexpr bool kGate = decltype(gated)::value;
-          constexpr int NB = J < 8 ? J : 8;
+          float kb[LB][1], vb[LB][1], o[LB][1], rg[LB];
+          Acc s1[1] = {st};
 #pragma unroll
-          for (int j0 = 0; j0 < J; j0 += NB) {
-            float kb[NB][1], vb[NB][1], ob[NB][1], rb[NB];
-#pragma unroll
-            for (int jj = 0; jj < NB; ++jj) {
-              kb[jj][0] = cok ? Elem<KV>::to_f32(kg[(size_t)(j0 + jj) * C]) : 0.f;
-              vb[jj][0] = cok ? Elem<KV>::to_f32(vg[(size_t)(j0 + jj) * C]) : 0.f;
-              if (kGate) rb[jj] = cok ? Elem<KV>::to_f32(rrow[(size_t)(j0 + jj) * C]) : 0.f;
-            }
-            step_tokens<NB, 1>(s1, kb, vb, w1, cb, ob);
-#pragma unroll
-            for (int jj = 0; jj < NB; ++jj) {
-              const float o[1] = {kGate ? gate(ob[jj][0], rb[jj]) : ob[jj][0]};
-              if (cok) stg_stream<OUT, 1>(orow + (size_t)(j0 + jj) * C, o);
-            }
+          for (int i = 0; i < LB; ++i) {
+            kb[i][0] = Elem<KV>::to_f32(ks[i * CG]);
+            vb[i][0] = Elem<KV>::to_f32(vs[i * CG]);
+            if (kGate) rg[i] = cok ? Elem<KV>::to_f32(rb[(size_t)i * C]) : 0.f;
           }
+          step_tokens<LB, 1>(s1, kb, vb, w1, cb, o);
+#pragma unroll
+          for (int i = 0; i < LB; ++i) {
+            const float oi[1] = {kGate ? gate(o[i][0], rg[i]) : o[i][0]};
+            if (cok) stg_stream<OUT, 1>(ob + (size_t)i * C, oi);
+          }
+          st = s1[0];
         };
-        if (rrow) {
-          span(Flag<true>{});
+        if (rb) {
+          run(Flag<true>{});
         } else {
-          span(Flag<false>{});
+          run(Flag<false>{});
         }
       } else {
-        for (int i = 0; i < nv; ++i) {
-          const float kk = cok ? Elem<KV>::to_f32(kg[(size_t)i * C]) : 0.f;
-          const float vv = cok ? Elem<KV>::to_f32(vg[(size_t)i * C]) : 0.f;
-          float o = out_token(s1[0], kk, vv, w, u);
-          add_token(s1[0], kk, vv, w);
-          if (rrow && cok) o = gate(o, Elem<KV>::to_f32(rrow[(size_t)i * C]));
-          if (cok) orow[(size_t)i * C] = Elem<OUT>::from_f32(o);
+        for (int i = 0; i < nt; ++i) {
+          const float kk = Elem<KV>::to_f32(ks[i * CG]);
+          const float vv = Elem<KV>::to_f32(vs[i * CG]);
+          float o = out_token(st, kk, vv, w, u);
+          add_token(st, kk, vv, w);
+          if (rb && cok) o = gate(o, Elem<KV>::to_f32(rb[(size_t)i * C]));
+          if (cok) ob[(size_t)i * C] = Elem<OUT>::from_f32(o);
         }
       }
-      st = s1[0];
+      release();
     }
     // the warp that holds the last token writes the state out
-    if (p.o_num && cok && ts + nv == T && WKV_IN(p.hdr, (size_t)b * C + c, (size_t)p.B * C)) {
+    if (ok && p.o_num && cok && ts + nv == T && WKV_IN(p.hdr, (size_t)b * C + c, (size_t)p.B * C)) {
       const size_t i = (size_t)b * C + c;
       p.o_num[i] = st.num;
       p.o_den[i] = st.den;
       p.o_max[i] = kWT ? acc_max_e_wt(st, lo) : acc_max_e(st, w);
     }
+  }
+  if (lane == 0) {
+    if (!ok) atomicOr(&p.hdr->status, kStatusWaitTimeout);
+    // copies still in flight (after a wait ran out, or a replay that did not
+    // run): a bounded chance to land before the CTA leaves
+    for (int x = n; x < issued; ++x) (void)mbar_wait(&bars[x % NS], (uint32_t)((x / NS) & 1), p.timeout_ns);
   }
   cluster_wait();
 }
