@@ -86,11 +86,12 @@ def test_workspace_size(L):
     assert 256 < a < b
     # cluster scan: a flag and a prefix per segment after the first and channel
     # group, and room for the single-launch scan that misaligned inputs take
-    o5, o2 = _abi.wkv_options(kernel=5), _abi.wkv_options(kernel=2)
+    o5, o3, o2 = (_abi.wkv_options(kernel=k) for k in (5, 3, 2))
     for T in (2048, 4096, 4097, 16384):
-        assert L.wkv_forward_workspace_size(8, T, 768, None) == L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o5))
-        assert L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o5)) >= \
-            L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o2))
+        assert L.wkv_forward_workspace_size(8, T, 768, None) == L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o3))
+        for o in (o5, o3):
+            assert L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o)) >= \
+                L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o2))
     assert L.wkv_forward_workspace_size(-1, 4, 4, None) == 0
     o = _abi.wkv_options(kernel=2, chunk_len=48)
     assert L.wkv_forward_workspace_size(1, 64, 64, ctypes.byref(o)) == 0
@@ -101,12 +102,12 @@ def test_workspace_size(L):
 def test_forward_kernel_choice(L):
     F32, BF16 = _abi.WKV_F32, _abi.WKV_BF16
     # many channels or short sequences: the sequential kernel; otherwise the
-    # cluster scan (any T)
+    # three-launch scan (in windows for long sequences)
     assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
-    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 5
-    assert L.wkv_forward_kernel(8, 2049, 768, F32, None) == 5
-    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 5
+    assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 3
+    assert L.wkv_forward_kernel(8, 2049, 768, F32, None) == 3
+    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 3
     assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 2  # rows TMA cannot address
     # an explicit choice stands, except that the TMA scans fall back to the
     # single-launch scan when a row pitch is not a multiple of 16 bytes
@@ -117,9 +118,13 @@ def test_forward_kernel_choice(L):
     for bad in (dict(cta_warps=3), dict(cta_warps=16), dict(cta_warps=32), dict(span=8), dict(span=16)):
         o = _abi.wkv_options(kernel=5, **bad)
         assert L.wkv_forward_kernel(2, 100, 64, F32, ctypes.byref(o)) == 0
-    assert L.wkv_forward_launches(8, 1024, 768, F32, None) == 1
-    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 1
-    assert L.wkv_forward_launches(1, 65536, 2048, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 3
+    assert L.wkv_forward_launches(8, 1024, 768, F32, ctypes.byref(_abi.wkv_options(kernel=5))) == 1
+    assert L.wkv_forward_launches(1, 65536, 2048, F32, ctypes.byref(_abi.wkv_options(kernel=3,
+                                                                                    window_tokens=-1))) == 3
+    # windows of 1536 tokens (24 MB of fp32 k and v) in 64-token chunks
+    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 3 * 43
+    for bad in (-2, -100):
+        assert L.wkv_forward_kernel(1, 4096, 64, F32, ctypes.byref(_abi.wkv_options(window_tokens=bad))) == 0
     assert L.wkv_forward_launches(2, 20, 64, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 2
     assert L.wkv_forward_launches(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(-1, 4, 4, F32, None) == 0

@@ -69,11 +69,11 @@ def _check_call(oracle, L, B, T, C, seed, with_state, misaligned, what):
 
 
 def test_noalloc_matches_oracle_on_calls_in_a_row(oracle):
-    """Calls in a row: the cluster scan with one segment (only the status word
-    in the scratch array) and several (the scratch holds each segment's flag
-    and prefix, which must start from a clean epoch on every call), and
-    misaligned inputs (the single-launch scan, whose flags share the array);
-    each against the oracle."""
+    """Calls in a row: the three-launch scan (chunk totals and incoming states
+    in the scratch array; as one window, since this entry point creates no
+    stream), misaligned inputs (the single-launch scan, whose flags share the
+    array and must start from a clean epoch on every call); each against the
+    oracle."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from wkv_recurrence_b200 import build

@@ -235,10 +235,13 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
     ok = __all_sync(0xffffffffu, got);
     return ok;
   };
-  auto release = [&]() {  // stage n-1 consumed: its slot takes copy n-1+NS
+  // Stage consumed: its slot takes the next copy. The warp's reads of the
+  // stage are ordered before the copy by __syncwarp (the consumer-release /
+  // producer-acquire pattern of TMA pipelines; no proxy fence is needed for a
+  // read followed by an asynchronous write).
+  auto release = [&]() {
     __syncwarp();
     if (lane == 0 && issued < nl) {
-      fence_proxy_async_smem();
       issue(issued);
       ++issued;
     }
@@ -275,9 +278,11 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
 #pragma unroll
       for (int i = 0; i < LB; ++i) wx[i] = ws[i * CG];
       float wb;
-      const Acc a = fold_regs_wt<LB>(kx, vx, wx, nt, wb);
+      const Acc a = nt == LB ? fold_regs_wt<LB>(kx, vx, wx, LB, wb) : fold_regs_wt<LB>(kx, vx, wx, nt, wb);
       agg = combine_wt(agg, a, wb);
       wsum += wb;
+    } else if (nt == LB) {
+      agg = combine(agg, fold_regs<LB>(kx, vx, LB, w), (float)LB, w);  // (full block: no per-token tests)
     } else {
       agg = combine(agg, fold_regs<LB>(kx, vx, nt, w), (float)nt, w);
     }
