@@ -125,16 +125,6 @@ typedef struct {
  *                   one replay warp walks (0 = choose; or 1, 2, 4)
  *   cta_warps       cluster scan (kernel 5): warps (spans) per CTA, 4 or 8
  *                   (0 = 8)
- *   window_tokens   three-launch scan (kernel 3): tokens per window (0 =
- *                   choose: about 24 MB of fp32 k and v; -1 = the whole
- *                   sequence as one window; otherwise rounded up to whole
- *                   replays). With more than one window, the chunk totals of
- *                   window w+1 are computed on a second stream of the
- *                   library's own while window w is scanned and replayed on
- *                   the caller's, which waits for everything before the call
- *                   returns its work; the replay's second read of k and v then
- *                   hits L2. Safe under stream capture once a first call on
- *                   the device has created that stream outside of capture.
  *   stages          shared-memory ring stages of the pipelined scan
  *                   (kernel 4): 0 = choose, otherwise 2..8 (must fit in one
  *                   CTA's shared memory, else WKV_ERR_INVALID_ARG at launch)
@@ -160,7 +150,6 @@ typedef struct {
     int32_t seq_vec;
     int32_t replay_chunks;
     int32_t cta_warps;
-    int32_t window_tokens;
 } wkv_options;
 
 /*

@@ -102,7 +102,7 @@ def test_workspace_size(L):
 def test_forward_kernel_choice(L):
     F32, BF16 = _abi.WKV_F32, _abi.WKV_BF16
     # many channels or short sequences: the sequential kernel; otherwise the
-    # three-launch scan (in windows for long sequences)
+    # three-launch scan
     assert L.wkv_forward_kernel(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
     assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 3
@@ -119,12 +119,7 @@ def test_forward_kernel_choice(L):
         o = _abi.wkv_options(kernel=5, **bad)
         assert L.wkv_forward_kernel(2, 100, 64, F32, ctypes.byref(o)) == 0
     assert L.wkv_forward_launches(8, 1024, 768, F32, ctypes.byref(_abi.wkv_options(kernel=5))) == 1
-    assert L.wkv_forward_launches(1, 65536, 2048, F32, ctypes.byref(_abi.wkv_options(kernel=3,
-                                                                                    window_tokens=-1))) == 3
-    # windows of 1536 tokens (24 MB of fp32 k and v) in 64-token chunks
-    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 3 * 43
-    for bad in (-2, -100):
-        assert L.wkv_forward_kernel(1, 4096, 64, F32, ctypes.byref(_abi.wkv_options(window_tokens=bad))) == 0
+    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 3
     assert L.wkv_forward_launches(2, 20, 64, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 2
     assert L.wkv_forward_launches(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(-1, 4, 4, F32, None) == 0

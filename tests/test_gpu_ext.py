@@ -1,5 +1,4 @@
-"""GPU parity of the cluster scan (kernel 5), of the three-launch scan in
-windows, and of the two optional inputs of
+"""GPU parity of the cluster scan (kernel 5) and of the two optional inputs of
 the RWKV-v6 time-mixing block ("RWKV-v6 Architecture: Attention-Free Linear
 Transformers"): per-token decays w_t (section "2. Dynamic Data-Dependent
 Decay") and the receptance gate out = sigmoid(r) * wkv. Everything through
@@ -127,79 +126,6 @@ def test_three_launch_is_the_automatic_choice_for_few_channels():
     assert W.forward_kernel(8, 1024, 768) == 3
     assert W.forward_kernel(1, 65536, 2048) == 3
     assert W.forward_kernel(16, 4096, 4096, torch.bfloat16) == 1
-
-
-# ---------------------------------------------------------------------------
-# the three-launch scan in windows (totals of window w+1 on the library's
-# second stream beside the scan and replay of window w)
-# ---------------------------------------------------------------------------
-
-WINDOWS = [{"kernel": 3, "window_tokens": 64}, {"kernel": 3, "window_tokens": 200},
-           {"kernel": 3, "window_tokens": 1024, "replay_chunks": 4}, {"kernel": 3, "window_tokens": 32,
-                                                                    "chunk_len": 32}]
-WIN_IDS = ["w64", "w200", "w1024r4", "w32c32"]
-
-
-@pytest.mark.parametrize("opts", WINDOWS, ids=WIN_IDS)
-@pytest.mark.parametrize("shape", [(2, 1000, 96), (1, 5000, 200), (3, 777, 64), (2, 4097, 128), (1, 64, 64),
-                                   (1, 65, 64)], ids=lambda s: "x".join(map(str, s)))
-def test_windowed_three_launch(oracle, opts, shape):
-    """Windows of one chunk up to many, ragged last windows and chunks, the
-    state in (read by the first window's scan) and out (written by the last
-    window's replay)."""
-    B, T, C = shape
-    k, v, w, u, st = I.random_case(B, T, C, seed=B * 11 + T + C, k_scale=2.0, k_spike=30.0,
-                                   w_range=(1e-4, 8.0), state=(T % 2 == 0))
-    compare_ext(oracle, k, v, w, u, st, options=opts)
-
-
-@pytest.mark.parametrize("kv", ["f32", "bf16"])
-def test_windowed_with_decay_and_gate(oracle, kv):
-    B, T, C = 2, 3000, 96
-    k, v, w, u, st = I.random_case(B, T, C, seed=77, k_spike=30.0, state=True)
-    wt, r = _wt((B, T, C), 78), _r((B, T, C), 79)
-    if kv == "bf16":
-        k, v, r = I.f32_to_bf16_bits(k), I.f32_to_bf16_bits(v), I.f32_to_bf16_bits(r)
-    compare_ext(oracle, k, v, w, u, st, kv=kv, options={"kernel": 3, "window_tokens": 256}, w_t=wt, r=r)
-
-
-def test_windowed_launch_count_and_default_windows():
-    o = {"kernel": 3, "window_tokens": 64, "chunk_len": 64}
-    assert W.forward_launches(1, 640, 64, options=o) == 3 * 9 + 2  # the last window: scan and replay only
-    assert W.forward_launches(1, 640, 64, options=dict(o, window_tokens=-1)) == 3
-    # the default keeps a window near 24 MB of fp32 k and v
-    assert W.forward_launches(8, 1024, 768) == 6
-    assert W.forward_launches(1, 65536, 2048) > 60
-
-
-def test_windowed_in_a_cuda_graph(oracle):
-    """The second stream joins a stream capture through the fork event and is
-    joined back before the capture ends; replays of the graph give the
-    oracle's result."""
-    B, T, C = 2, 3000, 64
-    k, v, w, u, st = I.random_case(B, T, C, seed=81, k_spike=30.0, state=True)
-    opts = {"kernel": 3, "window_tokens": 256}
-    K, V, Wt, U = dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u)
-    S = tuple(dev_f32(x) for x in st)
-    ws = W.make_workspace(B, T, C, options=opts)
-    out = torch.empty(B, T, C, device="cuda")
-    so = tuple(torch.empty(B, C, device="cuda") for _ in range(3))
-    s = torch.cuda.Stream()
-    with torch.cuda.stream(s):
-        W.forward(K, V, Wt, U, S, out=out, state_out=so, workspace=ws, options=opts)  # creates the second stream
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        W.forward(K, V, Wt, U, S, out=out, state_out=so, workspace=ws, options=opts)
-    out.fill_(float("nan"))
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize()
-    ref, rst = oracle.recurrence_forward(k, v, w, u, st)
-    sc, sst = oracle.abs_scale_forward(k, v, w, u, st)
-    assert_out(host(out), ref, sc, RTOL_F32)
-    assert_state(tuple(host(x) for x in so), rst, sst[0], RTOL_F32)
-    assert W.query_status(ws) == 0
 
 
 # ---------------------------------------------------------------------------

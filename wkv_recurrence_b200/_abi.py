@@ -50,7 +50,7 @@ class wkv_options(ctypes.Structure):
                 ("span", ctypes.c_int32), ("seq_threads", ctypes.c_int32),
                 ("scan_segments", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("seq_vec", ctypes.c_int32), ("replay_chunks", ctypes.c_int32),
-                ("cta_warps", ctypes.c_int32), ("window_tokens", ctypes.c_int32)]
+                ("cta_warps", ctypes.c_int32)]
 
 
 class wkv_ext(ctypes.Structure):

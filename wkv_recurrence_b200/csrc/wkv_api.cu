@@ -25,10 +25,6 @@ namespace wkv {
 namespace {
 
 constexpr int kMaxDevices = 64;
-// default window of the three-launch scan: this many bytes of fp32 k and v
-// (two windows, one being replayed and one being folded, stay well inside
-// the 126 MB L2 next to the outputs in flight)
-constexpr size_t kWindowBytes = 24u << 20;
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s
 
 // ---------------------------------------------------------------------------
@@ -57,7 +53,6 @@ struct Plan {
   int scan_segments;  // three-launch scan: segments per channel in the scan of chunk totals
   int replay_chunks;  // three-launch scan: consecutive chunks per replay CTA
   int replay_threads;  // three-launch scan: threads (channels) per replay CTA
-  int win_chunks;      // three-launch scan: chunks per window (>= nch: one window)
   int stages;       // pipelined chunked scan: ring stages (0 = choose at launch)
   int L;       // chunk length (chunk kernel)
   int J;       // tokens per warp (chunk kernel)
@@ -109,10 +104,9 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
     if (lanes >= 65536 || T <= 64) {
       kernel = 1;
     } else {
-      // the three-launch scan, in windows where the sequence does not fit in
-      // L2 (measured faster than the single-launch scans on every workload:
-      // layer 23.4 us against 29.8 for the cluster scan; long 436 against
-      // 438-490)
+      // the three-launch scan (measured faster than the single-launch scans
+      // on every workload: layer 23.4 us against 29.8 for the cluster scan;
+      // long 436 against 438-490)
       kernel = 3;
     }
   }
@@ -209,25 +203,6 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   // resident warps; layer: 23.8 us against 24.2 and 24.7 at 64 and 128; long:
   // within 1.5% at all three)
   pl->replay_threads = (o && o->seq_threads) ? o->seq_threads : 32;
-  // the three-launch scan in windows of chunks: the totals pass of window w+1
-  // (on a second stream) runs beside the scan and replay of window w, whose
-  // second read of k and v then hits L2; windows of about kWindowBytes of
-  // fp32 k and v by default
-  {
-    const int64_t wt_opt = o ? o->window_tokens : 0;
-    if (wt_opt < -1) return false;
-    const int64_t unit = (int64_t)L * pl->replay_chunks;  // tokens; windows are whole replays
-    int64_t wtok;
-    if (wt_opt == -1) {
-      wtok = T;
-    } else if (wt_opt > 0) {
-      wtok = wt_opt;
-    } else {
-      wtok = (int64_t)(kWindowBytes / (size_t)std::max<int64_t>(1, B * C * 8));
-    }
-    wtok = std::max<int64_t>(unit, (wtok + unit - 1) / unit * unit);
-    pl->win_chunks = (int)std::min<int64_t>(pl->nch, wtok / L);
-  }
   const long long BNG = (long long)B * pl->NG;
   pl->n_tiles = (long long)pl->nch * BNG;
   if (pl->n_tiles >= (1ll << 31)) return false;
@@ -507,36 +482,12 @@ wkv_status launch_seq_chunks(const FwdParams& p, const CUtensorMap& bk, const CU
   const size_t smem = (size_t)STAGES * seq_stage_bytes<KV, LT, TH, kWT>() + 64 * STAGES;
   int occ = 0;
   if (!kernel_setup(fb, dev, TH, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
-  const long long nseq = (p.chn + p.replay_chunks - 1) / p.replay_chunks;  // replays per row in the window
+  const long long nseq = (p.nch + p.replay_chunks - 1) / p.replay_chunks;
   const long long grid = (long long)p.B * nseq * ((p.C + TH - 1) / TH);
   if (grid >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
   PdlConfig cb(dim3((unsigned)grid), dim3(TH), smem, st);
   if (!cuda_ok(cudaLaunchKernelEx(&cb.cfg, fb, p, bk, bv, bw ? *bw : bv))) return WKV_ERR_CUDA;
   return launch_result();
-}
-
-// The library's second stream on a device, for the totals pass of the
-// windowed three-launch scan, and the events that fork it from the caller's
-// stream and order the two. Created on first use; one call at a time queues
-// work on them (mu), since the events are shared.
-struct AuxStream {
-  std::mutex mu;
-  bool ready = false;
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t a[2] = {nullptr, nullptr};  // totals pass of window w done (w % 2)
-  cudaEvent_t b[2] = {nullptr, nullptr};  // replay of window w done (w % 2)
-};
-AuxStream g_aux[kMaxDevices];
-
-bool aux_ready(AuxStream& x) {
-  if (x.ready) return true;
-  if (!cuda_ok(cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking))) return false;
-  cudaEvent_t* evs[5] = {&x.fork, &x.a[0], &x.a[1], &x.b[0], &x.b[1]};
-  for (cudaEvent_t* e : evs)
-    if (!cuda_ok(cudaEventCreateWithFlags(e, cudaEventDisableTiming))) return false;
-  x.ready = true;
-  return true;
 }
 
 template <typename KV, typename OUT, int NW, int J, bool kWT>
@@ -553,118 +504,68 @@ wkv_status launch_tile3(const Plan& pl, const FwdParams& p, const CUtensorMap& t
   int occ = 0;
   if (!kernel_setup(fa, dev, NW * 32, smem, &occ) || occ < 1) return WKV_ERR_CUDA;
   const long long BNG = (long long)p.B * p.NG;
-  // A: the totals of a window's chunks (all but the sequence's last chunk)
-  auto pass_a = [&](const FwdParams& q, cudaStream_t s) -> wkv_status {
-    const long long nt = std::min(q.ch0 + q.chn, q.nch - 1) - q.ch0;
-    if (nt <= 0) return WKV_OK;
-    fa<<<(unsigned)(nt * BNG), NW * 32, smem, s>>>(q, tk, tv, tw);
-    return launch_result();
-  };
-  // S: the incoming state of each chunk of a window; pdl = programmatic
-  // serialization behind A on the same stream
-  auto pass_s = [&](const FwdParams& q, cudaStream_t s, bool pdl) -> wkv_status {
-    const int ntot = std::min(q.ch0 + q.chn, q.nch - 1) - q.ch0;
-    // segments per channel in the scan: at most about 16 chunk totals each
-    int seg = pl.scan_segments;
-    if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 64 ? 4 : (ntot <= 256 ? 16 : 64));
-    const unsigned gs = (unsigned)(BNG * 4);  // 16 channels per CTA
-    PdlConfig cs(dim3(gs), dim3(16 * seg), 0, s);
-    if (!pdl) cs.cfg.numAttrs = 0;
-    cudaError_t e;
-    switch (seg) {
-      case 1: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<1, kWT>, q, L); break;
-      case 4: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<4, kWT>, q, L); break;
-      case 16: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<16, kWT>, q, L); break;
-      default: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<64, kWT>, q, L); break;
-    }
-    return (cuda_ok(e) && launch_result() == WKV_OK) ? WKV_OK : WKV_ERR_CUDA;
-  };
-  // B: the sequential kernel over every (batch row, replay of R chunks,
-  // 32-channel group) of a window, from the chunk's incoming state; one
-  // channel per thread, replay_threads channels per CTA (32 with per-token
-  // decays)
+  if (p.nch > 1) {
+    fa<<<(unsigned)((p.nch - 1) * BNG), NW * 32, smem, st>>>(p, tk, tv, tw);
+    if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  }
+  // segments per channel in the scan: at most about 16 chunk totals each
+  const int ntot = p.nch - 1;
+  int seg = pl.scan_segments;
+  if (seg == 0) seg = ntot <= 16 ? 1 : (ntot <= 64 ? 4 : (ntot <= 256 ? 16 : 64));
+  const unsigned gs = (unsigned)(BNG * 4);  // 16 channels per CTA
+  // programmatic serialization only behind A (an ordinary launch, so S is
+  // scheduled only after the launch ahead of the call has ended: S reads w
+  // before its own wait)
+  PdlConfig cs(dim3(gs), dim3(16 * seg), 0, st);
+  if (p.nch <= 1) cs.cfg.numAttrs = 0;
+  cudaError_t e;
+  switch (seg) {
+    case 1: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<1, kWT>, p, L); break;
+    case 4: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<4, kWT>, p, L); break;
+    case 16: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<16, kWT>, p, L); break;
+    default: e = cudaLaunchKernelEx(&cs.cfg, wkv_tile_scan<64, kWT>, p, L); break;
+  }
+  if (!cuda_ok(e) || launch_result() != WKV_OK) return WKV_ERR_CUDA;
+  // B: the sequential kernel over every (batch row, chunk, 32-channel group),
+  // from the chunk's incoming state; one channel per thread
   constexpr bool kF32 = sizeof(KV) == 4;
   constexpr int LT = kF32 ? 2 * kSeqLtF32 : 2 * kSeqLtBf16;
+  // one channel per thread, replay_threads channels per CTA (32 with
+  // per-token decays)
   const int th = kWT ? 32 : pl.replay_threads;
   CUtensorMap bk, bv, bw;
   if (!make_tmap(&bk, p.k, kvdt, p.B, p.T, p.C, LT, th) || !make_tmap(&bv, p.v, kvdt, p.B, p.T, p.C, LT, th))
     return WKV_ERR_CUDA;
-  if (kWT && !make_tmap(&bw, p.w_t, WKV_F32, p.B, p.T, p.C, LT, th)) return WKV_ERR_CUDA;
-  // a 32-token fp32 replay runs as one 32-token stage: one copy pair and one
-  // wait instead of two (layer: 23.5 against 23.8 us)
-  const bool one32 = !kWT && kF32 && pl.replay_chunks * L == 32 && th == 32;
-  CUtensorMap ck, cv;
-  if (one32 && (!make_tmap(&ck, p.k, kvdt, p.B, p.T, p.C, 32, th) ||
-                !make_tmap(&cv, p.v, kvdt, p.B, p.T, p.C, 32, th)))
-    return WKV_ERR_CUDA;
   // a replay of at most two stages is prefetched whole with 2 (more CTAs fit
   // per SM); longer ones stream through 3
-  const bool two = pl.replay_chunks * L <= 2 * LT;
-  auto pass_b = [&](const FwdParams& q, cudaStream_t s) -> wkv_status {
-    if (kWT) {
-      return two ? launch_seq_chunks<KV, OUT, 32, LT, 2, true>(q, bk, bv, s, dev, &bw)
-                 : launch_seq_chunks<KV, OUT, 32, LT, 3, true>(q, bk, bv, s, dev, &bw);
-    }
-    if (one32) return launch_seq_chunks<KV, OUT, 32, 32, 1>(q, ck, cv, s, dev);
-    switch (th) {
-      case 64:
-        return two ? launch_seq_chunks<KV, OUT, 64, LT, 2>(q, bk, bv, s, dev)
-                   : launch_seq_chunks<KV, OUT, 64, LT, 3>(q, bk, bv, s, dev);
-      case 128:
-        return two ? launch_seq_chunks<KV, OUT, 128, LT, 2>(q, bk, bv, s, dev)
-                   : launch_seq_chunks<KV, OUT, 128, LT, 3>(q, bk, bv, s, dev);
-      default:
-        return two ? launch_seq_chunks<KV, OUT, 32, LT, 2>(q, bk, bv, s, dev)
-                   : launch_seq_chunks<KV, OUT, 32, LT, 3>(q, bk, bv, s, dev);
-    }
-  };
   FwdParams q = p;
   q.replay_chunks = pl.replay_chunks;
-  const int cpw = std::max(1, pl.win_chunks);
-  const int nwin = (p.nch + cpw - 1) / cpw;
-  wkv_status r;
-  if (nwin <= 1) {
-    // one window, one stream: A, then S behind it (programmatic
-    // serialization: an ordinary launch for A, so that S is scheduled only
-    // after the launch ahead of the call has ended: S reads w before its own
-    // wait), then B behind S
-    q.ch0 = 0;
-    q.chn = p.nch;
-    if ((r = pass_a(q, st)) != WKV_OK) return r;
-    if ((r = pass_s(q, st, p.nch > 1)) != WKV_OK) return r;
-    return pass_b(q, st);
-  }
-  // windows: A(w+1) on the second stream beside S(w), B(w) on the caller's;
-  // A(w+1) waits for B(w-1) (at most two windows in L2), S(w) for A(w) and
-  // (same stream) for B(w-1), which has read the state S(w-1) left.
-  AuxStream& ax = g_aux[dev];
-  std::lock_guard<std::mutex> lk(ax.mu);
-  if (!aux_ready(ax)) return WKV_ERR_CUDA;
-  if (!cuda_ok(cudaEventRecord(ax.fork, st)) || !cuda_ok(cudaStreamWaitEvent(ax.s, ax.fork, 0)))
-    return WKV_ERR_CUDA;
-  auto window = [&](int w) {
-    FwdParams x = q;
-    x.ch0 = w * cpw;
-    x.chn = std::min(cpw, p.nch - x.ch0);
-    return x;
-  };
-  if ((r = pass_a(window(0), ax.s)) != WKV_OK) return r;
-  if (!cuda_ok(cudaEventRecord(ax.a[0], ax.s))) return WKV_ERR_CUDA;
-  for (int w = 0; w < nwin; ++w) {
-    if (w + 1 < nwin) {
-      if (w >= 1 && !cuda_ok(cudaStreamWaitEvent(ax.s, ax.b[(w - 1) & 1], 0))) return WKV_ERR_CUDA;
-      if ((r = pass_a(window(w + 1), ax.s)) != WKV_OK) return r;
-      if (!cuda_ok(cudaEventRecord(ax.a[(w + 1) & 1], ax.s))) return WKV_ERR_CUDA;
+  const bool two = pl.replay_chunks * L <= 2 * LT;
+  if (kWT) {
+    if (!make_tmap(&bw, p.w_t, WKV_F32, p.B, p.T, p.C, LT, th)) return WKV_ERR_CUDA;
+    return two ? launch_seq_chunks<KV, OUT, 32, LT, 2, true>(q, bk, bv, st, dev, &bw)
+               : launch_seq_chunks<KV, OUT, 32, LT, 3, true>(q, bk, bv, st, dev, &bw);
+  } else {
+    if (kF32 && pl.replay_chunks * L == 32 && th == 32) {
+      // a 32-token fp32 replay as one 32-token stage: one copy pair and one
+      // wait instead of two (layer: 23.5 against 23.8 us)
+      CUtensorMap ck, cv;
+      if (!make_tmap(&ck, p.k, kvdt, p.B, p.T, p.C, 32, th) || !make_tmap(&cv, p.v, kvdt, p.B, p.T, p.C, 32, th))
+        return WKV_ERR_CUDA;
+      return launch_seq_chunks<KV, OUT, 32, 32, 1>(q, ck, cv, st, dev);
     }
-    if (!cuda_ok(cudaStreamWaitEvent(st, ax.a[w & 1], 0))) return WKV_ERR_CUDA;
-    const FwdParams x = window(w);
-    if ((r = pass_s(x, st, false)) != WKV_OK) return r;
-    if ((r = pass_b(x, st)) != WKV_OK) return r;
-    if (w + 2 < nwin && !cuda_ok(cudaEventRecord(ax.b[w & 1], st))) return WKV_ERR_CUDA;
+    switch (th) {
+      case 64:
+        return two ? launch_seq_chunks<KV, OUT, 64, LT, 2>(q, bk, bv, st, dev)
+                   : launch_seq_chunks<KV, OUT, 64, LT, 3>(q, bk, bv, st, dev);
+      case 128:
+        return two ? launch_seq_chunks<KV, OUT, 128, LT, 2>(q, bk, bv, st, dev)
+                   : launch_seq_chunks<KV, OUT, 128, LT, 3>(q, bk, bv, st, dev);
+      default:
+        return two ? launch_seq_chunks<KV, OUT, 32, LT, 2>(q, bk, bv, st, dev)
+                   : launch_seq_chunks<KV, OUT, 32, LT, 3>(q, bk, bv, st, dev);
+    }
   }
-  // every launch on the second stream ended in an event the caller's stream
-  // waited for: the fork is joined
-  return WKV_OK;
 }
 
 template <typename KV, typename OUT>
@@ -1034,14 +935,7 @@ int32_t wkv_forward_launches(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype
   const size_t es = kv_dtype == WKV_F32 ? 4 : 2;
   Plan pl;
   if (!make_plan(B, T, C, opts, &pl, (C * (int64_t)es) % 16 == 0)) return 0;
-  if (pl.kernel == 3) {
-    // per window: chunk totals (when the window has a chunk before the
-    // sequence's last), scan, replay
-    const int cpw = std::max(1, pl.win_chunks);
-    int n = 0;
-    for (int c0 = 0; c0 < pl.nch; c0 += cpw) n += (std::min(c0 + cpw, pl.nch - 1) > c0 ? 3 : 2);
-    return n;
-  }
+  if (pl.kernel == 3) return pl.nch > 1 ? 3 : 2;  // chunk totals (when there is more than one chunk), scan, replay
   return 1;
 }
 
@@ -1122,8 +1016,6 @@ wkv_status wkv_forward_ext(int64_t B, int64_t T, int64_t C, const void* k, const
   } else if (pl.kernel >= 2) {
     p.NG = pl.NG;
     p.nch = pl.nch;
-    p.ch0 = 0;
-    p.chn = pl.nch;  // one window: launch_tile3 splits it
     p.G = pl.G;
     p.chunk_len = pl.L;
     p.n_tiles = (int)pl.n_tiles;
@@ -1318,8 +1210,6 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const void* k, const vo
   fp.C = (int)C;
   fp.NG = pl.NG;
   fp.nch = pl.nch;
-  fp.ch0 = 0;
-  fp.chn = pl.nch;
   fp.chunk_len = kBwdL;
   fp.k = k;
   fp.v = v;
@@ -1424,22 +1314,16 @@ wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, c
   const wkv_status chk =
       check_forward_args(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, nullptr);
   if (chk != WKV_OK) return chk;
-  // the default choices, but the three-launch scan as one window (windows
-  // would need the library's second stream, which this entry point does not
-  // create)
-  wkv_options o;
-  std::memset(&o, 0, sizeof o);
-  o.window_tokens = -1;
   Plan pl;
   const size_t kes = kv_dtype == WKV_BF16 ? 2 : 4;
-  if (!make_plan(B, T, C, &o, &pl, tma_usable(k, v, C, kes))) return WKV_ERR_INVALID_ARG;
+  if (!make_plan(B, T, C, nullptr, &pl, tma_usable(k, v, C, kes))) return WKV_ERR_INVALID_ARG;
   if (pl.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_WORKSPACE_TOO_SMALL;
   if (B * C == 0) {
     // nothing to compute: wkv_forward checks the other arguments and returns
     // before it would look at a workspace, so no device (and no scratch
     // address) is needed; 256 only satisfies its alignment check
     return wkv_forward(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out,
-                       reinterpret_cast<void*>(uintptr_t(256)), WKV_NOALLOC_SCRATCH_BYTES, stream, &o);
+                       reinterpret_cast<void*>(uintptr_t(256)), WKV_NOALLOC_SCRATCH_BYTES, stream, nullptr);
   }
   int dev = 0;
   if (!cuda_ok(cudaGetDevice(&dev))) return WKV_ERR_CUDA;
@@ -1451,7 +1335,7 @@ wkv_status wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, const void* k, c
   if (!cuda_ok(cudaMemsetAsync(scratch, 0, clear, reinterpret_cast<cudaStream_t>(stream))))
     return WKV_ERR_CUDA;
   return wkv_forward(B, T, C, k, v, kv_dtype, w, u, out, out_dtype, state_in, state_out, scratch,
-                     WKV_NOALLOC_SCRATCH_BYTES, stream, &o);
+                     WKV_NOALLOC_SCRATCH_BYTES, stream, nullptr);
 }
 
 }  // extern "C"

@@ -83,7 +83,6 @@ struct FwdParams {
   const float* w_t;    // per-token decay [B, T, C] in place of w, or NULL
   const void* r;       // receptance [B, T, C] (element type of k, v): out = sigmoid(r) wkv; or NULL
   float* wtot;         // three-launch scan with w_t: decay sum of each chunk total, [nch-1][B * NG][64]
-  int ch0, chn;        // three-launch scan: the chunks [ch0, ch0 + chn) this launch covers (a window)
 };
 
 // Programmatic dependent launch: let the next launch on the stream be
@@ -156,10 +155,9 @@ __device__ __forceinline__ void coop_load_tile(KV* dst, const KV* src, int b, in
 // ---------------------------------------------------------------------------
 // kChunked: the replay pass of the three-launch scan. A CTA then takes
 // R = p.replay_chunks consecutive chunks (R * p.chunk_len tokens) of one batch
-// row, inside the launch's window of chunks [p.ch0, p.ch0 + p.chn), and starts
-// from the incoming state of the first, which the scan pass wrote to p.x0
-// ([nch][B * NG][64] with p.NG 64-channel groups); the grid is
-// B * ceil(chn / R) * ceil(C / CG). It issues its first copies (inputs only)
+// row and starts from the incoming state of the first, which the scan pass
+// wrote to p.x0 ([nch][B * NG][64] with p.NG 64-channel groups); the grid is
+// B * ceil(nch / R) * ceil(C / CG). It issues its first copies (inputs only)
 // before waiting (griddepcontrol.wait) for the scan, and only the CTA that
 // ends the sequence writes the state out.
 template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA, bool kChunked,
@@ -183,12 +181,12 @@ __global__ void __launch_bounds__(THREADS)
   const int ngs = kChunked ? (C + CG - 1) / CG : p.NG;  // channel groups of this kernel
   const int bj = blockIdx.x / ngs;
   const int g = blockIdx.x % ngs;
-  const int nseq = kChunked ? (p.chn + p.replay_chunks - 1) / p.replay_chunks : 1;  // replays per row (window)
+  const int nseq = kChunked ? (p.nch + p.replay_chunks - 1) / p.replay_chunks : 1;  // replays per row
   const int b = kChunked ? bj / nseq : bj;
   const int js = kChunked ? bj % nseq : 0;  // replay
-  const int jc = kChunked ? p.ch0 + js * p.replay_chunks : 0;  // its first chunk
+  const int jc = js * (kChunked ? p.replay_chunks : 1);  // its first chunk
   const int tbeg = kChunked ? jc * p.chunk_len : 0;
-  const int tend = kChunked ? min(T, min(jc + p.replay_chunks, p.ch0 + p.chn) * p.chunk_len) : T;
+  const int tend = kChunked ? min(T, tbeg + p.replay_chunks * p.chunk_len) : T;
   const int c0 = g * CG + tid * VEC;
   const int ntile = (tend - tbeg + LT - 1) / LT;
 
@@ -348,7 +346,7 @@ __global__ void __launch_bounds__(THREADS)
     return;
   }
 
-  if (p.o_num && c0 < C && tend == T) {
+  if (p.o_num && c0 < C && (!kChunked || js == nseq - 1)) {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       const int c = c0 + e;
@@ -854,10 +852,9 @@ __device__ __forceinline__ float4 ldg_f4(const float4* q) {
   return r;
 }
 
-// Pass A. Grid: (chunks of the window but the last chunk of the sequence) *
-// B * NG CTAs of NW warps, in chunk-major order from chunk p.ch0. Every tile
-// here is a full chunk (the last chunk, which alone can be partial, has no
-// total to compute).
+// Pass A. Grid: (nch - 1) * B * NG CTAs of NW warps; tile = blockIdx.x in
+// chunk-major order. Every tile here is a full chunk (the last chunk, which
+// alone can be partial, has no total to compute).
 template <typename KV, int NW, int J, bool kWT>
 __global__ void __launch_bounds__(NW * 32)
     wkv_tile_totals(const FwdParams p, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -877,8 +874,8 @@ __global__ void __launch_bounds__(NW * 32)
   const int lane = threadIdx.x & 31;
   const int wp = threadIdx.x >> 5;
   const int BNG = p.B * p.NG;
-  const int j = p.ch0 + (int)(blockIdx.x / BNG), bg = (int)(blockIdx.x % BNG);
-  const size_t tile = (size_t)j * BNG + bg;  // chunk-major index of the total
+  const int tile = blockIdx.x;
+  const int j = tile / BNG, bg = tile % BNG;
   const int cl = lane * VEC;
   const int c0 = (bg % p.NG) * CG + cl;
   if (threadIdx.x == 0) {
@@ -937,12 +934,12 @@ __global__ void __launch_bounds__(NW * 32)
         }
       }
     }
-    float4* dst = p.agg_a + tile * CG + cl;
+    float4* dst = p.agg_a + (size_t)tile * CG + cl;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      if (!WKV_IN(p.hdr, tile * CG + cl + e, (size_t)(p.nch - 1) * BNG * CG)) continue;
+      if (!WKV_IN(p.hdr, (size_t)tile * CG + cl + e, (size_t)(p.nch - 1) * BNG * CG)) continue;
       dst[e] = acc_pack(t[e]);
-      if (kWT) p.wtot[tile * CG + cl + e] = wt[e];
+      if (kWT) p.wtot[(size_t)tile * CG + cl + e] = wt[e];
     }
   }
   if (!ok && threadIdx.x == 0) (void)mbar_wait(bar, 0, p.timeout_ns);  // bounded drain
@@ -972,16 +969,13 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   const int sg = threadIdx.x / CH;
   const int b = bg / p.NG, c = (bg % p.NG) * CG + cl;
   const float w = (!kWT && c < p.C) ? __ldg(p.w + c) : 0.f;
-  // the totals of the window's chunks [ch0, ch0 + ntot): all but the last
-  // chunk of the sequence
-  const int ntot = min(p.ch0 + p.chn, p.nch - 1) - p.ch0;
+  const int ntot = p.nch - 1;
   const int per = (ntot + SEG - 1) / SEG;
   const int q0 = min(ntot, sg * per), q1 = min(ntot, q0 + per);
   const float fL = (float)L;
+  const float4* tot_of = p.agg_a + (size_t)bg * CG + cl;  // chunk q's total at tot_of[q * BNG * CG]
+  const float* wtot_of = kWT ? p.wtot + (size_t)bg * CG + cl : nullptr;
   const size_t qs = (size_t)BNG * CG;
-  // the window's chunk q: its total at tot_of[q * qs], its incoming state at x0_of[q * qs]
-  const float4* tot_of = p.agg_a + (size_t)p.ch0 * qs + (size_t)bg * CG + cl;
-  const float* wtot_of = kWT ? p.wtot + (size_t)p.ch0 * qs + (size_t)bg * CG + cl : nullptr;
   const size_t n_x0 = (size_t)p.nch * qs;  // x0 entries (bounds-checked build)
   (void)n_x0;
   // one combine of a chunk total (its decay sum wq with per-token decays)
@@ -1036,10 +1030,7 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   __syncthreads();
   // 2. incoming state of every segment (state in, then the segments before)
   if (sg == 0) {
-    // the window's incoming state: the state in, or what the scan of the
-    // window before left for the window's first chunk
-    Acc x = p.ch0 == 0 ? state_in_acc(p, b, c)
-                       : acc_unpack(p.x0[(size_t)p.ch0 * qs + (size_t)bg * CG + cl]);
+    Acc x = state_in_acc(p, b, c);
     for (int k = 0; k < SEG; ++k) {
       const Acc t = acc_unpack(seg_st[k][ch]);
       const int kq0 = min(ntot, k * per), kq1 = min(ntot, kq0 + per);
@@ -1050,14 +1041,12 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
   __syncthreads();
   // 3. incoming state of every chunk of the segment (and of the last chunk)
   Acc x = acc_unpack(seg_st[sg][ch]);
-  float4* x0_of = p.x0 + (size_t)p.ch0 * qs + (size_t)bg * CG + cl;
-  const size_t xb = (size_t)p.ch0 * qs + (size_t)bg * CG + cl;  // x0_of's offset in p.x0
-  (void)xb;
+  float4* x0_of = p.x0 + (size_t)bg * CG + cl;
   if (cached) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       if (q0 + r < q1) {
-        if (WKV_IN(p.hdr, xb + (q0 + r) * qs, n_x0)) x0_of[(q0 + r) * qs] = acc_pack(x);
+        if (WKV_IN(p.hdr, (size_t)bg * CG + cl + (q0 + r) * qs, n_x0)) x0_of[(q0 + r) * qs] = acc_pack(x);
         x = comb(x, a0[r], w0[r]);
       }
     }
@@ -1075,13 +1064,14 @@ __global__ void __launch_bounds__(16 * SEG) wkv_tile_scan(const FwdParams p, int
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         if (qq + r < q1) {
-          if (WKV_IN(p.hdr, xb + (qq + r) * qs, n_x0)) x0_of[(qq + r) * qs] = acc_pack(x);
+          if (WKV_IN(p.hdr, (size_t)bg * CG + cl + (qq + r) * qs, n_x0)) x0_of[(qq + r) * qs] = acc_pack(x);
           x = comb(x, a[r], wa[r]);
         }
       }
     }
   }
-  if (((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) && WKV_IN(p.hdr, xb + (size_t)ntot * qs, n_x0))
+  if (((q0 < q1 && q1 == ntot) || (ntot == 0 && sg == 0)) &&
+      WKV_IN(p.hdr, (size_t)bg * CG + cl + (size_t)ntot * qs, n_x0))
     x0_of[ntot * qs] = acc_pack(x);
 }
 
