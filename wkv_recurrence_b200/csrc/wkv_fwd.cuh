@@ -102,7 +102,10 @@ __device__ __forceinline__ Acc state_in_acc(const FwdParams& p, int b, int c) {
 
 template <typename OUT, int VEC>
 __device__ __forceinline__ void store_out(OUT* row, int c0, int C, bool vec_ok, const float (&o)[VEC]) {
-  if (vec_ok && c0 + VEC <= C) {
+  if constexpr (VEC == 1) {
+    // one channel per thread: callers store only for c0 < C
+    row[c0] = Elem<OUT>::from_f32(o[0]);
+  } else if (vec_ok && c0 + VEC <= C) {
     store_vec<OUT, VEC>(row + c0, o);
   } else {
 #pragma unroll
