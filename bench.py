@@ -12,8 +12,9 @@ The headline workload is `long` (B=1, T=65536, C=2048 fp32, 1.6 GB per
 forward), the largest single-GPU configuration. At N=1 the same JSON line also
 carries one sub-record per other workload ("workloads": layer 8x1024x768 fp32,
 mixed 16x4096x4096 bf16, the 256-step batched decode of 4096 streams x 768,
-small 1x64x768), each with its own throughput, roofline fraction, clocks and
-CPU-oracle baseline.
+small 1x64x768, the backward pass on layer and long, and the RWKV-v6
+matrix-state forward 8x1024x12x64 in fp32 and bf16), each with its own
+throughput, roofline fraction, clocks and CPU-oracle baseline.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload long]
     python -m torch.distributed.run --nproc-per-node N bench.py --gpus N ...
