@@ -34,7 +34,8 @@
 //         tokens in reverse from rin, writing dk, dv and per-chunk partial sums
 //         of du, dw; chunk 0 also yields the state gradients;
 //   RED   wkv_bwd_reduce: du, dw as compensated sums of the partials over the
-//         chunks and batch rows (a warp per channel), in a fixed order.
+//         chunks and batch rows (a thread per channel, 8 warps over eighths
+//         of the partials), in a fixed order.
 // One 32-thread CTA per (batch row, chunk, 32 channels) in R1 and R2, the
 // chunk's k, v and g copied into shared memory by TMA. All orders of
 // accumulation depend on the shape only, so results are bitwise reproducible.
@@ -133,16 +134,25 @@ __device__ __forceinline__ float exp_exact(float n, float w, float a, float b, f
 // kExact: the current token's weight b = e^{D} (D < 0) evaluated from the
 // exact exponent (the gradient pass, where b multiplies dk and dv directly);
 // otherwise rounded like everywhere else.
+// Exponents of magnitude up to kExactFrom are evaluated rounded: a few
+// roundings at that magnitude cost at most ~2e-6 of relative accuracy. A warp
+// takes the exact evaluation when any of its lanes has a larger one.
+constexpr float kExactFrom = 8.0f;
+
+// (mask: the lanes of the warp taking part, for the kExact vote.)
 template <bool kExact = false>
-__device__ __forceinline__ OutStat out_stat(const Acc& s, float k, float v, float u, float w) {
+__device__ __forceinline__ OutStat out_stat(const Acc& s, float k, float v, float u, float w,
+                                            unsigned mask = 0xffffffffu) {
   // D = (k + u) - m, formed as (k - ma) + u + nf w
-  float D, Dlo = 0.f;
-  if constexpr (kExact) {
+  float D = fmaf(s.nf, w, (k - s.ma) + u);
+  float x;
+  if (kExact && __any_sync(mask, fabsf(D) > kExactFrom)) {
+    float Dlo;
     exponent_hl(s.nf, w, k, s.ma, u, D, Dlo);
+    x = exp_hl(-fabsf(D), D > 0.f ? -Dlo : Dlo);
   } else {
-    D = fmaf(s.nf, w, (k - s.ma) + u);
+    x = ex2(-fabsf(D) * kLog2e);
   }
-  const float x = kExact ? exp_hl(-fabsf(D), D > 0.f ? -Dlo : Dlo) : ex2(-fabsf(D) * kLog2e);
   const bool tok = D > 0.f;  // the current token carries the largest exponent
   const float a = tok ? x : 1.f;
   const float b = tok ? 1.f : x;
@@ -212,6 +222,8 @@ __device__ __forceinline__ RAcc racc_combine(const RAcc& a, const RAcc& b, float
 // The chunk's tiles in shared memory: k, v (element type KV) and g (fp32), L
 // tokens x 32 channels each, copied by TMA on one mbarrier. Returns false if
 // the copy did not land within the wait limit (the status word is set).
+// (Measured: reading g from global memory a few tokens ahead instead, for
+// more resident CTAs, was slower overall.)
 template <typename KV, int L>
 __host__ __device__ constexpr uint32_t bwd_tile_bytes() {
   return (uint32_t)(L * 32 * (2 * sizeof(KV) + sizeof(float)));
@@ -355,6 +367,7 @@ __global__ void __launch_bounds__(32)
   const int t0 = j * L;
   if (!bwd_load_tile<KV, L>(p, &tmk, &tmv, &tmg, smem, bar, gw, t0, b)) return;
   const int c = gw * 32 + lane;
+  const unsigned vm = __ballot_sync(0xffffffffu, c < p.C);  // the lanes that go on (votes below)
   if (c >= p.C) return;
   const float w = __ldg(p.w + c), u = __ldg(p.u + c);
   const int n = min(L, p.T - t0);
@@ -403,11 +416,14 @@ __global__ void __launch_bounds__(32)
     for (int q = 3; q >= 0; --q) {
       const int t = gi * 4 + q;
       if (t >= n) continue;
-      const OutStat o = out_stat<true>(st[q], kk[q], vv[q], u, w);
+      const OutStat o = out_stat<true>(st[q], kk[q], vv[q], u, w, vm);
       const float rz = rcp(o.z);
       const float pp = gg[q] * rz, qq = -gg[q] * o.out * rz;
       // the reverse accumulator stands at t+1: Q = -qk - qu u + qc w
-      const float E1 = exp_exact(r.qc, w, kk[q], r.qk, -r.qu * u);                     // e^{k_t + Q}
+      // e^{k_t + Q}, exact where the exponent is large in some lane
+      const float x1 = fmaf(r.qc, w, (kk[q] - r.qk) - r.qu * u);
+      const float E1 = __any_sync(vm, fabsf(x1) > kExactFrom) ? exp_exact(r.qc, w, kk[q], r.qk, -r.qu * u)
+                                                                : ex2(x1 * kLog2e);
       // (dw sums these over all tokens; its largest terms have exponents near
       // zero, so the rounded exponent suffices)
       const float E2 = ex2(fmaf(r.qc - st[q].nf - 1.f, w, (st[q].ma - r.qk) - r.qu * u) * kLog2e);  // e^{m_t + Q - w}
@@ -448,31 +464,47 @@ __global__ void __launch_bounds__(32)
 // (Kahan-Babuska), then a fixed shuffle tree: the order depends on the shape
 // only.
 __global__ void __launch_bounds__(256) wkv_bwd_reduce(const BwdParams p) {
-  const int lane = threadIdx.x & 31;
-  const long long c = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (c >= p.C) return;
-  float su = 0.f, cu = 0.f, sw = 0.f, cw = 0.f;
+  // a thread per channel (32 channels per CTA, coalesced rows of partials),
+  // the 8 warps each summing a contiguous eighth of the nch * B partials;
+  // then warp 0 combines the eighths in order
+  __shared__ float part[4][8][32];
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  const long long c = (long long)blockIdx.x * 32 + lane;
   const long long n = (long long)p.nch * p.B;
-  for (long long i = lane; i < n; i += 32) {
-    const float xu = p.pdu[i * p.C + c], xw = p.pdw[i * p.C + c];
-    float h, e;
-    two_sum(su, xu, h, e);
-    su = h;
-    cu += e;
-    two_sum(sw, xw, h, e);
-    sw = h;
-    cw += e;
+  const long long per = (n + 7) / 8;
+  const long long i0 = wp * per, i1 = min(n, i0 + per);
+  float su = 0.f, cu = 0.f, sw = 0.f, cw = 0.f;
+  if (c < p.C) {
+    for (long long i = i0; i < i1; ++i) {
+      const float xu = p.pdu[i * p.C + c], xw = p.pdw[i * p.C + c];
+      float h, e;
+      two_sum(su, xu, h, e);
+      su = h;
+      cu += e;
+      two_sum(sw, xw, h, e);
+      sw = h;
+      cw += e;
+    }
   }
-  su += cu;
-  sw += cw;
+  part[0][wp][lane] = su;
+  part[1][wp][lane] = cu;
+  part[2][wp][lane] = sw;
+  part[3][wp][lane] = cw;
+  __syncthreads();
+  if (wp == 0 && c < p.C) {
+    float tu = 0.f, ku = 0.f, tw = 0.f, kw = 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    su += __shfl_xor_sync(0xffffffffu, su, o);
-    sw += __shfl_xor_sync(0xffffffffu, sw, o);
-  }
-  if (lane == 0) {
-    p.du[c] = su;
-    p.dw[c] = sw;
+    for (int q = 0; q < 8; ++q) {
+      float h, e;
+      two_sum(tu, part[0][q][lane], h, e);
+      tu = h;
+      ku += e + part[1][q][lane];
+      two_sum(tw, part[2][q][lane], h, e);
+      tw = h;
+      kw += e + part[3][q][lane];
+    }
+    p.du[c] = tu + ku;
+    p.dw[c] = tw + kw;
   }
 }
 
