@@ -882,8 +882,8 @@ wkv_status launch_backward(const BwdPlan& pl, const FwdParams& fp, const BwdPara
   if (items >= (1ll << 31)) return WKV_ERR_INVALID_ARG;
   wkv_bwd_chunk<KV, kBwdL><<<(unsigned)items, 32, tsmem, st>>>(bp, rk, rv, rg);
   if (launch_result() != WKV_OK) return WKV_ERR_CUDA;
-  // RED: du, dw (a thread per channel)
-  wkv_bwd_reduce<<<(unsigned)((fp.C + 31) / 32), 256, 0, st>>>(bp);
+  // RED: du, dw (one warp per channel)
+  wkv_bwd_reduce<<<(unsigned)((fp.C + 7) / 8), 256, 0, st>>>(bp);
   return launch_result();
 }
 

@@ -34,8 +34,7 @@
 //         tokens in reverse from rin, writing dk, dv and per-chunk partial sums
 //         of du, dw; chunk 0 also yields the state gradients;
 //   RED   wkv_bwd_reduce: du, dw as compensated sums of the partials over the
-//         chunks and batch rows (a thread per channel, 8 warps over eighths
-//         of the partials), in a fixed order.
+//         chunks and batch rows (a warp per channel), in a fixed order.
 // One 32-thread CTA per (batch row, chunk, 32 channels) in R1 and R2, the
 // chunk's k, v and g copied into shared memory by TMA. All orders of
 // accumulation depend on the shape only, so results are bitwise reproducible.
@@ -464,47 +463,42 @@ __global__ void __launch_bounds__(32)
 // (Kahan-Babuska), then a fixed shuffle tree: the order depends on the shape
 // only.
 __global__ void __launch_bounds__(256) wkv_bwd_reduce(const BwdParams p) {
-  // a thread per channel (32 channels per CTA, coalesced rows of partials),
-  // the 8 warps each summing a contiguous eighth of the nch * B partials;
-  // then warp 0 combines the eighths in order
-  __shared__ float part[4][8][32];
-  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-  const long long c = (long long)blockIdx.x * 32 + lane;
-  const long long n = (long long)p.nch * p.B;
-  const long long per = (n + 7) / 8;
-  const long long i0 = wp * per, i1 = min(n, i0 + per);
+  // a warp per channel; lane l sums the partials of rows l, l + 32, ...
+  // (four rows in flight per round), then a fixed shuffle tree
+  const int lane = threadIdx.x & 31;
+  const long long c = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (c >= p.C) return;
   float su = 0.f, cu = 0.f, sw = 0.f, cw = 0.f;
-  if (c < p.C) {
-    for (long long i = i0; i < i1; ++i) {
-      const float xu = p.pdu[i * p.C + c], xw = p.pdw[i * p.C + c];
+  const long long n = (long long)p.nch * p.B;
+  for (long long i0 = lane; i0 < n; i0 += 4 * 32) {
+    float xu[4], xw[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const long long i = i0 + r * 32;
+      xu[r] = i < n ? p.pdu[i * p.C + c] : 0.f;
+      xw[r] = i < n ? p.pdw[i * p.C + c] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
       float h, e;
-      two_sum(su, xu, h, e);
+      two_sum(su, xu[r], h, e);
       su = h;
       cu += e;
-      two_sum(sw, xw, h, e);
+      two_sum(sw, xw[r], h, e);
       sw = h;
       cw += e;
     }
   }
-  part[0][wp][lane] = su;
-  part[1][wp][lane] = cu;
-  part[2][wp][lane] = sw;
-  part[3][wp][lane] = cw;
-  __syncthreads();
-  if (wp == 0 && c < p.C) {
-    float tu = 0.f, ku = 0.f, tw = 0.f, kw = 0.f;
+  su += cu;
+  sw += cw;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      float h, e;
-      two_sum(tu, part[0][q][lane], h, e);
-      tu = h;
-      ku += e + part[1][q][lane];
-      two_sum(tw, part[2][q][lane], h, e);
-      tw = h;
-      kw += e + part[3][q][lane];
-    }
-    p.du[c] = tu + ku;
-    p.dw[c] = tw + kw;
+  for (int o = 16; o > 0; o >>= 1) {
+    su += __shfl_xor_sync(0xffffffffu, su, o);
+    sw += __shfl_xor_sync(0xffffffffu, sw, o);
+  }
+  if (lane == 0) {
+    p.du[c] = su;
+    p.dw[c] = sw;
   }
 }
 
