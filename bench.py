@@ -706,6 +706,7 @@ def measure_v6(wl, args, device):
     call_ms = ms / (n_rep * R)
     tflops = flops / (call_ms / 1e3) / 1e12
     peak, peak_kind = measured_peaks()
+    traffic, _ = recorded_traffic("wkv6_fwd", wl.name)
     rec = {
         "workload": f"wkv_v6_forward {wl.kv_dtype} B={wl.B} T={wl.T} H={wl.H} D={wl.D} (matrix-valued state, "
                     "zero state in, state out)",
@@ -713,7 +714,7 @@ def measure_v6(wl, args, device):
         "steps": n_rep * R, "ms_per_step": call_ms,
         "roofline": {"bound": "alu", "kernel": "wkv6_fwd", "achieved": tflops, "peak": V6_FP32_PEAK_TFLOPS,
                      "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz", "unit": "TFLOP/s",
-                     "frac": tflops / V6_FP32_PEAK_TFLOPS, "traffic": None, "algorithmic_flops": flops,
+                     "frac": tflops / V6_FP32_PEAK_TFLOPS, "traffic": traffic, "algorithmic_flops": flops,
                      "hbm_achieved_gbs": hbm / (call_ms / 1e3) / 1e9, "hbm_frac_of_measured": hbm / (call_ms / 1e3) / 1e9 / peak,
                      "launch_ms": call_ms},
         "gpu_launches": n_rep * R, "clocks": clocks, "buffer_sets": R,
@@ -732,6 +733,16 @@ def run_ours(args):
     if world > 1:
         dist_init("nccl")
     options = json.loads(args.options) if args.options else None
+    if args.part:
+        # one sub-record alone (profiling): printed as its own JSON line
+        from wkv_recurrence_b200 import inputs as I
+        if args.part.startswith("backward_"):
+            rec = measure_backward(workload(args, args.part[len("backward_"):]), args, device)
+        else:
+            rec = measure_v6(I.V6_WORKLOADS[args.part], args, device)
+        if rank == 0:
+            print(json.dumps(rec), flush=True)
+        return
     wl = workload(args)
     main = measure_forward(wl, args, options, device, rank, world, headline=True)
 
@@ -749,11 +760,12 @@ def run_ours(args):
         for name in ("layer", "long"):
             subs[f"backward_{name}"] = measure_backward(workload(args, name), args, device)
         subs["v6"] = measure_v6(I.V6_WORKLOADS["v6"], args, device)
+        subs["v6_bf16"] = measure_v6(I.V6_WORKLOADS["v6_bf16"], args, device)
 
     if rank == 0 and world == 1 and not args.no_cpu:
         main["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds, one_core_s=args.cpu_seconds / 2)
         for name, rec in subs.items():
-            if name.startswith("backward_") or name == "v6":
+            if name.startswith("backward_") or name.startswith("v6"):
                 continue
             rec["cpu_baseline"] = cpu_baseline(workload(args, name), budget_s=args.cpu_seconds / 3,
                                                one_core_s=args.cpu_seconds / 4, decode=(name == "decode"))
@@ -761,7 +773,8 @@ def run_ours(args):
             subs[f"backward_{name}"]["cpu_baseline"] = cpu_baseline_backward(workload(args, name),
                                                                              budget_s=args.cpu_seconds / 3)
         from wkv_recurrence_b200 import inputs as I
-        subs["v6"]["cpu_baseline"] = cpu_baseline_v6(I.V6_WORKLOADS["v6"], budget_s=args.cpu_seconds / 3)
+        for name in ("v6", "v6_bf16"):
+            subs[name]["cpu_baseline"] = cpu_baseline_v6(I.V6_WORKLOADS[name], budget_s=args.cpu_seconds / 4)
 
     if rank == 0:
         bf16 = wl.kv_dtype == "bf16"
@@ -934,7 +947,7 @@ def cpu_baseline_v6(wl, budget_s=3.0):
     reps = 0
     t0 = time.perf_counter()
     while True:
-        V.recurrence(r, w, k, v)
+        V.recurrence(r, w, k, v, kv_dtype=wl.kv_dtype)
         reps += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -1000,6 +1013,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="headline workload only (no per-workload sub-records)")
+    ap.add_argument("--part", choices=["backward_layer", "backward_long", "v6", "v6_bf16"], default="",
+                    help="measure this sub-record alone and print it (profiling)")
     ap.add_argument("--no-clocks", action="store_true")
     args = ap.parse_args(argv)
     _, _, world = dist_env()
