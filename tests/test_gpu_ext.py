@@ -122,6 +122,19 @@ def test_cluster_in_place_state_and_determinism(oracle):
     assert torch.equal(a, b) and all(torch.equal(x, y) for x, y in zip(sa, sb))
 
 
+@pytest.mark.parametrize("name", ["layer", "long"])
+def test_cluster_workload_full_size(oracle, name):
+    """The cluster scan on the layer (one segment per channel group) and long
+    (16 chained segments, 1% key spikes of +-U(20, 60)) workloads: every output
+    and the final state against the float64 oracle."""
+    wl = I.WORKLOADS[name]
+    k, v = I.draw_kv(wl)
+    w, u = I.draw_w(wl), I.draw_u(wl)
+    st = I.draw_state(wl)
+    eo, es = compare_ext(oracle, k, v, w, u, st, kv=wl.kv_dtype, out_dtype=wl.out_dtype, options=CLUSTER)
+    print(f"{name} on the cluster scan: max normalised out error {eo:.2e}, state errors {es}")
+
+
 def test_three_launch_is_the_automatic_choice_for_few_channels():
     assert W.forward_kernel(8, 1024, 768) == 3
     assert W.forward_kernel(1, 65536, 2048) == 3
