@@ -122,13 +122,14 @@ def decode_desc(wl):
             f"prefix (wkv_forward), {wl.decode_steps} steps with fresh k, v")
 
 
-def workload(args, name=None):
-    """The named workload, with B and/or T overridden for profiling runs."""
+def workload(args, name=None, override=False):
+    """The named workload (the headline's when name is None), with B and/or T
+    overridden for profiling runs (the headline, or with override)."""
     import dataclasses
 
     from wkv_recurrence_b200 import inputs as I
     wl = I.WORKLOADS[name or args.workload]
-    if name is None and (args.batch or args.tokens):
+    if (name is None or override) and (args.batch or args.tokens):
         wl = dataclasses.replace(wl, B=args.batch or wl.B, T=args.tokens or wl.T)
     return wl
 
@@ -737,7 +738,7 @@ def run_ours(args):
         # one sub-record alone (profiling): printed as its own JSON line
         from wkv_recurrence_b200 import inputs as I
         if args.part.startswith("backward_"):
-            rec = measure_backward(workload(args, args.part[len("backward_"):]), args, device)
+            rec = measure_backward(workload(args, args.part[len("backward_"):], override=True), args, device)
         else:
             rec = measure_v6(I.V6_WORKLOADS[args.part], args, device)
         if rank == 0:
