@@ -205,6 +205,38 @@ WKV_API wkv_status wkv_forward(int64_t B, int64_t T, int64_t C,
                        void *stream, const wkv_options *opts);
 
 /*
+ * Sequence forward over HOST-resident k, v and out ([B, T, C] in host
+ * memory; page-locked for the copies to overlap), for inputs that live on the
+ * host: the sequence is cut into segments of seg_tokens tokens (0 = choose:
+ * about 64 MB of k and v per segment). Segment s is copied to the device on a
+ * stream of the library's own, computed by wkv_forward on `stream` from the
+ * state after segment s-1, and its outputs copied back on a second library
+ * stream; two segments are in flight, so the copies in, the compute and the
+ * copies back of neighbouring segments run side by side.
+ *   w, u, state_in, state_out  device arrays, as for wkv_forward
+ *   dev_buffer  device buffer of at least wkv_forward_host_buffer_size()
+ *               bytes, 256-byte aligned and zero-filled before its first use
+ *               (two segments of k, v and out, the carried state, and the
+ *               forward's workspace); owned by the caller
+ * Returns once the work is queued; it has all completed when `stream` has
+ * (the library's streams fork from `stream` at the call and join it before
+ * its end, also under stream capture once a first call on the device has
+ * created them outside of capture). The result equals wkv_forward's with the
+ * sequence split at the segment boundaries (the state handed from segment to
+ * segment as wkv_forward's state out). Errors as wkv_forward's, and
+ * WKV_ERR_WORKSPACE_TOO_SMALL for a dev_buffer below the size.
+ */
+WKV_API size_t wkv_forward_host_buffer_size(int64_t B, int64_t T, int64_t C, wkv_dtype kv_dtype,
+                                            wkv_dtype out_dtype, int64_t seg_tokens);
+WKV_API wkv_status wkv_forward_host(int64_t B, int64_t T, int64_t C,
+                            const void *k_host, const void *v_host, wkv_dtype kv_dtype,
+                            const float *w, const float *u,
+                            void *out_host, wkv_dtype out_dtype,
+                            const wkv_cstate *state_in, const wkv_state *state_out,
+                            void *dev_buffer, size_t dev_bytes, int64_t seg_tokens,
+                            void *stream);
+
+/*
  * Two optional inputs of the RWKV-v6 time-mixing block ("RWKV-v6
  * Architecture: Attention-Free Linear Transformers"), for wkv_forward_ext and
  * wkv_step_ext:

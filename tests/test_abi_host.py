@@ -76,6 +76,26 @@ def test_status_strings(L):
     assert L.wkv_last_cuda_error().decode().startswith("cuda")
 
 
+def test_forward_host_sizes_and_argument_checks(L):
+    F32, BF16 = _abi.WKV_F32, _abi.WKV_BF16
+    # two segments of k, v and out, the carried state, the forward's workspace
+    a = L.wkv_forward_host_buffer_size(1, 65536, 2048, F32, F32, 4096)
+    assert a >= 2 * 3 * 4096 * 2048 * 4 + 3 * 2048 * 4 + L.wkv_forward_workspace_size(1, 4096, 2048, None)
+    assert L.wkv_forward_host_buffer_size(1, 65536, 2048, F32, F32, 0) == a  # default: 64 MB of k and v
+    assert L.wkv_forward_host_buffer_size(1, 65536, 2048, BF16, BF16, 4096) < a
+    assert L.wkv_forward_host_buffer_size(1, 100, 64, 7, F32, 0) == 0
+    assert L.wkv_forward_host_buffer_size(-1, 100, 64, F32, F32, 0) == 0
+    # argument errors come back before anything is queued (no device needed)
+    assert L.wkv_forward_host(1, 10, 64, None, None, F32, None, None, None, F32, None, None, None, 0, 0,
+                              None) == _abi.WKV_ERR_INVALID_ARG
+    assert L.wkv_forward_host(1, 10, 64, None, None, 9, None, None, None, F32, None, None, None, 0, 0,
+                              None) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert L.wkv_forward_host(1, 10, 64, None, None, F32, None, None, None, BF16, None, None, None, 0, 0,
+                              None) == _abi.WKV_ERR_UNSUPPORTED_DTYPE
+    assert L.wkv_forward_host(1, 10, 64, None, None, F32, None, None, None, F32, None, None, None, 0, -5,
+                              None) == _abi.WKV_ERR_INVALID_ARG
+
+
 def test_workspace_size(L):
     # sequential kernel: the 256-byte header only
     assert L.wkv_forward_workspace_size(16, 4096, 4096, None) == 256

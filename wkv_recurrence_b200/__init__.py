@@ -7,6 +7,7 @@ without writing a CUDA kernel", section "The recurrence", carried as a
 binding:
 
     out, state = wkv_recurrence_b200.forward(k, v, w, u, state=None)
+    out, state = wkv_recurrence_b200.forward_host(k_host, v_host, w, u)  # k, v in host memory
     out, state = wkv_recurrence_b200.step(state, k, v, w, u)
 
 Importing the package does not load the library; the first call does, and
@@ -14,8 +15,9 @@ fails loudly if it is missing or no CUDA device is present.
 """
 
 from .api import (WKV, PreparedForward, PreparedStep, WkvError, backward, empty_state, forward,  # noqa: F401
-                  forward_kernel, forward_launches, make_workspace, query_status, step, v6_forward,
-                  workspace_size)
+                  forward_host, forward_host_buffer_size, forward_kernel, forward_launches, make_workspace,
+                  query_status, step, v6_forward, workspace_size)
 
-__all__ = ["forward", "step", "backward", "WKV", "v6_forward", "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
+__all__ = ["forward", "forward_host", "forward_host_buffer_size", "step", "backward", "WKV", "v6_forward",
+           "workspace_size", "forward_kernel", "forward_launches", "make_workspace", "query_status", "empty_state",
            "PreparedForward", "PreparedStep", "WkvError"]

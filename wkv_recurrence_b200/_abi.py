@@ -29,7 +29,7 @@ WKV_BF16 = 1
 EXPORTS = ("wkv_forward_workspace_size", "wkv_forward_kernel", "wkv_forward_launches", "wkv_forward",
            "wkv_forward_ext", "wkv_step", "wkv_step_ext", "wkv_query_status", "wkv_status_string", "wkv_version",
            "wkv_forward_noalloc", "wkv_last_cuda_error", "wkv_backward_workspace_size", "wkv_backward",
-           "wkv_v6_forward")
+           "wkv_v6_forward", "wkv_forward_host_buffer_size", "wkv_forward_host")
 
 # size of the library's built-in scratch array used by wkv_forward_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -101,6 +101,11 @@ def lib() -> ctypes.CDLL:
         L.wkv_forward_noalloc.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
                                           ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P]
         L.wkv_forward_noalloc.restype = I
+        L.wkv_forward_host_buffer_size.argtypes = [I64, I64, I64, I, I, I64]
+        L.wkv_forward_host_buffer_size.restype = SZ
+        L.wkv_forward_host.argtypes = [I64, I64, I64, P, P, I, P, P, P, I,
+                                       ctypes.POINTER(wkv_cstate), ctypes.POINTER(wkv_state), P, SZ, I64, P]
+        L.wkv_forward_host.restype = I
         L.wkv_backward_workspace_size.argtypes = [I64, I64, I64]
         L.wkv_backward_workspace_size.restype = SZ
         L.wkv_backward.argtypes = [I64, I64, I64, P, P, I, P, P, ctypes.POINTER(wkv_cstate), P,

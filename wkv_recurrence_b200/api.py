@@ -178,6 +178,79 @@ def forward(k: torch.Tensor, v: torch.Tensor, w: Optional[torch.Tensor], u: torc
     return out, state_out
 
 
+_host_buffers = {}
+
+
+def forward_host(k: torch.Tensor, v: torch.Tensor, w: torch.Tensor, u: torch.Tensor,
+                 state: Optional[State] = None, *, out_dtype: Optional[torch.dtype] = None,
+                 out: Optional[torch.Tensor] = None, state_out: Optional[State] = None,
+                 return_state: bool = True, seg_tokens: int = 0, buffer: Optional[torch.Tensor] = None):
+    """WKV over a sequence whose k, v (and out) live in host memory: k, v, out
+    are CPU tensors [B, T, C] (page-locked, e.g. ``.pin_memory()``, for the
+    copies to overlap the compute); w, u and the states are CUDA tensors as for
+    ``forward``. The library streams segments of seg_tokens tokens (0 =
+    choose) through the device, copies in, compute and copies back of
+    neighbouring segments side by side. Returns (out, state) like ``forward``;
+    the work is queued on the current stream (synchronise before reading out).
+    """
+    for t, name in ((k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if v.dtype != k.dtype or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, T, C] of one dtype")
+    _need_cuda(w, "w", torch.float32)
+    _need_cuda(u, "u", torch.float32)
+    B, T, C = k.shape
+    if w.shape != (C,) or u.shape != (C,):
+        raise ValueError("w and u must be [C]")
+    dev = w.device
+    out_dtype = out_dtype or k.dtype
+    if out is None:
+        out = torch.empty((B, T, C), dtype=out_dtype, pin_memory=True)
+    if out.is_cuda or not out.is_contiguous() or out.shape != (B, T, C) or out.dtype != out_dtype:
+        raise ValueError("out must be a contiguous CPU tensor [B, T, C] of out_dtype")
+    sin = None
+    if state is not None:
+        for i, x in enumerate(state):
+            _need_cuda(x, f"state[{i}]", torch.float32)
+            if x.shape != (B, C):
+                raise ValueError("state arrays must be [B, C]")
+        sin = _abi.wkv_cstate(*(x.data_ptr() for x in state))
+    sout = None
+    if return_state or state_out is not None:
+        if state_out is None:
+            state_out = tuple(torch.empty((B, C), dtype=torch.float32, device=dev) for _ in range(3))
+        for i, x in enumerate(state_out):
+            _need_cuda(x, f"state_out[{i}]", torch.float32)
+        sout = _abi.wkv_state(*(x.data_ptr() for x in state_out))
+    L = _abi.lib()
+    kvc, oc = _dtype_code(k, "k"), _dtype_code(out, "out")
+    need = L.wkv_forward_host_buffer_size(B, T, C, kvc, oc, int(seg_tokens))
+    if need == 0:
+        raise ValueError("invalid sizes")
+    if buffer is None:
+        key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
+        buffer = _host_buffers.get(key)
+        if buffer is None or buffer.numel() < need:
+            buffer = torch.zeros(need, dtype=torch.uint8, device=dev)
+            _host_buffers[key] = buffer
+    _need_cuda(buffer, "buffer")
+    code = L.wkv_forward_host(B, T, C, _ptr(k), _ptr(v), kvc, _ptr(w), _ptr(u), _ptr(out), oc,
+                              ctypes.byref(sin) if sin is not None else None,
+                              ctypes.byref(sout) if sout is not None else None,
+                              _ptr(buffer), buffer.numel(), int(seg_tokens), _stream())
+    _abi.check(code, "wkv_forward_host")
+    return out, state_out
+
+
+def forward_host_buffer_size(B: int, T: int, C: int, kv_dtype: torch.dtype = torch.float32,
+                             out_dtype: Optional[torch.dtype] = None, seg_tokens: int = 0) -> int:
+    """Bytes of the device buffer ``forward_host`` needs (host-only)."""
+    out_dtype = out_dtype or kv_dtype
+    return int(_abi.lib().wkv_forward_host_buffer_size(int(B), int(T), int(C), _DT[kv_dtype], _DT[out_dtype],
+                                                       int(seg_tokens)))
+
+
 def step(state: State, k: torch.Tensor, v: torch.Tensor, w: Optional[torch.Tensor], u: torch.Tensor, *,
          out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
          state_out: Optional[State] = None, inplace: bool = False,

@@ -21,6 +21,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC_DIR = os.path.join(HERE, "csrc")
 MAIN = os.path.join(SRC_DIR, "wkv_api.cu")
+HOST = os.path.join(SRC_DIR, "wkv_host.cpp")  # host-side streaming of host-resident sequences
 LIB = os.path.join(HERE, "_build", "libwkv.so")
 LIB_DEBUG = os.path.join(HERE, "_build", "libwkv_debug.so")
 HEADER = os.path.join(ROOT, "include", "wkv.h")
@@ -35,7 +36,7 @@ NVCC_FLAGS = [
 
 def _sources():
     return sorted(glob.glob(os.path.join(SRC_DIR, "*.cu")) + glob.glob(os.path.join(SRC_DIR, "*.cuh"))
-                  + [HEADER])
+                  + glob.glob(os.path.join(SRC_DIR, "*.cpp")) + [HEADER])
 
 
 def nvcc() -> str:
@@ -52,7 +53,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: boo
         return out
     os.makedirs(os.path.dirname(out), exist_ok=True)
     tmp = out + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-DWKV_DEBUG"] if debug else []), *extra_flags, "-o", tmp, MAIN]
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DWKV_DEBUG"] if debug else []), *extra_flags, "-o", tmp, MAIN, HOST]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
