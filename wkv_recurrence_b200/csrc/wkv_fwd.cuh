@@ -160,9 +160,10 @@ __device__ __forceinline__ void coop_load_tile(KV* dst, const KV* src, int b, in
 // R = p.replay_chunks consecutive chunks (R * p.chunk_len tokens) of one batch
 // row and starts from the incoming state of the first, which the scan pass
 // wrote to p.x0 ([nch][B * NG][64] with p.NG 64-channel groups); the grid is
-// B * ceil(nch / R) * ceil(C / CG). It issues its first copies (inputs only)
-// before waiting (griddepcontrol.wait) for the scan, and only the CTA that
-// ends the sequence writes the state out.
+// B * ceil(nch / R) * ceil(C / CG), replays taken from the sequence's end
+// (the chunks the totals pass read last are the ones still in L2). It issues
+// its first copies (inputs only) before waiting (griddepcontrol.wait) for the
+// scan, and only the CTA that ends the sequence writes the state out.
 template <typename KV, typename OUT, int VEC, int THREADS, int LT, int STAGES, bool kTMA, bool kChunked,
           bool kWT>
 __global__ void __launch_bounds__(THREADS)
@@ -185,8 +186,10 @@ __global__ void __launch_bounds__(THREADS)
   const int bj = blockIdx.x / ngs;
   const int g = blockIdx.x % ngs;
   const int nseq = kChunked ? (p.nch + p.replay_chunks - 1) / p.replay_chunks : 1;  // replays per row
-  const int b = kChunked ? bj / nseq : bj;
-  const int js = kChunked ? bj % nseq : 0;  // replay
+  // replays in reverse chunk order, batch rows inner: the totals pass read
+  // the chunks in order, so the last ones it read are the ones still in L2
+  const int b = kChunked ? bj % p.B : bj;
+  const int js = kChunked ? nseq - 1 - bj / p.B : 0;  // replay
   const int jc = js * (kChunked ? p.replay_chunks : 1);  // its first chunk
   const int tbeg = kChunked ? jc * p.chunk_len : 0;
   const int tend = kChunked ? min(T, tbeg + p.replay_chunks * p.chunk_len) : T;
