@@ -29,18 +29,19 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct HostPipe {
   std::mutex mu;
   bool ready = false;
-  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaStream_t s_in = nullptr, s_in2 = nullptr, s_out = nullptr;  // k in, v in, out back
   cudaEvent_t fork = nullptr;
-  cudaEvent_t loaded[2] = {}, computed[2] = {}, unloaded[2] = {};
+  cudaEvent_t loaded[2] = {}, loaded2[2] = {}, computed[2] = {}, unloaded[2] = {};
 };
 HostPipe g_pipe[kMaxDevices];
 
 bool pipe_ready(HostPipe& p) {
   if (p.ready) return true;
   if (cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaStreamCreateWithFlags(&p.s_in2, cudaStreamNonBlocking) != cudaSuccess) return false;
   if (cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking) != cudaSuccess) return false;
-  cudaEvent_t* evs[7] = {&p.fork, &p.loaded[0], &p.loaded[1], &p.computed[0], &p.computed[1], &p.unloaded[0],
-                         &p.unloaded[1]};
+  cudaEvent_t* evs[9] = {&p.fork,        &p.loaded[0],   &p.loaded[1],   &p.loaded2[0], &p.loaded2[1],
+                         &p.computed[0], &p.computed[1], &p.unloaded[0], &p.unloaded[1]};
   for (cudaEvent_t* e : evs)
     if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
   p.ready = true;
@@ -138,7 +139,7 @@ wkv_status wkv_forward_host(int64_t B, int64_t T, int64_t C, const void* k_host,
 
   // the copies follow everything queued on the caller's stream before the call
   if (!ok(cudaEventRecord(P.fork, st)) || !ok(cudaStreamWaitEvent(P.s_in, P.fork, 0)) ||
-      !ok(cudaStreamWaitEvent(P.s_out, P.fork, 0)))
+      !ok(cudaStreamWaitEvent(P.s_in2, P.fork, 0)) || !ok(cudaStreamWaitEvent(P.s_out, P.fork, 0)))
     return WKV_ERR_CUDA;
   for (int64_t s = 0; s < nseg; ++s) {
     const int slot = (int)(s & 1);
@@ -147,17 +148,22 @@ wkv_status wkv_forward_host(int64_t B, int64_t T, int64_t C, const void* k_host,
     void* vd = db + L.v[slot];
     void* od = db + L.o[slot];
     // host -> device: rows of len*C elements at pitch T*C (one 2-D copy per
-    // tensor); the slot's buffers are free once the compute of segment s-2 ended
-    if (s >= 2 && !ok(cudaStreamWaitEvent(P.s_in, P.computed[slot], 0))) return WKV_ERR_CUDA;
+    // tensor, k and v on two streams: two copy engines share the link, which
+    // is the limit either way: 21.6 against 21.7 ms per long-workload step);
+    // the slot's buffers are free once the compute of segment s-2 ended
+    if (s >= 2 && (!ok(cudaStreamWaitEvent(P.s_in, P.computed[slot], 0)) ||
+                   !ok(cudaStreamWaitEvent(P.s_in2, P.computed[slot], 0))))
+      return WKV_ERR_CUDA;
     const size_t wb = (size_t)(len * C) * kes, hp = (size_t)(T * C) * kes;
     if (!ok(cudaMemcpy2DAsync(kd, wb, static_cast<const unsigned char*>(k_host) + (size_t)(t0 * C) * kes, hp, wb,
                               (size_t)B, cudaMemcpyHostToDevice, P.s_in)) ||
         !ok(cudaMemcpy2DAsync(vd, wb, static_cast<const unsigned char*>(v_host) + (size_t)(t0 * C) * kes, hp, wb,
-                              (size_t)B, cudaMemcpyHostToDevice, P.s_in)) ||
-        !ok(cudaEventRecord(P.loaded[slot], P.s_in)))
+                              (size_t)B, cudaMemcpyHostToDevice, P.s_in2)) ||
+        !ok(cudaEventRecord(P.loaded[slot], P.s_in)) || !ok(cudaEventRecord(P.loaded2[slot], P.s_in2)))
       return WKV_ERR_CUDA;
     // compute on the caller's stream, from the state after segment s-1
-    if (!ok(cudaStreamWaitEvent(st, P.loaded[slot], 0))) return WKV_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(st, P.loaded[slot], 0)) || !ok(cudaStreamWaitEvent(st, P.loaded2[slot], 0)))
+      return WKV_ERR_CUDA;
     if (s >= 2 && !ok(cudaStreamWaitEvent(st, P.unloaded[slot], 0))) return WKV_ERR_CUDA;
     const wkv_cstate* sin = s == 0 ? state_in : &carry_in;
     const wkv_state* sout = s == nseg - 1 ? state_out : &carry_out;
