@@ -208,11 +208,11 @@ WKV_API wkv_status wkv_forward(int64_t B, int64_t T, int64_t C,
  * Sequence forward over HOST-resident k, v and out ([B, T, C] in host
  * memory; page-locked for the copies to overlap), for inputs that live on the
  * host: the sequence is cut into segments of seg_tokens tokens (0 = choose:
- * about 64 MB of k and v per segment). Segment s is copied to the device on a
- * stream of the library's own, computed by wkv_forward on `stream` from the
- * state after segment s-1, and its outputs copied back on a second library
- * stream; two segments are in flight, so the copies in, the compute and the
- * copies back of neighbouring segments run side by side.
+ * about 64 MB of k and v per segment). Segment s is copied to the device on
+ * streams of the library's own (k and v on one each), computed by wkv_forward
+ * on `stream` from the state after segment s-1, and its outputs copied back
+ * on a third library stream; two segments are in flight, so the copies in,
+ * the compute and the copies back of neighbouring segments run side by side.
  *   w, u, state_in, state_out  device arrays, as for wkv_forward
  *   dev_buffer  device buffer of at least wkv_forward_host_buffer_size()
  *               bytes, 256-byte aligned and zero-filled before its first use
