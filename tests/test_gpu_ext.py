@@ -135,6 +135,44 @@ def test_cluster_workload_full_size(oracle, name):
     print(f"{name} on the cluster scan: max normalised out error {eo:.2e}, state errors {es}")
 
 
+def test_cluster_mixed_full_size(oracle):
+    """The cluster scan on the mixed workload (16 x 4096 x 4096, bf16 k, v and
+    out, a state in): every output and the final state against the oracle."""
+    wl = I.WORKLOADS["mixed"]
+    k, v = I.draw_kv(wl)
+    w, u = I.draw_w(wl), I.draw_u(wl)
+    st = I.draw_state(wl)
+    eo, es = compare_ext(oracle, k, v, w, u, st, kv=wl.kv_dtype, out_dtype=wl.out_dtype, options=CLUSTER)
+    print(f"mixed on the cluster scan: max normalised out error {eo:.2e}, state errors {es}")
+
+
+def test_concurrent_calls_on_two_streams(oracle):
+    """Calls with their own workspaces on two streams at once (the three-launch
+    and the cluster scans, whose workspaces carry counters and flags): each
+    result equals the oracle's."""
+    cases = []
+    for i, opts in enumerate((TWO, CLUSTER)):
+        k, v, w, u, st = I.random_case(2, 3000 + 500 * i, 128, seed=90 + i, k_spike=30.0, state=True)
+        cases.append((k, v, w, u, st, opts))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    dev_in = [(dev_f32(k), dev_f32(v), dev_f32(w), dev_f32(u), tuple(dev_f32(x) for x in st), o)
+              for k, v, w, u, st, o in cases]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        outs = []
+        for s, (K, V, Wt, U, S, o) in zip(streams, dev_in):
+            with torch.cuda.stream(s):
+                ws = W.make_workspace(*K.shape, options=o)
+                outs.append(W.forward(K, V, Wt, U, S, workspace=ws, options=o))
+        torch.cuda.synchronize()
+    for (k, v, w, u, st, _), (out, so) in zip(cases, outs):
+        ref, rst = oracle.recurrence_forward(k, v, w, u, st)
+        sc, sst = oracle.abs_scale_forward(k, v, w, u, st)
+        assert_out(host(out), ref, sc, RTOL_F32)
+        assert_state(tuple(host(x) for x in so), rst, sst[0], RTOL_F32)
+
+
 def test_three_launch_is_the_automatic_choice_for_few_channels():
     assert W.forward_kernel(8, 1024, 768) == 3
     assert W.forward_kernel(1, 65536, 2048) == 3
