@@ -83,8 +83,10 @@ typedef struct {
 /*
  * Dispatch and test controls for wkv_forward. Pass NULL for the defaults; a
  * zero-filled struct also means "defaults".
- *   kernel          0 = choose by shape (sequential for many channels or short
- *                   sequences, otherwise the cluster scan),
+ *   kernel          0 = choose by shape: sequential for many channels
+ *                   (B*C >= 65536) or short sequences (T <= 64); otherwise the
+ *                   cluster scan above 2^24 elements of k (B*T*C; k and v
+ *                   larger than L2), else the three-launch scan,
  *                   1 = sequential-over-T kernel,
  *                   2 = chunked scan in one launch (look-back between CTAs),
  *                   3 = chunked scan in three launches (chunk totals, their
@@ -94,7 +96,7 @@ typedef struct {
  *                   pipeline their tiles (look-back of one tile overlapped
  *                   with the next tile's fold and later tiles' copies),
  *                   5 = chunked scan in thread-block clusters: a cluster of
- *                   up to 8 CTAs takes a segment of 8 x cta_warps x span
+ *                   up to 2 CTAs takes a segment of 2 x cta_warps x span
  *                   tokens of one (batch row, 32 channels); each warp streams
  *                   its span through its own TMA ring twice (fold, then
  *                   replay), the CTAs exchange their totals through

@@ -108,7 +108,8 @@ def test_workspace_size(L):
     # group, and room for the single-launch scan that misaligned inputs take
     o5, o3, o2 = (_abi.wkv_options(kernel=k) for k in (5, 3, 2))
     for T in (2048, 4096, 4097, 16384):
-        assert L.wkv_forward_workspace_size(8, T, 768, None) == L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o3))
+        auto = o3 if 8 * T * 768 <= 1 << 24 else o5  # the automatic choice
+        assert L.wkv_forward_workspace_size(8, T, 768, None) == L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(auto))
         for o in (o5, o3):
             assert L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o)) >= \
                 L.wkv_forward_workspace_size(8, T, 768, ctypes.byref(o2))
@@ -127,7 +128,12 @@ def test_forward_kernel_choice(L):
     assert L.wkv_forward_kernel(8, 64, 64, F32, None) == 1
     assert L.wkv_forward_kernel(8, 1024, 768, F32, None) == 3
     assert L.wkv_forward_kernel(8, 2049, 768, F32, None) == 3
-    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 3
+    # few channels and k, v larger than L2 (more than 2^24 elements each): the
+    # cluster scan
+    assert L.wkv_forward_kernel(1, 8192, 2048, F32, None) == 3
+    assert L.wkv_forward_kernel(1, 8193, 2048, F32, None) == 5
+    assert L.wkv_forward_kernel(8, 2049, 1024, BF16, None) == 5
+    assert L.wkv_forward_kernel(1, 65536, 2048, F32, None) == 5
     assert L.wkv_forward_kernel(1, 65536, 2049, F32, None) == 2  # rows TMA cannot address
     # an explicit choice stands, except that the TMA scans fall back to the
     # single-launch scan when a row pitch is not a multiple of 16 bytes
@@ -139,7 +145,8 @@ def test_forward_kernel_choice(L):
         o = _abi.wkv_options(kernel=5, **bad)
         assert L.wkv_forward_kernel(2, 100, 64, F32, ctypes.byref(o)) == 0
     assert L.wkv_forward_launches(8, 1024, 768, F32, ctypes.byref(_abi.wkv_options(kernel=5))) == 1
-    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 3
+    assert L.wkv_forward_launches(1, 65536, 2048, F32, None) == 1
+    assert L.wkv_forward_launches(1, 8192, 2048, F32, None) == 3
     assert L.wkv_forward_launches(2, 20, 64, F32, ctypes.byref(_abi.wkv_options(kernel=3))) == 2
     assert L.wkv_forward_launches(16, 4096, 4096, BF16, None) == 1
     assert L.wkv_forward_kernel(-1, 4, 4, F32, None) == 0

@@ -78,7 +78,7 @@ CLUSTER_IDS = ["w8j64", "w4j64", "w8j32", "w4j32"]
                                    (2, 2100, 64), (1, 9000, 40), (3, 4500, 200)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_cluster_random_f32(oracle, opts, shape):
-    """One segment (T up to 8 CTAs' worth) and several (the look-back between
+    """One segment (T up to 2 CTAs' worth) and several (the look-back between
     segments), ragged spans, ragged channel groups."""
     B, T, C = shape
     k, v, w, u, st = I.random_case(B, T, C, seed=B * 7 + T + C, k_scale=2.0, k_spike=30.0,
@@ -87,9 +87,10 @@ def test_cluster_random_f32(oracle, opts, shape):
 
 
 def test_cluster_segment_boundaries(oracle):
-    """T at, just below and just above multiples of a segment (8 CTAs x 8
-    spans x 64 tokens = 4096 tokens for the default shape)."""
-    for T in (4095, 4096, 4097, 8192, 8193, 12287):
+    """T at, just below and just above multiples of a segment (2 CTAs x 8
+    spans x 64 tokens = 1024 tokens for the default shape) and of a ring
+    stage (16 tokens)."""
+    for T in (1023, 1024, 1025, 2047, 2048, 2049, 4095, 4096, 4097, 8192, 8193, 12287, 1040, 1041, 1055):
         k, v, w, u, st = I.random_case(2, T, 64, seed=T, k_spike=40.0, w_range=(1e-4, 4.0), state=True)
         compare_ext(oracle, k, v, w, u, st, options=CLUSTER)
 
@@ -125,7 +126,7 @@ def test_cluster_in_place_state_and_determinism(oracle):
 @pytest.mark.parametrize("name", ["layer", "long"])
 def test_cluster_workload_full_size(oracle, name):
     """The cluster scan on the layer (one segment per channel group) and long
-    (16 chained segments, 1% key spikes of +-U(20, 60)) workloads: every output
+    (64 chained segments, 1% key spikes of +-U(20, 60)) workloads: every output
     and the final state against the float64 oracle."""
     wl = I.WORKLOADS[name]
     k, v = I.draw_kv(wl)
@@ -173,9 +174,14 @@ def test_concurrent_calls_on_two_streams(oracle):
         assert_state(tuple(host(x) for x in so), rst, sst[0], RTOL_F32)
 
 
-def test_three_launch_is_the_automatic_choice_for_few_channels():
+def test_automatic_choice_for_few_channels():
+    """Few channels: the three-launch scan while k and v fit in L2, the
+    cluster scan beyond (more than 2^24 elements of k)."""
     assert W.forward_kernel(8, 1024, 768) == 3
-    assert W.forward_kernel(1, 65536, 2048) == 3
+    assert W.forward_kernel(1, 8192, 2048) == 3
+    assert W.forward_kernel(1, 8193, 2048) == 5
+    assert W.forward_kernel(1, 65536, 2048) == 5
+    assert W.forward_kernel(1, 65536, 2048, torch.bfloat16) == 5
     assert W.forward_kernel(16, 4096, 4096, torch.bfloat16) == 1
 
 

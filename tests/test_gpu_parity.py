@@ -339,7 +339,7 @@ def test_bounded_wait_reports_timeout_and_recovers(oracle, kernel):
     k, v, w, u, _ = I.random_case(B, T, C, seed=41)
     opts = {"kernel": kernel, "chunk_len": 64, "lookback_group": 4, "wait_timeout_ns": 20_000_000,
             "inject_enable": 1, "inject_unpublished_tile": 9}
-    if kernel == 5:  # segments of 8 CTAs x 4 spans x 32 tokens = 1024 tokens; tickets 0-7 are segment 0
+    if kernel == 5:  # segments of 2 CTAs x 4 spans x 32 tokens = 256 tokens; tickets 0-7 are segment 0
         opts = {"kernel": 5, "cta_warps": 4, "span": 32, "wait_timeout_ns": 20_000_000, "inject_enable": 1,
                 "inject_unpublished_tile": 3}
     ws = W.make_workspace(B, T, C, options=opts)

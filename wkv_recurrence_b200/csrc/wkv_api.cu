@@ -41,6 +41,14 @@ constexpr int kChunkRW = 32, kChunkVec = 2, kChunkCG = kChunkRW * kChunkVec;
 // the automatic choice gives the sequential kernel one channel per thread below
 // this many channels (148 SMs x 16 warps x 64 channels)
 constexpr long long kSeqVec1MaxLanes = 148ll * 16 * 64;
+// Above this many elements of k (and as many of v: 128 MiB of both in fp32,
+// about the size of L2) the automatic choice for few channels is the cluster
+// scan, which reads k and v from HBM once, instead of the three-launch scan,
+// whose second read of k and v hits L2 only while they fit there (layer,
+// 8 x 1024 x 768: 23.5 us three-launch against 25.0 cluster; long,
+// 1 x 65536 x 2048: 426 against 364 us; the same at T = 16384: 114 against
+// 104 us).
+constexpr long long kClusterMinElems = 1ll << 24;
 
 struct Plan {
   int kernel;  // 1 seq, 2 chunked single launch, 3 chunked in three launches, 4 pipelined chunked, 5 cluster
@@ -95,8 +103,8 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   const int want = o ? o->kernel : 0;
   if (want < 0 || want > 5) return false;
   const int64_t lanes = B * C;
-  // the cluster scan's CTA shape: cw spans of cj tokens per CTA, up to 8 CTAs
-  // per cluster and segment
+  // the cluster scan's CTA shape: cw spans of cj tokens per CTA, up to
+  // kClusterMaxCTAs CTAs per cluster and segment
   if (o && o->cta_warps != 0 && o->cta_warps != 4 && o->cta_warps != 8) return false;
   const int cw = (o && o->cta_warps) ? o->cta_warps : 8;
   const int cj = (want == 5 && o && o->span) ? o->span : 64;
@@ -105,11 +113,10 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   if (kernel == 0) {
     if (lanes >= 65536 || T <= 64) {
       kernel = 1;
+    } else if (lanes * T > kClusterMinElems) {
+      kernel = 5;  // k and v larger than L2: read them once
     } else {
-      // the three-launch scan (measured faster than the single-launch scans
-      // on every workload: layer 23.4 us against 29.8 for the cluster scan;
-      // long 436 against 438-490)
-      kernel = 3;
+      kernel = 3;  // the three-launch scan (its second read of k and v hits L2)
     }
   }
   // per-token decays: the sequential, three-launch and cluster kernels only
@@ -121,7 +128,7 @@ bool make_plan(int64_t B, int64_t T, int64_t C, const wkv_options* o, Plan* pl, 
   pl->cj = cj;
   {
     const int64_t tpc = (int64_t)cw * cj;
-    pl->ncl = (int)std::min<int64_t>(8, std::max<int64_t>(1, (T + tpc - 1) / tpc));
+    pl->ncl = (int)std::min<int64_t>(kClusterMaxCTAs, std::max<int64_t>(1, (T + tpc - 1) / tpc));
     const int64_t seg_tokens = pl->ncl * tpc;
     pl->nseg = (int)std::max<int64_t>(1, (T + seg_tokens - 1) / seg_tokens);
   }

@@ -1,7 +1,7 @@
 // The chunked scan over T in thread-block clusters, reading k and v from HBM
 // once.
 //
-// A cluster of ncl CTAs (at most 8) takes one SEGMENT of ncl * NW * J tokens
+// A cluster of ncl CTAs (at most kClusterMaxCTAs) takes one SEGMENT of ncl * NW * J tokens
 // of one (batch row, 32-channel group); CTA `rank` holds tokens
 // [rank*TPC, (rank+1)*TPC) of the segment (TPC = NW*J), one span of J tokens
 // per warp, one channel per lane. Each warp streams its span through a ring of
@@ -49,8 +49,16 @@
 
 namespace wkv {
 
-constexpr int kClusterLB = 8;  // tokens per ring stage
-constexpr int kClusterNS = 4;  // ring stages per warp
+// Ring and cluster shape, measured on the long workload (1 x 65536 x 2048
+// fp32, 8-warp CTAs, 64-token spans). Clusters of up to 8 CTAs: rings of 4
+// stages of 8 tokens 488 us, 2 stages of 16 tokens 418 us (the same shared
+// memory in half as many copies), 4 stages of 16 tokens 725 us (twice the
+// shared memory, half the CTAs per SM). With 2 stages of 16 tokens, clusters
+// of up to 8, 4, 2 and 1 CTAs: 418, 392, 364 and 461 us (1: twice the
+// segments per channel group); up to 2 CTAs with 1 stage of 32 tokens: 372 us.
+constexpr int kClusterLB = 16;     // tokens per ring stage
+constexpr int kClusterNS = 2;      // ring stages per warp
+constexpr int kClusterMaxCTAs = 2; // CTAs per cluster (and segment), at most
 
 template <typename KV, bool kWT>
 __host__ __device__ constexpr uint32_t cluster_stage_bytes() {
