@@ -38,7 +38,10 @@
 // cluster barrier when there is one segment) runs after those reads, so the
 // two may alias. A second cluster barrier (arrive after the last remote read,
 // wait before exit) keeps every CTA's shared memory alive while others may
-// read it. All threads of every CTA take every barrier; no thread returns
+// read it. Only the threads whose accesses must be ordered before another
+// CTA's (the writes of the ticket and of a CTA's total, the first segment's
+// read of the state in) arrive with release semantics, the rest relaxed. All
+// threads of every CTA take every barrier; no thread returns
 // early, and a warp whose copy wait runs out stops consuming, reports
 // kStatusWaitTimeout, and before the end waits (bounded) for the copies it
 // still has in flight.
@@ -73,6 +76,7 @@ __host__ __device__ constexpr size_t cluster_smem_bytes() {
          + (size_t)NW * 32 * (16 + (kWT ? 4 : 0))                  // span aggregates (and decay sums)
          + 32 * (16 + 4)                                           // the CTA's total and decay sum
          + 32 * (16 + 4)                                           // the segment's incoming state
+         + 32 * 16                                                 // the totals of the CTAs before
          + 16;                                                     // the cluster's ticket
 }
 
@@ -170,8 +174,9 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
   float4* stot = reinterpret_cast<float4*>(swsum + (kWT ? NW * CG : 0));              // [CG]
   float* stotw = reinterpret_cast<float*>(stot + CG);                                 // [CG]
   float4* sx = reinterpret_cast<float4*>(stotw + CG);                                 // [CG] incoming state
-  float* sxw = reinterpret_cast<float*>(sx + CG);                                     // [CG] (spare, keeps alignment)
-  uint32_t* sticket = reinterpret_cast<uint32_t*>(sxw + CG);
+  float* sxw = reinterpret_cast<float*>(sx + CG);                                     // [CG] their decay sum (kWT)
+  float4* sxl = reinterpret_cast<float4*>(sxw + CG);                                  // [CG] CTAs before this one
+  uint32_t* sticket = reinterpret_cast<uint32_t*>(sxl + CG);
 
   const int T = p.T, C = p.C;
   const int ncl = p.cluster;
@@ -185,7 +190,11 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
   int cl_id;
   if (nseg > 1) {
     if (rank == 0 && threadIdx.x == 0) *sticket = atomicAdd(&p.hdr->ticket, 1u);
-    cluster_arrive();
+    if (rank == 0 && wp == 0) {
+      cluster_arrive();  // (release: the ticket)
+    } else {
+      cluster_arrive_relaxed();
+    }
     cluster_wait();
     cl_id = (int)ld_dsmem_u32(map_shared_rank(sticket, 0));
     if (rank == 0 && threadIdx.x == 0) {
@@ -326,22 +335,37 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
     stotw[lane] = wtot;
   }
 
-  // the totals of the CTAs before this one in the segment
-  cluster_arrive();
+  // the totals of the CTAs before this one in the segment, read by warp 0
+  // for the whole CTA. Only the warp that wrote this CTA's total releases at
+  // the barrier, and in the first segment warp 0, whose read of the state in
+  // must come before the state out is written (it may alias); a release in
+  // every thread and remote reads in every warp: 364 against 348 us on the
+  // long workload, 1 x 65536 x 2048
+  if (wp == NW - 1 || (wp == 0 && seg == 0 && p.s_num)) {
+    cluster_arrive();
+  } else {
+    cluster_arrive_relaxed();
+  }
   cluster_wait();
   Acc xl = acc_empty();
   float xlw = 0.f;
-  for (int r = 0; r < rank; ++r) {
-    const Acc t = acc_unpack(ld_dsmem_f4(map_shared_rank(&stot[lane], (uint32_t)r)));
-    if (kWT) {
-      const float wr = ld_dsmem_f32(map_shared_rank(&stotw[lane], (uint32_t)r));
-      xl = combine_wt(xl, t, wr);
-      xlw += wr;
-    } else {
-      xl = combine(xl, t, (float)TPC, w);
+  if (wp == 0) {
+    for (int r = 0; r < rank; ++r) {
+      const Acc t = acc_unpack(ld_dsmem_f4(map_shared_rank(&stot[lane], (uint32_t)r)));
+      if (kWT) {
+        const float wr = ld_dsmem_f32(map_shared_rank(&stotw[lane], (uint32_t)r));
+        xl = combine_wt(xl, t, wr);
+        xlw += wr;
+      } else {
+        xl = combine(xl, t, (float)TPC, w);
+      }
     }
+    sxl[lane] = acc_pack(xl);
+    sxw[lane] = xlw;
   }
-  cluster_arrive();  // done with the other CTAs' shared memory
+  // done with the other CTAs' shared memory: warp 0's remote loads have
+  // returned (their values are stored above), so no release is needed
+  cluster_arrive_relaxed();
 
   // the segment's incoming state; the last CTA publishes the segment's
   // inclusive prefix for the next segment
@@ -366,6 +390,10 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 ? 3 : 6))
   }
   __syncthreads();
   const Acc X = acc_unpack(sx[lane]);
+  if (wp != 0) {
+    xl = acc_unpack(sxl[lane]);
+    xlw = sxw[lane];
+  }
   if (rank == ncl - 1 && seg < nseg - 1 && wp == 0) {
     // the inclusive prefix of this (full) segment: X, then the CTAs before
     // this one, then this CTA's total

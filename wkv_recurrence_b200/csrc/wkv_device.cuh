@@ -543,6 +543,7 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 // (the non-.aligned forms: callers need not be converged)
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
 // shared-memory address of the same variable in CTA `rank` of this cluster
 __device__ __forceinline__ uint32_t map_shared_rank(const void* p, uint32_t rank) {
   uint32_t r;
