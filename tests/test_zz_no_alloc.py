@@ -86,6 +86,21 @@ def test_noalloc_matches_oracle_on_calls_in_a_row(oracle):
                     f"noalloc call {call + 1} ({'misaligned' if misaligned else 'aligned'})")
 
 
+def test_noalloc_runs_the_cluster_scan(oracle):
+    """A shape whose k and v exceed L2 takes the cluster scan (16 chained
+    segments per channel group here), whose flags live in the scratch array
+    and are cleared by every call: two calls in a row, each against the
+    oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L = _abi.lib()
+    B, T, C = 1, 16384, 2048
+    assert W.forward_kernel(B, T, C) == 5
+    assert W.workspace_size(B, T, C) <= _abi.NOALLOC_SCRATCH_BYTES
+    for call in range(2):
+        _check_call(oracle, L, B, T, C, 700 + call, call == 0, False, f"noalloc cluster scan, call {call + 1}")
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
